@@ -1,0 +1,105 @@
+/*
+ * Sparse-BitLinear CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously-correct host implementation of what the
+ * Sparse-BitLinear operator computes.  Only the test suite, the smoke check
+ * and the benchmark's CPU-baseline leg may load it; the CUDA library never
+ * links, includes or calls it, and it shares no code with the CUDA path.
+ *
+ * Citation legend.  All pages summarise the paper "Sparse-BitNet: 1.58-bit
+ * LLMs are Naturally Friendly to Semi-Structured Sparsity" (arXiv 2603.05168):
+ *   [ja]   gist.science, Japanese technical summary
+ *   [de]   gist.science, German technical summary
+ *   [ko]   gist.science, Korean technical summary
+ *   [fr]   gist.science, French technical summary
+ *   [abs]  fugumt.com, the English abstract
+ * followed by the section number on that page.  Steps the pages leave open
+ * are taken in their plainest reading; each such reading is marked READING.
+ *
+ * All pointers are host pointers.  Weights, activations and gradients are
+ * bfloat16 passed as their raw uint16 bit patterns.  Matrices are row-major:
+ *   W  [n_out, k]   master weights (nn.Linear convention)
+ *   X  [t, k]       activations
+ *   dY [t, n_out]   upstream gradient
+ * Groups of m run along k inside one row of W.
+ */
+#ifndef SBL_ORACLE_H
+#define SBL_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A1 (absmean).  gamma = RN_fp32( sum|w| / numel ), the sum taken exactly over
+ * ALL master weights (quantisation happens before masking, [de] §2, [fr] §2).
+ * Returns the fp32 bit pattern of gamma; 0x7fc00000 (NaN) if any w is not
+ * finite; 0 for numel == 0. */
+uint32_t sbo_absmean_bits(const uint16_t* w, int64_t numel);
+
+/* g = max(gamma, 1e-5f): READING, the eps clamp of the absmean scale. */
+float sbo_clamped_scale(float gamma);
+
+/* A2 (N:M mask, [ja] §2.1, [de] §2, [ko] §2.1).  For each row and each group of
+ * m consecutive weights along k, keep the n largest |w| (bf16 magnitude, i.e.
+ * bits & 0x7fff), ties to the lowest index.  mask[row*(k/m) + grp] has bit j
+ * set when position j of the group is kept.  Requires k % m == 0, 1<=n<=m<=8. */
+void sbo_nm_mask(const uint16_t* w, int64_t n_out, int64_t k, int n, int m,
+                 uint8_t* mask);
+
+/* A3 (ternarise): q = round-half-even(clip(w/g, -1, 1)), which is
+ * sign(w) when 2|w| > g and 0 otherwise ([de] §1, [fr] §1 ternary set). */
+void sbo_ternary(const uint16_t* w, int64_t numel, float g, int8_t* q);
+
+/* A3 (quant-then-mask, [ja] §2.1, [de] §2, [ko] §2.1):  weff = q * mask. */
+void sbo_apply_mask(const int8_t* q, const uint8_t* mask, int64_t n_out,
+                    int64_t k, int m, int8_t* weff);
+
+/* Canonical 2:4 packing of weff with its mask ("explicit N:M metadata",
+ * [ja] §2.1).  vals[row, k/2]: the two kept codes of each group of four, in
+ * index order.  meta[row, k/8]: one nibble per group (i0 in bits 1:0, i1 in
+ * bits 3:2, i0 < i1), group 2j in the low nibble of byte j. */
+void sbo_pack24(const int8_t* weff, const uint8_t* mask, int64_t n_out,
+                int64_t k, int8_t* vals, uint8_t* meta);
+
+/* A4 (per-token int8 absmax; not on the pages, READING): a = max_k |x|,
+ * a' = max(a, 1e-5f), xq = sign(x) * rne(fl32(127|x|) / a'), clamped to
+ * [-128, 127]; a_prime[t] = a'.  All fp32 IEEE operations. */
+void sbo_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq,
+                   float* a_prime);
+
+/* A5: acc[ti, o] = sum_k xq[ti,k] * weff[o,k] in int64, stored as int32.
+ * Returns 0, or -1 if some |acc| >= 2^31 (never for |codes| <= 127, k < 2^24). */
+int sbo_gemm_acc(const int8_t* xq, const int8_t* weff, int64_t t,
+                 int64_t n_out, int64_t k, int32_t* acc);
+
+/* One element of A5, for sampled checks at full size. */
+int32_t sbo_acc_at(const int8_t* xq_row, const int8_t* weff_row, int64_t k);
+
+/* A6 (dequant): y = (float)acc * ((g * a'_t) / 127), fp32, in that order. */
+void sbo_dequant(const int32_t* acc, const float* a_prime, float g, int64_t t,
+                 int64_t n_out, float* y);
+
+/* A7 (STE, [ja] §2.1, [de] §2, [ko] §2.2):  dX = g * (dY . weff), fp64. */
+void sbo_grad_x(const uint16_t* dy, const int8_t* weff, float g, int64_t t,
+                int64_t n_out, int64_t k, double* dx);
+double sbo_grad_x_at(const uint16_t* dy, const int8_t* weff, float g,
+                     int64_t n_out, int64_t k, int64_t ti, int64_t ki);
+
+/* A8 (dense gradient flow to every master, [de] §2, [ko] §2.2, [fr] §2):
+ * dW = dY^T . X, fp64; pruned weights receive their gradient too. */
+void sbo_grad_w(const uint16_t* dy, const uint16_t* x, int64_t t,
+                int64_t n_out, int64_t k, double* dw);
+double sbo_grad_w_at(const uint16_t* dy, const uint16_t* x, int64_t t,
+                     int64_t n_out, int64_t k, int64_t oi, int64_t ki);
+
+/* Round fp64 to bf16 (round to nearest, ties to even), bit patterns out. */
+void sbo_round_bf16(const double* in, int64_t count, uint16_t* out);
+
+/* Number of OpenMP threads the oracle runs with. */
+int sbo_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,422 @@
+"""Pins for the CPU oracle (runs without a GPU).
+
+Each test checks one oracle function against something other than the
+oracle itself: hand-derived golden cases, exact rational arithmetic with
+Python's ``fractions``, closed-form statistics, numpy library routines or
+brute-force enumeration.  A plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong rounding direction) fails
+at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_linear_layers_bitlinear_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bf16_bits(values):
+    return synth.bits(torch.tensor(values, dtype=torch.float32).to(torch.bfloat16))
+
+
+def _bf16_float(bits_u16):
+    """Exact float value of bf16 bit patterns (via the fp32 pattern)."""
+    return (np.asarray(bits_u16, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Independent exact rounding helpers (rational arithmetic, no shared code).
+# ---------------------------------------------------------------------------
+def _rne(q: Fraction) -> int:
+    return round(q)  # Fraction.__round__ rounds half to even
+
+
+def _fraction_to_f32(q: Fraction) -> np.float32:
+    """Nearest-even fp32 of a non-negative rational, via exact arithmetic."""
+    assert q >= 0
+    if q == 0:
+        return np.float32(0.0)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    if Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    lsb = max(e - 23, -149)
+    n = _rne(q / Fraction(2) ** lsb)
+    return np.float32(math.ldexp(n, lsb))
+
+
+def _fraction_to_bf16_value(q: Fraction) -> float:
+    sign = -1.0 if q < 0 else 1.0
+    q = abs(q)
+    if q == 0:
+        return 0.0
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    if Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    lsb = max(e - 7, -133)
+    n = _rne(q / Fraction(2) ** lsb)
+    v = math.ldexp(n, lsb)
+    if v >= 2.0 ** 128:
+        return sign * math.inf
+    return sign * v
+
+
+def _exact_mean_f32(w_bits) -> np.float32:
+    vals = _bf16_float(w_bits).ravel()
+    s = sum((Fraction(abs(float(v))) for v in vals), Fraction(0))
+    return _fraction_to_f32(s / len(vals))
+
+
+# ---------------------------------------------------------------------------
+# A1: absmean scale
+# ---------------------------------------------------------------------------
+def test_gamma_golden_cases():
+    for case in _golden("gamma_cases.json")["cases"]:
+        w = _bf16_bits(case["w"])
+        gamma = oracle.absmean_gamma(w)
+        assert gamma == np.float32(case["gamma"]), case
+        assert oracle.clamped_scale(gamma) == np.float32(case["g"]), case
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_gamma_equals_exact_rational_mean(seed):
+    rng = np.random.default_rng(seed)
+    n = 3001 + 997 * seed
+    # Mix of scales, including subnormal bf16 magnitudes and large exponents,
+    # so that the exact sum spans far more than 53 bits.
+    bits = rng.integers(0, 0x7F80, size=n, dtype=np.uint32).astype(np.uint16)
+    bits |= (rng.integers(0, 2, size=n, dtype=np.uint32) << 15).astype(np.uint16)
+    if seed % 2:
+        bits[: n // 3] &= 0x807F  # subnormal and zero magnitudes
+    assert oracle.absmean_gamma(bits) == _exact_mean_f32(bits)
+
+
+@pytest.mark.parametrize("seed", [5, 6])
+def test_gamma_gaussian_weights_exact(seed):
+    w = synth.master_weights(64, 96, seed)
+    assert oracle.absmean_gamma(w) == _exact_mean_f32(synth.bits(w))
+
+
+def test_gamma_constant_magnitude():
+    for c in [1.0, 0.015625, 3.0e38, 2.0 ** -133, 2.0 ** -126, 0.3]:
+        vals = np.full(777, c, dtype=np.float32)
+        vals[::3] *= -1
+        w = _bf16_bits(vals)
+        c_bf16 = float(_bf16_float(w[:1])[0])
+        c_bf16 = abs(c_bf16)
+        assert float(oracle.absmean_gamma(w)) == float(np.float32(c_bf16))
+
+
+def test_gamma_underflow_to_fp32_subnormal_and_zero():
+    w = np.zeros(1 << 16, dtype=np.uint16)
+    w[7] = 0x0001  # 2^-133, the smallest bf16 subnormal
+    # exact mean 2^-149 is the smallest fp32 subnormal
+    assert oracle.absmean_gamma(w) == np.float32(2.0 ** -149)
+    w2 = np.zeros(1 << 17, dtype=np.uint16)
+    w2[3] = 0x0001  # mean 2^-150: a tie between 0 and 2^-149, even gives 0
+    assert oracle.absmean_gamma(w2) == np.float32(0.0)
+    w3 = np.zeros(1 << 17, dtype=np.uint16)
+    w3[3] = 0x0001
+    w3[4] = 0x0001  # 2^-149 exactly
+    assert oracle.absmean_gamma(w3) == np.float32(2.0 ** -149)
+    assert oracle.clamped_scale(np.float32(0.0)) == np.float32(1e-5)
+
+
+def test_gamma_nonfinite_is_nan():
+    w = _bf16_bits([1.0, float("inf"), 2.0])
+    assert np.isnan(oracle.absmean_gamma(w))
+    w = _bf16_bits([1.0, float("nan")])
+    assert np.isnan(oracle.absmean_gamma(w))
+
+
+def test_gamma_gaussian_statistic():
+    # E|w| = sigma * sqrt(2/pi) for w ~ N(0, sigma^2); standard error of the
+    # mean is sigma * sqrt(1 - 2/pi) / sqrt(n).
+    w = synth.master_weights(1024, 1024, seed=11)
+    n = w.numel()
+    expect = 0.02 * math.sqrt(2 / math.pi)
+    se = 0.02 * math.sqrt(1 - 2 / math.pi) / math.sqrt(n)
+    assert abs(float(oracle.absmean_gamma(w)) - expect) < 6 * se + 1e-5 * expect
+
+
+# ---------------------------------------------------------------------------
+# A2: N:M mask
+# ---------------------------------------------------------------------------
+def test_mask_golden_cases():
+    for case in _golden("mask_cases.json")["cases"]:
+        w = _bf16_bits(case["w"]).reshape(1, -1)
+        mask = oracle.nm_mask(w, case["n"], case["m"])
+        assert int(mask[0, 0]) == case["mask"], case
+
+
+def _brute_force_mask(mags, n):
+    """The kept set is the unique size-n subset whose every member beats every
+    non-member under (magnitude descending, index ascending)."""
+    m = len(mags)
+    winners = []
+    for subset in itertools.combinations(range(m), n):
+        s = set(subset)
+        ok = all(
+            (mags[i] > mags[j]) or (mags[i] == mags[j] and i < j)
+            for i in s
+            for j in range(m)
+            if j not in s
+        )
+        if ok:
+            winners.append(subset)
+    assert len(winners) == 1
+    return sum(1 << i for i in winners[0])
+
+
+@pytest.mark.parametrize("n,m", [(1, 2), (2, 4), (1, 4), (3, 4), (6, 8), (4, 8), (3, 8), (2, 8), (5, 8)])
+def test_mask_brute_force(n, m):
+    rng = np.random.default_rng(100 * n + m)
+    rows, groups = 9, 13
+    # Draw from a small set of values so that ties (and +-0) are frequent.
+    pool = np.array([0.0, -0.0, 0.5, -0.5, 0.25, 1.0, -1.0, 0.125, 2.0], dtype=np.float32)
+    vals = pool[rng.integers(0, len(pool), size=rows * groups * m)].reshape(rows, groups * m)
+    w = _bf16_bits(vals)
+    mask = oracle.nm_mask(w, n, m)
+    mags = np.abs(_bf16_float(w))
+    for r in range(rows):
+        for g in range(groups):
+            want = _brute_force_mask(list(mags[r, g * m:(g + 1) * m]), n)
+            assert int(mask[r, g]) == want
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (4, 8), (8, 8)])
+def test_mask_invariants_gaussian(n, m):
+    w = synth.master_weights(40, 64, seed=3)
+    wb = synth.bits(w)
+    mask = oracle.nm_mask(wb, n, m)
+    mags = np.abs(_bf16_float(wb))
+    for r in range(wb.shape[0]):
+        for g in range(wb.shape[1] // m):
+            bits = int(mask[r, g])
+            kept = [j for j in range(m) if bits >> j & 1]
+            dropped = [j for j in range(m) if not bits >> j & 1]
+            assert len(kept) == n
+            grp = mags[r, g * m:(g + 1) * m]
+            for i in kept:
+                for j in dropped:
+                    assert grp[i] > grp[j] or (grp[i] == grp[j] and i < j)
+
+
+# ---------------------------------------------------------------------------
+# A3: ternary codes, quant-then-mask, packing
+# ---------------------------------------------------------------------------
+def test_ternary_golden_cases():
+    gold = _golden("ternary_cases.json")
+    w = _bf16_bits([c["w"] for c in gold["cases"]])
+    q = oracle.ternary(w, np.float32(gold["g"]))
+    assert list(q) == [c["q"] for c in gold["cases"]]
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_ternary_equals_rational_round_clip(seed):
+    w = synth.master_weights(32, 80, seed)
+    wb = synth.bits(w)
+    g = oracle.clamped_scale(oracle.absmean_gamma(wb))
+    q = oracle.ternary(wb, g)
+    gq = Fraction(float(g))
+    vals = _bf16_float(wb).ravel()
+    for v, code in zip(vals, q.ravel()):
+        r = Fraction(float(v)) / gq
+        r = max(Fraction(-1), min(Fraction(1), r))
+        assert _rne(r) == int(code)
+    # exact boundary |w| = g/2 maps to 0, just above maps to sign(w)
+    g2 = np.float32(0.03125)
+    wb2 = _bf16_bits([0.015625, -0.015625, 0.0157470703125, -0.0157470703125])
+    assert list(oracle.ternary(wb2, g2)) == [0, 0, 1, -1]
+
+
+def test_ternary_zero_fraction_closed_form():
+    # P(|w| <= g/2) for w ~ N(0, s^2) with g = s*sqrt(2/pi) is 2*Phi(sqrt(2/pi)/2) - 1.
+    w = synth.master_weights(1024, 1024, seed=21)
+    wb = synth.bits(w)
+    g = oracle.clamped_scale(oracle.absmean_gamma(wb))
+    q = oracle.ternary(wb, g)
+    z = math.sqrt(2 / math.pi) / 2
+    p = math.erf(z / math.sqrt(2))  # = 2*Phi(z) - 1
+    frac = float(np.mean(q == 0))
+    se = math.sqrt(p * (1 - p) / q.size)
+    assert abs(frac - p) < 6 * se + 2e-3, (frac, p)
+    assert abs(p - 0.3101) < 1e-3
+
+
+def test_quant_then_mask_and_dense_limit():
+    w = synth.master_weights(24, 64, seed=7)
+    for n, m in [(2, 4), (6, 8), (4, 8)]:
+        p = oracle.prepare(w, n, m)
+        q, mask, weff = p["q"], p["mask"], p["weff"]
+        expand = np.repeat(mask, m, axis=1)
+        pos = np.tile(np.arange(m), mask.shape[1])
+        kept = (expand >> pos) & 1
+        assert np.array_equal(weff, q * kept)
+        assert set(np.unique(weff)).issubset({-1, 0, 1})
+        # at most n non-zeros per group of m
+        nz = (weff != 0).reshape(weff.shape[0], -1, m).sum(-1)
+        assert nz.max() <= n
+    # N = M is plain ternary BitLinear: the mask keeps every weight
+    p = oracle.prepare(w, 4, 4)
+    assert np.array_equal(p["weff"], p["q"])
+
+
+def test_pack24_round_trip():
+    w = synth.master_weights(16, 64, seed=9)
+    p = oracle.prepare(w, 2, 4)
+    vals, meta = oracle.pack24(p["weff"], p["mask"])
+    rebuilt = np.zeros_like(p["weff"])
+    for r in range(16):
+        for g in range(16):
+            byte = int(meta[r, g // 2])
+            nib = (byte >> (4 * (g % 2))) & 0xF
+            i0, i1 = nib & 3, nib >> 2
+            assert i0 < i1
+            assert int(p["mask"][r, g]) == (1 << i0) | (1 << i1)
+            rebuilt[r, 4 * g + i0] = vals[r, 2 * g]
+            rebuilt[r, 4 * g + i1] = vals[r, 2 * g + 1]
+    assert np.array_equal(rebuilt, p["weff"])
+
+
+# ---------------------------------------------------------------------------
+# A4: activation quantisation
+# ---------------------------------------------------------------------------
+def test_act_quant_golden_cases():
+    for case in _golden("act_quant_cases.json")["cases"]:
+        x = _bf16_bits(case["x"]).reshape(1, -1)
+        xq, ap = oracle.act_quant(x)
+        assert list(xq[0]) == case["xq"], case
+        assert ap[0] == np.float32(case["a_prime"]), case
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_act_quant_equals_rational_rne(seed):
+    x = synth.activations(6, 200, seed)
+    xb = synth.bits(x)
+    xq, ap = oracle.act_quant(xb)
+    vals = _bf16_float(xb)
+    for r in range(vals.shape[0]):
+        a = max(abs(float(v)) for v in vals[r])
+        assert ap[r] == np.float32(max(a, np.float32(1e-5)))
+        A = Fraction(a)
+        for v, code in zip(vals[r], xq[r]):
+            n = _rne(127 * abs(Fraction(float(v))) / A)
+            n = min(n, 127)
+            want = -n if v < 0 else n
+            assert int(code) == want
+        assert np.max(np.abs(xq[r])) == 127  # the argmax element maps to +-127
+
+
+# ---------------------------------------------------------------------------
+# A5 / A6: integer product and dequant
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("t,n_out,k", [(1, 8, 16), (5, 12, 64), (17, 33, 96)])
+def test_gemm_acc_equals_numpy_int64(t, n_out, k):
+    rng = np.random.default_rng(t + n_out + k)
+    xq = rng.integers(-127, 128, size=(t, k), dtype=np.int64).astype(np.int8)
+    weff = rng.integers(-1, 2, size=(n_out, k), dtype=np.int64).astype(np.int8)
+    acc = oracle.gemm_acc(xq, weff)
+    ref = xq.astype(np.int64) @ weff.astype(np.int64).T
+    assert np.array_equal(acc.astype(np.int64), ref)
+    assert oracle.acc_at(xq, weff, t - 1, n_out - 1) == int(ref[-1, -1])
+
+
+def test_gemm_acc_extreme_range():
+    # |acc| = 127 * k at the extremes: no int32 overflow for realistic k
+    k = 8192
+    xq = np.full((2, k), 127, dtype=np.int8)
+    xq[1] = -127
+    weff = np.ones((3, k), dtype=np.int8)
+    weff[1] = -1
+    weff[2] = 0
+    acc = oracle.gemm_acc(xq, weff)
+    assert acc.tolist() == [[127 * k, -127 * k, 0], [-127 * k, 127 * k, 0]]
+
+
+def test_dequant_within_three_roundings_of_exact():
+    rng = np.random.default_rng(4)
+    acc = rng.integers(-400000, 400000, size=(7, 11), dtype=np.int64).astype(np.int32)
+    ap = rng.uniform(0.5, 6.0, size=7).astype(np.float32)
+    g = np.float32(0.0159)
+    y = oracle.dequant(acc, ap, g)
+    u = 2.0 ** -24
+    for i in range(7):
+        for j in range(11):
+            exact = Fraction(int(acc[i, j])) * Fraction(float(g)) * Fraction(float(ap[i])) / 127
+            err = abs(Fraction(float(y[i, j])) - exact)
+            assert err <= Fraction(4 * u) * abs(exact)
+    # g * a' = 127 makes the scale exactly 1
+    y1 = oracle.dequant(np.array([[254, -3, 0]], dtype=np.int32), np.array([127.0], np.float32), 1.0)
+    assert y1.tolist() == [[254.0, -3.0, 0.0]]
+
+
+def test_forward_end_to_end_small():
+    w = synth.master_weights(8, 32, seed=1)
+    x = synth.activations(3, 32, seed=2)
+    out = oracle.forward(w, x, 2, 4)
+    ref = out["xq"].astype(np.int64) @ out["weff"].astype(np.int64).T
+    assert np.array_equal(out["acc"], ref)
+    scale = (np.float32(out["g"]) * out["a_prime"]) / np.float32(127)
+    assert np.allclose(out["y"], ref * scale[:, None], rtol=1e-6, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# A7 / A8: STE gradients
+# ---------------------------------------------------------------------------
+def test_grad_x_equals_numpy_matmul():
+    w = synth.master_weights(24, 48, seed=3)
+    dy = synth.upstream_grad(5, 24, seed=4)
+    p = oracle.prepare(w, 2, 4)
+    dx = oracle.grad_x(dy, p["weff"], p["g"])
+    ref = float(p["g"]) * (_bf16_float(synth.bits(dy)) @ p["weff"].astype(np.float64))
+    assert np.allclose(dx, ref, rtol=1e-12, atol=1e-12)
+    assert math.isclose(oracle.grad_x_at(dy, p["weff"], p["g"], 4, 47), ref[4, 47], rel_tol=1e-12, abs_tol=1e-12)
+    # the gradient ignores pruned weights: changing a pruned code changes nothing
+    assert dx.shape == (5, 48)
+
+
+def test_grad_w_equals_numpy_matmul_and_is_dense():
+    dy = synth.upstream_grad(9, 20, seed=5)
+    x = synth.activations(9, 36, seed=6)
+    dw = oracle.grad_w(dy, x)
+    ref = _bf16_float(synth.bits(dy)).T @ _bf16_float(synth.bits(x))
+    assert np.allclose(dw, ref, rtol=1e-12, atol=1e-12)
+    assert math.isclose(oracle.grad_w_at(dy, x, 19, 35), ref[19, 35], rel_tol=1e-12, abs_tol=1e-12)
+    # dense gradient flow: every master weight gets a gradient, including pruned ones
+    assert np.count_nonzero(dw) == dw.size
+
+
+def test_round_bf16_matches_rational_rounding():
+    rng = np.random.default_rng(8)
+    vals = np.concatenate([
+        rng.normal(size=500) * 10.0 ** rng.integers(-40, 38, size=500),
+        np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -134, 3 * 2.0 ** -135,
+                  2.0 ** -140, 3.4e38, 3.3961e38, 0.0, -0.0]),
+    ])
+    out = oracle.round_bf16(vals)
+    got = _bf16_float(out)
+    for v, gv, b in zip(vals, got, out):
+        want = _fraction_to_bf16_value(Fraction(float(v)))
+        if math.isinf(want):
+            assert (int(b) & 0x7FFF) == 0x7F80
+        else:
+            assert gv == want, (v, gv, want)
+    # ties go to even
+    assert got[500] == 1.0 and got[501] == 1.0 + 2.0 ** -6 and got[502] == -1.0
