@@ -1,0 +1,183 @@
+/*
+ * sbl.h -- C ABI of the Sparse-BitLinear library for NVIDIA B200 (sm_100a).
+ *
+ * Sparse-BitLinear is the linear layer of Sparse-BitNet ("Sparse-BitNet:
+ * 1.58-bit LLMs are Naturally Friendly to Semi-Structured Sparsity",
+ * arXiv 2603.05168).  Citations below name the page and section:
+ *   [ja]  gist.science Japanese technical summary
+ *   [de]  gist.science German technical summary
+ *   [ko]  gist.science Korean technical summary
+ *   [fr]  gist.science French technical summary
+ *   [abs] fugumt.com English abstract
+ *
+ * The layer keeps bf16 master weights W [n_out, k] (row-major, nn.Linear
+ * convention).  Every step ([ja] 2.1, [ko] 2.2 "dynamic mask recompute") it
+ *   1. quantises all masters to ternary codes {-1, 0, +1} with the per-tensor
+ *      absmean scale g ([de] 1, [fr] 1),
+ *   2. recomputes an N:M mask from the master magnitudes: in each group of m
+ *      consecutive weights along k keep the n largest |w|, ties to the lowest
+ *      index ([ja] 2.1, [de] 2 "Maskengenerierung", [ko] 2.1),
+ *   3. applies the mask after quantisation, W_eff = q * mask ([de] 2
+ *      "Quant-then-Mask", [fr] 2),
+ *   4. quantises activations per token to int8 with absmax, multiplies them
+ *      with W_eff in int32 and rescales to fp32,
+ *   5. in the backward pass uses the dual straight-through estimator: dX goes
+ *      through the masked, scaled ternary weights and dW = dY^T X reaches
+ *      every master weight, pruned ones included ([de] 2 "Dual STE",
+ *      [ko] 2.2, [fr] 2 "Flot de Gradient Dense").
+ *
+ * Conventions for every entry point:
+ *  - Tensor arguments are DEVICE pointers on the current CUDA device, 16-byte
+ *    aligned, row-major and dense.  bf16 data is passed as `const void*`.
+ *  - The caller owns and allocates every buffer (cudaMalloc, torch, ...).  The
+ *    library allocates no device memory and keeps no state between calls.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Calls do not synchronise, except sbl_read_status.
+ *  - Arguments are validated before anything is enqueued; a rejected call
+ *    returns an error code and enqueues nothing.
+ *  - Errors that only the device can see (non-finite inputs, a bounded wait
+ *    that ran out) are OR-ed into the status word inside the prepared blob and
+ *    reported by sbl_read_status.  Outputs of a call that raised a device
+ *    error are unspecified.
+ */
+#ifndef SBL_H
+#define SBL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* sbl_stream_t;
+
+typedef enum sbl_status {
+  SBL_OK = 0,
+  SBL_ERR_INVALID_ARG = 1,    /* null pointer, negative size, unknown flag bit */
+  SBL_ERR_UNSUPPORTED_NM = 2, /* m not in {2, 4, 8}, or n < 1, or n > m */
+  SBL_ERR_SHAPE = 3,          /* k % 64 != 0, n_out % 8 != 0, n_out < 8, sizes too large */
+  SBL_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
+  SBL_ERR_CUDA = 5,           /* a CUDA call failed (launch error, no device, ...) */
+  SBL_ERR_NONFINITE = 6,      /* device saw a NaN/Inf master weight or activation */
+  SBL_ERR_TIMEOUT = 7,        /* a device-side bounded wait gave up */
+  SBL_ERR_DEVICE = 8          /* the current device is not sm_100 */
+} sbl_status;
+
+/* Flags of sbl_layer.flags (fixed at prepare time). */
+enum {
+  SBL_PACK_GEMV = 1u << 0 /* also write the 2-bit decode packing (2:4 only) */
+};
+
+/* Flags of sbl_backward's `flags` argument. */
+enum {
+  SBL_GRAD_F32 = 1u << 1, /* dx and dw are fp32 instead of bf16 */
+  SBL_NO_DX = 1u << 2,    /* skip dX (dx may be NULL) */
+  SBL_NO_DW = 1u << 3     /* skip dW (dw may be NULL) */
+};
+
+/* One Sparse-BitLinear layer: shapes, pattern and the caller-owned device
+ * blob that sbl_prepare_weights fills.  Plain data, no hidden state. */
+typedef struct sbl_layer {
+  int64_t n_out;   /* output features = rows of W; multiple of 8 */
+  int64_t k;       /* input features = columns of W; multiple of 64 */
+  int32_t n, m;    /* keep n of every m consecutive weights along k */
+  uint32_t flags;  /* SBL_PACK_* bits */
+  void* prepared;  /* device buffer of sbl_prepared_bytes() bytes, 256-byte aligned */
+} sbl_layer;
+
+/* Byte offsets of the sections inside the prepared blob (0 = absent). */
+typedef struct sbl_blob_layout {
+  uint64_t total_bytes;
+  uint64_t header;      /* 4096-byte header: shapes, gamma, g, status word, scratch */
+  uint64_t mask;        /* uint8 [n_out, k/m]: bit j = position j of the group kept */
+  uint64_t codes;       /* int8 [n_out, k]: W_eff codes (patterns other than 2:4) */
+  uint64_t weff_bf16;   /* bf16 [n_out, k]: W_eff as exact bf16 {-1, 0, 1} (backward) */
+  uint64_t sp_values;   /* int8 [n_out, k/2]: the two kept codes of each group of 4 (2:4) */
+  uint64_t sp_meta;     /* tensor-core metadata (2:4), sp_meta_bytes bytes; see below */
+  uint64_t sp_meta_bytes;
+  uint64_t gemv;        /* uint8 [n_out, k/4]: 2-bit decode packing (SBL_PACK_GEMV) */
+  uint64_t gamma;       /* float: exact absmean, rounded to fp32 */
+  uint64_t g;           /* float: max(gamma, 1e-5), the scale used everywhere */
+  uint64_t status;      /* uint32 device status word */
+} sbl_blob_layout;
+/* sp_meta layout: blocks of 128 rows x 128 k-positions, 2048 bytes each,
+ * ordered [row_block][k_block]; inside a block, row r's 16 bytes hold 32
+ * nibbles for its 32 groups of four in k order (group 2j in the low nibble
+ * of byte j); a nibble is (i0 | i1 << 2) with i0 < i1 the kept positions.
+ * Rows and k are padded up to 128 and 256 with nibble 0x4 over zero codes.
+ * gemv layout: one byte per group of four: the metadata nibble in the high
+ * half, the two kept codes in the low half (bits 1:0 the code at i0, bits 3:2
+ * the code at i1; 00 = 0, 01 = +1, 11 = -1). */
+
+/* Size and section offsets of the prepared blob.  Host only, no CUDA call.
+ * Returns SBL_ERR_* on unsupported shapes/patterns (out is then untouched). */
+sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t flags,
+                               sbl_blob_layout* out);
+
+/* Total bytes of the prepared blob, 0 for unsupported arguments. */
+size_t sbl_prepared_bytes(int64_t n_out, int64_t k, int n, int m, uint32_t flags);
+
+/* Bytes of scratch that sbl_forward needs when xq_out / xscale_out are NULL:
+ * t*k int8 codes plus t fp32 scales (256-byte aligned pieces). */
+size_t sbl_workspace_bytes(int64_t t, int64_t k);
+
+/* Steps 1-3 ([de] 2, [ja] 2.1, [ko] 2.1-2.2).  Reads the bf16 masters
+ * `w_master` [n_out, k] and fills layer->prepared: the exact absmean gamma
+ * (sum of all |w| computed exactly, rounded once to fp32), g = max(gamma,
+ * 1e-5), the N:M mask from the master magnitudes, the ternary codes
+ * q = sign(w) * [2|w| > g] with the mask applied after quantisation, and
+ * the packed forms the forward and backward kernels read.  Resets the blob's
+ * status word.  Raises SBL_ERR_NONFINITE (device) for NaN/Inf masters. */
+sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl_stream_t stream);
+
+/* Step 4.  x: bf16 [t, k] activations.  y: fp32 [t, n_out] output,
+ *   y[i, o] = (float)acc[i, o] * ((g * a'_i) / 127),
+ *   acc[i, o] = sum_k xq[i, k] * W_eff[o, k]   (int32),
+ *   a'_i = max(max_k |x[i, k]|, 1e-5),  xq = sign(x) * rne(127 |x| / a'_i).
+ * xq_out (int8 [t, k]) and xscale_out (fp32 [t], receives a'_i) may be NULL;
+ * then `workspace` (sbl_workspace_bytes(t, k) bytes) holds them.  acc_debug
+ * (int32 [t, n_out]) may be NULL; when given, the raw accumulators are
+ * written too.  t == 0 is a no-op.  2:4 layers run the 2:4-sparse int8
+ * tensor-core GEMM; other patterns the dense int8 one over W_eff codes. */
+sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
+                       float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
+
+/* Step 5 (dual STE).  x: bf16 [t, k] (the forward input), dy: bf16 [t, n_out].
+ *   dx [t, k]     = g * (dy . W_eff)          (straight through Q_w, Q_x, mask)
+ *   dw [n_out, k] = dy^T . x                  (dense: every master, pruned too)
+ * bf16 outputs (fp32 with SBL_GRAD_F32), fp32 accumulation on the tensor
+ * cores.  SBL_NO_DX / SBL_NO_DW skip one of the two products. */
+sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
+                        uint32_t flags, sbl_stream_t stream);
+
+/* Synchronises `stream`, then maps the layer's device status word to a code:
+ * SBL_OK, SBL_ERR_NONFINITE or SBL_ERR_TIMEOUT.  *bits_out (may be NULL)
+ * receives the raw word.  The word stays set until sbl_clear_status or the
+ * next sbl_prepare_weights. */
+sbl_status sbl_read_status(const sbl_layer* layer, sbl_stream_t stream, uint32_t* bits_out);
+sbl_status sbl_clear_status(const sbl_layer* layer, sbl_stream_t stream);
+
+/* Copies the fp32 gamma and g of a prepared layer to the host (synchronises). */
+sbl_status sbl_read_scale(const sbl_layer* layer, sbl_stream_t stream, float* gamma_out, float* g_out);
+
+/* Failure-path self test: launches one CTA whose mbarrier wait can never
+ * complete, bounded by `limit_ns`; the kernel then records SBL_STATUS_TIMEOUT
+ * in *status_dev (device uint32) and returns normally.  No fault, no hang. */
+sbl_status sbl_selftest_wait_timeout(uint32_t* status_dev, uint64_t limit_ns, sbl_stream_t stream);
+
+/* Bits of the device status word. */
+enum {
+  SBL_STATUS_NONFINITE_W = 1u << 0,
+  SBL_STATUS_NONFINITE_X = 1u << 1,
+  SBL_STATUS_TIMEOUT = 1u << 2
+};
+
+/* Library version string. */
+const char* sbl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SBL_H */

@@ -1,0 +1,256 @@
+// C ABI of the Sparse-BitLinear library: argument checks, prepared-blob
+// layout and dispatch to the kernels.  See include/sbl.h for the contract.
+#include <cstddef>
+#include <cstring>
+#include <mutex>
+
+#include "sbl_kernels.h"
+
+using namespace sbl;
+
+namespace {
+
+constexpr int64_t kMaxK = 131072;  // keeps |acc| <= 127 * k below 2^24: (float)acc is exact
+constexpr uint32_t kLayerFlags = SBL_PACK_GEMV;
+constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW;
+
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int num_sms = 0;
+};
+
+DeviceInfo g_devices[64];
+std::mutex g_dev_mutex;
+
+// Current device must be sm_100 (B200).  Cached per device ordinal.
+sbl_status current_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SBL_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.checked) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SBL_ERR_CUDA;
+    d.ok = (prop.major == 10 && prop.minor == 0);
+    d.num_sms = prop.multiProcessorCount;
+    d.checked = true;
+  }
+  if (!d.ok) return SBL_ERR_DEVICE;
+  *num_sms = d.num_sms;
+  return SBL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sbl_status check_shape(int64_t n_out, int64_t k, int n, int m, uint32_t flags) {
+  if ((flags & ~kLayerFlags) != 0u) return SBL_ERR_INVALID_ARG;
+  if (!(m == 2 || m == 4 || m == 8) || n < 1 || n > m) return SBL_ERR_UNSUPPORTED_NM;
+  if ((flags & SBL_PACK_GEMV) && !(n == 2 && m == 4)) return SBL_ERR_UNSUPPORTED_NM;
+  if (n_out < 8 || n_out % 8 != 0 || k < 64 || k % 64 != 0) return SBL_ERR_SHAPE;
+  if (k > kMaxK || n_out > (int64_t(1) << 30) || n_out * k > (int64_t(1) << 40)) return SBL_ERR_SHAPE;
+  return SBL_OK;
+}
+
+bool is_24(int n, int m) { return n == 2 && m == 4; }
+
+sbl_status check_layer(const sbl_layer* layer, sbl_blob_layout* L) {
+  if (layer == nullptr || layer->prepared == nullptr) return SBL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(layer->prepared) & 255u) != 0) return SBL_ERR_ALIGN;
+  return sbl_prepared_layout(layer->n_out, layer->k, layer->n, layer->m, layer->flags, L);
+}
+
+template <class T>
+T* at(const sbl_layer* layer, uint64_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(layer->prepared) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sbl_version(void) { return "sbl 0.1 (sm_100a)"; }
+
+sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t flags, sbl_blob_layout* out) {
+  if (out == nullptr) return SBL_ERR_INVALID_ARG;
+  const sbl_status st = check_shape(n_out, k, n, m, flags);
+  if (st != SBL_OK) return st;
+  sbl_blob_layout L;
+  std::memset(&L, 0, sizeof(L));
+  uint64_t off = 0;
+  L.header = off;
+  off += kHeaderBytes;
+  auto take = [&](uint64_t bytes) {
+    const uint64_t at_off = off;
+    off = align_up(off + bytes, 256);
+    return at_off;
+  };
+  L.mask = take(uint64_t(n_out) * uint64_t(k / m));
+  L.weff_bf16 = take(uint64_t(n_out) * uint64_t(k) * 2);
+  if (is_24(n, m)) {
+    L.sp_values = take(uint64_t(n_out) * uint64_t(k / 2));
+    L.sp_meta_bytes = uint64_t(meta_rows_padded(n_out)) * uint64_t(meta_k_padded(k) / 8);
+    L.sp_meta = take(L.sp_meta_bytes);
+    if (flags & SBL_PACK_GEMV) L.gemv = take(uint64_t(n_out) * uint64_t(k / 4));
+  } else {
+    L.codes = take(uint64_t(n_out) * uint64_t(k));
+  }
+  L.total_bytes = off;
+  L.gamma = L.header + offsetof(BlobHeader, gamma);
+  L.g = L.header + offsetof(BlobHeader, g);
+  L.status = L.header + offsetof(BlobHeader, status);
+  *out = L;
+  return SBL_OK;
+}
+
+size_t sbl_prepared_bytes(int64_t n_out, int64_t k, int n, int m, uint32_t flags) {
+  sbl_blob_layout L;
+  if (sbl_prepared_layout(n_out, k, n, m, flags, &L) != SBL_OK) return 0;
+  return static_cast<size_t>(L.total_bytes);
+}
+
+size_t sbl_workspace_bytes(int64_t t, int64_t k) {
+  if (t < 0 || k < 0) return 0;
+  return static_cast<size_t>(align_up(uint64_t(t) * uint64_t(k), 256) + align_up(uint64_t(t) * 4, 256));
+}
+
+sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (w_master == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(w_master)) return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  const cudaError_t e =
+      launch_prepare(static_cast<const uint16_t*>(w_master), layer->n_out, layer->k, layer->n, layer->m, layer->flags,
+                     static_cast<uint8_t*>(layer->prepared), L, sms, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out, float* xscale_out,
+                       int32_t* acc_debug, void* workspace, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (t < 0 || t > (int64_t(1) << 30)) return SBL_ERR_SHAPE;
+  if (t == 0) return SBL_OK;
+  if (x == nullptr || y == nullptr) return SBL_ERR_INVALID_ARG;
+  int8_t* xq = xq_out;
+  float* ap = xscale_out;
+  if (xq == nullptr || ap == nullptr) {
+    if (workspace == nullptr) return SBL_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SBL_ERR_ALIGN;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (xq == nullptr) xq = reinterpret_cast<int8_t*>(ws);
+    if (ap == nullptr) ap = reinterpret_cast<float*>(ws + align_up(uint64_t(t) * uint64_t(layer->k), 256));
+  }
+  if (!aligned16(x) || !aligned16(y) || !aligned16(xq) || !aligned16(ap) || !aligned16(acc_debug))
+    return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(layer, L.status);
+  const float* g = at<const float>(layer, L.g);
+  cudaError_t e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s);
+  if (e != cudaSuccess) return SBL_ERR_CUDA;
+  if (L.gemv != 0 && t <= 16) {
+    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), xq, ap, g, layer->n_out, t, layer->k, y, acc_debug, sms,
+                            s);
+  } else if (is_24(layer->n, layer->m)) {
+    e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
+                            static_cast<int>(meta_k_padded(layer->k) / 128), xq, ap, g, layer->n_out, t, layer->k, y,
+                            acc_debug, status, sms, s);
+  } else {
+    e = launch_forward_gemm(false, at<const int8_t>(layer, L.codes), nullptr, 0, xq, ap, g, layer->n_out, t, layer->k,
+                            y, acc_debug, status, sms, s);
+  }
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
+                        uint32_t flags, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if ((flags & ~kBackwardFlags) != 0u) return SBL_ERR_INVALID_ARG;
+  if (t < 0 || t > (int64_t(1) << 30)) return SBL_ERR_SHAPE;
+  const bool want_dx = !(flags & SBL_NO_DX), want_dw = !(flags & SBL_NO_DW);
+  const bool f32 = (flags & SBL_GRAD_F32) != 0u;
+  if ((want_dx && dx == nullptr) || (want_dw && dw == nullptr)) return SBL_ERR_INVALID_ARG;
+  if (t > 0 && ((want_dx || want_dw) && dy == nullptr)) return SBL_ERR_INVALID_ARG;
+  if (t > 0 && want_dw && x == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(dw)) return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t esize = f32 ? 4 : 2;
+  if (t == 0) {  // empty batch: dX is empty and dW = 0
+    if (want_dw && cudaMemsetAsync(dw, 0, size_t(layer->n_out) * size_t(layer->k) * esize, s) != cudaSuccess)
+      return SBL_ERR_CUDA;
+    return SBL_OK;
+  }
+  uint32_t* status = at<uint32_t>(layer, L.status);
+  if (want_dx) {
+    // dX[t, k] = g * dY[t, n_out] . W_eff[n_out, k]:  A = dY (K-major), B = W_eff stored [K][N].
+    const cudaError_t e = launch_bf16_gemm(false, true, f32, static_cast<const uint16_t*>(dy),
+                                           at<const uint16_t>(layer, L.weff_bf16), t, layer->k, layer->n_out,
+                                           at<const float>(layer, L.g), dx, status, sms, s);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+  }
+  if (want_dw) {
+    // dW[n_out, k] = dY^T . X:  A = dY stored [K=t][M=n_out], B = X stored [K=t][N=k].
+    const cudaError_t e = launch_bf16_gemm(true, true, f32, static_cast<const uint16_t*>(dy),
+                                           static_cast<const uint16_t*>(x), layer->n_out, layer->k, t, nullptr, dw,
+                                           status, sms, s);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+  }
+  return SBL_OK;
+}
+
+sbl_status sbl_read_status(const sbl_layer* layer, sbl_stream_t stream, uint32_t* bits_out) {
+  sbl_blob_layout L;
+  const sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t bits = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SBL_ERR_CUDA;
+  if (cudaMemcpy(&bits, at<uint32_t>(layer, L.status), 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SBL_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  if (bits & SBL_STATUS_TIMEOUT) return SBL_ERR_TIMEOUT;
+  if (bits & (SBL_STATUS_NONFINITE_W | SBL_STATUS_NONFINITE_X)) return SBL_ERR_NONFINITE;
+  return SBL_OK;
+}
+
+sbl_status sbl_clear_status(const sbl_layer* layer, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  const sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  return cudaMemsetAsync(at<uint32_t>(layer, L.status), 0, 4, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SBL_OK
+             : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_read_scale(const sbl_layer* layer, sbl_stream_t stream, float* gamma_out, float* g_out) {
+  sbl_blob_layout L;
+  const sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SBL_ERR_CUDA;
+  float v[2];
+  if (cudaMemcpy(v, at<float>(layer, L.gamma), 8, cudaMemcpyDeviceToHost) != cudaSuccess) return SBL_ERR_CUDA;
+  if (gamma_out) *gamma_out = v[0];
+  if (g_out) *g_out = v[1];
+  return SBL_OK;
+}
+
+sbl_status sbl_selftest_wait_timeout(uint32_t* status_dev, uint64_t limit_ns, sbl_stream_t stream) {
+  if (status_dev == nullptr) return SBL_ERR_INVALID_ARG;
+  int sms = 0;
+  const sbl_status st = current_device(&sms);
+  if (st != SBL_OK) return st;
+  return launch_selftest_wait(status_dev, limit_ns, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SBL_OK
+             : SBL_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,53 @@
+// Host-side launchers of the Sparse-BitLinear kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sbl_internal.h"
+
+namespace sbl {
+
+// Destinations of the pack pass (device pointers; optional ones may be null).
+struct PackOut {
+  uint8_t* mask;
+  int8_t* codes;
+  uint16_t* weff_bf16;
+  int8_t* sp_values;
+  uint8_t* sp_meta;
+  uint8_t* gemv;
+  int meta_kblocks;
+};
+
+cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags, uint8_t* blob,
+                           const sbl_blob_layout& L, int num_sms, cudaStream_t s);
+
+cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
+                             int num_sms, cudaStream_t s);
+
+// Forward GEMM + dequant.  sparse: codes = 2:4 kept values [n_out][k/2] and
+// meta = tensor-core metadata; dense: codes = W_eff int8 [n_out][k].
+cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,
+                                const int8_t* xq, const float* a_prime, const float* g, int64_t n_out, int64_t t,
+                                int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
+                                cudaStream_t s);
+
+// Decode GEMV for t <= 16 over the 2-bit packing.
+cudaError_t launch_forward_gemv(const uint8_t* gemv, const int8_t* xq, const float* a_prime, const float* g,
+                                int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out, int num_sms,
+                                cudaStream_t s);
+
+// out[M][N] = alpha * A . B^T in bf16 x bf16 -> fp32 (tensor cores).
+//   a_mn: A stored [K][M] (else [M][K]);  b_mn: B stored [K][N] (else [N][K]).
+cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t* A, const uint16_t* B, int64_t M,
+                             int64_t N, int64_t K, const float* alpha, void* out, uint32_t* status, int num_sms,
+                             cudaStream_t s);
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
+
+// cuTensorMapEncodeTiled, resolved through the runtime's driver entry point.
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+}  // namespace sbl

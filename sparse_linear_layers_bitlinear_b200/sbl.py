@@ -1,0 +1,241 @@
+"""ctypes binding of libsbl.so (include/sbl.h).
+
+Argument marshalling only: every step of the operator runs in the CUDA
+kernels of libsbl.so.  torch provides device memory and the current stream.
+If the library is missing the import fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsbl.so")
+
+# sbl_status
+SBL_OK = 0
+SBL_ERR_INVALID_ARG = 1
+SBL_ERR_UNSUPPORTED_NM = 2
+SBL_ERR_SHAPE = 3
+SBL_ERR_ALIGN = 4
+SBL_ERR_CUDA = 5
+SBL_ERR_NONFINITE = 6
+SBL_ERR_TIMEOUT = 7
+SBL_ERR_DEVICE = 8
+STATUS_NAMES = {
+    0: "SBL_OK", 1: "SBL_ERR_INVALID_ARG", 2: "SBL_ERR_UNSUPPORTED_NM", 3: "SBL_ERR_SHAPE",
+    4: "SBL_ERR_ALIGN", 5: "SBL_ERR_CUDA", 6: "SBL_ERR_NONFINITE", 7: "SBL_ERR_TIMEOUT", 8: "SBL_ERR_DEVICE",
+}
+# layer flags
+SBL_PACK_GEMV = 1 << 0
+# backward flags
+SBL_GRAD_F32 = 1 << 1
+SBL_NO_DX = 1 << 2
+SBL_NO_DW = 1 << 3
+# device status bits
+SBL_STATUS_NONFINITE_W = 1 << 0
+SBL_STATUS_NONFINITE_X = 1 << 1
+SBL_STATUS_TIMEOUT = 1 << 2
+
+
+class SblError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class sbl_layer(ctypes.Structure):
+    _fields_ = [
+        ("n_out", ctypes.c_int64),
+        ("k", ctypes.c_int64),
+        ("n", ctypes.c_int32),
+        ("m", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+        ("prepared", ctypes.c_void_p),
+    ]
+
+
+class sbl_blob_layout(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_uint64) for name in (
+        "total_bytes", "header", "mask", "codes", "weff_bf16", "sp_values", "sp_meta", "sp_meta_bytes",
+        "gemv", "gamma", "g", "status")]
+
+
+# Every entry point of include/sbl.h with its ctypes signature.
+_P, _I64, _I32, _U32, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint64
+_LP = ctypes.POINTER(sbl_layer)
+SIGNATURES = {
+    "sbl_prepared_layout": (_I32, [_I64, _I64, _I32, _I32, _U32, ctypes.POINTER(sbl_blob_layout)]),
+    "sbl_prepared_bytes": (ctypes.c_size_t, [_I64, _I64, _I32, _I32, _U32]),
+    "sbl_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "sbl_prepare_weights": (_I32, [_LP, _P, _P]),
+    "sbl_forward": (_I32, [_LP, _P, _I64, _P, _P, _P, _P, _P, _P]),
+    "sbl_backward": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P]),
+    "sbl_read_status": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "sbl_clear_status": (_I32, [_LP, _P]),
+    "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
+    "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
+    "sbl_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libsbl.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m sparse_linear_layers_bitlinear_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != SBL_OK:
+        raise SblError(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def prepared_layout(n_out: int, k: int, n: int, m: int, flags: int = 0) -> sbl_blob_layout:
+    out = sbl_blob_layout()
+    _check(lib().sbl_prepared_layout(n_out, k, n, m, flags, ctypes.byref(out)), "sbl_prepared_layout")
+    return out
+
+
+def prepared_bytes(n_out: int, k: int, n: int, m: int, flags: int = 0) -> int:
+    return int(lib().sbl_prepared_bytes(n_out, k, n, m, flags))
+
+
+def workspace_bytes(t: int, k: int) -> int:
+    return int(lib().sbl_workspace_bytes(t, k))
+
+
+@dataclass
+class Layer:
+    """A Sparse-BitLinear layer: shapes, N:M pattern and its prepared device blob."""
+
+    n_out: int
+    k: int
+    n: int
+    m: int
+    flags: int
+    blob: "object"  # torch.uint8 CUDA tensor
+
+    @classmethod
+    def allocate(cls, n_out: int, k: int, n: int, m: int, flags: int = 0, device="cuda"):
+        import torch
+
+        nbytes = prepared_bytes(n_out, k, n, m, flags)
+        if nbytes == 0:
+            prepared_layout(n_out, k, n, m, flags)  # raises with the reason
+        blob = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return cls(n_out, k, n, m, flags, blob)
+
+    def c(self) -> sbl_layer:
+        return sbl_layer(self.n_out, self.k, self.n, self.m, self.flags, self.blob.data_ptr())
+
+    def layout(self) -> sbl_blob_layout:
+        return prepared_layout(self.n_out, self.k, self.n, self.m, self.flags)
+
+    def section(self, name: str, nbytes: int):
+        off = getattr(self.layout(), name)
+        return self.blob[off:off + nbytes]
+
+
+def prepare_weights(layer: Layer, w_master, stream=None):
+    cl = layer.c()
+    _check(lib().sbl_prepare_weights(ctypes.byref(cl), _ptr(w_master), _stream(stream)), "sbl_prepare_weights")
+
+
+def forward(layer: Layer, x, t: int, y, xq_out=None, xscale_out=None, acc_debug=None, workspace=None, stream=None):
+    cl = layer.c()
+    _check(lib().sbl_forward(ctypes.byref(cl), _ptr(x), t, _ptr(y), _ptr(xq_out), _ptr(xscale_out), _ptr(acc_debug),
+                             _ptr(workspace), _stream(stream)), "sbl_forward")
+
+
+def backward(layer: Layer, x, dy, t: int, dx, dw, flags: int = 0, stream=None):
+    cl = layer.c()
+    _check(lib().sbl_backward(ctypes.byref(cl), _ptr(x), _ptr(dy), t, _ptr(dx), _ptr(dw), flags, _stream(stream)),
+           "sbl_backward")
+
+
+def read_status(layer: Layer, stream=None):
+    cl = layer.c()
+    bits = ctypes.c_uint32(0)
+    code = lib().sbl_read_status(ctypes.byref(cl), _stream(stream), ctypes.byref(bits))
+    return code, int(bits.value)
+
+
+def clear_status(layer: Layer, stream=None):
+    cl = layer.c()
+    _check(lib().sbl_clear_status(ctypes.byref(cl), _stream(stream)), "sbl_clear_status")
+
+
+def read_scale(layer: Layer, stream=None):
+    cl = layer.c()
+    gamma, g = ctypes.c_float(0), ctypes.c_float(0)
+    _check(lib().sbl_read_scale(ctypes.byref(cl), _stream(stream), ctypes.byref(gamma), ctypes.byref(g)),
+           "sbl_read_scale")
+    return gamma.value, g.value
+
+
+def selftest_wait_timeout(status_dev, limit_ns: int, stream=None):
+    _check(lib().sbl_selftest_wait_timeout(_ptr(status_dev), limit_ns, _stream(stream)), "sbl_selftest_wait_timeout")
+
+
+def version() -> str:
+    return lib().sbl_version().decode()
+
+
+class SparseBitLinear:
+    """Convenience wrapper: one layer, its blob and its forward/backward buffers.
+
+    All arithmetic happens in libsbl.so; this class only allocates torch
+    tensors and calls the C ABI.
+    """
+
+    def __init__(self, n_out: int, k: int, n: int = 2, m: int = 4, flags: int = 0, device="cuda"):
+        self.layer = Layer.allocate(n_out, k, n, m, flags, device)
+        self.device = device
+
+    def prepare(self, w_master):
+        prepare_weights(self.layer, w_master)
+
+    def forward(self, x, acc_debug: bool = False):
+        import torch
+
+        t = x.shape[0]
+        y = torch.empty((t, self.layer.n_out), dtype=torch.float32, device=self.device)
+        xq = torch.empty((t, self.layer.k), dtype=torch.int8, device=self.device)
+        ap = torch.empty((max(t, 1),), dtype=torch.float32, device=self.device)
+        acc = torch.empty((t, self.layer.n_out), dtype=torch.int32, device=self.device) if acc_debug else None
+        forward(self.layer, x, t, y, xq, ap, acc)
+        return y, xq, ap[:t], acc
+
+    def backward(self, x, dy, f32: bool = False):
+        import torch
+
+        t = dy.shape[0]
+        dt = torch.float32 if f32 else torch.bfloat16
+        dx = torch.empty((t, self.layer.k), dtype=dt, device=self.device)
+        dw = torch.empty((self.layer.n_out, self.layer.k), dtype=dt, device=self.device)
+        backward(self.layer, x, dy, t, dx, dw, SBL_GRAD_F32 if f32 else 0)
+        return dx, dw

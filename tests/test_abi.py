@@ -1,0 +1,113 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point
+that include/sbl.h declares, and its host-only functions and argument
+validation behave as documented (no compute is launched)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_linear_layers_bitlinear_b200 import build, sbl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sbl.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return sbl.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbl_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for required in ("sbl_prepare_weights", "sbl_forward", "sbl_backward", "sbl_prepared_bytes",
+                     "sbl_workspace_bytes", "sbl_read_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", sbl.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT (sbl_[a-z0-9_]+)$", out.stdout, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+    assert set(names) == set(sbl.SIGNATURES), "binding and header disagree"
+
+
+def test_version(lib):
+    assert "sm_100a" in sbl.version()
+
+
+def test_layout_sections_are_aligned_and_disjoint(lib):
+    for (n_out, k, n, m, flags) in [(6912, 2560, 2, 4, 0), (2560, 6912, 6, 8, 0), (264, 320, 2, 4, sbl.SBL_PACK_GEMV),
+                                    (8, 64, 1, 2, 0)]:
+        L = sbl.prepared_layout(n_out, k, n, m, flags)
+        spans = [("header", L.header, 4096), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
+        if (n, m) == (2, 4):
+            spans += [("sp_values", L.sp_values, n_out * k // 2), ("sp_meta", L.sp_meta, L.sp_meta_bytes)]
+            assert L.sp_meta_bytes == ((n_out + 127) // 128 * 128) * ((k + 255) // 256 * 256) // 8
+            assert L.codes == 0
+            if flags & sbl.SBL_PACK_GEMV:
+                spans.append(("gemv", L.gemv, n_out * k // 4))
+        else:
+            spans.append(("codes", L.codes, n_out * k))
+            assert L.sp_values == 0 and L.sp_meta == 0
+        spans.sort(key=lambda s: s[1])
+        for (_, off, size), (_, nxt, _) in zip(spans, spans[1:]):
+            assert off % 256 == 0 and off + size <= nxt
+        assert spans[-1][1] + spans[-1][2] <= L.total_bytes
+        assert sbl.prepared_bytes(n_out, k, n, m, flags) == L.total_bytes
+        assert L.header <= L.gamma < L.header + 4096 and L.g == L.gamma + 4
+
+
+@pytest.mark.parametrize("args,code", [
+    ((256, 256, 2, 3, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 256, 0, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 256, 5, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 256, 6, 8, sbl.SBL_PACK_GEMV), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 96, 2, 4, 0), sbl.SBL_ERR_SHAPE),
+    ((250, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),
+    ((0, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),
+    ((256, 256, 2, 4, 1 << 9), sbl.SBL_ERR_INVALID_ARG),
+])
+def test_layout_rejects_bad_arguments(lib, args, code):
+    out = sbl.sbl_blob_layout()
+    assert lib.sbl_prepared_layout(*args, ctypes.byref(out)) == code
+    assert sbl.prepared_bytes(*args) == 0
+
+
+def test_workspace_bytes(lib):
+    assert sbl.workspace_bytes(4096, 2560) == 4096 * 2560 + 4096 * 4
+    assert sbl.workspace_bytes(3, 64) == 256 + 256
+    assert sbl.workspace_bytes(0, 64) == 0
+
+
+def test_entry_points_validate_before_touching_the_device(lib):
+    # These return before any CUDA call, so they run on a machine without a GPU.
+    layer = sbl.sbl_layer(256, 256, 2, 4, 0, 0x1000)
+    assert lib.sbl_prepare_weights(None, ctypes.c_void_p(0x2000), None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_prepare_weights(ctypes.byref(layer), None, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_prepare_weights(ctypes.byref(layer), ctypes.c_void_p(0x2001), None) == sbl.SBL_ERR_ALIGN
+    misaligned = sbl.sbl_layer(256, 256, 2, 4, 0, 0x1010)
+    assert lib.sbl_prepare_weights(ctypes.byref(misaligned), ctypes.c_void_p(0x2000), None) == sbl.SBL_ERR_ALIGN
+    bad_nm = sbl.sbl_layer(256, 256, 3, 2, 0, 0x1000)
+    assert lib.sbl_prepare_weights(ctypes.byref(bad_nm), ctypes.c_void_p(0x2000), None) == sbl.SBL_ERR_UNSUPPORTED_NM
+    assert lib.sbl_forward(ctypes.byref(layer), None, -1, None, None, None, None, None, None) == sbl.SBL_ERR_SHAPE
+    assert lib.sbl_forward(ctypes.byref(layer), None, 0, None, None, None, None, None, None) == sbl.SBL_OK
+    assert lib.sbl_forward(ctypes.byref(layer), None, 8, None, None, None, None, None, None) == sbl.SBL_ERR_INVALID_ARG
+    # no workspace and no explicit xq / scale buffers
+    assert lib.sbl_forward(ctypes.byref(layer), ctypes.c_void_p(0x3000), 8, ctypes.c_void_p(0x4000), None, None, None,
+                           None, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 0, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 1 << 7, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_selftest_wait_timeout(None, 1000, None) == sbl.SBL_ERR_INVALID_ARG

@@ -1,0 +1,104 @@
+"""Full-size GPU parity at the benchmark workloads, through the same C ABI
+calls the benchmark times.  Whole-array checks where the oracle is fast
+(prepare outputs, activation codes), sampled outputs for the products."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_linear_layers_bitlinear_b200 import sbl, synth
+from tests import blob_decode as bd
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = [
+    # name, n_out, k, n, m, t
+    ("prefill 2:4, FFN up projection", 6912, 2560, 2, 4, 4096),
+    ("prefill 6:8, FFN down projection", 2560, 6912, 6, 8, 4096),
+]
+
+
+def _samples(rng, rows, cols, count):
+    r = rng.integers(0, rows, size=count)
+    c = rng.integers(0, cols, size=count)
+    edge_r = np.array([0, 127, 128, rows - 1, rows // 2] * 5)
+    edge_c = np.array([0, 127, 128, 255, 256, cols - 1, cols // 2] * 5)[: len(edge_r)]
+    return np.concatenate([r, edge_r]), np.concatenate([c, edge_c])
+
+
+@pytest.mark.parametrize("name,n_out,k,n,m,t", WORKLOADS)
+def test_fullsize_parity(name, n_out, k, n, m, t):
+    w_d = synth.master_weights(n_out, k, 0, device="cuda")
+    x_d = synth.activations(t, k, 1, device="cuda")
+    dy_d = synth.upstream_grad(t, n_out, 2, device="cuda")
+    w, x, dy = w_d.cpu(), x_d.cpu(), dy_d.cpu()
+
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, w_d)
+    torch.cuda.synchronize()
+    ref = oracle.prepare(w, n, m)
+    gamma, g, status = bd.header_scalars(layer)
+    assert status == 0
+    assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
+    assert np.float32(g) == ref["g"]
+    assert np.array_equal(bd.mask(layer), ref["mask"])
+    assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"])
+    if (n, m) == (2, 4):
+        vals, meta = oracle.pack24(ref["weff"], ref["mask"])
+        assert np.array_equal(bd.sp_values(layer), vals)
+        assert np.array_equal(bd.sp_meta_canonical(layer)[0], meta)
+    else:
+        assert np.array_equal(bd.codes(layer), ref["weff"])
+
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    sbl.forward(layer, x_d, t, y, xq, ap, acc)
+    dx = torch.empty((t, k), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
+    sbl.backward(layer, x_d, dy_d, t, dx, dw, 0)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+
+    rng = np.random.default_rng(7)
+    acc_h, y_h = acc.cpu().numpy(), y.cpu().numpy()
+    ti, oi = _samples(rng, t, n_out, 1500)
+    accs = np.array([oracle.acc_at(xq_ref, ref["weff"], a, b) for a, b in zip(ti, oi)], dtype=np.int32)
+    assert np.array_equal(acc_h[ti, oi], accs)
+    y_ref = oracle.dequant(accs.reshape(-1, 1), ap_ref[ti], ref["g"]).ravel()
+    assert np.array_equal(y_h[ti, oi].view(np.uint32), y_ref.view(np.uint32))
+
+    dx_h = bd.bf16_to_f64(dx)
+    ti, ki = _samples(rng, t, k, 600)
+    dxr = np.array([oracle.grad_x_at(dy, ref["weff"], ref["g"], a, b) for a, b in zip(ti, ki)])
+    err = np.abs(dx_h[ti, ki] - dxr)
+    assert (err <= 1e-2 + 2.0 ** -7 * np.abs(dxr)).all(), err.max()
+
+    dw_h = bd.bf16_to_f64(dw)
+    oi, ki = _samples(rng, n_out, k, 600)
+    dwr = np.array([oracle.grad_w_at(dy, x, a, b) for a, b in zip(oi, ki)])
+    err = np.abs(dw_h[oi, ki] - dwr)
+    assert (err <= 1e-2 + 2.0 ** -7 * np.abs(dwr)).all(), err.max()
+
+
+@pytest.mark.parametrize("t", [1, 4, 16])
+@pytest.mark.parametrize("n_out", [2560, 6912])
+def test_decode_gemv_fullsize(t, n_out):
+    k = 2560
+    w_d = synth.master_weights(n_out, k, 10, device="cuda")
+    x_d = synth.activations(t, k, 11, device="cuda")
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, w_d)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, x_d, t, y, acc_debug=acc, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle.forward(w_d.cpu(), x_d.cpu(), 2, 4)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))

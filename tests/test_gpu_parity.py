@@ -1,0 +1,213 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer, byte and index results (gamma bits, masks, codes, packed forms,
+int8 activations, int32 accumulators) must match bit for bit; y (fp32) is
+checked bit for bit too and, as the stated bound, within rel 1e-3 / abs 1e-2;
+gradients within rel 1e-3 / abs 1e-2 (fp32 mode) or one bf16 step plus abs
+1e-2 (bf16 mode) of the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_linear_layers_bitlinear_b200 import sbl, synth
+from tests import blob_decode as bd
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 1e-3, 1e-2
+BF16_REL = 2.0 ** -7  # one bf16 step, relative
+
+
+def _dev(t):
+    return t.to("cuda")
+
+
+def _close(gpu, ref, rtol=RTOL, atol=ATOL):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(gpu - ref)
+    bound = atol + rtol * np.abs(ref)
+    bad = err > bound
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside tolerance; worst err {err.max()}"
+
+
+def _check_prepared(layer, w, n, m):
+    ref = oracle.prepare(w, n, m)
+    gamma, g, status = bd.header_scalars(layer)
+    assert status == 0
+    assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
+    assert np.float32(g).view(np.uint32) == np.float32(ref["g"]).view(np.uint32)
+    assert np.array_equal(bd.mask(layer), ref["mask"])
+    assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"])
+    if (n, m) == (2, 4):
+        vals, meta = oracle.pack24(ref["weff"], ref["mask"])
+        assert np.array_equal(bd.sp_values(layer), vals)
+        canon, pad_rows, pad_cols = bd.sp_meta_canonical(layer)
+        assert np.array_equal(canon, meta)
+        assert (pad_rows == 0x44).all() and (pad_cols == 0x44).all()
+        if layer.flags & sbl.SBL_PACK_GEMV:
+            nib, c0, c1 = bd.decode_gemv(bd.gemv_bytes(layer))
+            mnib = np.stack([meta & 0xF, meta >> 4], axis=-1).reshape(meta.shape[0], -1)
+            assert np.array_equal(nib, mnib)
+            assert np.array_equal(c0, vals[:, 0::2]) and np.array_equal(c1, vals[:, 1::2])
+    else:
+        assert np.array_equal(bd.codes(layer), ref["weff"])
+    return ref
+
+
+CASES = [
+    # n_out, k, n, m, t
+    (256, 256, 2, 4, 16),     # the small single-forward workload
+    (264, 320, 2, 4, 300),    # ragged rows, k not a multiple of 128, ragged tokens
+    (136, 448, 6, 8, 77),
+    (128, 384, 4, 8, 129),
+    (520, 192, 1, 4, 33),
+    (64, 64, 3, 4, 3),
+    (8, 64, 2, 4, 5),
+    (384, 512, 8, 8, 260),    # N = M: plain ternary BitLinear
+    (200, 128, 1, 2, 50),
+    (392, 832, 3, 8, 513),
+]
+
+
+@pytest.mark.parametrize("n_out,k,n,m,t", CASES)
+def test_prepare_forward_backward_parity(n_out, k, n, m, t):
+    seed = n_out * 7 + k + 13 * n + m
+    w = synth.master_weights(n_out, k, seed)
+    x = synth.activations(t, k, seed + 1)
+    dy = synth.upstream_grad(t, n_out, seed + 2)
+
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    ref = _check_prepared(layer, w, n, m)
+
+    xd, dyd = _dev(x), _dev(dy)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    sbl.forward(layer, xd, t, y, xq, ap, acc)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    y_ref = oracle.dequant(acc_ref, ap_ref, ref["g"])
+    y_gpu = y.cpu().numpy()
+    _close(y_gpu, y_ref)
+    assert np.array_equal(y_gpu.view(np.uint32), y_ref.view(np.uint32))
+
+    # backward, fp32 outputs
+    dx = torch.empty((t, k), dtype=torch.float32, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, xd, dyd, t, dx, dw, sbl.SBL_GRAD_F32)
+    torch.cuda.synchronize()
+    dx_ref = oracle.grad_x(dy, ref["weff"], ref["g"])
+    dw_ref = oracle.grad_w(dy, x)
+    _close(dx.cpu().numpy(), dx_ref)
+    _close(dw.cpu().numpy(), dw_ref)
+
+    # backward, bf16 outputs: within one bf16 step of the rounded oracle
+    dx16 = torch.empty((t, k), dtype=torch.bfloat16, device="cuda")
+    dw16 = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
+    sbl.backward(layer, xd, dyd, t, dx16, dw16, 0)
+    torch.cuda.synchronize()
+    _close(bd.bf16_to_f64(dx16), dx_ref, rtol=BF16_REL, atol=ATOL)
+    _close(bd.bf16_to_f64(dw16), dw_ref, rtol=BF16_REL, atol=ATOL)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 7, 16])
+def test_gemv_path_parity(t):
+    n_out, k = 392, 640
+    w = synth.master_weights(n_out, k, 3)
+    x = synth.activations(t, k, 4)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    ref = _check_prepared(layer, w, 2, 4)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    y_ref = oracle.dequant(acc_ref, ap_ref, ref["g"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), y_ref.view(np.uint32))
+
+
+def test_workspace_path_matches_explicit_buffers():
+    n_out, k, t = 256, 512, 40
+    w = synth.master_weights(n_out, k, 8)
+    x = _dev(synth.activations(t, k, 9))
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(w))
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    y1 = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, x, t, y1, workspace=ws)
+    y2 = torch.empty_like(y1)
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, x, t, y2, xq, ap)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_empty_batch():
+    n_out, k = 64, 128
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 1)))
+    y = torch.empty((0, n_out), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, None, 0, y)
+    dw = torch.full((n_out, k), 7.0, dtype=torch.float32, device="cuda")
+    sbl.backward(layer, None, None, 0, None, dw, sbl.SBL_GRAD_F32 | sbl.SBL_NO_DX)
+    torch.cuda.synchronize()
+    assert (dw == 0).all()
+
+
+def test_nonfinite_inputs_raise_status():
+    n_out, k = 64, 128
+    w = synth.master_weights(n_out, k, 2)
+    w[3, 5] = float("nan")
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(w))
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_ERR_NONFINITE and bits & sbl.SBL_STATUS_NONFINITE_W
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 2)))
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    x = synth.activations(4, k, 3)
+    x[1, 7] = float("inf")
+    y = torch.empty((4, n_out), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(4, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), 4, y, workspace=ws)
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_ERR_NONFINITE and bits & sbl.SBL_STATUS_NONFINITE_X
+    sbl.clear_status(layer)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def test_bounded_wait_reports_timeout():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sbl.selftest_wait_timeout(status, 2_000_000)  # 2 ms on a barrier nothing arrives on
+    torch.cuda.synchronize()
+    assert int(status.item()) & sbl.SBL_STATUS_TIMEOUT
+    # the context is still usable afterwards
+    assert float(torch.ones(4, device="cuda").sum()) == 4.0
+
+
+def test_gamma_scale_readback():
+    w = synth.master_weights(128, 256, 5)
+    layer = sbl.Layer.allocate(128, 256, 6, 8)
+    sbl.prepare_weights(layer, _dev(w))
+    gamma, g = sbl.read_scale(layer)
+    assert np.float32(gamma) == oracle.absmean_gamma(w)
+    assert np.float32(g) == oracle.clamped_scale(oracle.absmean_gamma(w))
