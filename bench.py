@@ -1,0 +1,435 @@
+"""Sparse-BitLinear benchmark on B200.
+
+One step = the whole hot path of one Sparse-BitLinear layer over one batch:
+prepare the weights (exact absmean, N:M mask from the masters, ternarise and
+pack), the forward pass (per-token int8 activation quantisation, 2:4-sparse
+int8 tensor-core GEMM with the dequant epilogue) and the dual-STE backward
+(dX through the masked ternary weights, dense dW to every master).
+
+Workload: the prefill-shaped FFN up projection, T=4096 tokens, K=2560,
+N_out=6912, 2:4, bf16 masters ~N(0, 0.02), activations and upstream
+gradients ~N(0, 1), seeded synthetic data.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs an independent replica on its own GPU with its
+own token batch (no collective on the data path); the time is the max over
+ranks and `value` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Sparse-BitLinear fwd+bwd TOPS & tokens/s at 1 B200; % of sparse-int8/HBM roofline"
+UNIT = "tokens/s"
+WORKLOAD = dict(name="prefill 2:4 Sparse-BitLinear fwd+STE bwd, FFN up projection", tokens=4096, k=2560,
+                n_out=6912, n=2, m=4)
+ROTATE = 3  # distinct input sets cycled through the steps (3 x 112 MB > 126 MB L2)
+
+# Algorithmic work of one step at this workload (Measurement).
+def algorithmic(T, K, N):
+    dense_ops = 2.0 * T * K * N                    # one GEMM, dense-equivalent multiply-adds x 2
+    return {
+        "fwd_gemm_ops": dense_ops,                 # int8 x ternary, half of them skipped by 2:4
+        "bwd_flops_each": dense_ops,               # dX and dW, bf16 x bf16 -> fp32
+        "step_ops": 3.0 * dense_ops,
+        "prep_bytes": N * K * 2 + N * K // 2 + N * K // 8,   # read W; write 2:4 values + metadata
+        "actq_bytes": T * K * 2 + T * K + T * 4,            # read X; write xq + scales
+        "fwd_bytes": N * K // 2 + N * K // 8 + T * K + T * 4 + T * N * 4,  # read W_eff, xq; write fp32 Y
+        "dx_bytes": T * N * 2 + N * K * 2 + T * K * 2,
+        "dw_bytes": T * N * 2 + T * K * 2 + N * K * 2,
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_linear_layers_bitlinear_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec.get(kernel_key)
+        if ent and ent.get("source_sha") == kernel_source_sha():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML, every 20 ms)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        names = [v for k, v in self.REASONS.items() if self.reasons & k and k != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample, extrapolated linearly in tokens)
+# ---------------------------------------------------------------------------
+def oracle_sample(wb, xb, dyb, n, m, tokens):
+    import oracle
+
+    t0 = time.perf_counter()
+    p = oracle.prepare(wb, n, m)
+    xq, ap = oracle.act_quant(xb)
+    t_fixed = time.perf_counter() - t0  # prepare + act-quant over the whole batch
+    t1 = time.perf_counter()
+    acc = oracle.gemm_acc(xq[:tokens], p["weff"])
+    oracle.dequant(acc, ap[:tokens], p["g"])
+    oracle.grad_x(dyb[:tokens], p["weff"], p["g"])
+    oracle.grad_w(dyb[:tokens], xb[:tokens])
+    t_tok = (time.perf_counter() - t1) / tokens
+    return t_fixed, t_tok
+
+
+def cpu_baseline(T, K, N, n, m, target_s=15.0):
+    import oracle
+    from sparse_linear_layers_bitlinear_b200 import synth
+
+    wb = synth.bits(synth.master_weights(N, K, 0))
+    xb = synth.bits(synth.activations(T, K, 1))
+    dyb = synth.bits(synth.upstream_grad(T, N, 2))
+    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, 4)
+    tokens = int(max(4, min(T, (target_s - t_fixed) / max(t_tok, 1e-9))))
+    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, tokens)
+    step_s = t_fixed + T * t_tok
+    return {"value": T / step_s, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"prepare and act-quant over the full batch, then fwd + dX + dW for {tokens} of {T} tokens; "
+                      f"step time extrapolated linearly in tokens ({step_s:.1f} s per full step)"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm, timed on the host cores."""
+    import oracle
+    from sparse_linear_layers_bitlinear_b200 import synth
+
+    T, K, N, n, m = (WORKLOAD[k] for k in ("tokens", "k", "n_out", "n", "m"))
+    wb = synth.bits(synth.master_weights(N, K, 0))
+    xb = synth.bits(synth.activations(T, K, 1))
+    dyb = synth.bits(synth.upstream_grad(T, N, 2))
+    # size each step's token sample so the whole run stays within ~2 minutes
+    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, 2)
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    tokens = int(max(1, min(T, (per_step - t_fixed) / max(t_tok, 1e-9))))
+    for _ in range(args.warmup):
+        oracle_sample(wb, xb, dyb, n, m, tokens)
+    est = []
+    for _ in range(args.steps):
+        t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, tokens)
+        est.append(t_fixed + T * t_tok)
+    step_s = statistics.mean(est)
+    value = T / step_s
+    sample = (f"per step: prepare and act-quant over the full batch, fwd + dX + dW for {tokens} of {T} tokens; "
+              f"full-step time extrapolated linearly in tokens")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i64/f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "tokens": T, "k": K, "n_out": N, "n": n, "m": m},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T, K, N, n, m = (WORKLOAD[k] for k in ("tokens", "k", "n_out", "n", "m"))
+    A = algorithmic(T, K, N)
+    peaks = load_peaks()
+
+    # Inputs: ROTATE seeded sets, different per rank (independent batches).
+    sets = []
+    for r in range(ROTATE):
+        base = 1000 * rank + 10 * r
+        sets.append((synth.master_weights(N, K, base + 0, device=dev), synth.activations(T, K, base + 1, device=dev),
+                     synth.upstream_grad(T, N, base + 2, device=dev)))
+    layer = sbl.Layer.allocate(N, K, n, m, device=dev)
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        w, x, dy = sets[i % ROTATE]
+        if ev is not None:
+            ev[0].record(stream)
+        sbl.prepare_weights(layer, w)
+        if ev is not None:
+            ev[1].record(stream)
+        sbl.forward(layer, x, T, y, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        sbl.backward(layer, x, dy, T, dx, dw, sbl.SBL_NO_DW)
+        if ev is not None:
+            ev[3].record(stream)
+        sbl.backward(layer, x, dy, T, dx, dw, sbl.SBL_NO_DX)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_OK, (code, bits)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_total = start.elapsed_time(end)
+    ms_step = max_over_ranks(ms_total / args.steps, world)
+    phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(4)]
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_OK, (code, bits)
+
+    # End to end through the C ABI from pinned host buffers: H2D of the step's
+    # inputs, the step, D2H of its outputs, all inside the timed region.
+    w_h = [s[0].cpu().pin_memory() for s in sets]
+    x_h = [s[1].cpu().pin_memory() for s in sets]
+    dy_h = [s[2].cpu().pin_memory() for s in sets]
+    y_h = torch.empty((T, N), dtype=torch.float32).pin_memory()
+    dx_h = torch.empty((T, K), dtype=torch.bfloat16).pin_memory()
+    dw_h = torch.empty((N, K), dtype=torch.bfloat16).pin_memory()
+    w_d, x_d, dy_d = (torch.empty_like(t) for t in sets[0])
+
+    def e2e_step(i):
+        r = i % ROTATE
+        w_d.copy_(w_h[r], non_blocking=True)
+        x_d.copy_(x_h[r], non_blocking=True)
+        dy_d.copy_(dy_h[r], non_blocking=True)
+        sbl.prepare_weights(layer, w_d)
+        sbl.forward(layer, x_d, T, y, workspace=ws)
+        sbl.backward(layer, x_d, dy_d, T, dx, dw, 0)
+        y_h.copy_(y, non_blocking=True)
+        dx_h.copy_(dx, non_blocking=True)
+        dw_h.copy_(dw, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in sets[0])
+    d2h = y.numel() * 4 + dx.numel() * 2 + dw.numel() * 2
+
+    # Rooflines: each phase's bound at the measured peaks.
+    hbm = peaks["hbm_gbs"] * 1e9
+    bf16 = peaks["bf16_tflops"] * 1e12
+    i8_sparse = 4.0 * bf16  # dense-equivalent int8 2:4 peak: bf16 x (int8 2x, sparsity 2x) nominal ratio
+    bound_ms = {
+        "prepare": A["prep_bytes"] / hbm * 1e3,
+        "forward": max(A["fwd_gemm_ops"] / i8_sparse, (A["actq_bytes"] + A["fwd_bytes"]) / hbm) * 1e3,
+        "dx": max(A["bwd_flops_each"] / bf16, A["dx_bytes"] / hbm) * 1e3,
+        "dw": max(A["bwd_flops_each"] / bf16, A["dw_bytes"] / hbm) * 1e3,
+    }
+    names = ["prepare", "forward", "dx", "dw"]
+    dom = max(range(4), key=lambda j: phase_ms[j])
+    dom_name = names[dom]
+    if dom_name in ("dx", "dw"):
+        achieved = A["bwd_flops_each"] / (phase_ms[dom] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": ncu_traffic("bf16_gemm_" + dom_name),
+                "kernel": f"k_gemm_tc<CfgBf16> ({dom_name})",
+                "peak_note": f"{peaks['source']} bf16 burst figure (kernel timed inside a short step loop)"}
+    else:
+        by = {"prepare": A["prep_bytes"], "forward": A["actq_bytes"] + A["fwd_bytes"]}[dom_name]
+        achieved = by / (phase_ms[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(dom_name), "kernel": dom_name,
+                "peak_note": f"{peaks['source']} HBM copy bandwidth"}
+
+    tokens_per_s = world * T / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8xternary->i32 fwd, bf16->f32 bwd", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "tokens": T, "k": K, "n_out": N, "n": n, "m": m,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotate over {ROTATE} seeded sets (3 x 112 MB > 126 MB L2)"},
+        "tops": A["step_ops"] * world / (ms_step * 1e-3) / 1e12,
+        "phase_ms": dict(zip(names, phase_ms)),
+        "phase_roofline_ms": bound_ms,
+        "step_roofline_frac": sum(bound_ms.values()) / ms_step,
+        "roofline": roof,
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clocks.summary(),
+        "peaks": peaks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
