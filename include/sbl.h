@@ -62,7 +62,8 @@ typedef enum sbl_status {
   SBL_ERR_CUDA = 5,           /* a CUDA call failed (launch error, no device, ...) */
   SBL_ERR_NONFINITE = 6,      /* device saw a NaN/Inf master weight or activation */
   SBL_ERR_TIMEOUT = 7,        /* a device-side bounded wait gave up */
-  SBL_ERR_DEVICE = 8          /* the current device is not sm_100 */
+  SBL_ERR_DEVICE = 8,         /* the current device is not sm_100 */
+  SBL_ERR_SCRATCH = 9         /* sbl_forward_noalloc: t * k exceeds its fixed scratch */
 } sbl_status;
 
 /* Flags of sbl_layer.flags (fixed at prepare time). */
@@ -143,6 +144,34 @@ sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl
  * tensor-core GEMM; other patterns the dense int8 one over W_eff codes. */
 sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
                        float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
+
+/* Forward pass for callers that cannot allocate device memory.  The paper has
+ * no counterpart: this is a deployment convenience, not a step of the method.
+ *
+ * Same arithmetic and outputs as sbl_forward, but the int8 activation codes
+ * and per-token scales go to a fixed scratch array that the library itself
+ * holds in device memory, so the caller supplies only x, y (and optionally
+ * acc_debug).  Meant for code that has no way to obtain a workspace: plugins
+ * whose enqueue hook must not allocate, processes whose device memory belongs
+ * to an allocator they cannot reach, and latency-critical loops that cannot
+ * pay for cudaMalloc's implicit synchronisation.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Limit: align256(t * k) + align256(4 * t) <= SBL_NOALLOC_SCRATCH_BYTES
+ * (16 MiB; e.g. t = 4096 tokens at k = 2560); larger requests return
+ * SBL_ERR_SCRATCH and enqueue nothing.  Every device that loads the library's
+ * device code keeps those 16 MiB until the process exits.
+ *
+ * The first call with t > 0 on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls on a device share the one array and it keeps the
+ * last call's contents, so calls that can overlap on the GPU (two streams,
+ * two host threads) race on it: serialise them.  Nothing in the array needs to
+ * start at zero; each call writes everything it reads.  Errors: as
+ * sbl_forward, plus SBL_ERR_SCRATCH. */
+#define SBL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+sbl_status sbl_forward_noalloc(const sbl_layer* layer, const void* x, int64_t t, float* y, int32_t* acc_debug,
+                               sbl_stream_t stream);
 
 /* Step 5 (dual STE).  x: bf16 [t, k] (the forward input), dy: bf16 [t, n_out].
  *   dx [t, k]     = g * (dy . W_eff)          (straight through Q_w, Q_x, mask)

@@ -23,10 +23,14 @@ SBL_ERR_CUDA = 5
 SBL_ERR_NONFINITE = 6
 SBL_ERR_TIMEOUT = 7
 SBL_ERR_DEVICE = 8
+SBL_ERR_SCRATCH = 9
 STATUS_NAMES = {
     0: "SBL_OK", 1: "SBL_ERR_INVALID_ARG", 2: "SBL_ERR_UNSUPPORTED_NM", 3: "SBL_ERR_SHAPE",
     4: "SBL_ERR_ALIGN", 5: "SBL_ERR_CUDA", 6: "SBL_ERR_NONFINITE", 7: "SBL_ERR_TIMEOUT", 8: "SBL_ERR_DEVICE",
+    9: "SBL_ERR_SCRATCH",
 }
+# Fixed scratch of sbl_forward_noalloc (SBL_NOALLOC_SCRATCH_BYTES in include/sbl.h).
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 # layer flags
 SBL_PACK_GEMV = 1 << 0
 # backward flags
@@ -72,6 +76,7 @@ SIGNATURES = {
     "sbl_prepare_weights": (_I32, [_LP, _P, _P]),
     "sbl_forward": (_I32, [_LP, _P, _I64, _P, _P, _P, _P, _P, _P]),
     "sbl_backward": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P]),
+    "sbl_forward_noalloc": (_I32, [_LP, _P, _I64, _P, _P, _P]),
     "sbl_read_status": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "sbl_clear_status": (_I32, [_LP, _P]),
     "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
@@ -169,6 +174,14 @@ def forward(layer: Layer, x, t: int, y, xq_out=None, xscale_out=None, acc_debug=
     cl = layer.c()
     _check(lib().sbl_forward(ctypes.byref(cl), _ptr(x), t, _ptr(y), _ptr(xq_out), _ptr(xscale_out), _ptr(acc_debug),
                              _ptr(workspace), _stream(stream)), "sbl_forward")
+
+
+def forward_noalloc(layer: Layer, x, t: int, y, acc_debug=None, stream=None):
+    """sbl_forward_noalloc: the forward pass without any caller-provided scratch,
+    for callers that cannot allocate device memory (see include/sbl.h)."""
+    cl = layer.c()
+    _check(lib().sbl_forward_noalloc(ctypes.byref(cl), _ptr(x), t, _ptr(y), _ptr(acc_debug), _stream(stream)),
+           "sbl_forward_noalloc")
 
 
 def backward(layer: Layer, x, dy, t: int, dx, dw, flags: int = 0, stream=None):
