@@ -91,7 +91,7 @@ typedef struct sbl_layer {
 /* Byte offsets of the sections inside the prepared blob (0 = absent). */
 typedef struct sbl_blob_layout {
   uint64_t total_bytes;
-  uint64_t header;      /* 4096-byte header: shapes, gamma, g, status word, scratch */
+  uint64_t header;      /* 4096-byte header: shapes, gamma, g, status word */
   uint64_t mask;        /* uint8 [n_out, k/m]: bit j = position j of the group kept */
   uint64_t codes;       /* int8 [n_out, k]: W_eff codes (patterns other than 2:4) */
   uint64_t weff_bf16;   /* bf16 [n_out, k]: W_eff as exact bf16 {-1, 0, 1} (backward) */
@@ -102,6 +102,7 @@ typedef struct sbl_blob_layout {
   uint64_t gamma;       /* float: exact absmean, rounded to fp32 */
   uint64_t g;           /* float: max(gamma, 1e-5), the scale used everywhere */
   uint64_t status;      /* uint32 device status word */
+  uint64_t scratch;     /* partial sums of the exact absmean (written and read by sbl_prepare_weights) */
 } sbl_blob_layout;
 /* sp_meta layout: blocks of 128 rows x 128 k-positions, 2048 bytes each,
  * ordered [row_block][k_block]; inside a block, row r's 16 bytes hold 32

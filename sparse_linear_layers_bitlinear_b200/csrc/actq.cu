@@ -2,76 +2,157 @@
 // The Sparse-BitNet pages do not spell out the activation quantiser; this is
 // the BitNet b1.58 convention: a' = max(max_k |x|, 1e-5), and
 // xq = sign(x) * rne(fl32(127 |x|) / a') clamped to [-128, 127].
+//
+// One block of 128 threads per token row.  Each thread keeps its R 16-byte
+// vectors of the row in registers, so the row is read from memory once: the
+// block reduces the absmax, then every thread quantises what it holds.  Rows
+// longer than 128 * 8 * kMaxR elements take a two-pass, warp-per-row kernel.
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
 
 namespace sbl {
 
-constexpr int kActWarps = 8;  // one warp per token row
+constexpr int kActThreads = 128;
+constexpr int kMaxR = 16;  // rows up to 16384 elements stay in registers
 
 __device__ __forceinline__ float bf16_abs_value(uint32_t bits16) { return __uint_as_float((bits16 & 0x7FFFu) << 16); }
 
-__global__ void __launch_bounds__(kActWarps * 32)
-    k_act_quant(const uint16_t* __restrict__ x, int64_t t, int64_t k, int8_t* __restrict__ xq,
-                float* __restrict__ a_prime, uint32_t* status) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t nvec = k / 8;  // 16-byte vectors per row
-  for (int64_t row = int64_t(blockIdx.x) * kActWarps + warp; row < t; row += int64_t(gridDim.x) * kActWarps) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + row * k);
+// 8 bf16 values -> 8 int8 codes (two words).
+__device__ __forceinline__ uint2 quantise8(const uint4 v, float ap) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t b = (words[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+    const float q = __fdiv_rn(__fmul_rn(127.0f, bf16_abs_value(b)), ap);
+    const int n = min(__float2int_rn(q), 127);  // nearest, ties to even
+    const int code = (b & 0x8000u) ? -n : n;
+    packed[e >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (e & 3));
+  }
+  return make_uint2(packed[0], packed[1]);
+}
+
+__device__ __forceinline__ void scan8(const uint4 v, float& amax, uint32_t& bad) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t b = (words[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+    bad |= ((b & 0x7F80u) == 0x7F80u);
+    amax = fmaxf(amax, bf16_abs_value(b));
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(kActThreads)
+    k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
+                     float* __restrict__ a_prime, uint32_t* status) {
+  __shared__ float s_max[kActThreads / 32];
+  __shared__ uint32_t s_bad[kActThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int64_t row = blockIdx.x; row < t; row += gridDim.x) {
+    const uint4* src = x + row * nvec;
+    uint4 v[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = int64_t(r) * kActThreads + tid;
+      v[r] = (i < nvec) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    }
     float amax = 0.0f;
     uint32_t bad = 0;
-    auto scan = [&](const uint4 v) {
-      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t b = (words[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-        bad |= ((b & 0x7F80u) == 0x7F80u);
-        amax = fmaxf(amax, bf16_abs_value(b));
-      }
-    };
+    for (int r = 0; r < R; ++r) scan8(v[r], amax, bad);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      bad |= __shfl_xor_sync(0xffffffffu, bad, off);
+    }
+    if (lane == 0) {
+      s_max[warp] = amax;
+      s_bad[warp] = bad;
+    }
+    __syncthreads();
+    amax = s_max[0];
+    bad = s_bad[0];
+#pragma unroll
+    for (int w = 1; w < kActThreads / 32; ++w) {
+      amax = fmaxf(amax, s_max[w]);
+      bad |= s_bad[w];
+    }
+    __syncthreads();  // s_max is rewritten by the next row
+    const float ap = fmaxf(amax, 1e-5f);
+    if (tid == 0) {
+      a_prime[row] = ap;
+      if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
+    }
+    uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = int64_t(r) * kActThreads + tid;
+      if (i < nvec) dst[i] = quantise8(v[r], ap);
+    }
+  }
+}
+
+// Long rows: one warp per row, absmax pass then a second (L1/L2) pass.
+constexpr int kActWarps = 8;
+
+__global__ void __launch_bounds__(kActWarps * 32)
+    k_act_quant_long(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
+                     float* __restrict__ a_prime, uint32_t* status) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t row = int64_t(blockIdx.x) * kActWarps + warp; row < t; row += int64_t(gridDim.x) * kActWarps) {
+    const uint4* src = x + row * nvec;
+    float amax = 0.0f;
+    uint32_t bad = 0;
     int64_t i = lane;
     for (; i + 96 < nvec; i += 128) {
       const uint4 v0 = __ldg(src + i), v1 = __ldg(src + i + 32), v2 = __ldg(src + i + 64), v3 = __ldg(src + i + 96);
-      scan(v0);
-      scan(v1);
-      scan(v2);
-      scan(v3);
+      scan8(v0, amax, bad);
+      scan8(v1, amax, bad);
+      scan8(v2, amax, bad);
+      scan8(v3, amax, bad);
     }
-    for (; i < nvec; i += 32) scan(__ldg(src + i));
+    for (; i < nvec; i += 32) scan8(__ldg(src + i), amax, bad);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (__any_sync(0xffffffffu, bad != 0) && lane == 0) raise_status(status, SBL_STATUS_NONFINITE_X);
     const float ap = fmaxf(amax, 1e-5f);
     if (lane == 0) a_prime[row] = ap;
-
-    uint2* dst = reinterpret_cast<uint2*>(xq + row * k);
-    for (int64_t j = lane; j < nvec; j += 32) {
-      const uint4 v = __ldg(src + j);  // second read hits L1/L2
-      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-      uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t b = (words[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-        const float ax = bf16_abs_value(b);
-        const float q = __fdiv_rn(__fmul_rn(127.0f, ax), ap);
-        int n = __float2int_rn(q);  // nearest, ties to even
-        n = min(n, 127);
-        const int code = (b & 0x8000u) ? -n : n;
-        packed[e >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (e & 3));
-      }
-      dst[j] = make_uint2(packed[0], packed[1]);
-    }
+    uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
+    for (int64_t j = lane; j < nvec; j += 32) dst[j] = quantise8(__ldg(src + j), ap);
   }
+}
+
+template <int R>
+static void launch_rows(const uint4* x, int64_t t, int64_t nvec, int8_t* xq, float* ap, uint32_t* status,
+                        int num_sms, cudaStream_t s) {
+  int64_t blocks = t;
+  const int64_t cap = int64_t(num_sms) * 64;
+  if (blocks > cap) blocks = cap;
+  k_act_quant_rows<R><<<static_cast<unsigned>(blocks), kActThreads, 0, s>>>(x, t, nvec, xq, ap, status);
 }
 
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
                              int num_sms, cudaStream_t s) {
   if (t <= 0) return cudaSuccess;
-  int64_t blocks = (t + kActWarps - 1) / kActWarps;
-  const int64_t cap = int64_t(num_sms) * 16;
-  if (blocks > cap) blocks = cap;
-  k_act_quant<<<static_cast<unsigned>(blocks), kActWarps * 32, 0, s>>>(x, t, k, xq, a_prime, status);
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  const int64_t nvec = k / 8;
+  const int64_t r = (nvec + kActThreads - 1) / kActThreads;
+  if (r <= 1) launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 2) launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 3) launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 4) launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 6) launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 8) launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= 12) launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else if (r <= kMaxR) launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  else {
+    int64_t blocks = (t + kActWarps - 1) / kActWarps;
+    const int64_t cap = int64_t(num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    k_act_quant_long<<<static_cast<unsigned>(blocks), kActWarps * 32, 0, s>>>(xv, t, nvec, xq, a_prime, status);
+  }
   return cudaGetLastError();
 }
 

@@ -78,19 +78,22 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
   p.meta_kblocks = meta_kblocks;
   p.status = status;
   CUtensorMap ta, tb;
+  const bool acc = acc_out != nullptr;
   if (sparse) {
     if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k / 2, n_out, k / 2, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdSparse::BN,
+        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdSparse<false>::BN,
                         CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-    return launch_tc<CfgFwdSparse>(ta, tb, p, p.n_out, p.T, num_sms, s);
+    return acc ? launch_tc<CfgFwdSparse<true>>(ta, tb, p, p.n_out, p.T, num_sms, s)
+               : launch_tc<CfgFwdSparse<false>>(ta, tb, p, p.n_out, p.T, num_sms, s);
   }
   if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k, n_out, k, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdDense::BN,
+      !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdDense<false>::BN,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  return launch_tc<CfgFwdDense>(ta, tb, p, p.n_out, p.T, num_sms, s);
+  return acc ? launch_tc<CfgFwdDense<true>>(ta, tb, p, p.n_out, p.T, num_sms, s)
+             : launch_tc<CfgFwdDense<false>>(ta, tb, p, p.n_out, p.T, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------

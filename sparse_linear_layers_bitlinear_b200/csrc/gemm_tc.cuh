@@ -304,25 +304,48 @@ struct FwdParams {
   uint32_t* status;
 };
 
+// One 32-token chunk of the forward epilogue.  The thread owns output row o
+// (a TMEM lane) and holds its 32 int32 accumulators for tokens t0..t0+31;
+// lane j computes token t0+j's scale (g * a') / 127 and shares it with a
+// shuffle.  For each token the warp stores 32 consecutive floats of y.
+template <bool ACC_OUT>
 __device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uint32_t (&r)[32], int o, int t0,
                                                    int lane, float g) {
-  // Each lane fetches one token's scale; lane j's value is broadcast for column j.
   const int tl = t0 + lane;
   const float f_mine = (tl < p.T) ? __fdiv_rn(__fmul_rn(g, p.a_prime[tl]), 127.0f) : 0.0f;
   const bool row_ok = o < p.n_out;
+  const int64_t ld = p.n_out;
+  float* yp = p.y + int64_t(t0) * ld + o;
+  int32_t* ap = ACC_OUT ? p.acc_out + int64_t(t0) * ld + o : nullptr;
+  if (t0 + 32 <= p.T) {  // full chunk: no per-token bound
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float f = __shfl_sync(0xffffffffu, f_mine, j);
-    const int t = t0 + j;
-    if (row_ok && t < p.T) {
+    for (int j = 0; j < 32; ++j) {
+      const float f = __shfl_sync(0xffffffffu, f_mine, j);
       const int32_t a = static_cast<int32_t>(r[j]);
-      p.y[int64_t(t) * p.n_out + o] = __fmul_rn(static_cast<float>(a), f);
-      if (p.acc_out) p.acc_out[int64_t(t) * p.n_out + o] = a;
+      if (row_ok) {
+        *yp = __fmul_rn(static_cast<float>(a), f);
+        if (ACC_OUT) *ap = a;
+      }
+      yp += ld;
+      if (ACC_OUT) ap += ld;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float f = __shfl_sync(0xffffffffu, f_mine, j);
+      const int32_t a = static_cast<int32_t>(r[j]);
+      if (row_ok && t0 + j < p.T) {
+        *yp = __fmul_rn(static_cast<float>(a), f);
+        if (ACC_OUT) *ap = a;
+      }
+      yp += ld;
+      if (ACC_OUT) ap += ld;
     }
   }
 }
 
 // Dense int8: A = W_eff codes [n_out][K], B = xq [T][K]; UMMA 128 x 256 x 32.
+template <bool ACC_OUT>
 struct CfgFwdDense {
   using Params = FwdParams;
   static constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
@@ -362,8 +385,8 @@ struct CfgFwdDense {
       __syncwarp();
       tmem_load_32x32b_x32(t_acc + c * 32, r);
       tmem_load_wait();
-      if (n0 + c * 32 >= p.T) continue;  // uniform across the warp  // uniform across the warp
-      fwd_epilogue_chunk(p, r, row, n0 + c * 32, lane, g);
+      if (n0 + c * 32 >= p.T) continue;  // uniform across the warp
+      fwd_epilogue_chunk<ACC_OUT>(p, r, row, n0 + c * 32, lane, g);
     }
   }
 };
@@ -371,6 +394,7 @@ struct CfgFwdDense {
 // 2:4 sparse int8: A = kept codes [n_out][K/2] plus metadata, B = xq [T][K].
 // One stage covers 256 logical k: A 128 x 128 bytes, B 2 x [128 rows][128
 // bytes], metadata 2 blocks of 128 rows x 16 bytes.  UMMA 128 x 128 x 64.
+template <bool ACC_OUT>
 struct CfgFwdSparse {
   using Params = FwdParams;
   static constexpr int BM = 128, BN = 128, BK = 256, STAGES = 4;
@@ -420,7 +444,7 @@ struct CfgFwdSparse {
       tmem_load_32x32b_x32(t_acc + c * 32, r);
       tmem_load_wait();
       if (n0 + c * 32 >= p.T) continue;  // uniform across the warp
-      fwd_epilogue_chunk(p, r, row, n0 + c * 32, lane, g);
+      fwd_epilogue_chunk<ACC_OUT>(p, r, row, n0 + c * 32, lane, g);
     }
   }
 };

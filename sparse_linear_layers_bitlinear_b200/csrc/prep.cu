@@ -6,6 +6,16 @@
 // Semi-Structured Sparsity" -- gist.science German technical summary §2
 // (magnitude mask from the masters, quantise then mask), Korean summary
 // §2.1-2.2 (per-step recompute), French summary §2.
+//
+// Three kernels:
+//   k_absmean_partials  streams W once, adds every |w| exactly into per-block
+//                       integer bins
+//   k_gamma_finalize    one block: folds the bins, rounds the exact mean once to
+//                       fp32, writes gamma, g and the header
+//   k_prep_pack<M>      re-reads W (from L2), masks, ternarises and writes every
+//                       packed section
+// The last two are launched with programmatic stream serialisation, so their
+// launches overlap the tail of the kernel before them.
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
@@ -13,289 +23,438 @@
 namespace sbl {
 
 // ---------------------------------------------------------------------------
-// Header reset: shapes, zeroed exact-sum bins, cleared status.
-// ---------------------------------------------------------------------------
-__global__ void k_prep_header(BlobHeader* h, int64_t n_out, int64_t k, int n, int m, uint32_t flags) {
-  const int i = threadIdx.x;
-  if (i < 32) h->bins[i] = 0ull;
-  if (i == 0) {
-    h->magic = kMagic;
-    h->version = 1;
-    h->n_out = n_out;
-    h->k = k;
-    h->n = n;
-    h->m = m;
-    h->flags = flags;
-    h->gamma = 0.0f;
-    h->g = 0.0f;
-    h->status = 0u;
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Exact sum of |w| (absmean numerator).
 //
 // In units of 2^-133 a bf16 magnitude (biased exponent e, mantissa f) is the
-// integer sig << s with sig = (e ? 128 + f : f) and s = max(e, 1) - 1.  Each
-// lane keeps 32 private 32-bit bins in shared memory, bin b = s >> 3 holding
-// sum(sig << (s & 7)) (< 2^15 per add, so 2^17 adds per lane cannot
-// overflow); the block folds its bins into 64-bit global bins.  The exact
-// total is sum_b bins[b] << 8b, formed in k_gamma_finalize.
+// integer sig << s with sig = (e ? 128 + f : f) and s = max(e, 1) - 1 <= 253,
+// i.e. sig - s * 128 = mag - s * 128 with mag = e * 128 + f.  Each lane keeps
+// 32 private 32-bit bins in shared memory, bin b = s >> 3 collecting
+// sig << (s & 7) (< 2^15 per add).  A round lets each lane add at most 2^16
+// weights, so no bin overflows; after each round the block folds its lanes'
+// bins into 64-bit totals.  A slot bin b is an integer in units of 2^(8b-133).
 // ---------------------------------------------------------------------------
-constexpr int kBinWarps = 8;
+constexpr int kAbsThreads = 1024;
+constexpr int kAbsWarps = kAbsThreads / 32;
+constexpr int kLaneBins = 32;
+constexpr int64_t kRoundVecs = 8192;  // 16-byte vectors per thread per round (8 weights each)
 
-__global__ void __launch_bounds__(kBinWarps * 32) k_absmean_bins(const uint4* __restrict__ w, int64_t nvec,
-                                                                 BlobHeader* h) {
-  __shared__ uint32_t bins[kBinWarps][32][32];  // [warp][bin][lane]
+__global__ void __launch_bounds__(kAbsThreads, 1)
+    k_absmean_partials(const uint4* __restrict__ w, int64_t nvec, uint64_t* __restrict__ slot_bins,
+                       uint32_t* __restrict__ slot_flags) {
+  extern __shared__ uint32_t lane_bins[];  // [warp][bin][lane]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int b = 0; b < 32; ++b) bins[warp][b][lane] = 0u;
+  uint32_t* my = lane_bins + warp * (kLaneBins * 32) + lane;
 
-  uint32_t bad = 0;
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t emax = 0;
   auto consume = [&](const uint4 v) {
     const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const uint32_t mag = (words[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
       const uint32_t e = mag >> 7;
-      bad |= (e == 0xFFu);
-      const uint32_t sig = (mag & 0x7Fu) | (e ? 0x80u : 0u);
-      const uint32_t s = (e ? e : 1u) - 1u;
-      bins[warp][(s >> 3) & 31u][lane] += sig << (s & 7u);
+      emax = max(emax, e);
+      const uint32_t s = max(e, 1u) - 1u;
+      const uint32_t sig = mag - (s << 7);
+      my[(s >> 3) * 32] += sig << (s & 7u);
     }
   };
-  // Four independent 16-byte loads in flight per thread.
-  for (; i + 3 * stride < nvec; i += 4 * stride) {
-    // default caching: the pack pass re-reads W right after this one
-    const uint4 v0 = __ldg(w + i);
-    const uint4 v1 = __ldg(w + i + stride);
-    const uint4 v2 = __ldg(w + i + 2 * stride);
-    const uint4 v3 = __ldg(w + i + 3 * stride);
-    consume(v0);
-    consume(v1);
-    consume(v2);
-    consume(v3);
-  }
-  for (; i < nvec; i += stride) consume(__ldg(w + i));
 
-  __syncthreads();
-  // Thread (bin = tid / 8, part = tid % 8) sums warp `part`'s 32 lanes of that bin.
-  const int bin = threadIdx.x >> 3, part = threadIdx.x & 7;
-  unsigned long long sum = 0ull;
-#pragma unroll 4
-  for (int l = 0; l < 32; ++l) sum += bins[part][bin][(l + lane) & 31];
-  sum += __shfl_down_sync(0xffffffffu, sum, 4, 8);
-  sum += __shfl_down_sync(0xffffffffu, sum, 2, 8);
-  sum += __shfl_down_sync(0xffffffffu, sum, 1, 8);
-  if (part == 0 && sum != 0ull) atomicAdd(&h->bins[bin], sum);
-  if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(&h->status, SBL_STATUS_NONFINITE_W);
-}
-
-// ---------------------------------------------------------------------------
-// gamma = RN_fp32(S * 2^-133 / numel), S = sum_b bins[b] << 8b (exact).
-// Limb-wise long division of S * 2^128 by numel, then nearest-even rounding
-// of the quotient to fp32 (normal or subnormal) from its bits plus sticky.
-// ---------------------------------------------------------------------------
-__device__ void add_limb(uint64_t* x, int nlimbs, int i, uint64_t v) {
-  while (v != 0ull && i < nlimbs) {
-    const uint64_t before = x[i];
-    x[i] += v;
-    v = (x[i] < before) ? 1ull : 0ull;
-    ++i;
-  }
-}
-
-__global__ void k_gamma_finalize(BlobHeader* h, int64_t numel) {
-  if (threadIdx.x != 0) return;
-  // X = S << 128 in seven 64-bit limbs (S < 2^312).
-  uint64_t X[7] = {0, 0, 0, 0, 0, 0, 0};
-  for (int b = 0; b < 32; ++b) {
-    const uint64_t v = h->bins[b];
-    if (v == 0ull) continue;
-    const int shift = 8 * b + 128;
-    const int li = shift >> 6, off = shift & 63;
-    add_limb(X, 7, li, v << off);
-    if (off != 0) add_limb(X, 7, li + 1, v >> (64 - off));
-  }
-  float gamma = 0.0f;
-  bool nonzero = false;
-  for (int i = 0; i < 7; ++i) nonzero |= (X[i] != 0ull);
-  if (h->status & SBL_STATUS_NONFINITE_W) {
-    gamma = __int_as_float(0x7fc00000);
-  } else if (nonzero) {
-    const uint64_t n = static_cast<uint64_t>(numel);
-    uint64_t Q[7];
-    unsigned __int128 rem = 0;
-    for (int i = 6; i >= 0; --i) {
-      const unsigned __int128 cur = (rem << 64) | X[i];
-      Q[i] = static_cast<uint64_t>(cur / n);
-      rem = cur % n;
+  const int64_t stride = int64_t(gridDim.x) * kAbsThreads;
+  const int64_t round = stride * kRoundVecs;
+  uint64_t total = 0;  // thread (bin = warp, part = lane) keeps the block total of its bin
+  for (int64_t r0 = 0; r0 < nvec; r0 += round) {
+#pragma unroll
+    for (int b = 0; b < kLaneBins; ++b) my[b * 32] = 0u;
+    const int64_t r1 = (nvec - r0 < round) ? nvec : r0 + round;
+    int64_t i = r0 + int64_t(blockIdx.x) * kAbsThreads + threadIdx.x;
+    // Four independent 16-byte loads in flight per thread (default caching:
+    // the pack kernel re-reads W right after this one).
+    for (; i + 3 * stride < r1; i += 4 * stride) {
+      const uint4 v0 = __ldg(w + i);
+      const uint4 v1 = __ldg(w + i + stride);
+      const uint4 v2 = __ldg(w + i + 2 * stride);
+      const uint4 v3 = __ldg(w + i + 3 * stride);
+      consume(v0);
+      consume(v1);
+      consume(v2);
+      consume(v3);
     }
-    // Q = floor(S * 2^128 / n); bit j of Q has real weight 2^(j - 261).
-    int top = -1;
-    for (int i = 6; i >= 0 && top < 0; --i)
-      if (Q[i]) top = 64 * i + 63 - __clzll(static_cast<long long>(Q[i]));
-    auto qbit = [&](int j) -> uint32_t { return static_cast<uint32_t>((Q[j >> 6] >> (j & 63)) & 1ull); };
-    const int e = top - 261;
-    const int lsb = max(e - 23, -149);
-    const int lsb_pos = lsb + 261;  // >= 112
-    uint32_t mant = 0;
-    for (int j = top; j >= lsb_pos; --j) mant = (mant << 1) | qbit(j);
-    const uint32_t round_bit = qbit(lsb_pos - 1);
-    bool sticky = (rem != 0);
-    for (int j = lsb_pos - 2; j >= 0 && !sticky; --j) sticky = qbit(j) != 0u;
-    if (round_bit && (sticky || (mant & 1u))) ++mant;
-    // value = mant * 2^lsb; the pattern below covers subnormals and the carry.
-    gamma = __uint_as_float((static_cast<uint32_t>(lsb + 149) << 23) + mant);
-  }
-  h->gamma = gamma;
-  h->g = (gamma > 1e-5f) ? gamma : 1e-5f;  // NaN gamma gives 1e-5; the status word says why
-}
-
-// ---------------------------------------------------------------------------
-// Mask, ternarise, pack.  One thread per 32 consecutive weights of a row.
-// ---------------------------------------------------------------------------
-template <int M>
-__global__ void __launch_bounds__(256) k_prep_pack(const uint16_t* __restrict__ w, int64_t n_out, int64_t k, int n,
-                                                   const BlobHeader* __restrict__ h, PackOut out) {
-  const float g = h->g;
-  const int64_t chunks_per_row = k / 32;
-  const int64_t total = n_out * chunks_per_row;
-  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-       idx += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = idx / chunks_per_row, c = idx % chunks_per_row;
-    const uint4* src = reinterpret_cast<const uint4*>(w + r * k + 32 * c);
-    uint32_t wv[16];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 x = __ldcs(src + v);
-      wv[4 * v + 0] = x.x;
-      wv[4 * v + 1] = x.y;
-      wv[4 * v + 2] = x.z;
-      wv[4 * v + 3] = x.w;
-    }
-    auto bits_of = [&](int j) -> uint32_t { return (wv[j >> 1] >> (16 * (j & 1))) & 0xFFFFu; };
-
-    // Ternary code of every weight: sign(w) when 2|w| > g (exact fp32), else 0.
-    int code[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t b = bits_of(j);
-      const float v = __uint_as_float(b << 16);
-      code[j] = (__fmul_rn(2.0f, fabsf(v)) > g) ? ((b & 0x8000u) ? -1 : 1) : 0;
-    }
-    // N:M selection on the magnitude bits: keep rank < n, where rank counts
-    // larger magnitudes plus equal ones at lower index.
-    uint32_t kept = 0;  // bit j: weight j of the chunk is kept
-#pragma unroll
-    for (int gi = 0; gi < 32 / M; ++gi) {
-#pragma unroll
-      for (int a = 0; a < M; ++a) {
-        const uint32_t ka = bits_of(gi * M + a) & 0x7FFFu;
-        int rank = 0;
-#pragma unroll
-        for (int b = 0; b < M; ++b) {
-          if (b == a) continue;
-          const uint32_t kb = bits_of(gi * M + b) & 0x7FFFu;
-          rank += (kb > ka) || (kb == ka && b < a);
-        }
-        if (rank < n) kept |= 1u << (gi * M + a);
-      }
-    }
-
-    // mask bytes: 32/M groups, each M bits
+    for (; i < r1; i += stride) consume(__ldg(w + i));
+    __syncthreads();
+    // Warp `bin` folds bin `bin`: lane p sums the 32 lanes of warp p.
     {
-      uint8_t mb[32 / M];
+      const int bin = warp, part = lane;
+      const uint32_t* src = lane_bins + part * (kLaneBins * 32) + bin * 32;
+      uint64_t sum = 0;
+#pragma unroll 8
+      for (int l = 0; l < 32; ++l) sum += src[(l + lane) & 31];
 #pragma unroll
-      for (int gi = 0; gi < 32 / M; ++gi) mb[gi] = static_cast<uint8_t>((kept >> (gi * M)) & ((1u << M) - 1u));
-      uint8_t* dst = out.mask + r * (k / M) + c * (32 / M);
-#pragma unroll
-      for (int gi = 0; gi < 32 / M; ++gi) dst[gi] = mb[gi];
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      total += sum;
     }
-    // W_eff as exact bf16 (+1 = 0x3F80, -1 = 0xBF80, 0)
-    {
-      uint32_t pk[16];
+    __syncthreads();
+  }
+  if (lane == 0) slot_bins[int64_t(blockIdx.x) * kExactBins + warp] = total;
+  if (threadIdx.x < kExactBins - kLaneBins) slot_bins[int64_t(blockIdx.x) * kExactBins + kLaneBins + threadIdx.x] = 0ull;
+  const int bad = __syncthreads_or(emax == 0xFFu);
+  if (threadIdx.x == 0) slot_flags[blockIdx.x] = bad ? SBL_STATUS_NONFINITE_W : 0u;
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// gamma = RN_fp32(S * 2^-133 / numel) with S = sum_b bins[b] << 8b exactly.
+// S (< 2^310) is assembled in six 64-bit limbs, normalised to a 128-bit
+// integer N with its top bit at 127 (bits shifted out only feed the sticky
+// bit), one 128/64 division gives a quotient of at least 86 bits, and that
+// quotient is rounded to nearest-even at the fp32 precision (24 bits, or the
+// 2^-149 step for subnormal results).  Straight-line code on registers.
+// ---------------------------------------------------------------------------
+constexpr int kLimbs = 6;
+
+__device__ float exact_mean_fp32(const uint64_t* bins, uint64_t numel) {
+  unsigned __int128 T[kLimbs];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        uint32_t lo = 0, hi = 0;
-        const int c0 = (kept >> (2 * j)) & 1u ? code[2 * j] : 0;
-        const int c1 = (kept >> (2 * j + 1)) & 1u ? code[2 * j + 1] : 0;
-        lo = c0 == 0 ? 0u : (c0 > 0 ? 0x3F80u : 0xBF80u);
-        hi = c1 == 0 ? 0u : (c1 > 0 ? 0x3F80u : 0xBF80u);
-        pk[j] = lo | (hi << 16);
-      }
-      uint4* dst = reinterpret_cast<uint4*>(out.weff_bf16 + r * k + 32 * c);
+  for (int L = 0; L < kLimbs; ++L) T[L] = 0;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  for (int b = 0; b < kExactBins; ++b) {
+    const uint64_t v = bins[b];  // < 2^60
+    const int sh = 8 * b, L = sh >> 6, off = sh & 63;
+    T[L] += static_cast<unsigned __int128>(v << off);
+    if (off != 0 && L + 1 < kLimbs) T[L + 1] += static_cast<unsigned __int128>(v >> (64 - off));
+  }
+  uint64_t S[kLimbs];
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L) {
+    S[L] = static_cast<uint64_t>(T[L]);
+    if (L + 1 < kLimbs) T[L + 1] += T[L] >> 64;
+  }
+  int topS = -1;
+#pragma unroll
+  for (int L = kLimbs - 1; L >= 0; --L)
+    if (topS < 0 && S[L] != 0ull) topS = 64 * L + 63 - __clzll(static_cast<long long>(S[L]));
+  if (topS < 0) return 0.0f;
+  // the 64 bits of S starting at bit pos (pos may be negative: zeros below bit 0)
+  auto get64 = [&](int pos) -> uint64_t {
+    uint64_t r = 0;
+#pragma unroll
+    for (int L = 0; L < kLimbs; ++L) {
+      const int d = 64 * L - pos;
+      if (d >= 0 && d < 64) r |= S[L] << d;
+      else if (d < 0 && d > -64) r |= S[L] >> (-d);
     }
-    if (out.codes != nullptr) {  // dense int8 W_eff codes
-      uint32_t pk[8];
+    return r;
+  };
+  const int low = topS - 127;  // bit of S that lands at bit 0 of N
+  const unsigned __int128 N = (static_cast<unsigned __int128>(get64(low + 64)) << 64) | get64(low);
+  bool sticky0 = false;
+#pragma unroll
+  for (int L = 0; L < kLimbs; ++L) {
+    const int lim = low - 64 * L;  // bits of limb L below `low`
+    if (lim >= 64) sticky0 |= S[L] != 0ull;
+    else if (lim > 0) sticky0 |= (S[L] & ((1ull << lim) - 1ull)) != 0ull;
+  }
+  const unsigned __int128 q = N / numel;
+  const bool rem_nz = (N % numel) != 0;
+  // bit j of q has weight 2^(j + topS - 260); q >= 2^86
+  const uint64_t q_hi = static_cast<uint64_t>(q >> 64), q_lo = static_cast<uint64_t>(q);
+  const int topq = q_hi ? 127 - __clzll(static_cast<long long>(q_hi)) : 63 - __clzll(static_cast<long long>(q_lo));
+  const int E = topq + topS - 260;
+  const int lsb = (E - 23 > -149) ? E - 23 : -149;
+  const int sh = lsb - (topS - 260);  // bit of q that becomes the last mantissa bit; 63 <= sh <= 111
+  uint64_t mant = static_cast<uint64_t>(q >> sh);
+  const int rpos = sh - 1;
+  const uint32_t round_bit = static_cast<uint32_t>((q >> rpos) & 1u);
+  const bool below = (q & ((static_cast<unsigned __int128>(1) << rpos) - 1u)) != 0;
+  const bool sticky = sticky0 || rem_nz || below;
+  if (round_bit && (sticky || (mant & 1ull))) ++mant;
+  // value = mant * 2^lsb: the pattern covers subnormals and the rounding carry.
+  return __uint_as_float((static_cast<uint32_t>(lsb + 149) << 23) + static_cast<uint32_t>(mant));
+}
+
+// ---------------------------------------------------------------------------
+// Fold the per-block partial sums, compute gamma and g, write the header.
+// One block.  It lets the pack kernel start launching right away (that kernel
+// waits for this one to complete before it reads g), then waits for the
+// partial sums.
+// ---------------------------------------------------------------------------
+constexpr int kFinGroups = 25;                       // slot groups
+constexpr int kFinThreads = kFinGroups * kExactBins;  // 1000 threads: (group, bin) pairs
+
+__global__ void __launch_bounds__(1024) k_gamma_finalize(const uint64_t* slot_bins, const uint32_t* slot_flags,
+                                                         int nslots, BlobHeader* h, int64_t n_out, int64_t k, int n,
+                                                         int m, uint32_t layer_flags) {
+  __shared__ uint64_t s_part[kFinGroups][kExactBins];
+  __shared__ uint64_t s_bins[kExactBins];
+  __shared__ uint32_t s_flags;
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x;
+  if (tid == 0) s_flags = 0u;
+  if (tid < kFinThreads) {
+    // Group grp folds slots grp, grp + 25, ...: all its loads are issued before
+    // any add, so the fold costs one memory round trip.
+    const int bin = tid % kExactBins, grp = tid / kExactBins;
+    const int per = (nslots - grp + kFinGroups - 1) / kFinGroups;  // slots of this group
+    uint64_t v[8];
+    uint64_t a = 0;
+    for (int j0 = 0; j0 < per; j0 += 8) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int idx2 = 4 * j + e;
-          const int cv = ((kept >> idx2) & 1u) ? code[idx2] : 0;
-          word |= (static_cast<uint32_t>(cv) & 0xFFu) << (8 * e);
-        }
-        pk[j] = word;
+        const int slot = grp + (j0 + j) * kFinGroups;
+        v[j] = (j0 + j < per) ? __ldcg(slot_bins + int64_t(slot) * kExactBins + bin) : 0ull;
       }
-      uint4* dst = reinterpret_cast<uint4*>(out.codes + r * k + 32 * c);
-      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a += v[j];
     }
-    if (M == 4 && out.sp_values != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
-      uint32_t vals[4] = {0, 0, 0, 0};
-      uint32_t meta = 0;
-      uint32_t gemv[2] = {0, 0};
+    s_part[grp][bin] = a;
+  }
+  __syncthreads();
+  uint32_t f = 0;
+  for (int i = tid; i < nslots; i += blockDim.x) f |= __ldcg(slot_flags + i);
+  if (f) atomicOr(&s_flags, f);
+  if (tid < kExactBins) {
+    uint64_t t = 0;
+#pragma unroll 5
+    for (int g2 = 0; g2 < kFinGroups; ++g2) t += s_part[g2][tid];
+    s_bins[tid] = t;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t flags = s_flags;
+    const bool bad = (flags & SBL_STATUS_NONFINITE_W) != 0u;
+    const float gamma = bad ? __int_as_float(0x7fc00000) : exact_mean_fp32(s_bins, uint64_t(n_out) * uint64_t(k));
+    h->magic = kMagic;
+    h->version = 2;
+    h->n_out = n_out;
+    h->k = k;
+    h->n = n;
+    h->m = m;
+    h->flags = layer_flags;
+    h->gamma = gamma;
+    h->g = (gamma > 1e-5f) ? gamma : 1e-5f;  // a NaN gamma gives 1e-5; the status word says why
+    h->status = flags;                        // a new prepare resets the status word
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Mask, ternarise, pack.  Lane = 8 consecutive weights of a row (one 16-byte
+// vector); a warp covers 256 consecutive weights, so every load and most
+// stores are contiguous across the warp.  k is a multiple of 64, so a row has
+// a multiple of 8 lanes' worth of weights and no group or quad of lanes
+// straddles two rows.
+//
+// Bit tricks (all exact):
+//  * code != 0  <=>  2|w| > g  <=>  |w| > g/2 (g/2 is exact)  <=>  the 15-bit
+//    magnitude field exceeds bits(g/2) >> 16, compared two at a time with
+//    __vcmpgtu2 on the packed bf16 pairs;
+//  * W_eff as bf16 is (sign | 0x3F80) masked by (kept & code != 0);
+//  * the int8 code byte of a bf16 W_eff value h is (h bit 13) | 0xFE * (h bit 15).
+// ---------------------------------------------------------------------------
+constexpr int kPackThreads = 512;
+
+// (i0 | i1 << 2) for each 4-bit kept pattern with exactly two bits set.
+constexpr uint64_t kPairNibble = (uint64_t(0x4) << (4 * 0x3)) | (uint64_t(0x8) << (4 * 0x5)) |
+                                 (uint64_t(0x9) << (4 * 0x6)) | (uint64_t(0xC) << (4 * 0x9)) |
+                                 (uint64_t(0xD) << (4 * 0xA)) | (uint64_t(0xE) << (4 * 0xC));
+
+// Keep-bits of one group of M magnitudes: position a is kept when fewer than
+// n positions beat it, where b beats a if |w_b| > |w_a|, or if they are equal
+// and b < a.  For b < a that is |w_b| >= |w_a|.
+template <int M>
+__device__ __forceinline__ uint32_t keep_bits(const uint32_t (&mag)[8], int base, int n) {
+  int rank[M];
 #pragma unroll
-      for (int gi = 0; gi < 8; ++gi) {
-        const uint32_t bits = (kept >> (4 * gi)) & 0xFu;
-        // two lowest set bits, ascending (exactly two are set for n == 2)
-        const int i0 = __ffs(bits) - 1;
-        const int i1 = __ffs(bits & (bits - 1u)) - 1;
-        const int v0 = code[4 * gi + i0], v1 = code[4 * gi + i1];
-        const uint32_t nib = uint32_t(i0) | (uint32_t(i1) << 2);
-        meta |= nib << (4 * gi);
-        vals[gi >> 1] |= ((uint32_t(v0) & 0xFFu) | ((uint32_t(v1) & 0xFFu) << 8)) << (16 * (gi & 1));
-        const uint32_t gb = (nib << 4) | (uint32_t(v0) & 3u) | ((uint32_t(v1) & 3u) << 2);
-        gemv[gi >> 2] |= gb << (8 * (gi & 3));
+  for (int a = 0; a < M; ++a) rank[a] = 0;
+#pragma unroll
+  for (int i = 0; i < M; ++i)
+#pragma unroll
+    for (int j = i + 1; j < M; ++j) {
+      const int i_wins = mag[base + i] >= mag[base + j] ? 1 : 0;  // i < j: ties go to i
+      rank[j] += i_wins;
+      rank[i] += 1 - i_wins;
+    }
+  uint32_t kept = 0;
+#pragma unroll
+  for (int a = 0; a < M; ++a) kept |= (rank[a] < n ? 1u : 0u) << a;
+  return kept;
+}
+
+// Groups of four: the six pairwise outcomes c_ij = (|w_i| >= |w_j|), i < j,
+// index a 64-entry table whose byte holds the keep pattern (bits 0..3) and,
+// for n == 2, the metadata nibble i0 | i1 << 2 (bits 4..7).
+__device__ __forceinline__ uint32_t pair_outcomes4(const uint32_t (&mag)[8], int base) {
+  const uint32_t a = mag[base], b = mag[base + 1], c = mag[base + 2], d = mag[base + 3];
+  return (a >= b ? 1u : 0u) | (a >= c ? 2u : 0u) | (a >= d ? 4u : 0u) | (b >= c ? 8u : 0u) | (b >= d ? 16u : 0u) |
+         (c >= d ? 32u : 0u);
+}
+
+__device__ __forceinline__ uint32_t select4_entry(uint32_t cbits, int n) {
+  const uint32_t c01 = cbits & 1u, c02 = (cbits >> 1) & 1u, c03 = (cbits >> 2) & 1u;
+  const uint32_t c12 = (cbits >> 3) & 1u, c13 = (cbits >> 4) & 1u, c23 = (cbits >> 5) & 1u;
+  const uint32_t r0 = 3u - c01 - c02 - c03;
+  const uint32_t r1 = c01 + 2u - c12 - c13;
+  const uint32_t r2 = c02 + c12 + 1u - c23;
+  const uint32_t r3 = c03 + c13 + c23;
+  const uint32_t kept = (r0 < uint32_t(n) ? 1u : 0u) | (r1 < uint32_t(n) ? 2u : 0u) | (r2 < uint32_t(n) ? 4u : 0u) |
+                        (r3 < uint32_t(n) ? 8u : 0u);
+  const uint32_t nib = static_cast<uint32_t>(kPairNibble >> (4 * kept)) & 0xFu;
+  return kept | (nib << 4);
+}
+
+// int8 codes (+1 = 0x01, -1 = 0xFF, 0) of four bf16 W_eff values held in two
+// words: their high bytes are 0x3F, 0xBF or 0x00.
+__device__ __forceinline__ uint32_t code_bytes4(uint32_t weff_lo, uint32_t weff_hi) {
+  const uint32_t hb = __byte_perm(weff_lo, weff_hi, 0x7531);
+  return ((hb >> 5) & 0x01010101u) | (((hb >> 7) & 0x01010101u) * 0xFEu);
+}
+
+template <int M>
+__global__ void __launch_bounds__(kPackThreads)
+    k_prep_pack(const uint4* __restrict__ w, int64_t n_out, int64_t k, int n, const BlobHeader* h, PackOut out) {
+  __shared__ uint32_t s_sel[64];  // M == 4: keep pattern and nibble per comparison outcome
+  if (M == 4 && threadIdx.x < 64) s_sel[threadIdx.x] = select4_entry(threadIdx.x, n);
+  __syncthreads();
+  pdl_wait();  // g comes from k_gamma_finalize (a kernel that may overlap this one: coherent load)
+  const float g = __ldcg(&h->g);
+  // code != 0 <=> 15-bit magnitude > thr; adding (0x7FFF - thr) to each half
+  // sets that half's bit 15 exactly then (no carry leaves a half).
+  const uint32_t thr = __float_as_uint(__fmul_rn(g, 0.5f)) >> 16;
+  const uint32_t bias2 = (0x7FFFu - thr) * 0x00010001u;
+  pdl_trigger();
+
+  const int lane = threadIdx.x & 31;
+  const int upr = static_cast<int>(k / 8);  // lanes' worth of weights per row (multiple of 8)
+  const int64_t gwarp = int64_t(blockIdx.x) * (kPackThreads / 32) + (threadIdx.x >> 5);
+  const int64_t nwarps = int64_t(gridDim.x) * (kPackThreads / 32);
+  for (int64_t row = gwarp; row < n_out; row += nwarps) {
+    const uint4* wrow = w + row * upr;
+    uint4* weff_row = reinterpret_cast<uint4*>(out.weff_bf16) + row * upr;
+    // Four 16-byte loads in flight per lane, then process them one by one.
+    for (int c0 = 0; c0 < upr; c0 += 4 * 32) {
+      uint4 vbuf[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int cq = c0 + 32 * q + lane;
+        vbuf[q] = (cq < upr) ? __ldcs(wrow + cq) : make_uint4(0, 0, 0, 0);
       }
-      *reinterpret_cast<uint4*>(out.sp_values + r * (k / 2) + 16 * c) = make_uint4(vals[0], vals[1], vals[2], vals[3]);
-      // tensor-core metadata: [row_block][k_block][128 rows][16 bytes]
-      const int64_t rb = r >> 7, rr = r & 127;
-      const int64_t kblk = (32 * c) >> 7;
-      const int64_t byte_in_row = ((32 * c) & 127) >> 3;  // 4 bytes per 32 weights
-      uint8_t* mdst = out.sp_meta + ((rb * out.meta_kblocks + kblk) * 128 + rr) * 16 + byte_in_row;
-      *reinterpret_cast<uint32_t*>(mdst) = meta;
-      if (out.gemv != nullptr)
-        *reinterpret_cast<uint2*>(out.gemv + r * (k / 4) + 8 * c) = make_uint2(gemv[0], gemv[1]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (c0 + 32 * q >= upr) break;  // uniform across the warp
+        const int c = c0 + 32 * q + lane;
+        const bool active = c < upr;  // upr is a multiple of 8: quads are all-or-nothing
+        const uint32_t wd[4] = {vbuf[q].x, vbuf[q].y, vbuf[q].z, vbuf[q].w};
+        uint32_t mag[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          mag[2 * j] = wd[j] & 0x7FFFu;
+          mag[2 * j + 1] = wd[j] >> 16 & 0x7FFFu;
+        }
+        uint32_t kept = 0, sel0 = 0, sel1 = 0;
+        if (M == 4) {
+          sel0 = s_sel[pair_outcomes4(mag, 0)];
+          sel1 = s_sel[pair_outcomes4(mag, 4)];
+          kept = (sel0 & 0xFu) | ((sel1 & 0xFu) << 4);
+        } else {
+#pragma unroll
+          for (int gi = 0; gi < 8 / M; ++gi) kept |= keep_bits<M>(mag, gi * M, n) << (gi * M);
+        }
+
+        // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and code != 0.
+        uint32_t weff[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t nz = ((((wd[j] & 0x7FFF7FFFu) + bias2) >> 15) & 0x00010001u) * 0xFFFFu;
+          const uint32_t kp = (kept >> (2 * j)) & 3u;
+          const uint32_t km = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
+          weff[j] = ((wd[j] & 0x80008000u) | 0x3F803F80u) & nz & km;
+        }
+        const uint32_t codes_lo = code_bytes4(weff[0], weff[1]);  // weights 0..3
+        const uint32_t codes_hi = code_bytes4(weff[2], weff[3]);  // weights 4..7
+
+        if (active) {
+          if (M == 2) {
+            const uint32_t mw = (kept & 3u) | (((kept >> 2) & 3u) << 8) | (((kept >> 4) & 3u) << 16) |
+                                (((kept >> 6) & 3u) << 24);
+            reinterpret_cast<uint32_t*>(out.mask + row * (k / 2))[c] = mw;
+          } else if (M == 4) {
+            const uint32_t mw = (kept & 0xFu) | (((kept >> 4) & 0xFu) << 8);
+            reinterpret_cast<uint16_t*>(out.mask + row * (k / 4))[c] = static_cast<uint16_t>(mw);
+          } else {
+            out.mask[row * (k / 8) + c] = static_cast<uint8_t>(kept);
+          }
+          weff_row[c] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
+          if (out.codes != nullptr) reinterpret_cast<uint2*>(out.codes + row * k)[c] = make_uint2(codes_lo, codes_hi);
+        }
+        if (M == 4 && out.sp_values != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
+          const uint32_t nib0 = sel0 >> 4, nib1 = sel1 >> 4;
+          // the two kept codes of each group, in index order
+          const uint32_t v0 = __byte_perm(codes_lo, 0u, (nib0 & 3u) | ((nib0 >> 2) << 4));
+          const uint32_t v1 = __byte_perm(codes_hi, 0u, (nib1 & 3u) | ((nib1 >> 2) << 4));
+          const uint32_t vals = (v0 & 0xFFFFu) | (v1 << 16);
+          const uint32_t meta = nib0 | (nib1 << 4);
+          // tensor-core metadata: [row_block][k_block][128 rows][16 bytes]; this
+          // lane's byte is byte (c % 16) of the row's 16 bytes in k block c / 16.
+          uint32_t word = meta << (8 * (lane & 3));
+          word |= __shfl_xor_sync(0xffffffffu, word, 1);
+          word |= __shfl_xor_sync(0xffffffffu, word, 2);
+          if (active) {
+            reinterpret_cast<uint32_t*>(out.sp_values + row * (k / 2))[c] = vals;
+            if ((lane & 3) == 0) {
+              uint8_t* mrow = out.sp_meta + ((row >> 7) * out.meta_kblocks * 128 + (row & 127)) * 16;
+              *reinterpret_cast<uint32_t*>(mrow + (c >> 4) * 2048 + (c & 15)) = word;
+            }
+            if (out.gemv != nullptr) {
+              const uint32_t g0 = (nib0 << 4) | (v0 & 3u) | (((v0 >> 8) & 3u) << 2);
+              const uint32_t g1 = (nib1 << 4) | (v1 & 3u) | (((v1 >> 8) & 3u) << 2);
+              reinterpret_cast<uint16_t*>(out.gemv + row * (k / 4))[c] = static_cast<uint16_t>(g0 | (g1 << 8));
+            }
+          }
+        }
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Host launchers
+// Host launcher
 // ---------------------------------------------------------------------------
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
                            uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s) {
   BlobHeader* h = reinterpret_cast<BlobHeader*>(blob + L.header);
-  k_prep_header<<<1, 64, 0, s>>>(h, n_out, k, n, m, flags);
+  uint64_t* slot_bins = reinterpret_cast<uint64_t*>(blob + L.scratch);
+  uint32_t* slot_flags = reinterpret_cast<uint32_t*>(blob + L.scratch + uint64_t(kPrepSlots) * kExactBins * 8);
   if (L.sp_meta && (n_out % 128 != 0 || k % 256 != 0)) {
     cudaError_t e = cudaMemsetAsync(blob + L.sp_meta, 0x44, L.sp_meta_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  const int64_t numel = n_out * k;
-  const int64_t nvec = numel / 8;
-  // Enough blocks that no lane adds more than 2^16 weights into one bin.
-  int64_t blocks = int64_t(num_sms) * 2;
-  const int64_t min_blocks = (numel + (int64_t(256) << 16) - 1) / (int64_t(256) << 16);
-  if (blocks < min_blocks) blocks = min_blocks;
-  k_absmean_bins<<<static_cast<unsigned>(blocks), kBinWarps * 32, 0, s>>>(reinterpret_cast<const uint4*>(w), nvec, h);
-  k_gamma_finalize<<<1, 32, 0, s>>>(h, numel);
+  const int64_t nvec = n_out * k / 8;
+  int slots = num_sms < kPrepSlots ? num_sms : kPrepSlots;
+  const int64_t need = (nvec + kAbsThreads - 1) / kAbsThreads;
+  if (need < slots) slots = static_cast<int>(need);
+  constexpr int abs_smem = kAbsWarps * kLaneBins * 32 * 4;  // 128 KB of lane bins
+  static const cudaError_t attr_err =
+      cudaFuncSetAttribute(k_absmean_partials, cudaFuncAttributeMaxDynamicSharedMemorySize, abs_smem);
+  if (attr_err != cudaSuccess) return attr_err;
+  k_absmean_partials<<<slots, kAbsThreads, abs_smem, s>>>(reinterpret_cast<const uint4*>(w), nvec, slot_bins,
+                                                          slot_flags);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
 
   PackOut out;
   out.mask = blob + L.mask;
@@ -305,15 +464,22 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   out.sp_meta = L.sp_meta ? blob + L.sp_meta : nullptr;
   out.gemv = L.gemv ? blob + L.gemv : nullptr;
   out.meta_kblocks = static_cast<int>(meta_k_padded(k) / 128);
-  const int64_t chunks = n_out * (k / 32);
-  const int64_t pblocks = (chunks + 255) / 256;
-  const unsigned grid = static_cast<unsigned>(pblocks < int64_t(num_sms) * 64 ? pblocks : int64_t(num_sms) * 64);
+  e = launch_pdl(k_gamma_finalize, dim3(1), dim3(kFinThreads), 0, s, slot_bins, slot_flags, slots, h, n_out, k, n, m, flags);
+  if (e != cudaSuccess) return e;
+  // Rows are spread over warps; pick the warp count so every warp gets the
+  // same number of rows (within one) and the grid stays within two blocks/SM.
+  const int64_t max_warps = int64_t(num_sms) * 2 * (kPackThreads / 32);
+  const int64_t rounds = (n_out + max_warps - 1) / max_warps;
+  const int64_t warps = (n_out + rounds - 1) / rounds;
+  const int64_t blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(kPackThreads);
+  const uint4* wv = reinterpret_cast<const uint4*>(w);
+  const BlobHeader* hc = h;
   switch (m) {
-    case 2: k_prep_pack<2><<<grid, 256, 0, s>>>(w, n_out, k, n, h, out); break;
-    case 4: k_prep_pack<4><<<grid, 256, 0, s>>>(w, n_out, k, n, h, out); break;
-    default: k_prep_pack<8><<<grid, 256, 0, s>>>(w, n_out, k, n, h, out); break;
+    case 2: return launch_pdl(k_prep_pack<2>, grid, block, 0, s, wv, n_out, k, n, hc, out);
+    case 4: return launch_pdl(k_prep_pack<4>, grid, block, 0, s, wv, n_out, k, n, hc, out);
+    default: return launch_pdl(k_prep_pack<8>, grid, block, 0, s, wv, n_out, k, n, hc, out);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace sbl

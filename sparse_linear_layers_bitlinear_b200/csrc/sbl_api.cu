@@ -80,6 +80,8 @@ sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t 
   uint64_t off = 0;
   L.header = off;
   off += kHeaderBytes;
+  L.scratch = off;
+  off = align_up(off + kScratchBytes, 256);
   auto take = [&](uint64_t bytes) {
     const uint64_t at_off = off;
     off = align_up(off + bytes, 256);

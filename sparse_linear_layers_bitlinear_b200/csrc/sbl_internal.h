@@ -18,11 +18,15 @@ struct BlobHeader {
   float g;            // max(gamma, 1e-5)
   uint32_t status;    // SBL_STATUS_* bits
   uint32_t pad0;
-  // Exact sum of |w|: 32 bins; bin b accumulates sig << (s & 7) for every
-  // weight whose fixed-point shift s (see prep.cu) has s >> 3 == b.
-  unsigned long long bins[32];
 };
 static_assert(sizeof(BlobHeader) <= 4096, "header must fit its 4 KB slot");
+
+// Per-block partial sums of the exact absmean: the first prepare kernel writes
+// one slot per block, the second folds them.  Bin b of a slot is an integer in
+// units of 2^(8b - 133); the exact sum of |w| is sum_b bin[b] * 2^(8b - 133).
+constexpr int kPrepSlots = 1024;
+constexpr int kExactBins = 40;
+constexpr uint64_t kScratchBytes = uint64_t(kPrepSlots) * kExactBins * 8 + uint64_t(kPrepSlots) * 4;
 
 constexpr uint32_t kMagic = 0x314C4253u;  // "SBL1"
 constexpr uint64_t kHeaderBytes = 4096;

@@ -63,7 +63,7 @@ class sbl_layer(ctypes.Structure):
 class sbl_blob_layout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_uint64) for name in (
         "total_bytes", "header", "mask", "codes", "weff_bf16", "sp_values", "sp_meta", "sp_meta_bytes",
-        "gemv", "gamma", "g", "status")]
+        "gemv", "gamma", "g", "status", "scratch")]
 
 
 # Every entry point of include/sbl.h with its ctypes signature.

@@ -211,3 +211,53 @@ def test_gamma_scale_readback():
     gamma, g = sbl.read_scale(layer)
     assert np.float32(gamma) == oracle.absmean_gamma(w)
     assert np.float32(g) == oracle.clamped_scale(oracle.absmean_gamma(w))
+
+
+@pytest.mark.parametrize("kind", ["bf16_subnormal", "all_exponents", "near_max", "constant", "gauss_few_tiny"])
+def test_gamma_and_codes_at_extreme_magnitudes(kind):
+    """The exact absmean over inputs that reach the corners of the bf16 range:
+    subnormal masters (gamma lands in the fp32 subnormal range or rounds to 0),
+    magnitudes spread over every finite exponent (every partial-sum bin in
+    use), magnitudes near the bf16 maximum, and a constant magnitude."""
+    n_out, k, n, m = 136, 320, 2, 4
+    rng = np.random.default_rng({"bf16_subnormal": 1, "all_exponents": 2, "near_max": 3, "constant": 4,
+                                 "gauss_few_tiny": 5}[kind])
+    size = (n_out, k)
+    if kind == "bf16_subnormal":
+        mag = rng.integers(0, 0x80, size=size)
+    elif kind == "all_exponents":
+        mag = rng.integers(0, 0x7F80, size=size)
+    elif kind == "near_max":
+        mag = rng.integers(0x7E00, 0x7F80, size=size)
+    elif kind == "constant":
+        mag = np.full(size, 0x3C00)
+    else:  # Gaussian masters with a few subnormal and tiny ones mixed in
+        mag = synth.bits(synth.master_weights(n_out, k, 77)).astype(np.int64) & 0x7FFF
+        idx = rng.integers(0, mag.size, size=40)
+        mag.ravel()[idx[:20]] = rng.integers(1, 0x80, size=20)
+        mag.ravel()[idx[20:]] = rng.integers(0x0800, 0x1000, size=20)
+    sign = rng.integers(0, 2, size=size) << 15
+    bits = (mag | sign).astype(np.uint16)
+    w = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    _check_prepared(layer, w, n, m)
+
+
+@pytest.mark.parametrize("k", [64, 1088, 2560, 4160, 6912, 12352, 16384, 16448])
+def test_act_quant_row_lengths(k):
+    """Activation codes and scales for row lengths that exercise every
+    register-resident variant of the act-quant kernel and its long-row path."""
+    n_out, t = 8, 5
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 50)))
+    x = synth.activations(t, k, 51)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
