@@ -108,7 +108,7 @@ typedef struct sbl_blob_layout {
  * ordered [row_block][k_block]; inside a block, row r's 16 bytes hold 32
  * nibbles for its 32 groups of four in k order (group 2j in the low nibble
  * of byte j); a nibble is (i0 | i1 << 2) with i0 < i1 the kept positions.
- * Rows and k are padded up to 128 and 256 with nibble 0x4 over zero codes.
+ * Rows and k are padded up to multiples of 256 with nibble 0x4 over zero codes.
  * gemv layout: one byte per group of four: the metadata nibble in the high
  * half, the two kept codes in the low half (bits 1:0 the code at i0, bits 3:2
  * the code at i1; 00 = 0, 01 = +1, 11 = -1). */

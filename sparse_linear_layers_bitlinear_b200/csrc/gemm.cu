@@ -3,7 +3,7 @@
 // self test.
 #include <mutex>
 
-#include "gemm_tc.cuh"
+#include "gemm_pair.cuh"
 #include "sbl_kernels.h"
 
 namespace sbl {
@@ -59,13 +59,50 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, const t
   return cudaGetLastError();
 }
 
+// Pair kernels: grid = two CTAs per concurrently resident cluster, capped by
+// the tile count.
+template <class Cfg>
+static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
+                               const typename Cfg::Params& p, int m_rows, int n_cols, int num_sms, cudaStream_t s) {
+  constexpr int smem = pair_smem_bytes<Cfg>();
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
+  std::call_once(once, [num_sms] {
+    attr_err = cudaFuncSetAttribute(k_gemm_pair<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms & ~1);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    attr_err = cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<Cfg>, &cfg);
+    max_clusters = n;
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
+  const int tiles = ((m_rows + 255) / 256) * ((n_cols + Cfg::BN - 1) / Cfg::BN);
+  const int pairs = tiles < max_clusters ? tiles : max_clusters;
+  if (pairs <= 0) return cudaSuccess;
+  k_gemm_pair<Cfg><<<2 * pairs, kGemmThreads, smem, s>>>(a, b, e, p);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // Forward int8 GEMM
 // ---------------------------------------------------------------------------
 cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,
-                                const int8_t* xq, const float* a_prime, const float* g, int64_t n_out, int64_t t,
-                                int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
-                                cudaStream_t s) {
+                                uint64_t meta_bytes, const int8_t* xq, const float* a_prime, const float* g,
+                                int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out, uint32_t* status,
+                                int num_sms, cudaStream_t s) {
   FwdParams p;
   p.n_out = static_cast<int>(n_out);
   p.T = static_cast<int>(t);
@@ -77,16 +114,20 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
   p.meta = meta;
   p.meta_kblocks = meta_kblocks;
   p.status = status;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, te;
   const bool acc = acc_out != nullptr;
   if (sparse) {
+    // A: compressed codes [n_out][k/2]; B: xq [t][k], 112-token halves; E:
+    // the metadata section viewed as rows of 256 bytes.
     if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k / 2, n_out, k / 2, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdSparse<false>::BN,
-                        CU_TENSOR_MAP_SWIZZLE_128B))
+        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgPairSparse<false>::BN / 2,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 256, meta_bytes / 256, 256, 256, 16,
+                        CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
-    return acc ? launch_tc<CfgFwdSparse<true>>(ta, tb, p, p.n_out, p.T, num_sms, s)
-               : launch_tc<CfgFwdSparse<false>>(ta, tb, p, p.n_out, p.T, num_sms, s);
+    return acc ? launch_pair<CfgPairSparse<true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s)
+               : launch_pair<CfgPairSparse<false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s);
   }
   if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k, n_out, k, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, CfgFwdDense<false>::BN,
@@ -102,13 +143,14 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
 template <bool A_MN, bool B_MN, bool F32>
 static cudaError_t bf16_dispatch(const uint16_t* A, const uint16_t* B, int64_t M, int64_t N, int64_t K,
                                  const float* alpha, void* out, uint32_t* status, int num_sms, cudaStream_t s) {
-  using Cfg = CfgBf16<A_MN, B_MN, F32>;
+  using Cfg = CfgPairBf16<A_MN, B_MN, F32>;
   CUtensorMap ta, tb;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // Per CTA: A 128 rows, B 128 columns (half of the pair's 256).
   const bool ok_a = A_MN ? encode_tmap_2d(&ta, bf, A, M, K, M * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)
                          : encode_tmap_2d(&ta, bf, A, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   const bool ok_b = B_MN ? encode_tmap_2d(&tb, bf, B, N, K, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)
-                         : encode_tmap_2d(&tb, bf, B, K, N, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B);
+                         : encode_tmap_2d(&tb, bf, B, K, N, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   Bf16Params p;
   p.M = static_cast<int>(M);
@@ -118,7 +160,7 @@ static cudaError_t bf16_dispatch(const uint16_t* A, const uint16_t* B, int64_t M
   p.out = out;
   p.ldo = N;
   p.status = status;
-  return launch_tc<Cfg>(ta, tb, p, p.M, p.N, num_sms, s);
+  return launch_pair<Cfg>(ta, tb, tb, p, p.M, p.N, num_sms, s);
 }
 
 cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t* A, const uint16_t* B, int64_t M,

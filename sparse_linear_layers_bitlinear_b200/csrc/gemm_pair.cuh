@@ -1,0 +1,311 @@
+// Persistent, warp-specialised tcgen05 GEMM on CTA pairs (sm_100a).
+//
+// A cluster of two CTAs on two SMs computes one 256-row output tile with the
+// 2-SM MMA (tcgen05.mma.cta_group::2): CTA r holds rows 128r..128r+127 of the
+// A tile and half of the B tile in its shared memory, and receives its 128
+// rows of the accumulator in its own tensor memory.  Per SM that halves the B
+// traffic of a 128-row tile with the same N, which is what keeps the tensor
+// pipe fed from L2.
+//
+//   warp 0      TMA producer, in both CTAs: its copies land in its own shared
+//               memory and count on the even (leader) CTA's "full" barrier
+//   warp 1      allocates tensor memory (both CTAs); in the leader, lane 0
+//               issues the MMAs and commits to the "empty" and accumulator
+//               barriers of both CTAs at once
+//   warps 2..5  epilogue, in both CTAs: drain this CTA's accumulator rows,
+//               then arrive on the leader's "accumulator empty" barrier
+//
+// Every wait is bounded; a CTA whose wait runs out records SBL_STATUS_TIMEOUT
+// and winds down, and its partner's waits run out in turn.  Both CTAs always
+// reach the final cluster barrier, so neither frees memory the other can
+// still signal.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace sbl {
+
+struct PairSmemTail {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <class Cfg>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmE, const typename Cfg::Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smA = smem;
+  uint8_t* smB = smA + Cfg::STAGES * Cfg::A_BYTES;
+  uint8_t* smE = smB + Cfg::STAGES * Cfg::B_BYTES;
+  PairSmemTail* tail = reinterpret_cast<PairSmemTail*>(smE + Cfg::STAGES * Cfg::E_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  uint32_t* status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&tail->full[s], 2);   // leader: its expect-tx arrive + the partner's arrive
+      mbar_init(&tail->empty[s], 1);  // one MMA commit, sent to both CTAs
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->acc_full[b], 1);
+      mbar_init(&tail->acc_empty[b], 8);  // 4 epilogue warps in each CTA
+    }
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (Cfg::E_BYTES) prefetch_tensormap(&tmE);
+  }
+  cluster_sync_all();  // barriers initialised in both CTAs before any remote use
+  if (warp == 1) tmem_alloc_pair(&tail->tmem_base, Cfg::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+
+  const uint32_t tmem_base = tail->tmem_base;
+  volatile int* abort_flag = &tail->abort_flag;
+  const int m_blocks = (Cfg::rows_M(p) + 255) / 256;
+  const int n_blocks = (Cfg::cols_N(p) + Cfg::BN - 1) / Cfg::BN;
+  const int num_tiles = m_blocks * n_blocks;
+  const int k_blocks = Cfg::k_blocks(p);
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      const uint32_t leader_full0 = map_to_rank(&tail->full[0], 0);
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const int m0 = (tile % m_blocks) * 256 + 128 * int(rank);
+        const int n0 = (tile / m_blocks) * Cfg::BN + int(rank) * (Cfg::BN / 2);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&tail->empty[stage], phase ^ 1u, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          Cfg::load_stage(&tmA, &tmB, &tmE, p, smA + stage * Cfg::A_BYTES, smB + stage * Cfg::B_BYTES,
+                          smE + stage * Cfg::E_BYTES, m0, n0, kb, &tail->full[stage]);
+          if (leader) {
+            mbar_arrive_expect_tx(&tail->full[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES + Cfg::E_BYTES));
+          } else {
+            mbar_arrive_remote(leader_full0 + stage * 8u);
+          }
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader only) ----------------
+    if (leader && lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t local = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++local) {
+        const uint32_t ab = local & 1u;
+        const uint32_t aphase = (local >> 1) & 1u;
+        if (!mbar_wait(&tail->acc_empty[ab], aphase ^ 1u, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * Cfg::ACC_COLS;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&tail->full[stage], phase, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          Cfg::mma_stage(p, d_tmem, tmem_base + Cfg::E_COL0 + (stage & 1u) * Cfg::E_COLS, smA + stage * Cfg::A_BYTES,
+                         smB + stage * Cfg::B_BYTES, smE + stage * Cfg::E_BYTES, kb == 0);
+          mma_commit_pair(&tail->empty[stage]);  // frees the stage in both CTAs once these MMAs have read it
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tail->acc_full[ab]);  // accumulator complete in both CTAs
+      }
+      // No MMA may still run when tensor memory is released.
+      mma_commit_pair(&tail->drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&tail->drain, 0)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          raise_status(status, SBL_STATUS_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const uint32_t leader_acc_empty0 = map_to_rank(&tail->acc_empty[0], 0);
+    uint32_t local = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
+      const uint32_t ab = local & 1u;
+      const uint32_t aphase = (local >> 1) & 1u;
+      bool ready = true;
+      if (lane == 0) ready = mbar_wait(&tail->acc_full[ab], aphase, abort_flag, status);
+      ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+      if (!ready) break;
+      tc_fence_after();
+      const int m0 = (tile % m_blocks) * 256 + 128 * int(rank);
+      const int n0 = (tile / m_blocks) * Cfg::BN;
+      const uint32_t t_acc = tmem_base + ab * Cfg::ACC_COLS + (uint32_t(quarter * 32) << 16);
+      Cfg::epilogue(p, t_acc, m0 + quarter * 32 + lane, n0, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_acc_empty0 + ab * 8u);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the partner no longer signals this CTA's barriers
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+template <class Cfg>
+constexpr int pair_smem_bytes() {
+  return 1024 + Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES + Cfg::E_BYTES) + int(sizeof(PairSmemTail));
+}
+
+// ---------------------------------------------------------------------------
+// bf16 backward on pairs: tile 256 (M) x 256 (N), K 64 per stage.  Each CTA
+// holds A 128 x 64 and B 128 x 64 (its half of N); output as CfgBf16.
+// ---------------------------------------------------------------------------
+template <bool A_MN, bool B_MN, bool OUT_F32>
+struct CfgPairBf16 {
+  using Params = Bf16Params;
+  static constexpr int BN = 256, BK = 64, STAGES = 6;
+  static constexpr int A_BYTES = 128 * BK * 2;        // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB
+  static constexpr int E_BYTES = 0;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int E_COL0 = 0, E_COLS = 0;
+  static constexpr uint32_t IDESC = idesc_bf16(256, BN, A_MN, B_MN);
+
+  __device__ static int rows_M(const Params& p) { return p.M; }
+  __device__ static int cols_N(const Params& p) { return p.N; }
+  __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
+
+  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap*, const Params&,
+                                    uint8_t* sA, uint8_t* sB, uint8_t*, int m0, int n0, int kb, uint64_t* bar) {
+    const int k0 = kb * BK;
+    if (A_MN) {  // two boxes of [64 k][64 m]
+      tma_load_2d_pair(sA, tA, m0, k0, bar);
+      tma_load_2d_pair(sA + 8192, tA, m0 + 64, k0, bar);
+    } else {  // one box of [128 m][64 k]
+      tma_load_2d_pair(sA, tA, k0, m0, bar);
+    }
+    if (B_MN) {  // two boxes of [64 k][64 n]
+      tma_load_2d_pair(sB, tB, n0, k0, bar);
+      tma_load_2d_pair(sB + 8192, tB, n0 + 64, k0, bar);
+    } else {  // one box of [128 n][64 k]
+      tma_load_2d_pair(sB, tB, k0, n0, bar);
+    }
+  }
+
+  __device__ static void mma_stage(const Params&, uint32_t d_tmem, uint32_t, uint8_t* sA, uint8_t* sB, uint8_t*,
+                                   bool first) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+    for (int kk = 0; kk < BK / 16; ++kk) {
+      const uint64_t ad = A_MN ? smem_desc(a0 + kk * 2048, 8192, 1024, 2) : smem_desc(a0 + kk * 32, 16, 1024, 2);
+      const uint64_t bd = B_MN ? smem_desc(b0 + kk * 2048, 8192, 1024, 2) : smem_desc(b0 + kk * 32, 16, 1024, 2);
+      mma_bf16_pair(d_tmem, ad, bd, IDESC, (first && kk == 0) ? 0u : 1u);
+    }
+  }
+
+  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int lane) {
+    CfgBf16<A_MN, B_MN, OUT_F32>::epilogue(p, t_acc, row, n0, lane);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// 2:4 sparse int8 forward on pairs: tile 256 W rows x 224 tokens, 256 logical
+// k per stage.  Each CTA holds its 128 rows of compressed codes (128 x 128
+// bytes), 112 tokens of xq (2 boxes of [112 rows][128 bytes]) and its rows'
+// metadata (2 blocks of 128 rows x 16 bytes, copied to tensor memory).
+// ---------------------------------------------------------------------------
+template <bool ACC_OUT>
+struct CfgPairSparse {
+  using Params = FwdParams;
+  static constexpr int BN = 224, BK = 256, STAGES = 4;
+  static constexpr int A_BYTES = 128 * BK / 2;      // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK;     // 28 KB
+  static constexpr int E_BYTES = 2 * 2048;          // 4 KB
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int E_COL0 = 2 * BN;             // metadata after the two accumulators
+  static constexpr int E_COLS = 8;                  // 2 blocks x 4 columns, two slots
+  static constexpr uint32_t IDESC = idesc_i8(256, BN, true);
+  static_assert(E_COL0 + 2 * E_COLS <= TMEM_COLS, "tensor memory budget");
+
+  __device__ static int rows_M(const Params& p) { return p.n_out; }
+  __device__ static int cols_N(const Params& p) { return p.T; }
+  __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
+
+  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tE,
+                                    const Params& p, uint8_t* sA, uint8_t* sB, uint8_t* sE, int m0, int n0, int kb,
+                                    uint64_t* bar) {
+    tma_load_2d_pair(sA, tA, kb * (BK / 2), m0, bar);              // compressed columns
+    tma_load_2d_pair(sB, tB, kb * BK, n0, bar);                    // logical k 0..127 of the stage
+    tma_load_2d_pair(sB + (BN / 2) * 128, tB, kb * BK + 128, n0, bar);  // logical k 128..255
+    // metadata: 2 consecutive 2 KB blocks = 16 rows of 256 bytes in the section
+    const int row = ((m0 / 128) * p.meta_kblocks + kb * 2) * 8;
+    tma_load_2d_pair(sE, tE, 0, row, bar);
+  }
+
+  __device__ static void mma_stage(const Params&, uint32_t d_tmem, uint32_t e_tmem, uint8_t* sA, uint8_t* sB,
+                                   uint8_t* sE, bool first) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB), e0 = smem_u32(sE);
+    tmem_copy_128x128b_pair(e_tmem, smem_desc(e0, 2048, 128, 0));
+    tmem_copy_128x128b_pair(e_tmem + 4, smem_desc(e0 + 2048, 2048, 128, 0));
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024, 2);  // 32 compressed bytes = 64 logical k
+      const uint32_t bsub = (kk >> 1) * ((BN / 2) * 128) + (kk & 1) * 64;
+      const uint64_t bd = smem_desc(b0 + bsub, 16, 1024, 2);
+      mma_sp_i8_pair(d_tmem, ad, bd, e_tmem + 2 * kk, IDESC, (first && kk == 0) ? 0u : 1u);
+    }
+  }
+
+  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int lane) {
+    const float g = *p.g;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      __syncwarp();
+      tmem_load_32x32b_x32(t_acc + c * 32, r);
+      tmem_load_wait();
+      if (n0 + c * 32 >= p.T) continue;  // uniform across the warp
+      fwd_epilogue_chunk<ACC_OUT>(p, r, row, n0 + c * 32, lane, g);
+    }
+  }
+};
+
+}  // namespace sbl

@@ -439,7 +439,7 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   BlobHeader* h = reinterpret_cast<BlobHeader*>(blob + L.header);
   uint64_t* slot_bins = reinterpret_cast<uint64_t*>(blob + L.scratch);
   uint32_t* slot_flags = reinterpret_cast<uint32_t*>(blob + L.scratch + uint64_t(kPrepSlots) * kExactBins * 8);
-  if (L.sp_meta && (n_out % 128 != 0 || k % 256 != 0)) {
+  if (L.sp_meta && (n_out % 256 != 0 || k % 256 != 0)) {
     cudaError_t e = cudaMemsetAsync(blob + L.sp_meta, 0x44, L.sp_meta_bytes, s);
     if (e != cudaSuccess) return e;
   }

@@ -161,10 +161,11 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
                             s);
   } else if (is_24(layer->n, layer->m)) {
     e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
-                            static_cast<int>(meta_k_padded(layer->k) / 128), xq, ap, g, layer->n_out, t, layer->k, y,
+                            static_cast<int>(meta_k_padded(layer->k) / 128), L.sp_meta_bytes, xq, ap, g, layer->n_out,
+                            t, layer->k, y,
                             acc_debug, status, sms, s);
   } else {
-    e = launch_forward_gemm(false, at<const int8_t>(layer, L.codes), nullptr, 0, xq, ap, g, layer->n_out, t, layer->k,
+    e = launch_forward_gemm(false, at<const int8_t>(layer, L.codes), nullptr, 0, 0, xq, ap, g, layer->n_out, t, layer->k,
                             y, acc_debug, status, sms, s);
   }
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;

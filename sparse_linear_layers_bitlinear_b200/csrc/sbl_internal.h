@@ -34,7 +34,8 @@ constexpr uint64_t kHeaderBytes = 4096;
 inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
 
 // Padded extents of the tensor-core metadata section.
-inline int64_t meta_rows_padded(int64_t n_out) { return (n_out + 127) / 128 * 128; }
+// Rows pad to 256: the pair GEMM reads the metadata of two 128-row blocks per tile.
+inline int64_t meta_rows_padded(int64_t n_out) { return (n_out + 255) / 256 * 256; }
 inline int64_t meta_k_padded(int64_t k) { return (k + 255) / 256 * 256; }
 
 }  // namespace sbl

@@ -29,7 +29,7 @@ cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq
 // Forward GEMM + dequant.  sparse: codes = 2:4 kept values [n_out][k/2] and
 // meta = tensor-core metadata; dense: codes = W_eff int8 [n_out][k].
 cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,
-                                const int8_t* xq, const float* a_prime, const float* g, int64_t n_out, int64_t t,
+                                uint64_t meta_bytes, const int8_t* xq, const float* a_prime, const float* g, int64_t n_out, int64_t t,
                                 int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
                                 cudaStream_t s);
 

@@ -57,7 +57,7 @@ def sp_meta_canonical(layer):
     L = layer.layout()
     raw = section(layer, "sp_meta", int(L.sp_meta_bytes))
     kpad = (k + 255) // 256 * 256
-    rpad = (n_out + 127) // 128 * 128
+    rpad = (n_out + 255) // 256 * 256
     kblocks = kpad // 128
     # [row_block][k_block][128 rows][16 bytes] -> [rpad][kpad/8]
     blocks = raw.reshape(rpad // 128, kblocks, 128, 16)

@@ -55,7 +55,7 @@ def test_layout_sections_are_aligned_and_disjoint(lib):
         spans = [("header", L.header, 4096), ("scratch", L.scratch, 1024 * 32 * 8 + 1024 * 4), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
         if (n, m) == (2, 4):
             spans += [("sp_values", L.sp_values, n_out * k // 2), ("sp_meta", L.sp_meta, L.sp_meta_bytes)]
-            assert L.sp_meta_bytes == ((n_out + 127) // 128 * 128) * ((k + 255) // 256 * 256) // 8
+            assert L.sp_meta_bytes == ((n_out + 255) // 256 * 256) * ((k + 255) // 256 * 256) // 8
             assert L.codes == 0
             if flags & sbl.SBL_PACK_GEMV:
                 spans.append(("gemv", L.gemv, n_out * k // 4))
