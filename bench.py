@@ -36,6 +36,9 @@ UNIT = "tokens/s"
 WORKLOAD = dict(name="prefill 2:4 Sparse-BitLinear fwd+STE bwd, FFN up projection", tokens=4096, k=2560,
                 n_out=6912, n=2, m=4)
 ROTATE = 3  # distinct input sets cycled through the steps (3 x 112 MB > 126 MB L2)
+# Library kernels per step: prepare (exact-sum partials, finalize, pack),
+# forward (act-quant, 2:4 GEMM), backward (dX and dW in one launch).
+LAUNCHES_PER_STEP = 6
 
 # Algorithmic work of one step at this workload (Measurement).
 def algorithmic(T, K, N):
@@ -309,12 +312,9 @@ def main():
         sbl.forward(layer, x, T, y, workspace=ws)
         if ev is not None:
             ev[2].record(stream)
-        sbl.backward(layer, x, dy, T, dx, dw, sbl.SBL_NO_DW)
+        sbl.backward(layer, x, dy, T, dx, dw, 0)  # dX and dW in one launch
         if ev is not None:
             ev[3].record(stream)
-        sbl.backward(layer, x, dy, T, dx, dw, sbl.SBL_NO_DX)
-        if ev is not None:
-            ev[4].record(stream)
 
     for i in range(args.warmup):
         step(i)
@@ -322,7 +322,7 @@ def main():
     code, bits = sbl.read_status(layer)
     assert code == sbl.SBL_OK, (code, bits)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -335,7 +335,7 @@ def main():
     barrier(world)
     ms_total = start.elapsed_time(end)
     ms_step = max_over_ranks(ms_total / args.steps, world)
-    phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(4)]
+    phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
     code, bits = sbl.read_status(layer)
     assert code == sbl.SBL_OK, (code, bits)
 
@@ -382,18 +382,17 @@ def main():
     bound_ms = {
         "prepare": A["prep_bytes"] / hbm * 1e3,
         "forward": max(A["fwd_gemm_ops"] / i8_sparse, (A["actq_bytes"] + A["fwd_bytes"]) / hbm) * 1e3,
-        "dx": max(A["bwd_flops_each"] / bf16, A["dx_bytes"] / hbm) * 1e3,
-        "dw": max(A["bwd_flops_each"] / bf16, A["dw_bytes"] / hbm) * 1e3,
+        "backward": max(2 * A["bwd_flops_each"] / bf16, (A["dx_bytes"] + A["dw_bytes"]) / hbm) * 1e3,
     }
-    names = ["prepare", "forward", "dx", "dw"]
-    dom = max(range(4), key=lambda j: phase_ms[j])
+    names = ["prepare", "forward", "backward"]
+    dom = max(range(3), key=lambda j: phase_ms[j])
     dom_name = names[dom]
-    if dom_name in ("dx", "dw"):
-        achieved = A["bwd_flops_each"] / (phase_ms[dom] * 1e-3) / 1e12
+    if dom_name == "backward":
+        achieved = 2 * A["bwd_flops_each"] / (phase_ms[dom] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
-                "traffic": ncu_traffic("bf16_gemm_" + dom_name),
-                "kernel": f"k_gemm_tc<CfgBf16> ({dom_name})",
+                "traffic": ncu_traffic("bf16_backward"),
+                "kernel": "k_gemm_pair<CfgPairDualBf16> (dX and dW, one launch)",
                 "peak_note": f"{peaks['source']} bf16 burst figure (kernel timed inside a short step loop)"}
     else:
         by = {"prepare": A["prep_bytes"], "forward": A["actq_bytes"] + A["fwd_bytes"]}[dom_name]
@@ -417,7 +416,7 @@ def main():
         "roofline": roof,
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "peaks": peaks,
     }

@@ -1,7 +1,11 @@
 // Launchers for the tensor-core GEMMs (forward int8, dense or 2:4 sparse;
 // backward bf16), the decode GEMV, the tensor-map encoder and the bounded-wait
 // self test.
+#include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "gemm_pair.cuh"
 #include "sbl_kernels.h"
@@ -62,8 +66,7 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, const t
 // Pair kernels: grid = two CTAs per concurrently resident cluster, capped by
 // the tile count.
 template <class Cfg>
-static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
-                               const typename Cfg::Params& p, int m_rows, int n_cols, int num_sms, cudaStream_t s) {
+static cudaError_t pair_setup(int num_sms, int* max_clusters_out) {
   constexpr int smem = pair_smem_bytes<Cfg>();
   static_assert(smem <= 227 * 1024, "shared memory budget");
   static std::once_flag once;
@@ -89,10 +92,20 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const
   });
   if (attr_err != cudaSuccess) return attr_err;
   if (max_clusters <= 0) return cudaErrorInvalidConfiguration;
+  *max_clusters_out = max_clusters;
+  return cudaSuccess;
+}
+
+template <class Cfg>
+static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
+                               const typename Cfg::Params& p, int m_rows, int n_cols, int num_sms, cudaStream_t s) {
+  int max_clusters = 0;
+  const cudaError_t err = pair_setup<Cfg>(num_sms, &max_clusters);
+  if (err != cudaSuccess) return err;
   const int tiles = ((m_rows + 255) / 256) * ((n_cols + Cfg::BN - 1) / Cfg::BN);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
   if (pairs <= 0) return cudaSuccess;
-  k_gemm_pair<Cfg><<<2 * pairs, kGemmThreads, smem, s>>>(a, b, e, p);
+  k_gemm_pair<Cfg><<<2 * pairs, kGemmThreads, pair_smem_bytes<Cfg>(), s>>>(a, b, e, e, p);
   return cudaGetLastError();
 }
 
@@ -177,6 +190,108 @@ cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t*
     case 6: return bf16_dispatch<true, true, false>(A, B, M, N, K, alpha, out, status, num_sms, s);
     default: return bf16_dispatch<true, true, true>(A, B, M, N, K, alpha, out, status, num_sms, s);
   }
+}
+
+// ---------------------------------------------------------------------------
+// dX and dW in one launch
+// ---------------------------------------------------------------------------
+namespace {
+
+struct DualSchedule {
+  std::vector<uint16_t> off, ids;
+};
+
+// Longest-processing-time-first: tiles by depth (k blocks), deepest first,
+// each to the pair with the least work so far.  Cached per shape.
+const DualSchedule& dual_schedule(int tiles0, int kb0, int tiles1, int kb1, int npairs) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int>, DualSchedule> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(tiles0, kb0, tiles1, kb1, npairs);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  std::vector<int> order;
+  order.reserve(tiles0 + tiles1);
+  const bool first0 = kb0 >= kb1;
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool prob0 = (pass == 0) == first0;
+    const int base = prob0 ? 0 : tiles0, n = prob0 ? tiles0 : tiles1;
+    for (int i = 0; i < n; ++i) order.push_back(base + i);
+  }
+  std::vector<std::vector<uint16_t>> per(npairs);
+  std::vector<long long> load(npairs, 0);
+  for (int id : order) {
+    const int cost = id < tiles0 ? kb0 : kb1;
+    int best = 0;
+    for (int q = 1; q < npairs; ++q)
+      if (load[q] < load[best]) best = q;
+    per[best].push_back(static_cast<uint16_t>(id));
+    load[best] += cost;
+  }
+  DualSchedule sch;
+  sch.off.push_back(0);
+  for (int q = 0; q < npairs; ++q) {
+    sch.ids.insert(sch.ids.end(), per[q].begin(), per[q].end());
+    sch.off.push_back(static_cast<uint16_t>(sch.ids.size()));
+  }
+  return cache.emplace(key, std::move(sch)).first->second;
+}
+
+template <bool F32>
+cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16_t* x, int64_t t, int64_t n_out,
+                          int64_t k, const float* g, void* dx, void* dw, uint32_t* status, int num_sms,
+                          cudaStream_t s, bool* done) {
+  using Cfg = CfgPairDualBf16<F32>;
+  *done = false;
+  int max_clusters = 0;
+  cudaError_t err = pair_setup<Cfg>(num_sms, &max_clusters);
+  if (err != cudaSuccess) return err;
+  const int nb = static_cast<int>((k + 255) / 256);
+  const int mb0 = static_cast<int>((t + 255) / 256), mb1 = static_cast<int>((n_out + 255) / 256);
+  const int tiles0 = mb0 * nb, tiles1 = mb1 * nb;
+  if (tiles0 + tiles1 > kDualMaxTiles) return cudaSuccess;  // caller runs two launches
+  int npairs = std::min(std::min(max_clusters, kDualMaxPairs), tiles0 + tiles1);
+  const int kb0 = static_cast<int>((n_out + 63) / 64), kb1 = static_cast<int>((t + 63) / 64);
+  const DualSchedule& sch = dual_schedule(tiles0, kb0, tiles1, kb1, npairs);
+
+  CUtensorMap a0, b0, a1, b1;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // dX: A0 = dY [t][n_out] K-major, B0 = W_eff [n_out][k] MN-major
+  // dW: A1 = dY [t][n_out] MN-major (M = n_out), B1 = X [t][k] MN-major
+  if (!encode_tmap_2d(&a0, bf, dy, n_out, t, n_out * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&b0, bf, weff, k, n_out, k * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&a1, bf, dy, n_out, t, n_out * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_2d(&b1, bf, x, k, t, k * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  DualBf16Params p;
+  p.M[0] = static_cast<int>(t);
+  p.M[1] = static_cast<int>(n_out);
+  p.N = static_cast<int>(k);
+  p.K[0] = static_cast<int>(n_out);
+  p.K[1] = static_cast<int>(t);
+  p.mblocks[0] = mb0;
+  p.mblocks[1] = mb1;
+  p.tiles0 = tiles0;
+  p.alpha[0] = g;
+  p.alpha[1] = nullptr;
+  p.out[0] = dx;
+  p.out[1] = dw;
+  p.status = status;
+  std::copy(sch.off.begin(), sch.off.end(), p.sched_off);
+  std::copy(sch.ids.begin(), sch.ids.end(), p.sched);
+  k_gemm_pair<Cfg><<<2 * npairs, kGemmThreads, pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
+  err = cudaGetLastError();
+  *done = err == cudaSuccess;
+  return err;
+}
+
+}  // namespace
+
+cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const uint16_t* weff, const uint16_t* x,
+                                      int64_t t, int64_t n_out, int64_t k, const float* g, void* dx, void* dw,
+                                      uint32_t* status, int num_sms, cudaStream_t s, bool* done) {
+  return out_f32 ? dual_dispatch<true>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done)
+                 : dual_dispatch<false>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done);
 }
 
 // ---------------------------------------------------------------------------

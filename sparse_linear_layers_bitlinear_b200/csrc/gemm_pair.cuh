@@ -25,6 +25,26 @@
 
 namespace sbl {
 
+// One output tile of a pair: problem index (for multi-problem launches),
+// 256-row block, BN-column block and its number of k blocks.
+struct PairTile {
+  int prob, mb, nb, kblocks;
+};
+
+// Default schedule: tiles of one problem striped over the pairs, M fastest.
+template <class Cfg>
+struct StripedTiles {
+  __device__ static int count(const typename Cfg::Params& p, int pair, int npairs) {
+    const int nt = ((Cfg::rows_M(p) + 255) / 256) * ((Cfg::cols_N(p) + Cfg::BN - 1) / Cfg::BN);
+    return pair < nt ? (nt - pair + npairs - 1) / npairs : 0;
+  }
+  __device__ static PairTile at(const typename Cfg::Params& p, int pair, int npairs, int i) {
+    const int mb = (Cfg::rows_M(p) + 255) / 256;
+    const int t = pair + i * npairs;
+    return PairTile{0, t % mb, t / mb, Cfg::k_blocks(p)};
+  }
+};
+
 struct PairSmemTail {
   uint64_t full[8];
   uint64_t empty[8];
@@ -38,7 +58,8 @@ struct PairSmemTail {
 template <class Cfg>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmE, const typename Cfg::Params p) {
+                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
+                const typename Cfg::Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smA = smem;
@@ -68,7 +89,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    if (Cfg::E_BYTES) prefetch_tensormap(&tmE);
+    if (Cfg::MAPS > 2) prefetch_tensormap(&tmE);
+    if (Cfg::MAPS > 3) prefetch_tensormap(&tmF);
   }
   cluster_sync_all();  // barriers initialised in both CTAs before any remote use
   if (warp == 1) tmem_alloc_pair(&tail->tmem_base, Cfg::TMEM_COLS);
@@ -78,11 +100,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
-  const int m_blocks = (Cfg::rows_M(p) + 255) / 256;
-  const int n_blocks = (Cfg::cols_N(p) + Cfg::BN - 1) / Cfg::BN;
-  const int num_tiles = m_blocks * n_blocks;
-  const int k_blocks = Cfg::k_blocks(p);
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int ntiles = Cfg::Tiles::count(p, pair, npairs);
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -90,15 +109,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       const uint32_t leader_full0 = map_to_rank(&tail->full[0], 0);
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        const int m0 = (tile % m_blocks) * 256 + 128 * int(rank);
-        const int n0 = (tile / m_blocks) * Cfg::BN + int(rank) * (Cfg::BN / 2);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
+        const int m0 = t.mb * 256 + 128 * int(rank);
+        const int n0 = t.nb * Cfg::BN + int(rank) * (Cfg::BN / 2);
+        for (int kb = 0; kb < t.kblocks; ++kb) {
           if (!mbar_wait(&tail->empty[stage], phase ^ 1u, abort_flag, status)) {
             ok = false;
             break;
           }
-          Cfg::load_stage(&tmA, &tmB, &tmE, p, smA + stage * Cfg::A_BYTES, smB + stage * Cfg::B_BYTES,
+          Cfg::load_stage(&tmA, &tmB, &tmE, &tmF, p, t.prob, smA + stage * Cfg::A_BYTES, smB + stage * Cfg::B_BYTES,
                           smE + stage * Cfg::E_BYTES, m0, n0, kb, &tail->full[stage]);
           if (leader) {
             mbar_arrive_expect_tx(&tail->full[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES + Cfg::E_BYTES));
@@ -116,25 +136,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ---------------- MMA issuer (leader only) ----------------
     if (leader && lane == 0) {
       uint32_t stage = 0, phase = 0;
-      uint32_t local = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++local) {
-        const uint32_t ab = local & 1u;
-        const uint32_t aphase = (local >> 1) & 1u;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
+        const uint32_t ab = uint32_t(i) & 1u;
+        const uint32_t aphase = (uint32_t(i) >> 1) & 1u;
         if (!mbar_wait(&tail->acc_empty[ab], aphase ^ 1u, abort_flag, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * Cfg::ACC_COLS;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        for (int kb = 0; kb < t.kblocks; ++kb) {
           if (!mbar_wait(&tail->full[stage], phase, abort_flag, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          Cfg::mma_stage(p, d_tmem, tmem_base + Cfg::E_COL0 + (stage & 1u) * Cfg::E_COLS, smA + stage * Cfg::A_BYTES,
-                         smB + stage * Cfg::B_BYTES, smE + stage * Cfg::E_BYTES, kb == 0);
+          Cfg::mma_stage(p, t.prob, d_tmem, tmem_base + Cfg::E_COL0 + (stage & 1u) * Cfg::E_COLS,
+                         smA + stage * Cfg::A_BYTES, smB + stage * Cfg::B_BYTES, smE + stage * Cfg::E_BYTES, kb == 0);
           mma_commit_pair(&tail->empty[stage]);  // frees the stage in both CTAs once these MMAs have read it
           if (++stage == Cfg::STAGES) {
             stage = 0;
@@ -158,19 +178,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ---------------- epilogue (warps 2..5, both CTAs) ----------------
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const uint32_t leader_acc_empty0 = map_to_rank(&tail->acc_empty[0], 0);
-    uint32_t local = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++local) {
-      const uint32_t ab = local & 1u;
-      const uint32_t aphase = (local >> 1) & 1u;
+    for (int i = 0; i < ntiles; ++i) {
+      const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
+      const uint32_t ab = uint32_t(i) & 1u;
+      const uint32_t aphase = (uint32_t(i) >> 1) & 1u;
       bool ready = true;
       if (lane == 0) ready = mbar_wait(&tail->acc_full[ab], aphase, abort_flag, status);
       ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
       if (!ready) break;
       tc_fence_after();
-      const int m0 = (tile % m_blocks) * 256 + 128 * int(rank);
-      const int n0 = (tile / m_blocks) * Cfg::BN;
+      const int m0 = t.mb * 256 + 128 * int(rank);
+      const int n0 = t.nb * Cfg::BN;
       const uint32_t t_acc = tmem_base + ab * Cfg::ACC_COLS + (uint32_t(quarter * 32) << 16);
-      Cfg::epilogue(p, t_acc, m0 + quarter * 32 + lane, n0, lane);
+      Cfg::epilogue(p, t.prob, t_acc, m0 + quarter * 32 + lane, n0, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_acc_empty0 + ab * 8u);
@@ -199,6 +219,8 @@ constexpr int pair_smem_bytes() {
 template <bool A_MN, bool B_MN, bool OUT_F32>
 struct CfgPairBf16 {
   using Params = Bf16Params;
+  using Tiles = StripedTiles<CfgPairBf16>;
+  static constexpr int MAPS = 2;
   static constexpr int BN = 256, BK = 64, STAGES = 6;
   static constexpr int A_BYTES = 128 * BK * 2;        // 16 KB
   static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB
@@ -212,8 +234,9 @@ struct CfgPairBf16 {
   __device__ static int cols_N(const Params& p) { return p.N; }
   __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
 
-  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap*, const Params&,
-                                    uint8_t* sA, uint8_t* sB, uint8_t*, int m0, int n0, int kb, uint64_t* bar) {
+  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap*,
+                                    const CUtensorMap*, const Params&, int, uint8_t* sA, uint8_t* sB, uint8_t*, int m0,
+                                    int n0, int kb, uint64_t* bar) {
     const int k0 = kb * BK;
     if (A_MN) {  // two boxes of [64 k][64 m]
       tma_load_2d_pair(sA, tA, m0, k0, bar);
@@ -229,8 +252,8 @@ struct CfgPairBf16 {
     }
   }
 
-  __device__ static void mma_stage(const Params&, uint32_t d_tmem, uint32_t, uint8_t* sA, uint8_t* sB, uint8_t*,
-                                   bool first) {
+  __device__ static void mma_stage(const Params&, int, uint32_t d_tmem, uint32_t, uint8_t* sA, uint8_t* sB,
+                                   uint8_t*, bool first) {
     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
     for (int kk = 0; kk < BK / 16; ++kk) {
@@ -240,8 +263,96 @@ struct CfgPairBf16 {
     }
   }
 
-  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int lane) {
+  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane) {
     CfgBf16<A_MN, B_MN, OUT_F32>::epilogue(p, t_acc, row, n0, lane);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Both STE backward products in one launch, tiles of 256 x 256:
+//   problem 0 (dX):  out0[M0][N] = alpha0 * A0 . B0,  A0 K-major [M0][K0], B0 MN-major [K0][N]
+//   problem 1 (dW):  out1[M1][N] = A1^T . B1,          A1 MN-major [K1][M1], B1 MN-major [K1][N]
+// The host orders the tiles of both problems longest first over the pairs
+// (the two problems have different depths), so the launch ends with all
+// pairs close to even instead of two separate tails.
+// ---------------------------------------------------------------------------
+constexpr int kDualMaxPairs = 96;
+constexpr int kDualMaxTiles = 1280;
+
+struct DualBf16Params {
+  int M[2], N, K[2];
+  int mblocks[2];           // 256-row blocks per problem
+  int tiles0;               // tile ids below this are problem 0
+  const float* alpha[2];    // device scalars or nullptr for 1
+  void* out[2];
+  uint32_t* status;
+  uint16_t sched_off[kDualMaxPairs + 1];  // pair p runs sched[sched_off[p] .. sched_off[p+1])
+  uint16_t sched[kDualMaxTiles];
+};
+
+template <bool OUT_F32>
+struct CfgPairDualBf16 {
+  using Params = DualBf16Params;
+  static constexpr int MAPS = 4;
+  static constexpr int BN = 256, BK = 64, STAGES = 6;
+  static constexpr int A_BYTES = 128 * BK * 2;        // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB
+  static constexpr int E_BYTES = 0;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int E_COL0 = 0, E_COLS = 0;
+  static constexpr uint32_t IDESC0 = idesc_bf16(256, BN, false, true);
+  static constexpr uint32_t IDESC1 = idesc_bf16(256, BN, true, true);
+
+  struct Tiles {
+    __device__ static int count(const Params& p, int pair, int) { return p.sched_off[pair + 1] - p.sched_off[pair]; }
+    __device__ static PairTile at(const Params& p, int pair, int, int i) {
+      const int id = p.sched[p.sched_off[pair] + i];
+      const int prob = id >= p.tiles0 ? 1 : 0;
+      const int local = id - (prob ? p.tiles0 : 0);
+      const int mb = p.mblocks[prob];
+      return PairTile{prob, local % mb, local / mb, (p.K[prob] + BK - 1) / BK};
+    }
+  };
+
+  // Maps: A0, B0, A1, B1.
+  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tA1,
+                                    const CUtensorMap* tB1, const Params&, int prob, uint8_t* sA, uint8_t* sB,
+                                    uint8_t*, int m0, int n0, int kb, uint64_t* bar) {
+    const int k0 = kb * BK;
+    if (prob == 0) {
+      tma_load_2d_pair(sA, tA, k0, m0, bar);  // [128 m][64 k]
+      tma_load_2d_pair(sB, tB, n0, k0, bar);
+      tma_load_2d_pair(sB + 8192, tB, n0 + 64, k0, bar);
+    } else {
+      tma_load_2d_pair(sA, tA1, m0, k0, bar);  // [64 k][64 m] x 2
+      tma_load_2d_pair(sA + 8192, tA1, m0 + 64, k0, bar);
+      tma_load_2d_pair(sB, tB1, n0, k0, bar);
+      tma_load_2d_pair(sB + 8192, tB1, n0 + 64, k0, bar);
+    }
+  }
+
+  __device__ static void mma_stage(const Params&, int prob, uint32_t d_tmem, uint32_t, uint8_t* sA, uint8_t* sB,
+                                   uint8_t*, bool first) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+    for (int kk = 0; kk < BK / 16; ++kk) {
+      const uint64_t ad = prob ? smem_desc(a0 + kk * 2048, 8192, 1024, 2) : smem_desc(a0 + kk * 32, 16, 1024, 2);
+      const uint64_t bd = smem_desc(b0 + kk * 2048, 8192, 1024, 2);
+      mma_bf16_pair(d_tmem, ad, bd, prob ? IDESC1 : IDESC0, (first && kk == 0) ? 0u : 1u);
+    }
+  }
+
+  __device__ static void epilogue(const Params& p, int prob, uint32_t t_acc, int row, int n0, int lane) {
+    Bf16Params q;
+    q.M = p.M[prob];
+    q.N = p.N;
+    q.K = p.K[prob];
+    q.alpha = p.alpha[prob];
+    q.out = p.out[prob];
+    q.ldo = p.N;
+    q.status = p.status;
+    CfgBf16<false, true, OUT_F32>::epilogue(q, t_acc, row, n0, lane);
   }
 };
 
@@ -254,6 +365,8 @@ struct CfgPairBf16 {
 template <bool ACC_OUT>
 struct CfgPairSparse {
   using Params = FwdParams;
+  using Tiles = StripedTiles<CfgPairSparse>;
+  static constexpr int MAPS = 3;
   static constexpr int BN = 224, BK = 256, STAGES = 4;
   static constexpr int A_BYTES = 128 * BK / 2;      // 16 KB
   static constexpr int B_BYTES = (BN / 2) * BK;     // 28 KB
@@ -270,8 +383,8 @@ struct CfgPairSparse {
   __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
 
   __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tE,
-                                    const Params& p, uint8_t* sA, uint8_t* sB, uint8_t* sE, int m0, int n0, int kb,
-                                    uint64_t* bar) {
+                                    const CUtensorMap*, const Params& p, int, uint8_t* sA, uint8_t* sB, uint8_t* sE,
+                                    int m0, int n0, int kb, uint64_t* bar) {
     tma_load_2d_pair(sA, tA, kb * (BK / 2), m0, bar);              // compressed columns
     tma_load_2d_pair(sB, tB, kb * BK, n0, bar);                    // logical k 0..127 of the stage
     tma_load_2d_pair(sB + (BN / 2) * 128, tB, kb * BK + 128, n0, bar);  // logical k 128..255
@@ -280,7 +393,7 @@ struct CfgPairSparse {
     tma_load_2d_pair(sE, tE, 0, row, bar);
   }
 
-  __device__ static void mma_stage(const Params&, uint32_t d_tmem, uint32_t e_tmem, uint8_t* sA, uint8_t* sB,
+  __device__ static void mma_stage(const Params&, int, uint32_t d_tmem, uint32_t e_tmem, uint8_t* sA, uint8_t* sB,
                                    uint8_t* sE, bool first) {
     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB), e0 = smem_u32(sE);
     tmem_copy_128x128b_pair(e_tmem, smem_desc(e0, 2048, 128, 0));
@@ -294,7 +407,7 @@ struct CfgPairSparse {
     }
   }
 
-  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int lane) {
+  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane) {
     const float g = *p.g;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {

@@ -194,6 +194,14 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
     return SBL_OK;
   }
   uint32_t* status = at<uint32_t>(layer, L.status);
+  if (want_dx && want_dw) {
+    bool done = false;
+    const cudaError_t e = launch_bf16_backward_dual(
+        f32, static_cast<const uint16_t*>(dy), at<const uint16_t>(layer, L.weff_bf16), static_cast<const uint16_t*>(x),
+        t, layer->n_out, layer->k, at<const float>(layer, L.g), dx, dw, status, sms, s, &done);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+    if (done) return SBL_OK;
+  }
   if (want_dx) {
     // dX[t, k] = g * dY[t, n_out] . W_eff[n_out, k]:  A = dY (K-major), B = W_eff stored [K][N].
     const cudaError_t e = launch_bf16_gemm(false, true, f32, static_cast<const uint16_t*>(dy),

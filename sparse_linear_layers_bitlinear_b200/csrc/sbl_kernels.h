@@ -44,6 +44,12 @@ cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t*
                              int64_t N, int64_t K, const float* alpha, void* out, uint32_t* status, int num_sms,
                              cudaStream_t s);
 
+// dX = g * dY . W_eff and dW = dY^T . X in one launch.  Sets *done = false
+// (and enqueues nothing) when the tile count exceeds the launch's schedule.
+cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const uint16_t* weff, const uint16_t* x,
+                                      int64_t t, int64_t n_out, int64_t k, const float* g, void* dx, void* dw,
+                                      uint32_t* status, int num_sms, cudaStream_t s, bool* done);
+
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 // cuTensorMapEncodeTiled, resolved through the runtime's driver entry point.
