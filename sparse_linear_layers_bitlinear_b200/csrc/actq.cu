@@ -7,6 +7,11 @@
 // vectors of the row in registers, so the row is read from memory once: the
 // block reduces the absmax, then every thread quantises what it holds.  Rows
 // longer than 128 * 8 * kMaxR elements take a two-pass, warp-per-row kernel.
+//
+// The kernel reads only x and writes only its own outputs, so it is launched
+// with programmatic stream serialisation: right after a weight prepare it
+// runs alongside the pack kernel.  It waits for its predecessor before it
+// touches the status word it shares with the prepare and before it exits.
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
@@ -83,7 +88,10 @@ __global__ void __launch_bounds__(kActThreads)
     const float ap = fmaxf(amax, 1e-5f);
     if (tid == 0) {
       a_prime[row] = ap;
-      if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
+      if (bad) {
+        pdl_wait();  // a prepare before this kernel resets the status word
+        raise_status(status, SBL_STATUS_NONFINITE_X);
+      }
     }
     uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
 #pragma unroll
@@ -92,6 +100,7 @@ __global__ void __launch_bounds__(kActThreads)
       if (i < nvec) dst[i] = quantise8(v[r], ap);
     }
   }
+  pdl_wait();
 }
 
 // Long rows: one warp per row, absmax pass then a second (L1/L2) pass.
@@ -116,21 +125,26 @@ __global__ void __launch_bounds__(kActWarps * 32)
     for (; i < nvec; i += 32) scan8(__ldg(src + i), amax, bad);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) raise_status(status, SBL_STATUS_NONFINITE_X);
+    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) {
+      pdl_wait();  // a prepare before this kernel resets the status word
+      raise_status(status, SBL_STATUS_NONFINITE_X);
+    }
     const float ap = fmaxf(amax, 1e-5f);
     if (lane == 0) a_prime[row] = ap;
     uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
     for (int64_t j = lane; j < nvec; j += 32) dst[j] = quantise8(__ldg(src + j), ap);
   }
+  pdl_wait();
 }
 
 template <int R>
-static void launch_rows(const uint4* x, int64_t t, int64_t nvec, int8_t* xq, float* ap, uint32_t* status,
-                        int num_sms, cudaStream_t s) {
+static cudaError_t launch_rows(const uint4* x, int64_t t, int64_t nvec, int8_t* xq, float* ap, uint32_t* status,
+                               int num_sms, cudaStream_t s) {
   int64_t blocks = t;
   const int64_t cap = int64_t(num_sms) * 64;
   if (blocks > cap) blocks = cap;
-  k_act_quant_rows<R><<<static_cast<unsigned>(blocks), kActThreads, 0, s>>>(x, t, nvec, xq, ap, status);
+  return launch_pdl(k_act_quant_rows<R>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t, nvec,
+                    xq, ap, status);
 }
 
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
@@ -139,21 +153,19 @@ cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const int64_t nvec = k / 8;
   const int64_t r = (nvec + kActThreads - 1) / kActThreads;
-  if (r <= 1) launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 2) launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 3) launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 4) launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 6) launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 8) launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= 12) launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else if (r <= kMaxR) launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  else {
-    int64_t blocks = (t + kActWarps - 1) / kActWarps;
-    const int64_t cap = int64_t(num_sms) * 16;
-    if (blocks > cap) blocks = cap;
-    k_act_quant_long<<<static_cast<unsigned>(blocks), kActWarps * 32, 0, s>>>(xv, t, nvec, xq, a_prime, status);
-  }
-  return cudaGetLastError();
+  if (r <= 1) return launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 2) return launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 3) return launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 4) return launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 6) return launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 8) return launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 12) return launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= kMaxR) return launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  int64_t blocks = (t + kActWarps - 1) / kActWarps;
+  const int64_t cap = int64_t(num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(k_act_quant_long, dim3(static_cast<unsigned>(blocks)), dim3(kActWarps * 32), 0, s, xv, t, nvec, xq,
+                    a_prime, status);
 }
 
 }  // namespace sbl

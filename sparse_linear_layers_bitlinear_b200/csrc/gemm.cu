@@ -77,7 +77,7 @@ static cudaError_t pair_setup(int num_sms, int* max_clusters_out) {
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms & ~1);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(pair_threads<Cfg>());
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -105,7 +105,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const
   const int tiles = ((m_rows + 255) / 256) * ((n_cols + Cfg::BN - 1) / Cfg::BN);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
   if (pairs <= 0) return cudaSuccess;
-  k_gemm_pair<Cfg><<<2 * pairs, kGemmThreads, pair_smem_bytes<Cfg>(), s>>>(a, b, e, e, p);
+  k_gemm_pair<Cfg><<<2 * pairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a, b, e, e, p);
   return cudaGetLastError();
 }
 
@@ -279,7 +279,7 @@ cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16
   p.status = status;
   std::copy(sch.off.begin(), sch.off.end(), p.sched_off);
   std::copy(sch.ids.begin(), sch.ids.end(), p.sched);
-  k_gemm_pair<Cfg><<<2 * npairs, kGemmThreads, pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
+  k_gemm_pair<Cfg><<<2 * npairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
   err = cudaGetLastError();
   *done = err == cudaSuccess;
   return err;

@@ -56,7 +56,12 @@ struct PairSmemTail {
 };
 
 template <class Cfg>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+constexpr int pair_threads() {
+  return 64 + 32 * Cfg::EPI_WARPS;
+}
+
+template <class Cfg>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<Cfg>(), 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmF,
                 const typename Cfg::Params p) {
@@ -80,7 +85,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->acc_full[b], 1);
-      mbar_init(&tail->acc_empty[b], 8);  // 4 epilogue warps in each CTA
+      mbar_init(&tail->acc_empty[b], 2 * Cfg::EPI_WARPS);  // every epilogue warp of both CTAs
     }
     mbar_init(&tail->drain, 1);
     tail->abort_flag = 0;
@@ -175,8 +180,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    // ---------------- epilogue (warps 2.., both CTAs) ----------------
+    // Warp w reads TMEM lanes 32*(w%4)..+31; with 8 epilogue warps two warps
+    // share a lane quarter and split its 32-column chunks.
+    const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2, parts = Cfg::EPI_WARPS / 4;
     const uint32_t leader_acc_empty0 = map_to_rank(&tail->acc_empty[0], 0);
     for (int i = 0; i < ntiles; ++i) {
       const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
@@ -190,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int m0 = t.mb * 256 + 128 * int(rank);
       const int n0 = t.nb * Cfg::BN;
       const uint32_t t_acc = tmem_base + ab * Cfg::ACC_COLS + (uint32_t(quarter * 32) << 16);
-      Cfg::epilogue(p, t.prob, t_acc, m0 + quarter * 32 + lane, n0, lane);
+      Cfg::epilogue(p, t.prob, t_acc, m0 + quarter * 32 + lane, n0, lane, part, parts);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_acc_empty0 + ab * 8u);
@@ -221,6 +229,7 @@ struct CfgPairBf16 {
   using Params = Bf16Params;
   using Tiles = StripedTiles<CfgPairBf16>;
   static constexpr int MAPS = 2;
+  static constexpr int EPI_WARPS = 4;
   static constexpr int BN = 256, BK = 64, STAGES = 6;
   static constexpr int A_BYTES = 128 * BK * 2;        // 16 KB
   static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB
@@ -263,8 +272,9 @@ struct CfgPairBf16 {
     }
   }
 
-  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane) {
-    CfgBf16<A_MN, B_MN, OUT_F32>::epilogue(p, t_acc, row, n0, lane);
+  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane, int part,
+                                  int parts) {
+    CfgBf16<A_MN, B_MN, OUT_F32>::epilogue(p, t_acc, row, n0, lane, part, parts);
   }
 };
 
@@ -294,6 +304,7 @@ template <bool OUT_F32>
 struct CfgPairDualBf16 {
   using Params = DualBf16Params;
   static constexpr int MAPS = 4;
+  static constexpr int EPI_WARPS = 4;
   static constexpr int BN = 256, BK = 64, STAGES = 6;
   static constexpr int A_BYTES = 128 * BK * 2;        // 16 KB
   static constexpr int B_BYTES = (BN / 2) * BK * 2;   // 16 KB
@@ -343,7 +354,8 @@ struct CfgPairDualBf16 {
     }
   }
 
-  __device__ static void epilogue(const Params& p, int prob, uint32_t t_acc, int row, int n0, int lane) {
+  __device__ static void epilogue(const Params& p, int prob, uint32_t t_acc, int row, int n0, int lane, int part,
+                                  int parts) {
     Bf16Params q;
     q.M = p.M[prob];
     q.N = p.N;
@@ -352,7 +364,7 @@ struct CfgPairDualBf16 {
     q.out = p.out[prob];
     q.ldo = p.N;
     q.status = p.status;
-    CfgBf16<false, true, OUT_F32>::epilogue(q, t_acc, row, n0, lane);
+    CfgBf16<false, true, OUT_F32>::epilogue(q, t_acc, row, n0, lane, part, parts);
   }
 };
 
@@ -367,6 +379,7 @@ struct CfgPairSparse {
   using Params = FwdParams;
   using Tiles = StripedTiles<CfgPairSparse>;
   static constexpr int MAPS = 3;
+  static constexpr int EPI_WARPS = 8;  // the fp32 output is the heavy part of this epilogue
   static constexpr int BN = 224, BK = 256, STAGES = 4;
   static constexpr int A_BYTES = 128 * BK / 2;      // 16 KB
   static constexpr int B_BYTES = (BN / 2) * BK;     // 28 KB
@@ -407,10 +420,11 @@ struct CfgPairSparse {
     }
   }
 
-  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane) {
+  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane, int part,
+                                  int parts) {
     const float g = *p.g;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = part; c < BN / 32; c += parts) {
       uint32_t r[32];
       __syncwarp();
       tmem_load_32x32b_x32(t_acc + c * 32, r);

@@ -244,10 +244,11 @@ struct CfgBf16 {
     }
   }
 
-  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int) {
+  __device__ static void epilogue(const Params& p, uint32_t t_acc, int row, int n0, int, int part = 0,
+                                  int parts = 1) {
     const float alpha = p.alpha ? *p.alpha : 1.0f;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = part; c < BN / 32; c += parts) {
       uint32_t r[32];
       __syncwarp();
       tmem_load_32x32b_x32(t_acc + c * 32, r);
