@@ -15,43 +15,21 @@
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
+#include "actq_math.cuh"
 
 namespace sbl {
 
 constexpr int kActThreads = 128;
 constexpr int kMaxR = 16;  // rows up to 16384 elements stay in registers
 
-__device__ __forceinline__ float bf16_abs_value(uint32_t bits16) { return __uint_as_float((bits16 & 0x7FFFu) << 16); }
-
-// 8 bf16 values -> 8 int8 codes (two words).
-__device__ __forceinline__ uint2 quantise8(const uint4 v, float ap) {
-  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-  uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const uint32_t b = (words[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-    const float q = __fdiv_rn(__fmul_rn(127.0f, bf16_abs_value(b)), ap);
-    const int n = min(__float2int_rn(q), 127);  // nearest, ties to even
-    const int code = (b & 0x8000u) ? -n : n;
-    packed[e >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (e & 3));
-  }
-  return make_uint2(packed[0], packed[1]);
-}
-
-__device__ __forceinline__ void scan8(const uint4 v, float& amax, uint32_t& bad) {
-  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t b = (words[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-    bad |= ((b & 0x7F80u) == 0x7F80u);
-    amax = fmaxf(amax, bf16_abs_value(b));
-  }
-}
-
 template <int R>
 __global__ void __launch_bounds__(kActThreads)
     k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
-                     float* __restrict__ a_prime, uint32_t* status) {
+                     float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
+  if (early_trigger) {
+    pdl_wait();
+    pdl_trigger();
+  }
   __shared__ float s_max[kActThreads / 32];
   __shared__ uint32_t s_bad[kActThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -108,7 +86,11 @@ constexpr int kActWarps = 8;
 
 __global__ void __launch_bounds__(kActWarps * 32)
     k_act_quant_long(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
-                     float* __restrict__ a_prime, uint32_t* status) {
+                     float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
+  if (early_trigger) {
+    pdl_wait();
+    pdl_trigger();
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int64_t row = int64_t(blockIdx.x) * kActWarps + warp; row < t; row += int64_t(gridDim.x) * kActWarps) {
     const uint4* src = x + row * nvec;
@@ -139,33 +121,34 @@ __global__ void __launch_bounds__(kActWarps * 32)
 
 template <int R>
 static cudaError_t launch_rows(const uint4* x, int64_t t, int64_t nvec, int8_t* xq, float* ap, uint32_t* status,
-                               int num_sms, cudaStream_t s) {
+                               int num_sms, cudaStream_t s, int early) {
   int64_t blocks = t;
   const int64_t cap = int64_t(num_sms) * 64;
   if (blocks > cap) blocks = cap;
   return launch_pdl(k_act_quant_rows<R>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t, nvec,
-                    xq, ap, status);
+                    xq, ap, status, early);
 }
 
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
-                             int num_sms, cudaStream_t s) {
+                             int num_sms, cudaStream_t s, bool early_trigger) {
+  const int early = early_trigger ? 1 : 0;
   if (t <= 0) return cudaSuccess;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const int64_t nvec = k / 8;
   const int64_t r = (nvec + kActThreads - 1) / kActThreads;
-  if (r <= 1) return launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 2) return launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 3) return launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 4) return launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 6) return launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 8) return launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= 12) return launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s);
-  if (r <= kMaxR) return launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s);
+  if (r <= 1) return launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 2) return launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 3) return launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 4) return launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 6) return launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 8) return launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 12) return launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= kMaxR) return launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
   int64_t blocks = (t + kActWarps - 1) / kActWarps;
   const int64_t cap = int64_t(num_sms) * 16;
   if (blocks > cap) blocks = cap;
   return launch_pdl(k_act_quant_long, dim3(static_cast<unsigned>(blocks)), dim3(kActWarps * 32), 0, s, xv, t, nvec, xq,
-                    a_prime, status);
+                    a_prime, status, early);
 }
 
 }  // namespace sbl

@@ -1,6 +1,5 @@
 // Launchers for the tensor-core GEMMs (forward int8, dense or 2:4 sparse;
-// backward bf16), the decode GEMV, the tensor-map encoder and the bounded-wait
-// self test.
+// backward bf16), the tensor-map encoder and the bounded-wait self test.
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -292,128 +291,6 @@ cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const ui
                                       uint32_t* status, int num_sms, cudaStream_t s, bool* done) {
   return out_f32 ? dual_dispatch<true>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done)
                  : dual_dispatch<false>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done);
-}
-
-// ---------------------------------------------------------------------------
-// Decode GEMV (t <= 16) over the 2-bit packing: one byte per group of four,
-// metadata nibble high (i0 | i1 << 2), codes low (2 bits each: 00 0, 01 +1,
-// 11 -1).  The group byte expands through a 256-entry table into the four
-// int8 weights of the group; dp4a multiplies them with four activation codes.
-// Each warp owns 4 rows; lanes stride over 16-weight words of the rows.
-// ---------------------------------------------------------------------------
-constexpr int kGemvRows = 4;
-
-template <int TP>  // token count rounded up to a power of two
-__global__ void __launch_bounds__(256) k_gemv(const uint32_t* __restrict__ packed, const int8_t* __restrict__ xq,
-                                              const float* __restrict__ a_prime, const float* __restrict__ gptr,
-                                              int n_out, int t, int k, float* __restrict__ y,
-                                              int32_t* __restrict__ acc_out) {
-  extern __shared__ uint32_t smem_u[];
-  uint32_t* lut = smem_u;                // 256 entries
-  uint32_t* sx = smem_u + 256;           // [TP][k/4]
-  const int kw = k / 4;                  // 32-bit words of activation codes per token
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-    auto code_of = [](int two_bits) { return two_bits == 1 ? 1 : (two_bits == 3 ? -1 : 0); };
-    const int c0 = code_of(i & 3), c1 = code_of((i >> 2) & 3);
-    const int i0 = (i >> 4) & 3, i1 = (i >> 6) & 3;
-    lut[i] = ((static_cast<uint32_t>(c0) & 0xFFu) << (8 * i0)) | ((static_cast<uint32_t>(c1) & 0xFFu) << (8 * i1));
-  }
-  const uint32_t* xw = reinterpret_cast<const uint32_t*>(xq);
-  for (int i = threadIdx.x; i < TP * kw; i += blockDim.x) {
-    const int tt = i / kw;
-    sx[i] = (tt < t) ? __ldg(xw + int64_t(tt) * kw + (i % kw)) : 0u;
-  }
-  __syncthreads();
-  const float g = *gptr;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int words_per_row = k / 16;  // packed 32-bit words per row (4 groups each)
-  const int warps_total = gridDim.x * (blockDim.x >> 5);
-  for (int row0 = (blockIdx.x * (blockDim.x >> 5) + warp) * kGemvRows; row0 < n_out; row0 += warps_total * kGemvRows) {
-    int acc[kGemvRows][TP];
-#pragma unroll
-    for (int r = 0; r < kGemvRows; ++r)
-#pragma unroll
-      for (int tt = 0; tt < TP; ++tt) acc[r][tt] = 0;
-    for (int q = lane; q < words_per_row; q += 32) {
-      uint32_t wexp[kGemvRows][4];
-#pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) {
-        const uint32_t word = (row0 + r < n_out) ? __ldcs(packed + int64_t(row0 + r) * words_per_row + q) : 0u;
-#pragma unroll
-        for (int gi = 0; gi < 4; ++gi) wexp[r][gi] = lut[(word >> (8 * gi)) & 0xFFu];
-      }
-#pragma unroll
-      for (int tt = 0; tt < TP; ++tt) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(sx + tt * kw + 4 * q);
-#pragma unroll
-        for (int r = 0; r < kGemvRows; ++r) {
-          acc[r][tt] = __dp4a(static_cast<int>(wexp[r][0]), static_cast<int>(xv.x), acc[r][tt]);
-          acc[r][tt] = __dp4a(static_cast<int>(wexp[r][1]), static_cast<int>(xv.y), acc[r][tt]);
-          acc[r][tt] = __dp4a(static_cast<int>(wexp[r][2]), static_cast<int>(xv.z), acc[r][tt]);
-          acc[r][tt] = __dp4a(static_cast<int>(wexp[r][3]), static_cast<int>(xv.w), acc[r][tt]);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kGemvRows; ++r)
-#pragma unroll
-      for (int tt = 0; tt < TP; ++tt) {
-        int v = acc[r][tt];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        acc[r][tt] = v;
-      }
-#pragma unroll
-    for (int base = 0; base < kGemvRows * TP; base += 32) {
-      const int pair = base + lane;  // pair -> (row r, token tt)
-      if (pair < kGemvRows * TP) {
-        // pick the reduced value without dynamic register indexing
-        int v = 0;
-#pragma unroll
-        for (int r = 0; r < kGemvRows; ++r)
-#pragma unroll
-          for (int tt = 0; tt < TP; ++tt)
-            if (pair == r * TP + tt) v = acc[r][tt];
-        const int r = pair / TP, tt = pair % TP;
-        const int row = row0 + r;
-        if (row < n_out && tt < t) {
-          const float f = __fdiv_rn(__fmul_rn(g, a_prime[tt]), 127.0f);
-          y[int64_t(tt) * n_out + row] = __fmul_rn(static_cast<float>(v), f);
-          if (acc_out) acc_out[int64_t(tt) * n_out + row] = v;
-        }
-      }
-    }
-  }
-}
-
-template <int TP>
-static cudaError_t gemv_tp(const uint8_t* gemv, const int8_t* xq, const float* a_prime, const float* g, int64_t n_out,
-                           int64_t t, int64_t k, float* y, int32_t* acc_out, int num_sms, cudaStream_t s) {
-  const size_t smem = (256 + size_t(TP) * size_t(k / 4)) * 4;
-  if (smem > 200 * 1024) return cudaErrorInvalidValue;
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    err = cudaFuncSetAttribute(k_gemv<TP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  });
-  if (err != cudaSuccess) return err;
-  const int64_t warps_needed = (n_out + kGemvRows - 1) / kGemvRows;
-  int64_t blocks = (warps_needed + 7) / 8;
-  if (blocks > num_sms) blocks = num_sms;
-  k_gemv<TP><<<static_cast<unsigned>(blocks), 256, smem, s>>>(reinterpret_cast<const uint32_t*>(gemv), xq, a_prime, g,
-                                                              static_cast<int>(n_out), static_cast<int>(t),
-                                                              static_cast<int>(k), y, acc_out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_forward_gemv(const uint8_t* gemv, const int8_t* xq, const float* a_prime, const float* g,
-                                int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out, int num_sms,
-                                cudaStream_t s) {
-  if (t <= 1) return gemv_tp<1>(gemv, xq, a_prime, g, n_out, t, k, y, acc_out, num_sms, s);
-  if (t <= 2) return gemv_tp<2>(gemv, xq, a_prime, g, n_out, t, k, y, acc_out, num_sms, s);
-  if (t <= 4) return gemv_tp<4>(gemv, xq, a_prime, g, n_out, t, k, y, acc_out, num_sms, s);
-  if (t <= 8) return gemv_tp<8>(gemv, xq, a_prime, g, n_out, t, k, y, acc_out, num_sms, s);
-  return gemv_tp<16>(gemv, xq, a_prime, g, n_out, t, k, y, acc_out, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -154,12 +154,21 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(layer, L.status);
   const float* g = at<const float>(layer, L.g);
+  if (L.gemv != 0 && gemv_fits(t, layer->k)) {
+    // decode: the 2-bit weight stream
+    const bool fused = gemv_fuses_act_quant(t);
+    if (!fused &&
+        launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true) != cudaSuccess)
+      return SBL_ERR_CUDA;
+    const cudaError_t e =
+        launch_forward_gemv(at<const uint8_t>(layer, L.gemv), static_cast<const uint16_t*>(x), xq, ap, g,
+                            layer->n_out, t, layer->k, y, acc_debug, fused ? xq_out : nullptr,
+                            fused ? xscale_out : nullptr, status, sms, s);
+    return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+  }
   cudaError_t e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s);
   if (e != cudaSuccess) return SBL_ERR_CUDA;
-  if (L.gemv != 0 && t <= 16) {
-    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), xq, ap, g, layer->n_out, t, layer->k, y, acc_debug, sms,
-                            s);
-  } else if (is_24(layer->n, layer->m)) {
+  if (is_24(layer->n, layer->m)) {
     e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
                             static_cast<int>(meta_k_padded(layer->k) / 128), L.sp_meta_bytes, xq, ap, g, layer->n_out,
                             t, layer->k, y,

@@ -42,8 +42,10 @@ struct PackOut {
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags, uint8_t* blob,
                            const sbl_blob_layout& L, int num_sms, cudaStream_t s);
 
+// early_trigger: wait for the predecessor, then let the next kernel launch at
+// once (it must wait for this one before reading xq / a_prime).
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
-                             int num_sms, cudaStream_t s);
+                             int num_sms, cudaStream_t s, bool early_trigger = false);
 
 // Forward GEMM + dequant.  sparse: codes = 2:4 kept values [n_out][k/2] and
 // meta = tensor-core metadata; dense: codes = W_eff int8 [n_out][k].
@@ -52,10 +54,16 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
                                 int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
                                 cudaStream_t s);
 
-// Decode GEMV for t <= 16 over the 2-bit packing.
-cudaError_t launch_forward_gemv(const uint8_t* gemv, const int8_t* xq, const float* a_prime, const float* g,
-                                int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out, int num_sms,
-                                cudaStream_t s);
+// Decode forward for 1 <= t <= 16 over the 2-bit packing.  For t up to 4 the
+// kernel quantises the activations itself (xq_out / ap_out, when given,
+// receive the codes and scales); for larger t the act-quant kernel runs first
+// with its early trigger and xq_in / ap_in are its outputs.  gemv_fits() says
+// whether the token rows fit the kernel's shared memory.
+bool gemv_fits(int64_t t, int64_t k);
+bool gemv_fuses_act_quant(int64_t t);
+cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const int8_t* xq_in, const float* ap_in,
+                                const float* g, int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out,
+                                int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms, cudaStream_t s);
 
 // out[M][N] = alpha * A . B^T in bf16 x bf16 -> fp32 (tensor cores).
 //   a_mn: A stored [K][M] (else [M][K]);  b_mn: B stored [K][N] (else [N][K]).

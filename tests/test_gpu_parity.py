@@ -123,7 +123,7 @@ def test_prepare_forward_backward_parity(n_out, k, n, m, t):
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
 
 
-@pytest.mark.parametrize("t", [1, 2, 4, 7, 16])
+@pytest.mark.parametrize("t", [1, 2, 3, 4, 5, 7, 8, 9, 16])
 def test_gemv_path_parity(t):
     n_out, k = 392, 640
     w = synth.master_weights(n_out, k, 3)
@@ -138,7 +138,10 @@ def test_gemv_path_parity(t):
     ap = torch.empty((t,), dtype=torch.float32, device="cuda")
     sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
     torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
     xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
     acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     y_ref = oracle.dequant(acc_ref, ap_ref, ref["g"])
