@@ -256,6 +256,122 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Other workloads, reported beside the headline line
+# ---------------------------------------------------------------------------
+def bench_decode(dev, hbm_gbs, reps=10):
+    """Decode-shaped forward over the 2-bit weight packing: T in {1, 4, 16},
+    K = 2560, N_out in {2560, 6912}.  One replay = 64 forward calls in a CUDA
+    graph over distinct weight blobs (more than 2 x L2 of weights in total),
+    so every call streams its weights from HBM.  The per-call time includes the
+    launch of each call inside the graph."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    K = 2560
+    out = []
+    for N in (2560, 6912):
+        nblob = max(8, int(2 * 126e6 / (N * K / 4)) + 1)
+        layers = []
+        for i in range(nblob):
+            L = sbl.Layer.allocate(N, K, 2, 4, sbl.SBL_PACK_GEMV, device=dev)
+            sbl.prepare_weights(L, synth.master_weights(N, K, 5000 + i, device=dev))
+            layers.append(L)
+        for T in (1, 4, 16):
+            x = synth.activations(T, K, 7, device=dev)
+            y = torch.empty((T, N), dtype=torch.float32, device=dev)
+            ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+            s = torch.cuda.Stream(dev)
+            with torch.cuda.stream(s):
+                for i in range(3):
+                    sbl.forward(layers[i % nblob], x, T, y, workspace=ws, stream=s)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for i in range(64):
+                    sbl.forward(layers[i % nblob], x, T, y, workspace=ws, stream=s)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) / (64 * reps) * 1e3
+            by = N * K / 4 + 2 * T * K + 4 * T * N
+            out.append({"n_out": N, "k": K, "tokens": T, "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
+                        "gbs": by / (us * 1e-6) / 1e9, "hbm_frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+                        "bytes_per_call": by})
+            del g
+        del layers
+        torch.cuda.empty_cache()
+    return {"workload": "decode 2:4 forward, 2-bit packed weights, K=2560",
+            "timing": "CUDA graph of 64 calls over distinct weight blobs (> 2 x L2), per-call time incl. launch",
+            "points": out}
+
+
+def bench_prefill68(dev, peaks, steps=20):
+    """The 6:8 FFN down projection: T=4096, K=6912, N_out=2560, prepare +
+    forward (dense int8 over W_eff codes) + dual-STE backward per step."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    T, K, N = 4096, 6912, 2560
+    sets = [(synth.master_weights(N, K, 20 + 10 * r, device=dev), synth.activations(T, K, 21 + 10 * r, device=dev),
+             synth.upstream_grad(T, N, 22 + 10 * r, device=dev)) for r in range(ROTATE)]
+    layer = sbl.Layer.allocate(N, K, 6, 8, device=dev)
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def step(i, rec=False):
+        w, x, dy = sets[i % ROTATE]
+        if rec:
+            ev[0].record()
+        sbl.prepare_weights(layer, w)
+        if rec:
+            ev[1].record()
+        sbl.forward(layer, x, T, y, workspace=ws)
+        if rec:
+            ev[2].record()
+        sbl.backward(layer, x, dy, T, dx, dw, 0)
+        if rec:
+            ev[3].record()
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    ph = [0.0, 0.0, 0.0]
+    for i in range(5):
+        step(i, True)
+        torch.cuda.synchronize(dev)
+        for j in range(3):
+            ph[j] += ev[j].elapsed_time(ev[j + 1]) / 5
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_OK, (code, bits)
+    dense_ops = 2.0 * T * K * N
+    i8_dense = 2.0 * peaks["bf16_tflops"] * 1e12
+    return {"workload": "prefill 6:8 Sparse-BitLinear fwd+STE bwd, FFN down projection", "tokens": T, "k": K,
+            "n_out": N, "n": 6, "m": 8, "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3),
+            "phase_ms": {"prepare": ph[0], "forward": ph[1], "backward": ph[2]},
+            "fwd_dense_int8_tops": dense_ops / (ph[1] * 1e-3) / 1e12,
+            "fwd_frac_of_dense_int8_peak": dense_ops / (ph[1] * 1e-3) / i8_dense,
+            "bwd_tflops": 2 * dense_ops / (ph[2] * 1e-3) / 1e12}
+
+
+# ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
 def main():
@@ -266,6 +382,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode and 6:8 workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -429,6 +546,9 @@ def main():
         "clocks": clocks.summary(),
         "peaks": peaks,
     }
+    if not args.no_extras:
+        line["decode_gemv"] = bench_decode(dev, peaks["hbm_gbs"])
+        line["prefill_6of8"] = bench_prefill68(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
     if rank == 0:

@@ -435,4 +435,62 @@ struct CfgPairSparse {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Dense int8 forward on pairs (every N:M pattern other than 2:4): tile 256 W
+// rows x BN tokens, 128 k per stage.  Each CTA holds 128 rows of W_eff codes
+// (128 x 128 bytes) and BN/2 tokens of xq.
+// ---------------------------------------------------------------------------
+template <bool ACC_OUT, int BN_>
+struct CfgPairDense {
+  using Params = FwdParams;
+  using Tiles = StripedTiles<CfgPairDense>;
+  static constexpr int MAPS = 2;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int BN = BN_, BK = 128;
+  static constexpr int A_BYTES = 128 * BK;        // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK;   // 16 KB at BN = 256
+  static constexpr int E_BYTES = 0;
+  static constexpr int STAGES = (200 * 1024) / (A_BYTES + B_BYTES) < 8 ? (200 * 1024) / (A_BYTES + B_BYTES) : 8;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int E_COL0 = 0, E_COLS = 0;
+  static constexpr uint32_t IDESC = idesc_i8(256, BN, false);
+  static_assert((BN / 2) % 8 == 0 && 2 * BN <= TMEM_COLS, "tile");
+
+  __device__ static int rows_M(const Params& p) { return p.n_out; }
+  __device__ static int cols_N(const Params& p) { return p.T; }
+  __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
+
+  __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap*,
+                                    const CUtensorMap*, const Params&, int, uint8_t* sA, uint8_t* sB, uint8_t*, int m0,
+                                    int n0, int kb, uint64_t* bar) {
+    tma_load_2d_pair(sA, tA, kb * BK, m0, bar);  // [128 rows][128 bytes]
+    tma_load_2d_pair(sB, tB, kb * BK, n0, bar);  // [BN/2 rows][128 bytes]
+  }
+
+  __device__ static void mma_stage(const Params&, int, uint32_t d_tmem, uint32_t, uint8_t* sA, uint8_t* sB, uint8_t*,
+                                   bool first) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+    for (int kk = 0; kk < BK / 32; ++kk) {
+      mma_i8_pair(d_tmem, smem_desc(a0 + kk * 32, 16, 1024, 2), smem_desc(b0 + kk * 32, 16, 1024, 2), IDESC,
+                  (first && kk == 0) ? 0u : 1u);
+    }
+  }
+
+  __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane, int part,
+                                  int parts) {
+    const float g = *p.g;
+#pragma unroll 1
+    for (int c = part; c < BN / 32; c += parts) {
+      uint32_t r[32];
+      __syncwarp();
+      tmem_load_32x32b_x32(t_acc + c * 32, r);
+      tmem_load_wait();
+      if (n0 + c * 32 >= p.T) continue;  // uniform across the warp
+      fwd_epilogue_chunk<ACC_OUT>(p, r, row, n0 + c * 32, lane, g);
+    }
+  }
+};
+
 }  // namespace sbl
