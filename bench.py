@@ -371,6 +371,78 @@ def bench_prefill68(dev, peaks, steps=20):
             "bwd_tflops": 2 * dense_ops / (ph[2] * 1e-3) / 1e12}
 
 
+def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
+    """One training step's linear layers: 30 x {q, k, v, o: 2560 x 2560;
+    gate, up: 2560 -> 6912; down: 6912 -> 2560} at 8192 tokens.  Per step every
+    linear re-prepares its weights (mask and codes from its masters) and runs
+    its forward; then every backward runs, last layer first.  Each linear has
+    its own masters, activations and upstream gradient; the whole step is one
+    CUDA graph."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    H, F, T = 2560, 6912, tokens
+    shapes = [("q", H, H), ("k", H, H), ("v", H, H), ("o", H, H), ("gate", F, H), ("up", F, H), ("down", H, F)]
+    lin = []
+    for l in range(layers):
+        for j, (name, n_out, k) in enumerate(shapes):
+            seed = 1000 * l + 10 * j
+            lin.append(dict(
+                layer=sbl.Layer.allocate(n_out, k, n, m, device=dev),
+                w=synth.master_weights(n_out, k, seed, device=dev),
+                x=synth.activations(T, k, seed + 1, device=dev),
+                dy=synth.upstream_grad(T, n_out, seed + 2, device=dev), n_out=n_out, k=k))
+    # outputs reuse one buffer per shape (their values are not read within the step)
+    y = {n_out: torch.empty((T, n_out), dtype=torch.float32, device=dev) for n_out in (H, F)}
+    ws = {k: torch.empty(sbl.workspace_bytes(T, k), dtype=torch.uint8, device=dev) for k in (H, F)}
+    dx = {k: torch.empty((T, k), dtype=torch.bfloat16, device=dev) for k in (H, F)}
+    dw = {(o, k): torch.empty((o, k), dtype=torch.bfloat16, device=dev) for (_, o, k) in shapes}
+    s = torch.cuda.Stream(dev)
+
+    def step():
+        for d in lin:
+            sbl.prepare_weights(d["layer"], d["w"], stream=s)
+            sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], workspace=ws[d["k"]], stream=s)
+        for d in reversed(lin):
+            sbl.backward(d["layer"], d["x"], d["dy"], T, dx[d["k"]], dw[(d["n_out"], d["k"])], 0, stream=s)
+
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    for d in lin[:7]:
+        code, bits = sbl.read_status(d["layer"])
+        assert code == sbl.SBL_OK, (code, bits)
+    # roofline of the step at the measured peaks
+    hbm, bf16 = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
+    i8 = (4.0 if (n, m) == (2, 4) else 2.0) * bf16
+    bound = 0.0
+    for (_, n_out, k) in shapes:
+        ops = 2.0 * T * n_out * k
+        prep_b = n_out * k * 2 + n_out * k * (0.625 if (n, m) == (2, 4) else 1.0)
+        fwd_b = T * k * 2 + T * k + T * n_out * 4
+        bound += layers * (prep_b / hbm + max(ops / i8, fwd_b / hbm) + 2 * ops / bf16)
+    del g
+    del lin
+    torch.cuda.empty_cache()
+    return {"workload": f"training step, {layers} layers x 7 linears, {n}:{m}", "tokens": T, "n": n, "m": m,
+            "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "roofline_ms": bound * 1e3,
+            "roofline_frac": bound * 1e3 / ms, "peak_note": "sustained bf16 peak (seconds-long step)",
+            "timing": f"one CUDA graph per step, {steps} replays after one warm-up"}
+
+
 # ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
@@ -549,6 +621,7 @@ def main():
     if not args.no_extras:
         line["decode_gemv"] = bench_decode(dev, peaks["hbm_gbs"])
         line["prefill_6of8"] = bench_prefill68(dev, peaks)
+        line["train_step"] = [bench_train_step(dev, peaks, 2, 4), bench_train_step(dev, peaks, 4, 8)]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
     if rank == 0:
