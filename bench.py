@@ -176,14 +176,21 @@ def barrier(world):
 
 
 def max_over_ranks(value: float, world: int) -> float:
+    """The slowest rank's value (NCCL needs a device tensor, gloo a host one)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(rank: int, rotation: int, tensor: int) -> int:
+    """Seed of one input tensor: every rank draws its own batch (weak scaling)."""
+    return 1000 * rank + 10 * rotation + tensor
 
 
 # ---------------------------------------------------------------------------
@@ -481,9 +488,9 @@ def main():
     # Inputs: ROTATE seeded sets, different per rank (independent batches).
     sets = []
     for r in range(ROTATE):
-        base = 1000 * rank + 10 * r
-        sets.append((synth.master_weights(N, K, base + 0, device=dev), synth.activations(T, K, base + 1, device=dev),
-                     synth.upstream_grad(T, N, base + 2, device=dev)))
+        sets.append((synth.master_weights(N, K, replica_seed(rank, r, 0), device=dev),
+                     synth.activations(T, K, replica_seed(rank, r, 1), device=dev),
+                     synth.upstream_grad(T, N, replica_seed(rank, r, 2), device=dev)))
     layer = sbl.Layer.allocate(N, K, n, m, device=dev)
     y = torch.empty((T, N), dtype=torch.float32, device=dev)
     ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)

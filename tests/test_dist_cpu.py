@@ -1,0 +1,56 @@
+"""Multi-rank plumbing of bench.py on CPU: two gloo ranks on 127.0.0.1.
+
+bench.py runs one independent replica per GPU (no collective on the data
+path): each rank draws its own inputs, the ranks meet at a barrier around the
+timed region, and the reported time is the slowest rank's.  These tests run
+that host logic with world size 2 and no GPU.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        # each rank reports a different per-step time; all must agree on the max
+        mx = bench.max_over_ranks(1.5 + rank, world)
+        seeds = [bench.replica_seed(rank, r, j) for r in range(bench.ROTATE) for j in range(3)]
+        gathered = [None] * world
+        dist.all_gather_object(gathered, seeds)
+        out[rank] = (mx, gathered)
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_time_and_draw_distinct_inputs():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 2.5
+    seeds0, seeds1 = res[0][1]
+    assert len(set(seeds0)) == len(seeds0) and not set(seeds0) & set(seeds1)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+    bench.barrier(1)
