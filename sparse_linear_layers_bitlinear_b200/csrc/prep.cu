@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(1024) k_gamma_finalize(const uint64_t* slot_bi
 //  * W_eff as bf16 is (sign | 0x3F80) masked by (kept & code != 0);
 //  * the int8 code byte of a bf16 W_eff value h is (h bit 13) | 0xFE * (h bit 15).
 // ---------------------------------------------------------------------------
-constexpr int kPackThreads = 512;
+constexpr int kPackThreads = 256;
+constexpr int kPackDepth = 8;  // 16-byte loads in flight per lane
 
 // (i0 | i1 << 2) for each 4-bit kept pattern with exactly two bits set.
 constexpr uint64_t kPairNibble = (uint64_t(0x4) << (4 * 0x3)) | (uint64_t(0x8) << (4 * 0x5)) |
@@ -279,15 +280,33 @@ __device__ __forceinline__ uint32_t keep_bits(const uint32_t (&mag)[8], int base
   return kept;
 }
 
+// Packed bf16 compares: 0xFFFF in each half where a > b (a >= b).  Inputs here
+// are magnitudes (sign bits cleared), so the float order is the order of the
+// 15-bit magnitude fields.
+__device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_ge_mask(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// The six outcomes c_ij = |w_i| >= |w_j| (i < j) of a group of four held as
+// two words of magnitudes (m0 | m1 << 16, m2 | m3 << 16), in the table-index
+// bit order c01, c02, c03, c12, c13, c23.
+__device__ __forceinline__ uint32_t pair_outcomes4_packed(uint32_t m01, uint32_t m23) {
+  const uint32_t rA = bf16x2_ge_mask(__byte_perm(m01, m23, 0x5410), __byte_perm(m01, m23, 0x7632));  // c01 | c23
+  const uint32_t rB = bf16x2_ge_mask(m01, m23);                                                       // c02 | c13
+  const uint32_t rC = bf16x2_ge_mask(m01, __byte_perm(m23, m23, 0x1032));                             // c03 | c12
+  return (rA & 1u) | (rB & 2u) | (rC & 4u) | ((rC >> 13) & 8u) | ((rB >> 12) & 16u) | ((rA >> 11) & 32u);
+}
+
 // Groups of four: the six pairwise outcomes c_ij = (|w_i| >= |w_j|), i < j,
 // index a 64-entry table whose byte holds the keep pattern (bits 0..3) and,
 // for n == 2, the metadata nibble i0 | i1 << 2 (bits 4..7).
-__device__ __forceinline__ uint32_t pair_outcomes4(const uint32_t (&mag)[8], int base) {
-  const uint32_t a = mag[base], b = mag[base + 1], c = mag[base + 2], d = mag[base + 3];
-  return (a >= b ? 1u : 0u) | (a >= c ? 2u : 0u) | (a >= d ? 4u : 0u) | (b >= c ? 8u : 0u) | (b >= d ? 16u : 0u) |
-         (c >= d ? 32u : 0u);
-}
-
 __device__ __forceinline__ uint32_t select4_entry(uint32_t cbits, int n) {
   const uint32_t c01 = cbits & 1u, c02 = (cbits >> 1) & 1u, c03 = (cbits >> 2) & 1u;
   const uint32_t c12 = (cbits >> 3) & 1u, c13 = (cbits >> 4) & 1u, c23 = (cbits >> 5) & 1u;
@@ -311,15 +330,22 @@ __device__ __forceinline__ uint32_t code_bytes4(uint32_t weff_lo, uint32_t weff_
 template <int M>
 __global__ void __launch_bounds__(kPackThreads)
     k_prep_pack(const uint4* __restrict__ w, int64_t n_out, int64_t k, int n, const BlobHeader* h, PackOut out) {
-  __shared__ uint32_t s_sel[64];  // M == 4: keep pattern and nibble per comparison outcome
-  if (M == 4 && threadIdx.x < 64) s_sel[threadIdx.x] = select4_entry(threadIdx.x, n);
+  // M == 4: per comparison outcome, the keep masks of the group's two words
+  // (0xFFFF per kept weight) and the byte keep pattern | nibble << 4.
+  __shared__ uint4 s_sel[64];
+  if (M == 4 && threadIdx.x < 64) {
+    const uint32_t e = select4_entry(threadIdx.x, n), kp = e & 0xFu;
+    const uint32_t km_lo = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
+    const uint32_t km_hi = (((kp >> 2) & 1u) | (((kp >> 2) & 2u) << 15)) * 0xFFFFu;
+    s_sel[threadIdx.x] = make_uint4(km_lo, km_hi, e, 0u);
+  }
   __syncthreads();
   pdl_wait();  // g comes from k_gamma_finalize (a kernel that may overlap this one: coherent load)
   const float g = __ldcg(&h->g);
-  // code != 0 <=> 15-bit magnitude > thr; adding (0x7FFF - thr) to each half
-  // sets that half's bit 15 exactly then (no carry leaves a half).
+  // code != 0 <=> 2|w| > g <=> |w| > g/2 (exact) <=> the 15-bit magnitude
+  // exceeds bits(g/2) >> 16, i.e. |w| > that bf16 value as a float compare.
   const uint32_t thr = __float_as_uint(__fmul_rn(g, 0.5f)) >> 16;
-  const uint32_t bias2 = (0x7FFFu - thr) * 0x00010001u;
+  const uint32_t thr2 = thr | (thr << 16);
   pdl_trigger();
 
   const int lane = threadIdx.x & 31;
@@ -329,44 +355,57 @@ __global__ void __launch_bounds__(kPackThreads)
   for (int64_t row = gwarp; row < n_out; row += nwarps) {
     const uint4* wrow = w + row * upr;
     uint4* weff_row = reinterpret_cast<uint4*>(out.weff_bf16) + row * upr;
-    // Four 16-byte loads in flight per lane, then process them one by one.
-    for (int c0 = 0; c0 < upr; c0 += 4 * 32) {
-      uint4 vbuf[4];
+    // kPackDepth 16-byte loads in flight per lane, then process them one by one.
+    for (int c0 = 0; c0 < upr; c0 += kPackDepth * 32) {
+      uint4 vbuf[kPackDepth];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kPackDepth; ++q) {
         const int cq = c0 + 32 * q + lane;
         vbuf[q] = (cq < upr) ? __ldcs(wrow + cq) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kPackDepth; ++q) {
         if (c0 + 32 * q >= upr) break;  // uniform across the warp
         const int c = c0 + 32 * q + lane;
         const bool active = c < upr;  // upr is a multiple of 8: quads are all-or-nothing
         const uint32_t wd[4] = {vbuf[q].x, vbuf[q].y, vbuf[q].z, vbuf[q].w};
-        uint32_t mag[8];
+        uint32_t mw[4];  // magnitudes, two per word
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          mag[2 * j] = wd[j] & 0x7FFFu;
-          mag[2 * j + 1] = wd[j] >> 16 & 0x7FFFu;
-        }
+        for (int j = 0; j < 4; ++j) mw[j] = wd[j] & 0x7FFF7FFFu;
         uint32_t kept = 0, sel0 = 0, sel1 = 0;
+        uint32_t km[4];  // 0xFFFF per kept weight
         if (M == 4) {
-          sel0 = s_sel[pair_outcomes4(mag, 0)];
-          sel1 = s_sel[pair_outcomes4(mag, 4)];
+          const uint4 e0 = s_sel[pair_outcomes4_packed(mw[0], mw[1])];
+          const uint4 e1 = s_sel[pair_outcomes4_packed(mw[2], mw[3])];
+          km[0] = e0.x;
+          km[1] = e0.y;
+          km[2] = e1.x;
+          km[3] = e1.y;
+          sel0 = e0.z;
+          sel1 = e1.z;
           kept = (sel0 & 0xFu) | ((sel1 & 0xFu) << 4);
         } else {
+          uint32_t mag[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            mag[2 * j] = mw[j] & 0xFFFFu;
+            mag[2 * j + 1] = mw[j] >> 16;
+          }
 #pragma unroll
           for (int gi = 0; gi < 8 / M; ++gi) kept |= keep_bits<M>(mag, gi * M, n) << (gi * M);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t kp = (kept >> (2 * j)) & 3u;
+            km[j] = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
+          }
         }
 
         // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and code != 0.
         uint32_t weff[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint32_t nz = ((((wd[j] & 0x7FFF7FFFu) + bias2) >> 15) & 0x00010001u) * 0xFFFFu;
-          const uint32_t kp = (kept >> (2 * j)) & 3u;
-          const uint32_t km = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
-          weff[j] = ((wd[j] & 0x80008000u) | 0x3F803F80u) & nz & km;
+          const uint32_t nz = bf16x2_gt_mask(mw[j], thr2);
+          weff[j] = ((wd[j] & 0x80008000u) | 0x3F803F80u) & nz & km[j];
         }
         const uint32_t codes_lo = code_bytes4(weff[0], weff[1]);  // weights 0..3
         const uint32_t codes_hi = code_bytes4(weff[2], weff[3]);  // weights 4..7
@@ -451,8 +490,8 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   e = launch_pdl(k_gamma_finalize, dim3(1), dim3(kFinThreads), 0, s, slot_bins, slot_flags, slots, h, n_out, k, n, m, flags);
   if (e != cudaSuccess) return e;
   // Rows are spread over warps; pick the warp count so every warp gets the
-  // same number of rows (within one) and the grid stays within two blocks/SM.
-  const int64_t max_warps = int64_t(num_sms) * 2 * (kPackThreads / 32);
+  // same number of rows (within one) and the grid stays within three blocks/SM.
+  const int64_t max_warps = int64_t(num_sms) * 3 * (kPackThreads / 32);
   const int64_t rounds = (n_out + max_warps - 1) / max_warps;
   const int64_t warps = (n_out + rounds - 1) / rounds;
   const int64_t blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
