@@ -7,98 +7,130 @@
 // (magnitude mask from the masters, quantise then mask), Korean summary
 // §2.1-2.2 (per-step recompute), French summary §2.
 //
-// Three kernels:
-//   k_absmean_partials  streams W once, adds every |w| exactly into per-block
-//                       integer bins
-//   k_gamma_finalize    one block: folds the bins, rounds the exact mean once to
-//                       fp32, writes gamma, g and the header
-//   k_prep_pack<M>      re-reads W (from L2), masks, ternarises and writes every
-//                       packed section
-// The last two are launched with programmatic stream serialisation, so their
-// launches overlap the tail of the kernel before them.
+// One cooperative launch, one CTA per SM.  Each CTA owns a contiguous range
+// of W (in 16-byte vectors of eight weights) and streams it twice through a
+// ring of shared-memory stages filled by bulk copies (one producer warp,
+// sixteen consumer warps):
+//   phase 1  from HBM: every |w| is added exactly (below); W stays in L2;
+//   barrier  every CTA publishes its partial sum and waits for the others
+//            (bounded wait on per-CTA arrival words);
+//   phase 2  from L2: every CTA folds all partial sums and rounds the exact
+//            mean once to fp32 (so all CTAs hold the same g) while the first
+//            stages refill, then masks, ternarises and writes every packed
+//            section.
+// The kernel lets its successor (the activation quantiser, launched with
+// programmatic stream serialisation) start at once, so the two HBM streams
+// overlap.
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
 
 namespace sbl {
 
+constexpr int kPrepConsumers = 512;                    // 16 consumer warps
+constexpr int kPrepConsumerWarps = kPrepConsumers / 32;
+constexpr int kPrepThreads = kPrepConsumers + 32;      // + one producer warp
+constexpr int kVecsPerThread = 2;                      // 16-byte vectors per consumer per stage
+constexpr int kChunkVecs = kVecsPerThread * kPrepConsumers;  // 24 KB per stage
+constexpr int kPrepStages = 12;
+constexpr size_t kPrepTailBytes = 4096;
+constexpr size_t kSelBytes = 64 * 32 * 8;  // 64 entries x 32 lane copies x 8 bytes
+constexpr size_t kPrepSmem = size_t(kPrepStages) * kChunkVecs * 16 + kSelBytes + kPrepTailBytes;
+
 // ---------------------------------------------------------------------------
 // Exact sum of |w| (absmean numerator).
 //
-// In units of 2^-133 a bf16 magnitude (biased exponent e, mantissa f) is the
-// integer sig << s with sig = (e ? 128 + f : f) and s = max(e, 1) - 1 <= 253,
-// i.e. sig - s * 128 = mag - s * 128 with mag = e * 128 + f.  Each lane keeps
-// 32 private 32-bit bins in shared memory, bin b = s >> 3 collecting
-// sig << (s & 7) (< 2^15 per add).  A round lets each lane add at most 2^16
-// weights, so no bin overflows; after each round the block folds its lanes'
-// bins into 64-bit totals.  A slot bin b is an integer in units of 2^(8b-133).
+// Fast path, exact by construction: a bf16 magnitude field `mag` (biased
+// exponent e, 7-bit fraction f) shifted left by 13 is the high word of the
+// fp64 number |w| * 2^-896 (the fp64 exponent field takes e, the top fraction
+// bits take f).  For 2^-30 <= |w| < 2^6 every such number
+// is an integer multiple of 2^(-37-896) below 2^(6-896), so a sum of up to
+// 64 of them stays below 2^49 units and fp64 adds it without rounding.  After
+// each stage (16 weights per thread) a thread converts its fp64 sum (scaled by 2^933) to
+// an exact integer in units of 2^-37 and adds it to a 128-bit integer.
+//
+// Slow path, for any vector holding a weight outside that window (below
+// 2^-30, zero included, at or above 2^6, Inf or NaN): in units of 2^-133 the magnitude
+// is sig << s with sig = (e ? 128 + f : f) and s = max(e, 1) - 1 <= 253;
+// shared 64-bit bin b = s >> 3 collects sig << (s & 7).  Bin b is an integer
+// in units of 2^(8b - 133); the fast path's units 2^-37 are bin 12.
 // ---------------------------------------------------------------------------
-constexpr int kAbsThreads = 1024;
-constexpr int kAbsWarps = kAbsThreads / 32;
-constexpr int kLaneBins = 32;
-constexpr int64_t kRoundVecs = 8192;  // 16-byte vectors per thread per round (8 weights each)
+constexpr uint32_t kWinLo = 97u << 7;   // magnitude field of 2^-30
+constexpr uint32_t kWinSpan = 36u << 7;  // up to, not including, 2^6
+constexpr int kFastBin = 12;             // 8 * 12 - 133 = -37
+constexpr int kFastBinHi = 19;           // 2^56 units of bin 12
 
-__global__ void __launch_bounds__(kAbsThreads, 1)
-    k_absmean_partials(const uint4* __restrict__ w, int64_t nvec, uint64_t* __restrict__ slot_bins,
-                       uint32_t* __restrict__ slot_flags) {
-  extern __shared__ uint32_t lane_bins[];  // [warp][bin][lane]
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t* my = lane_bins + warp * (kLaneBins * 32) + lane;
+__device__ __forceinline__ double fp64_of_hi_word(uint32_t hi_word) {
+  return __hiloint2double(static_cast<int>(hi_word), 0);
+}
 
-  uint32_t emax = 0;
-  auto consume = [&](const uint4 v) {
-    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t mag = (words[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
-      const uint32_t e = mag >> 7;
-      emax = max(emax, e);
-      const uint32_t s = max(e, 1u) - 1u;
-      const uint32_t sig = mag - (s << 7);
-      my[(s >> 3) * 32] += sig << (s & 7u);
-    }
-  };
+__device__ __forceinline__ uint32_t bf16x2_max_nan(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_lt_mask(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.lt.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_ge_mask_(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 
-  const int64_t stride = int64_t(gridDim.x) * kAbsThreads;
-  const int64_t round = stride * kRoundVecs;
-  uint64_t total = 0;  // thread (bin = warp, part = lane) keeps the block total of its bin
-  for (int64_t r0 = 0; r0 < nvec; r0 += round) {
-#pragma unroll
-    for (int b = 0; b < kLaneBins; ++b) my[b * 32] = 0u;
-    const int64_t r1 = (nvec - r0 < round) ? nvec : r0 + round;
-    int64_t i = r0 + int64_t(blockIdx.x) * kAbsThreads + threadIdx.x;
-    // Four independent 16-byte loads in flight per thread (default caching:
-    // the pack kernel re-reads W right after this one).
-    for (; i + 3 * stride < r1; i += 4 * stride) {
-      const uint4 v0 = __ldg(w + i);
-      const uint4 v1 = __ldg(w + i + stride);
-      const uint4 v2 = __ldg(w + i + 2 * stride);
-      const uint4 v3 = __ldg(w + i + 3 * stride);
-      consume(v0);
-      consume(v1);
-      consume(v2);
-      consume(v3);
+// All eight magnitudes (four words of two, sign bits clear) inside the fast
+// window: the packed maximum (NaN propagating) below 2^6 and the packed
+// minimum at least 2^-30.  Zeros take the slow path too.
+__device__ __forceinline__ bool in_window(const uint32_t (&mw)[4]) {
+  const uint32_t mx = bf16x2_max_nan(bf16x2_max_nan(mw[0], mw[1]), bf16x2_max_nan(mw[2], mw[3]));
+  const uint32_t mn = bf16x2_min(bf16x2_min(mw[0], mw[1]), bf16x2_min(mw[2], mw[3]));
+  constexpr uint32_t kHi2 = (kWinLo + kWinSpan) | ((kWinLo + kWinSpan) << 16), kLo2 = kWinLo | (kWinLo << 16);
+  return (bf16x2_lt_mask(mx, kHi2) & bf16x2_ge_mask_(mn, kLo2)) == 0xFFFFFFFFu;
+}
+
+__device__ __noinline__ void add_slow(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3,
+                                      unsigned long long* s_bins, uint32_t* s_flags) {
+  const uint32_t mw[4] = {m0, m1, m2, m3};
+  uint32_t bad = 0;
+#pragma unroll 1
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t mag = (mw[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
+    const uint32_t e = mag >> 7;
+    if (e == 0xFFu) {
+      bad = 1u;
+      continue;
     }
-    for (; i < r1; i += stride) consume(__ldg(w + i));
-    __syncthreads();
-    // Warp `bin` folds bin `bin`: lane p sums the 32 lanes of warp p.
-    {
-      const int bin = warp, part = lane;
-      const uint32_t* src = lane_bins + part * (kLaneBins * 32) + bin * 32;
-      uint64_t sum = 0;
-#pragma unroll 8
-      for (int l = 0; l < 32; ++l) sum += src[(l + lane) & 31];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      total += sum;
-    }
-    __syncthreads();
+    const uint32_t s = max(e, 1u) - 1u;
+    const uint32_t sig = mag - (s << 7);
+    if (sig != 0u) atomicAdd(&s_bins[s >> 3], static_cast<unsigned long long>(sig << (s & 7u)));
   }
-  if (lane == 0) slot_bins[int64_t(blockIdx.x) * kExactBins + warp] = total;
-  if (threadIdx.x < kExactBins - kLaneBins) slot_bins[int64_t(blockIdx.x) * kExactBins + kLaneBins + threadIdx.x] = 0ull;
-  const int bad = __syncthreads_or(emax == 0xFFu);
-  if (threadIdx.x == 0) slot_flags[blockIdx.x] = bad ? SBL_STATUS_NONFINITE_W : 0u;
-  pdl_trigger();
+  atomicOr(s_flags, 2u | bad);  // bit 1: the bins are in use; bit 0: a non-finite weight
+}
+
+// Correct rounding without a division.  q approximates a positive value v
+// within 2^-51 relative.  If q is farther than that from the fp32 rounding
+// midpoint on its side of RN_fp32(q), then v lies on the same side and
+// RN_fp32(v) = RN_fp32(q).  Returns false when q is too close to decide (an
+// exact or near tie) or too small (the fp32 subnormal range is left to the
+// exact path).
+__device__ __forceinline__ bool round_fp32_if_clear(double q, float* out) {
+  if (!(q > 0x1p-120)) return false;
+  const float f = __double2float_rn(q);
+  const double fd = static_cast<double>(f);
+  const double nb = (q >= fd) ? static_cast<double>(nextafterf(f, 3.0e38f)) : static_cast<double>(nextafterf(f, 0.0f));
+  const double mid = 0.5 * (fd + nb);  // exact: both are fp32 values
+  if (fabs(q - mid) > q * 0x1p-48) {
+    *out = f;
+    return true;
+  }
+  return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -144,6 +176,12 @@ __device__ float exact_mean_fp32(const uint64_t* bins, uint64_t numel) {
     }
     return r;
   };
+  {
+    // division-free attempt: the top 64 bits of S (truncated) in fp64
+    float r;
+    const double ds = ldexp(static_cast<double>(get64(topS - 63)), topS - 63 - 133);
+    if (round_fp32_if_clear(ds / static_cast<double>(numel), &r)) return r;
+  }
   const int low = topS - 127;  // bit of S that lands at bit 0 of N
   const unsigned __int128 N = (static_cast<unsigned __int128>(get64(low + 64)) << 64) | get64(low);
   bool sticky0 = false;
@@ -171,92 +209,17 @@ __device__ float exact_mean_fp32(const uint64_t* bins, uint64_t numel) {
   return __uint_as_float((static_cast<uint32_t>(lsb + 149) << 23) + static_cast<uint32_t>(mant));
 }
 
-// ---------------------------------------------------------------------------
-// Fold the per-block partial sums, compute gamma and g, write the header.
-// One block.  It lets the pack kernel start launching right away (that kernel
-// waits for this one to complete before it reads g), then waits for the
-// partial sums.
-// ---------------------------------------------------------------------------
-constexpr int kFinGroups = 25;                       // slot groups
-constexpr int kFinThreads = kFinGroups * kExactBins;  // 1000 threads: (group, bin) pairs
 
-__global__ void __launch_bounds__(1024) k_gamma_finalize(const uint64_t* slot_bins, const uint32_t* slot_flags,
-                                                         int nslots, BlobHeader* h, int64_t n_out, int64_t k, int n,
-                                                         int m, uint32_t layer_flags) {
-  __shared__ uint64_t s_part[kFinGroups][kExactBins];
-  __shared__ uint64_t s_bins[kExactBins];
-  __shared__ uint32_t s_flags;
-  pdl_trigger();
-  pdl_wait();
-  const int tid = threadIdx.x;
-  if (tid == 0) s_flags = 0u;
-  if (tid < kFinThreads) {
-    // Group grp folds slots grp, grp + 25, ...: all its loads are issued before
-    // any add, so the fold costs one memory round trip.
-    const int bin = tid % kExactBins, grp = tid / kExactBins;
-    const int per = (nslots - grp + kFinGroups - 1) / kFinGroups;  // slots of this group
-    uint64_t v[8];
-    uint64_t a = 0;
-    for (int j0 = 0; j0 < per; j0 += 8) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int slot = grp + (j0 + j) * kFinGroups;
-        v[j] = (j0 + j < per) ? __ldcg(slot_bins + int64_t(slot) * kExactBins + bin) : 0ull;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) a += v[j];
-    }
-    s_part[grp][bin] = a;
+// gamma = RN_fp32(S * 2^-37 / numel) for a sum S held as a 128-bit integer
+// (hi, lo), from an fp64 quotient (one rounding of S, one of the division).
+__device__ bool mean_fp32_fast(uint64_t lo, uint64_t hi, uint64_t numel, float* out) {
+  const double s = __ull2double_rn(hi) * 0x1p64 + __ull2double_rn(lo);  // hi * 2^64 is exact
+  if (s == 0.0) {
+    *out = 0.0f;
+    return true;
   }
-  __syncthreads();
-  uint32_t f = 0;
-  for (int i = tid; i < nslots; i += blockDim.x) f |= __ldcg(slot_flags + i);
-  if (f) atomicOr(&s_flags, f);
-  if (tid < kExactBins) {
-    uint64_t t = 0;
-#pragma unroll 5
-    for (int g2 = 0; g2 < kFinGroups; ++g2) t += s_part[g2][tid];
-    s_bins[tid] = t;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t flags = s_flags;
-    const bool bad = (flags & SBL_STATUS_NONFINITE_W) != 0u;
-    const float gamma = bad ? __int_as_float(0x7fc00000) : exact_mean_fp32(s_bins, uint64_t(n_out) * uint64_t(k));
-    h->magic = kMagic;
-    h->version = 2;
-    h->n_out = n_out;
-    h->k = k;
-    h->n = n;
-    h->m = m;
-    h->flags = layer_flags;
-    h->gamma = gamma;
-    h->g = (gamma > 1e-5f) ? gamma : 1e-5f;  // a NaN gamma gives 1e-5; the status word says why
-    h->status = flags;                        // a new prepare resets the status word
-  }
+  return round_fp32_if_clear(__ddiv_rn(s, __ull2double_rn(numel)) * 0x1p-37, out);
 }
-
-// ---------------------------------------------------------------------------
-// Mask, ternarise, pack.  Lane = 8 consecutive weights of a row (one 16-byte
-// vector); a warp covers 256 consecutive weights, so every load and most
-// stores are contiguous across the warp.  k is a multiple of 64, so a row has
-// a multiple of 8 lanes' worth of weights and no group or quad of lanes
-// straddles two rows.
-//
-// Bit tricks (all exact):
-//  * code != 0  <=>  2|w| > g  <=>  |w| > g/2 (g/2 is exact)  <=>  the 15-bit
-//    magnitude field exceeds bits(g/2) >> 16, compared two at a time with
-//    __vcmpgtu2 on the packed bf16 pairs;
-//  * W_eff as bf16 is (sign | 0x3F80) masked by (kept & code != 0);
-//  * the int8 code byte of a bf16 W_eff value h is (h bit 13) | 0xFE * (h bit 15).
-// ---------------------------------------------------------------------------
-constexpr int kPackThreads = 256;
-constexpr int kPackDepth = 8;  // 16-byte loads in flight per lane
-
-// (i0 | i1 << 2) for each 4-bit kept pattern with exactly two bits set.
-constexpr uint64_t kPairNibble = (uint64_t(0x4) << (4 * 0x3)) | (uint64_t(0x8) << (4 * 0x5)) |
-                                 (uint64_t(0x9) << (4 * 0x6)) | (uint64_t(0xC) << (4 * 0x9)) |
-                                 (uint64_t(0xD) << (4 * 0xA)) | (uint64_t(0xE) << (4 * 0xC));
 
 // Keep-bits of one group of M magnitudes: position a is kept when fewer than
 // n positions beat it, where b beats a if |w_b| > |w_a|, or if they are equal
@@ -295,213 +258,562 @@ __device__ __forceinline__ uint32_t bf16x2_ge_mask(uint32_t a, uint32_t b) {
 }
 
 // The six outcomes c_ij = |w_i| >= |w_j| (i < j) of a group of four held as
-// two words of magnitudes (m0 | m1 << 16, m2 | m3 << 16), in the table-index
-// bit order c01, c02, c03, c12, c13, c23.
-__device__ __forceinline__ uint32_t pair_outcomes4_packed(uint32_t m01, uint32_t m23) {
+// two words of magnitudes (m0 | m1 << 16, m2 | m3 << 16), as a 6-bit table
+// index: bit 0 c01, bit 1 c02, bit 2 c03, bit 3 c23, bit 4 c13, bit 5 c12.
+// Each packed compare gives 0xFFFF per true half, so the low halves supply
+// bits 0-2 and the high halves bits 3-5 (taken from bits 19-21).
+__device__ __forceinline__ uint32_t outcomes4_index(uint32_t m01, uint32_t m23) {
   const uint32_t rA = bf16x2_ge_mask(__byte_perm(m01, m23, 0x5410), __byte_perm(m01, m23, 0x7632));  // c01 | c23
   const uint32_t rB = bf16x2_ge_mask(m01, m23);                                                       // c02 | c13
   const uint32_t rC = bf16x2_ge_mask(m01, __byte_perm(m23, m23, 0x1032));                             // c03 | c12
-  return (rA & 1u) | (rB & 2u) | (rC & 4u) | ((rC >> 13) & 8u) | ((rB >> 12) & 16u) | ((rA >> 11) & 32u);
+  const uint32_t u = (rA & 0x00080001u) | (rB & 0x00100002u) | (rC & 0x00200004u);
+  return (u >> 16) | (u & 7u);
 }
 
-// Groups of four: the six pairwise outcomes c_ij = (|w_i| >= |w_j|), i < j,
-// index a 64-entry table whose byte holds the keep pattern (bits 0..3) and,
-// for n == 2, the metadata nibble i0 | i1 << 2 (bits 4..7).
-__device__ __forceinline__ uint32_t select4_entry(uint32_t cbits, int n) {
-  const uint32_t c01 = cbits & 1u, c02 = (cbits >> 1) & 1u, c03 = (cbits >> 2) & 1u;
-  const uint32_t c12 = (cbits >> 3) & 1u, c13 = (cbits >> 4) & 1u, c23 = (cbits >> 5) & 1u;
-  const uint32_t r0 = 3u - c01 - c02 - c03;
+// Table entry for one outcome index (8 bytes, replicated per lane so that a
+// warp's random lookups never share a bank):
+//   x  the keep bit of position p in the sign bit of byte p (a byte permute
+//      with sign replication turns it into the 0xFFFF-per-kept-weight masks)
+//   y  bits 0-3 the kept pattern, bits 4-7 the 2:4 metadata nibble
+//      i0 | i1 << 2, bits 8-15 the byte-permute selector nibbles i0, i1 that
+//      pick the two kept high bytes (i0 < i1 are the first two kept positions)
+__device__ uint2 select4_entry(uint32_t idx, int n) {
+  const uint32_t c01 = idx & 1u, c02 = (idx >> 1) & 1u, c03 = (idx >> 2) & 1u;
+  const uint32_t c23 = (idx >> 3) & 1u, c13 = (idx >> 4) & 1u, c12 = (idx >> 5) & 1u;
+  const uint32_t r0 = 3u - c01 - c02 - c03;  // positions that beat position 0
   const uint32_t r1 = c01 + 2u - c12 - c13;
   const uint32_t r2 = c02 + c12 + 1u - c23;
   const uint32_t r3 = c03 + c13 + c23;
   const uint32_t kept = (r0 < uint32_t(n) ? 1u : 0u) | (r1 < uint32_t(n) ? 2u : 0u) | (r2 < uint32_t(n) ? 4u : 0u) |
                         (r3 < uint32_t(n) ? 8u : 0u);
-  const uint32_t nib = static_cast<uint32_t>(kPairNibble >> (4 * kept)) & 0xFu;
-  return kept | (nib << 4);
+  uint32_t i0 = 0, i1 = 0;
+  {
+    int found = 0;
+    for (uint32_t p = 0; p < 4; ++p)
+      if (kept & (1u << p)) {
+        if (found == 0) i0 = p;
+        else if (found == 1) i1 = p;
+        ++found;
+      }
+  }
+  const uint32_t x = ((kept & 1u) << 7) | ((kept & 2u) << 14) | ((kept & 4u) << 21) | ((kept & 8u) << 28);
+  const uint32_t y = kept | ((i0 | (i1 << 2)) << 4) | ((i0 | (i1 << 4)) << 8);
+  return make_uint2(x, y);
 }
 
-// int8 codes (+1 = 0x01, -1 = 0xFF, 0) of four bf16 W_eff values held in two
-// words: their high bytes are 0x3F, 0xBF or 0x00.
-__device__ __forceinline__ uint32_t code_bytes4(uint32_t weff_lo, uint32_t weff_hi) {
-  const uint32_t hb = __byte_perm(weff_lo, weff_hi, 0x7531);
-  return ((hb >> 5) & 0x01010101u) | (((hb >> 7) & 0x01010101u) * 0xFEu);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// int8 codes (+1 = 0x01, -1 = 0xFF, 0) of four W_eff values given by their
+// bf16 high bytes (0x3F, 0xBF or 0x00): the sign byte replicated, or bit 5.
+__device__ __forceinline__ uint32_t codes_of_high_bytes(uint32_t hb) {
+  // prmt with selector bit 3 set replicates the sign bit of the chosen byte
+  return prmt(hb, 0u, 0xBA98u) | ((hb >> 5) & 0x01010101u);
+}
+
+// ---------------------------------------------------------------------------
+// Grid barrier on the blob's scratch: a generation word `gen` and each CTA's
+// tagged partial-sum words.  Every CTA reads gen (= G) before it publishes,
+// tags its words with G + 1, and waits until all CTAs' words carry G + 1;
+// CTA 0 then stores G + 1 to gen (plain stores, so gen wraps like the tags).  Nothing needs initialising: a blob holds
+// the tag G + 1 in every word only by accident of its previous contents,
+// which a completed launch never leaves behind (it leaves tags equal to gen).
+// A wait that gives up raises the timeout bit and stores G + 2 to gen, so
+// stale words of that launch cannot satisfy the next one.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ ulonglong2 ld_relaxed_v2u64(const ulonglong2* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kPrepConsumers) : "memory"); }
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+struct PrepArgs {
+  const uint4* w;
+  int64_t n_out, k;
+  int n, m;
+  uint32_t layer_flags;
+  BlobHeader* h;
+  uint64_t* slot_fast;  // [grid][4]: tagged pieces of the 128-bit fast sum, tagged flags
+  uint64_t* slot_bins;  // [grid][kExactBins], written only when the slow path ran
+  uint64_t* gen;
+  PackOut out;
+};
+
+struct PrepTail {
+  uint64_t full[kPrepStages];
+  uint64_t empty[kPrepStages];
+  unsigned long long bins[kExactBins];
+  unsigned long long fold_bins[kExactBins];
+  uint64_t warp_lo[kPrepConsumerWarps], warp_hi[kPrepConsumerWarps];
+  uint64_t gen;
+  uint32_t flags;       // bit 0 non-finite, bit 1 slow bins in use (this CTA)
+  float g;
+  int abort_flag;
+};
+static_assert(sizeof(PrepTail) <= kPrepTailBytes, "prepare kernel's shared tail overflows its slot");
+
+// The exact path of the scale: add the 128-bit fast sum (L, H) to the folded
+// slow-path bins of all CTAs, then round the exact mean once.  Kept out of line: it runs only for ties, tiny means or
+// magnitudes outside the fast window.
+__device__ __noinline__ float gamma_exact(const unsigned long long* slow_bins, uint64_t L, uint64_t H, uint64_t numel) {
+  uint64_t bins[kExactBins];
+#pragma unroll
+  for (int b = 0; b < kExactBins; ++b) bins[b] = slow_bins[b];
+  bins[kFastBin] += L & ((1ull << 56) - 1ull);
+  bins[kFastBinHi] += (L >> 56) | (H << 8);
+  return exact_mean_fp32(bins, numel);
 }
 
 template <int M>
-__global__ void __launch_bounds__(kPackThreads)
-    k_prep_pack(const uint4* __restrict__ w, int64_t n_out, int64_t k, int n, const BlobHeader* h, PackOut out) {
-  // M == 4: per comparison outcome, the keep masks of the group's two words
-  // (0xFFFF per kept weight) and the byte keep pattern | nibble << 4.
-  __shared__ uint4 s_sel[64];
-  if (M == 4 && threadIdx.x < 64) {
-    const uint32_t e = select4_entry(threadIdx.x, n), kp = e & 0xFu;
-    const uint32_t km_lo = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
-    const uint32_t km_hi = (((kp >> 2) & 1u) | (((kp >> 2) & 2u) << 15)) * 0xFFFFu;
-    s_sel[threadIdx.x] = make_uint4(km_lo, km_hi, e, 0u);
+__global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint4* ring = reinterpret_cast<uint4*>(smem);
+  uint2* sel = reinterpret_cast<uint2*>(smem + size_t(kPrepStages) * kChunkVecs * 16);  // [64][32 lanes]
+  PrepTail* tail = reinterpret_cast<PrepTail*>(smem + size_t(kPrepStages) * kChunkVecs * 16 + kSelBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = static_cast<int>(gridDim.x), blk = static_cast<int>(blockIdx.x);
+  uint32_t* status = &a.h->status;
+  volatile int* abort_flag = &tail->abort_flag;
+  // The successor only reads its own inputs before it waits for this kernel.
+  pdl_trigger();
+
+  // This CTA's vectors [v0, v1): equal shares rounded to 32 vectors.
+  const int64_t nvec = a.n_out * a.k / 8;
+  const int64_t share = ((nvec + G - 1) / G + 31) / 32 * 32;
+  const int64_t v0 = share * blk < nvec ? share * blk : nvec;
+  const int64_t v1 = v0 + share < nvec ? v0 + share : nvec;
+  const int nch = static_cast<int>((v1 - v0 + kChunkVecs - 1) / kChunkVecs);
+
+  if (tid < kExactBins) {
+    tail->bins[tid] = 0ull;
+    tail->fold_bins[tid] = 0ull;
+  }
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kPrepStages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], kPrepConsumerWarps);
+    }
+    fence_mbar_init();
+    tail->gen = ld_relaxed_u64(a.gen);
+    tail->flags = 0u;
+    tail->abort_flag = 0;
+    if (blk == 0) *status = 0u;  // a new prepare resets the status word
+  }
+  if (M == 4) {
+    for (int i = tid; i < 64 * 32; i += kPrepThreads) sel[i] = select4_entry(static_cast<uint32_t>(i >> 5), a.n);
   }
   __syncthreads();
-  pdl_wait();  // g comes from k_gamma_finalize (a kernel that may overlap this one: coherent load)
-  const float g = __ldcg(&h->g);
+
+  if (warp == kPrepConsumerWarps) {
+    // ---- producer: phase 1 chunks from HBM, then phase 2 chunks from L2 (W
+    // does not depend on the scale, so refills need not wait for the barrier)
+    if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
+      for (int J = 0; J < 2 * nch; ++J) {
+        const int j = J < nch ? J : J - nch;
+        const int s = J % kPrepStages;
+        if (J >= kPrepStages && !mbar_wait(&tail->empty[s], ((J / kPrepStages) - 1) & 1, abort_flag, status)) break;
+        const int64_t c0 = v0 + int64_t(j) * kChunkVecs;
+        const int64_t cnt = (v1 - c0 < kChunkVecs) ? v1 - c0 : kChunkVecs;
+        const uint32_t bytes = static_cast<uint32_t>(cnt) * 16u;
+        mbar_arrive_expect_tx(&tail->full[s], bytes);
+        bulk_load_hint(ring + size_t(s) * kChunkVecs, a.w + c0, bytes, &tail->full[s], J < nch ? keep : drop);
+      }
+    }
+    return;
+  }
+
+  // ---- consumers, phase 1: exact sum of |w| ----
+  uint64_t lo = 0, hi = 0;
+  for (int j = 0; j < nch; ++j) {
+    const int s = j % kPrepStages;
+    if (!mbar_wait(&tail->full[s], (j / kPrepStages) & 1, abort_flag, status)) break;
+    const int64_t rem = v1 - v0 - int64_t(j) * kChunkVecs;
+    const int cnt = rem < kChunkVecs ? static_cast<int>(rem) : kChunkVecs;
+    const uint4* st = ring + size_t(s) * kChunkVecs;
+    double acc[kVecsPerThread];
+#pragma unroll
+    for (int h2 = 0; h2 < kVecsPerThread; ++h2) {
+      acc[h2] = 0.0;
+      const int e = tid + h2 * kPrepConsumers;
+      if (e < cnt) {
+        const uint4 v = st[e];
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t mw[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+        if (in_window(mw)) {
+          // the high words of |w| * 2^-896 in fp64, read straight off the bf16
+          // bits (the masks drop the sign and the neighbouring weight)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[h2] += fp64_of_hi_word((wd[q] << 13) & 0x0FFFE000u);
+            acc[h2] += fp64_of_hi_word((wd[q] >> 3) & 0x0FFFE000u);
+          }
+        } else {
+          add_slow(mw[0], mw[1], mw[2], mw[3], tail->bins, &tail->flags);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
+    double tot = acc[0];
+#pragma unroll
+    for (int h2 = 1; h2 < kVecsPerThread; ++h2) tot += acc[h2];
+    const uint64_t units = __double2ull_rn(tot * 0x1p933);  // exact: an integer below 2^48
+    lo += units;
+    hi += (lo < units) ? 1ull : 0ull;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t olo = __shfl_xor_sync(0xffffffffu, lo, off), ohi = __shfl_xor_sync(0xffffffffu, hi, off);
+    lo += olo;
+    hi += ohi + ((lo < olo) ? 1ull : 0ull);
+  }
+  if (lane == 0) {
+    tail->warp_lo[warp] = lo;
+    tail->warp_hi[warp] = hi;
+  }
+  consumers_sync();
+
+  // ---- grid barrier and fold in one (warp 0) ----
+  // Each CTA publishes its partial sum as four 64-bit words, each carrying
+  // the generation tag G + 1 in its upper half (a 64-bit store is seen whole
+  // or not at all): the 128-bit sum in three 32-bit pieces and the flags.
+  // Warp 0 of every CTA polls all CTAs' words until every tag reads G + 1,
+  // summing the pieces as it goes, so the wait and the fold cost one pass.
+  const uint64_t gen0 = tail->gen;
+  if (warp == 0) {
+    uint64_t L = lane < kPrepConsumerWarps ? tail->warp_lo[lane] : 0ull;
+    uint64_t H = lane < kPrepConsumerWarps ? tail->warp_hi[lane] : 0ull;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t olo = __shfl_xor_sync(0xffffffffu, L, off), ohi = __shfl_xor_sync(0xffffffffu, H, off);
+      L += olo;
+      H += ohi + ((L < olo) ? 1ull : 0ull);
+    }
+    const uint32_t fl_own = tail->flags;
+    if (fl_own & 2u) {  // slow bins in use: publish them first
+      for (int b = lane; b < kExactBins; b += 32) a.slot_bins[int64_t(blk) * kExactBins + b] = tail->bins[b];
+      __threadfence();
+    }
+    __syncwarp();
+    const uint32_t tagv = static_cast<uint32_t>(gen0 + 1);
+    const uint64_t tag = uint64_t(tagv) << 32;
+    if (lane == 0) {  // H < 2^32: a CTA holds at most 2^40 weights below 2^6, i.e. below 2^83 units
+      uint64_t* sf = a.slot_fast + int64_t(blk) * 4;
+      st_relaxed_u64(sf + 0, tag | (L & 0xFFFFFFFFull));
+      st_relaxed_u64(sf + 1, tag | (L >> 32));
+      st_relaxed_u64(sf + 2, tag | (H & 0xFFFFFFFFull));
+      st_release_u64(sf + 3, tag | fl_own);
+    }
+    uint64_t s0 = 0, s1 = 0, s2 = 0;
+    uint32_t fl = 0, slow_r = 0;  // slow_r: bit r set when CTA lane + 32 r used its slow bins
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+      bool all = true;
+      s0 = s1 = s2 = 0;
+      fl = slow_r = 0;
+      auto take = [&](int c, int r) {
+        const ulonglong2* sf = reinterpret_cast<const ulonglong2*>(a.slot_fast + int64_t(c) * 4);
+        const ulonglong2 p01 = ld_relaxed_v2u64(sf), p23 = ld_relaxed_v2u64(sf + 1);
+        all &= ((p01.x >> 32) == tagv) & ((p01.y >> 32) == tagv) & ((p23.x >> 32) == tagv) & ((p23.y >> 32) == tagv);
+        s0 += p01.x & 0xFFFFFFFFull;
+        s1 += p01.y & 0xFFFFFFFFull;
+        s2 += p23.x & 0xFFFFFFFFull;
+        fl |= static_cast<uint32_t>(p23.y);
+        if (r < 32 && (p23.y & 2u)) slow_r |= 1u << r;
+      };
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (lane + 32 * r < G) take(lane + 32 * r, r);
+      for (int c = lane + 256, r = 8; c < G; c += 32, ++r) take(c, r);
+      if (__all_sync(0xffffffffu, all)) break;
+      __nanosleep(128);
+      if ((it & 7u) == 7u) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+          if (lane == 0) {
+            raise_status(status, SBL_STATUS_TIMEOUT);
+            st_relaxed_u64(a.gen, gen0 + 2);
+          }
+          break;
+        }
+      }
+    }
+    __threadfence();  // acquire: the slow bins behind the tags are visible from here on
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      fl |= __shfl_xor_sync(0xffffffffu, fl, off);
+    }
+    if (fl & 2u) {  // rare: fold the slow bins of the CTAs that used them, lanes over bins
+      for (int r = 0; 32 * r < G && r < 32; ++r) {
+        uint32_t slow = __ballot_sync(0xffffffffu, (slow_r >> r) & 1u);
+        while (slow) {
+          const int c = 32 * r + __ffs(slow) - 1;
+          slow &= slow - 1u;
+          const unsigned long long* src = reinterpret_cast<const unsigned long long*>(a.slot_bins + int64_t(c) * kExactBins);
+          const unsigned long long v0 = __ldcg(src + lane);
+          const unsigned long long v1 = (lane + 32 < kExactBins) ? __ldcg(src + lane + 32) : 0ull;
+          if (v0) atomicAdd(&tail->fold_bins[lane], v0);
+          if (v1) atomicAdd(&tail->fold_bins[lane + 32], v1);
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      if (blk == 0) st_relaxed_u64(a.gen, gen0 + 1);
+      // the 128-bit total: s0 + s1 * 2^32 + s2 * 2^64 (each below 2^42)
+      const uint64_t t1 = s1 << 32;
+      const uint64_t Lt = s0 + t1;
+      const uint64_t Ht = s2 + (s1 >> 32) + ((Lt < t1) ? 1ull : 0ull);
+      const uint64_t numel = uint64_t(a.n_out) * uint64_t(a.k);
+      float gamma;
+      if (fl & 1u) {
+        gamma = __int_as_float(0x7fc00000);
+      } else if ((fl & 2u) || !mean_fp32_fast(Lt, Ht, numel, &gamma)) {
+        gamma = gamma_exact(tail->fold_bins, Lt, Ht, numel);
+      }
+      const float g = (gamma > 1e-5f) ? gamma : 1e-5f;  // a NaN gamma gives 1e-5; the status word says why
+      tail->g = g;
+      if (blk == 0) {
+        BlobHeader* h = a.h;
+        h->magic = kMagic;
+        h->version = 3;
+        h->n_out = a.n_out;
+        h->k = a.k;
+        h->n = a.n;
+        h->m = a.m;
+        h->flags = a.layer_flags;
+        h->gamma = gamma;
+        h->g = g;
+        if (fl & 1u) raise_status(status, SBL_STATUS_NONFINITE_W);
+      }
+    }
+  }
+  consumers_sync();
+  const float g = tail->g;
   // code != 0 <=> 2|w| > g <=> |w| > g/2 (exact) <=> the 15-bit magnitude
   // exceeds bits(g/2) >> 16, i.e. |w| > that bf16 value as a float compare.
   const uint32_t thr = __float_as_uint(__fmul_rn(g, 0.5f)) >> 16;
   const uint32_t thr2 = thr | (thr << 16);
-  pdl_trigger();
 
-  const int lane = threadIdx.x & 31;
-  const int upr = static_cast<int>(k / 8);  // lanes' worth of weights per row (multiple of 8)
-  const int64_t gwarp = int64_t(blockIdx.x) * (kPackThreads / 32) + (threadIdx.x >> 5);
-  const int64_t nwarps = int64_t(gridDim.x) * (kPackThreads / 32);
-  for (int64_t row = gwarp; row < n_out; row += nwarps) {
-    const uint4* wrow = w + row * upr;
-    uint4* weff_row = reinterpret_cast<uint4*>(out.weff_bf16) + row * upr;
-    // kPackDepth 16-byte loads in flight per lane, then process them one by one.
-    for (int c0 = 0; c0 < upr; c0 += kPackDepth * 32) {
-      uint4 vbuf[kPackDepth];
+  // ---- consumers, phase 2: mask, ternarise, pack ----
+  const int n = a.n;
+  const int upr = static_cast<int>(a.k / 8);  // vectors per row (multiple of 8)
+  // (row, column-vector) of this thread's vectors in the current chunk
+  int64_t row[kVecsPerThread];
+  int col[kVecsPerThread];
 #pragma unroll
-      for (int q = 0; q < kPackDepth; ++q) {
-        const int cq = c0 + 32 * q + lane;
-        vbuf[q] = (cq < upr) ? __ldcs(wrow + cq) : make_uint4(0, 0, 0, 0);
+  for (int h2 = 0; h2 < kVecsPerThread; ++h2) {
+    const int64_t i = v0 + tid + h2 * kPrepConsumers;
+    row[h2] = i / upr;
+    col[h2] = static_cast<int>(i - row[h2] * upr);
+  }
+  const int64_t meta_rb_bytes = int64_t(a.out.meta_kblocks) * 2048;  // one 128-row block of metadata
+  const int step_rows = kChunkVecs / upr, step_cols = kChunkVecs % upr;  // one chunk, in (rows, vectors)
+  for (int j = 0; j < nch; ++j) {
+    const int J = nch + j, s = J % kPrepStages;
+    if (!mbar_wait(&tail->full[s], (J / kPrepStages) & 1, abort_flag, status)) break;
+    const uint4* st = ring + size_t(s) * kChunkVecs;
+#pragma unroll
+    for (int h2 = 0; h2 < kVecsPerThread; ++h2) {
+      const int e = tid + h2 * kPrepConsumers;
+      const int64_t i = v0 + int64_t(j) * kChunkVecs + e;
+      const bool active = i < v1;  // quads of lanes are all-or-nothing (v1 - v0 and upr are multiples of 8)
+      const uint4 vv = active ? st[e] : make_uint4(0, 0, 0, 0);
+      const uint32_t wd[4] = {vv.x, vv.y, vv.z, vv.w};
+      uint32_t mw[4];  // magnitudes, two per word
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mw[q] = wd[q] & 0x7FFF7FFFu;
+      uint32_t km[4];  // 0xFFFF per kept weight
+      // Z: bits 0-3 / 8-11 kept pattern of group 0 / 1 (the mask section's
+      // u16), bits 16-19 / 20-23 their 2:4 metadata nibbles; W: byte-permute
+      // selector of the four kept high bytes.
+      uint32_t Z = 0, W = 0;
+      if (M == 4) {
+        const uint2 e0 = sel[outcomes4_index(mw[0], mw[1]) * 32 + lane];
+        const uint2 e1 = sel[outcomes4_index(mw[2], mw[3]) * 32 + lane];
+        km[0] = prmt(e0.x, 0u, 0x9988u);
+        km[1] = prmt(e0.x, 0u, 0xBBAAu);
+        km[2] = prmt(e1.x, 0u, 0x9988u);
+        km[3] = prmt(e1.x, 0u, 0xBBAAu);
+        Z = (e0.y & 0x0Fu) | ((e1.y & 0x0Fu) << 8) | ((e0.y & 0xF0u) << 12) | ((e1.y & 0xF0u) << 16);
+        W = ((e0.y >> 8) & 0xFFu) | ((((e1.y >> 8) & 0xFFu) + 0x44u) << 8);
+      } else {
+        uint32_t mag[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          mag[2 * q] = mw[q] & 0xFFFFu;
+          mag[2 * q + 1] = mw[q] >> 16;
+        }
+        uint32_t kept = 0;
+#pragma unroll
+        for (int gi = 0; gi < 8 / M; ++gi) kept |= keep_bits<M>(mag, gi * M, n) << (gi * M);
+        Z = kept;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t kp = (kept >> (2 * q)) & 3u;
+          km[q] = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
+        }
       }
+
+      // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and
+      // code != 0 (code != 0 <=> |w| > g/2, a packed bf16 compare).
+      uint32_t weff[4];
 #pragma unroll
-      for (int q = 0; q < kPackDepth; ++q) {
-        if (c0 + 32 * q >= upr) break;  // uniform across the warp
-        const int c = c0 + 32 * q + lane;
-        const bool active = c < upr;  // upr is a multiple of 8: quads are all-or-nothing
-        const uint32_t wd[4] = {vbuf[q].x, vbuf[q].y, vbuf[q].z, vbuf[q].w};
-        uint32_t mw[4];  // magnitudes, two per word
-#pragma unroll
-        for (int j = 0; j < 4; ++j) mw[j] = wd[j] & 0x7FFF7FFFu;
-        uint32_t kept = 0, sel0 = 0, sel1 = 0;
-        uint32_t km[4];  // 0xFFFF per kept weight
-        if (M == 4) {
-          const uint4 e0 = s_sel[pair_outcomes4_packed(mw[0], mw[1])];
-          const uint4 e1 = s_sel[pair_outcomes4_packed(mw[2], mw[3])];
-          km[0] = e0.x;
-          km[1] = e0.y;
-          km[2] = e1.x;
-          km[3] = e1.y;
-          sel0 = e0.z;
-          sel1 = e1.z;
-          kept = (sel0 & 0xFu) | ((sel1 & 0xFu) << 4);
+      for (int q = 0; q < 4; ++q) weff[q] = ((wd[q] | 0x3F803F80u) & 0xBF80BF80u) & bf16x2_gt_mask(mw[q], thr2) & km[q];
+      const uint32_t hb_lo = __byte_perm(weff[0], weff[1], 0x7531);  // high bytes of weights 0..3
+      const uint32_t hb_hi = __byte_perm(weff[2], weff[3], 0x7531);  // weights 4..7
+
+      // Every section except the tensor-core metadata is laid out in the
+      // order of the 16-byte weight vectors, so vector i writes at index i.
+      if (active) {
+        if (M == 2) {
+          const uint32_t kept = Z;
+          reinterpret_cast<uint32_t*>(a.out.mask)[i] =
+              (kept & 3u) | (((kept >> 2) & 3u) << 8) | (((kept >> 4) & 3u) << 16) | (((kept >> 6) & 3u) << 24);
+        } else if (M == 4) {
+          reinterpret_cast<uint16_t*>(a.out.mask)[i] = static_cast<uint16_t>(Z);
         } else {
-          uint32_t mag[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            mag[2 * j] = mw[j] & 0xFFFFu;
-            mag[2 * j + 1] = mw[j] >> 16;
-          }
-#pragma unroll
-          for (int gi = 0; gi < 8 / M; ++gi) kept |= keep_bits<M>(mag, gi * M, n) << (gi * M);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t kp = (kept >> (2 * j)) & 3u;
-            km[j] = ((kp & 1u) | ((kp & 2u) << 15)) * 0xFFFFu;
-          }
+          a.out.mask[i] = static_cast<uint8_t>(Z);
         }
-
-        // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and code != 0.
-        uint32_t weff[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t nz = bf16x2_gt_mask(mw[j], thr2);
-          weff[j] = ((wd[j] & 0x80008000u) | 0x3F803F80u) & nz & km[j];
-        }
-        const uint32_t codes_lo = code_bytes4(weff[0], weff[1]);  // weights 0..3
-        const uint32_t codes_hi = code_bytes4(weff[2], weff[3]);  // weights 4..7
-
+        reinterpret_cast<uint4*>(a.out.weff_bf16)[i] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
+        if (a.out.codes != nullptr)
+          reinterpret_cast<uint2*>(a.out.codes)[i] = make_uint2(codes_of_high_bytes(hb_lo), codes_of_high_bytes(hb_hi));
+      }
+      if (M == 4 && a.out.sp_values != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
+        const uint32_t vals = codes_of_high_bytes(__byte_perm(hb_lo, hb_hi, W));  // the kept codes, index order
+        // tensor-core metadata: [row_block][k_block][128 rows][16 bytes]; this
+        // lane's byte is byte (col % 16) of the row's 16 bytes in k block col / 16.
+        uint32_t word = (Z >> 16) << (8 * (lane & 3));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
         if (active) {
-          if (M == 2) {
-            const uint32_t mw = (kept & 3u) | (((kept >> 2) & 3u) << 8) | (((kept >> 4) & 3u) << 16) |
-                                (((kept >> 6) & 3u) << 24);
-            reinterpret_cast<uint32_t*>(out.mask + row * (k / 2))[c] = mw;
-          } else if (M == 4) {
-            const uint32_t mw = (kept & 0xFu) | (((kept >> 4) & 0xFu) << 8);
-            reinterpret_cast<uint16_t*>(out.mask + row * (k / 4))[c] = static_cast<uint16_t>(mw);
-          } else {
-            out.mask[row * (k / 8) + c] = static_cast<uint8_t>(kept);
+          reinterpret_cast<uint32_t*>(a.out.sp_values)[i] = vals;
+          if ((lane & 3) == 0) {
+            const int64_t r = row[h2];
+            const int c = col[h2];
+            *reinterpret_cast<uint32_t*>(a.out.sp_meta + (r >> 7) * meta_rb_bytes + (r & 127) * 16 + (c >> 4) * 2048 +
+                                         (c & 15)) = word;
           }
-          weff_row[c] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
-          if (out.codes != nullptr) reinterpret_cast<uint2*>(out.codes + row * k)[c] = make_uint2(codes_lo, codes_hi);
-        }
-        if (M == 4 && out.sp_values != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
-          const uint32_t nib0 = sel0 >> 4, nib1 = sel1 >> 4;
-          // the two kept codes of each group, in index order
-          const uint32_t v0 = __byte_perm(codes_lo, 0u, (nib0 & 3u) | ((nib0 >> 2) << 4));
-          const uint32_t v1 = __byte_perm(codes_hi, 0u, (nib1 & 3u) | ((nib1 >> 2) << 4));
-          const uint32_t vals = (v0 & 0xFFFFu) | (v1 << 16);
-          const uint32_t meta = nib0 | (nib1 << 4);
-          // tensor-core metadata: [row_block][k_block][128 rows][16 bytes]; this
-          // lane's byte is byte (c % 16) of the row's 16 bytes in k block c / 16.
-          uint32_t word = meta << (8 * (lane & 3));
-          word |= __shfl_xor_sync(0xffffffffu, word, 1);
-          word |= __shfl_xor_sync(0xffffffffu, word, 2);
-          if (active) {
-            reinterpret_cast<uint32_t*>(out.sp_values + row * (k / 2))[c] = vals;
-            if ((lane & 3) == 0) {
-              uint8_t* mrow = out.sp_meta + ((row >> 7) * out.meta_kblocks * 128 + (row & 127)) * 16;
-              *reinterpret_cast<uint32_t*>(mrow + (c >> 4) * 2048 + (c & 15)) = word;
-            }
-            if (out.gemv != nullptr) {
-              const uint32_t g0 = (nib0 << 4) | (v0 & 3u) | (((v0 >> 8) & 3u) << 2);
-              const uint32_t g1 = (nib1 << 4) | (v1 & 3u) | (((v1 >> 8) & 3u) << 2);
-              reinterpret_cast<uint16_t*>(out.gemv + row * (k / 4))[c] = static_cast<uint16_t>(g0 | (g1 << 8));
-            }
+          if (a.out.gemv != nullptr) {
+            // per group: the two kept 2-bit codes (01 = +1, 11 = -1) low, the metadata nibble high
+            uint32_t t = vals & 0x03030303u;
+            t |= t >> 6;
+            const uint32_t nibs = ((Z >> 12) & 0xF0u) | ((Z >> 8) & 0xF000u);
+            reinterpret_cast<uint16_t*>(a.out.gemv)[i] = static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
           }
         }
+      }
+      row[h2] += step_rows;
+      col[h2] += step_cols;
+      if (col[h2] >= upr) {
+        col[h2] -= upr;
+        ++row[h2];
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
   }
 }
 
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
+template <int M>
+static cudaError_t launch_prepare_m(const cudaLaunchConfig_t& cfg, const PrepArgs& a) {
+  static const cudaError_t attr_err =
+      cudaFuncSetAttribute(k_prepare<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kPrepSmem));
+  if (attr_err != cudaSuccess) return attr_err;
+  return cudaLaunchKernelEx(&cfg, k_prepare<M>, a);
+}
+
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
                            uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s) {
-  BlobHeader* h = reinterpret_cast<BlobHeader*>(blob + L.header);
-  uint64_t* slot_bins = reinterpret_cast<uint64_t*>(blob + L.scratch);
-  uint32_t* slot_flags = reinterpret_cast<uint32_t*>(blob + L.scratch + uint64_t(kPrepSlots) * kExactBins * 8);
   if (L.sp_meta && (n_out % 256 != 0 || k % 256 != 0)) {
     cudaError_t e = cudaMemsetAsync(blob + L.sp_meta, 0x44, L.sp_meta_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  const int64_t nvec = n_out * k / 8;
-  int slots = num_sms < kPrepSlots ? num_sms : kPrepSlots;
-  const int64_t need = (nvec + kAbsThreads - 1) / kAbsThreads;
-  if (need < slots) slots = static_cast<int>(need);
-  constexpr int abs_smem = kAbsWarps * kLaneBins * 32 * 4;  // 128 KB of lane bins
-  static const cudaError_t attr_err =
-      cudaFuncSetAttribute(k_absmean_partials, cudaFuncAttributeMaxDynamicSharedMemorySize, abs_smem);
-  if (attr_err != cudaSuccess) return attr_err;
-  k_absmean_partials<<<slots, kAbsThreads, abs_smem, s>>>(reinterpret_cast<const uint4*>(w), nvec, slot_bins,
-                                                          slot_flags);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  PrepArgs a;
+  a.w = reinterpret_cast<const uint4*>(w);
+  a.n_out = n_out;
+  a.k = k;
+  a.n = n;
+  a.m = m;
+  a.layer_flags = flags;
+  a.h = reinterpret_cast<BlobHeader*>(blob + L.header);
+  a.slot_fast = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchSlotFast);
+  a.slot_bins = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchSlotBins);
+  a.gen = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchGen);
+  a.out.mask = blob + L.mask;
+  a.out.codes = L.codes ? reinterpret_cast<int8_t*>(blob + L.codes) : nullptr;
+  a.out.weff_bf16 = reinterpret_cast<uint16_t*>(blob + L.weff_bf16);
+  a.out.sp_values = L.sp_values ? reinterpret_cast<int8_t*>(blob + L.sp_values) : nullptr;
+  a.out.sp_meta = L.sp_meta ? blob + L.sp_meta : nullptr;
+  a.out.gemv = L.gemv ? blob + L.gemv : nullptr;
+  a.out.meta_kblocks = static_cast<int>(meta_k_padded(k) / 128);
 
-  PackOut out;
-  out.mask = blob + L.mask;
-  out.codes = L.codes ? reinterpret_cast<int8_t*>(blob + L.codes) : nullptr;
-  out.weff_bf16 = reinterpret_cast<uint16_t*>(blob + L.weff_bf16);
-  out.sp_values = L.sp_values ? reinterpret_cast<int8_t*>(blob + L.sp_values) : nullptr;
-  out.sp_meta = L.sp_meta ? blob + L.sp_meta : nullptr;
-  out.gemv = L.gemv ? blob + L.gemv : nullptr;
-  out.meta_kblocks = static_cast<int>(meta_k_padded(k) / 128);
-  e = launch_pdl(k_gamma_finalize, dim3(1), dim3(kFinThreads), 0, s, slot_bins, slot_flags, slots, h, n_out, k, n, m, flags);
-  if (e != cudaSuccess) return e;
-  // Rows are spread over warps; pick the warp count so every warp gets the
-  // same number of rows (within one) and the grid stays within three blocks/SM.
-  const int64_t max_warps = int64_t(num_sms) * 3 * (kPackThreads / 32);
-  const int64_t rounds = (n_out + max_warps - 1) / max_warps;
-  const int64_t warps = (n_out + rounds - 1) / rounds;
-  const int64_t blocks = (warps + kPackThreads / 32 - 1) / (kPackThreads / 32);
-  const dim3 grid(static_cast<unsigned>(blocks)), block(kPackThreads);
-  const uint4* wv = reinterpret_cast<const uint4*>(w);
-  const BlobHeader* hc = h;
+  // One CTA per SM (fewer for small matrices: at least one 16 KB stage of
+  // weights per CTA), all resident at once for the grid barrier.
+  const int64_t nvec = n_out * k / 8;
+  int64_t grid = (nvec + kChunkVecs - 1) / kChunkVecs;
+  if (grid > num_sms) grid = num_sms;
+  if (grid > kPrepSlots) grid = kPrepSlots;
+  if (grid < 1) grid = 1;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kPrepThreads);
+  cfg.dynamicSmemBytes = kPrepSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   switch (m) {
-    case 2: return launch_pdl(k_prep_pack<2>, grid, block, 0, s, wv, n_out, k, n, hc, out);
-    case 4: return launch_pdl(k_prep_pack<4>, grid, block, 0, s, wv, n_out, k, n, hc, out);
-    default: return launch_pdl(k_prep_pack<8>, grid, block, 0, s, wv, n_out, k, n, hc, out);
+    case 2: return launch_prepare_m<2>(cfg, a);
+    case 4: return launch_prepare_m<4>(cfg, a);
+    default: return launch_prepare_m<8>(cfg, a);
   }
 }
 

@@ -21,12 +21,17 @@ struct BlobHeader {
 };
 static_assert(sizeof(BlobHeader) <= 4096, "header must fit its 4 KB slot");
 
-// Per-block partial sums of the exact absmean: the first prepare kernel writes
-// one slot per block, the second folds them.  Bin b of a slot is an integer in
-// units of 2^(8b - 133); the exact sum of |w| is sum_b bin[b] * 2^(8b - 133).
+// Scratch of the prepare kernel inside the blob: per-CTA partial sums of the
+// exact absmean (a 128-bit sum in units of 2^-37 and a flags word, as four
+// generation-tagged words, and, when a CTA met magnitudes outside that
+// format, 40 bins where bin b is an integer in units of 2^(8b - 133)), and
+// the grid barrier's generation word.
 constexpr int kPrepSlots = 1024;
 constexpr int kExactBins = 40;
-constexpr uint64_t kScratchBytes = uint64_t(kPrepSlots) * kExactBins * 8 + uint64_t(kPrepSlots) * 4;
+constexpr uint64_t kScratchSlotBins = 0;
+constexpr uint64_t kScratchSlotFast = kScratchSlotBins + uint64_t(kPrepSlots) * kExactBins * 8;
+constexpr uint64_t kScratchGen = kScratchSlotFast + uint64_t(kPrepSlots) * 32;
+constexpr uint64_t kScratchBytes = kScratchGen + 256;
 
 constexpr uint32_t kMagic = 0x314C4253u;  // "SBL1"
 constexpr uint64_t kHeaderBytes = 4096;

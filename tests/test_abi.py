@@ -52,7 +52,7 @@ def test_layout_sections_are_aligned_and_disjoint(lib):
     for (n_out, k, n, m, flags) in [(6912, 2560, 2, 4, 0), (2560, 6912, 6, 8, 0), (264, 320, 2, 4, sbl.SBL_PACK_GEMV),
                                     (8, 64, 1, 2, 0)]:
         L = sbl.prepared_layout(n_out, k, n, m, flags)
-        spans = [("header", L.header, 4096), ("scratch", L.scratch, 1024 * 32 * 8 + 1024 * 4), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
+        spans = [("header", L.header, 4096), ("scratch", L.scratch, 1024 * 40 * 8 + 1024 * 32 + 256), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
         if (n, m) == (2, 4):
             spans += [("sp_values", L.sp_values, n_out * k // 2), ("sp_meta", L.sp_meta, L.sp_meta_bytes)]
             assert L.sp_meta_bytes == ((n_out + 255) // 256 * 256) * ((k + 255) // 256 * 256) // 8

@@ -248,6 +248,27 @@ def test_gamma_and_codes_at_extreme_magnitudes(kind):
     _check_prepared(layer, w, n, m)
 
 
+@pytest.mark.parametrize("fill", ["random", "ones", "zeros"])
+def test_prepare_on_uninitialised_blob_and_repeats(fill):
+    """The prepare kernel's grid barrier keeps its state in the blob's scratch
+    and needs no initialisation: a blob holding arbitrary bytes prepares
+    correctly, and so does every later prepare of the same blob."""
+    n_out, k, n, m = 520, 1024, 2, 4
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    if fill == "random":
+        gen = torch.Generator().manual_seed(11)
+        layer.blob.copy_(torch.randint(0, 256, layer.blob.shape, dtype=torch.uint8, generator=gen))
+    elif fill == "ones":
+        layer.blob.fill_(0xFF)
+    else:
+        layer.blob.zero_()
+    for rep in range(3):
+        w = synth.master_weights(n_out, k, 100 + rep)
+        sbl.prepare_weights(layer, _dev(w))
+        torch.cuda.synchronize()
+        _check_prepared(layer, w, n, m)
+
+
 @pytest.mark.parametrize("k", [64, 1088, 2560, 4160, 6912, 12352, 16384, 16448])
 def test_act_quant_row_lengths(k):
     """Activation codes and scales for row lengths that exercise every
