@@ -8,10 +8,10 @@
 // block reduces the absmax, then every thread quantises what it holds.  Rows
 // longer than 128 * 8 * kMaxR elements take a two-pass, warp-per-row kernel.
 //
-// The kernel reads only x and writes only its own outputs, so it is launched
-// with programmatic stream serialisation: right after a weight prepare it
-// runs alongside the pack kernel.  It waits for its predecessor before it
-// touches the status word it shares with the prepare and before it exits.
+// Launched with programmatic stream serialisation: its launch overlaps the
+// kernel before it, and it waits for that kernel (which may have written x,
+// or reset the status word) before it reads anything.  With early_trigger it
+// then lets the next kernel (the decode GEMV) launch at once.
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
@@ -26,10 +26,13 @@ template <int R>
 __global__ void __launch_bounds__(kActThreads)
     k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
                      float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
-  if (early_trigger) {
-    pdl_wait();
-    pdl_trigger();
-  }
+  // x may be the output of the kernel before this one: bring this block's
+  // rows towards L2 while that kernel runs, then wait for it.
+  if (threadIdx.x == 0)
+    for (int64_t row = blockIdx.x; row < t; row += gridDim.x)
+      bulk_prefetch_l2(x + row * nvec, static_cast<uint32_t>(nvec * 16));
+  pdl_wait();
+  if (early_trigger) pdl_trigger();
   __shared__ float s_max[kActThreads / 32];
   __shared__ uint32_t s_bad[kActThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -66,10 +69,7 @@ __global__ void __launch_bounds__(kActThreads)
     const float ap = fmaxf(amax, 1e-5f);
     if (tid == 0) {
       a_prime[row] = ap;
-      if (bad) {
-        pdl_wait();  // a prepare before this kernel resets the status word
-        raise_status(status, SBL_STATUS_NONFINITE_X);
-      }
+      if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
     uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
 #pragma unroll
@@ -78,7 +78,6 @@ __global__ void __launch_bounds__(kActThreads)
       if (i < nvec) dst[i] = quantise8(v[r], ap);
     }
   }
-  pdl_wait();
 }
 
 // Long rows: one warp per row, absmax pass then a second (L1/L2) pass.
@@ -87,10 +86,8 @@ constexpr int kActWarps = 8;
 __global__ void __launch_bounds__(kActWarps * 32)
     k_act_quant_long(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
                      float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
-  if (early_trigger) {
-    pdl_wait();
-    pdl_trigger();
-  }
+  pdl_wait();  // x may be the output of the kernel before this one
+  if (early_trigger) pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int64_t row = int64_t(blockIdx.x) * kActWarps + warp; row < t; row += int64_t(gridDim.x) * kActWarps) {
     const uint4* src = x + row * nvec;
@@ -107,16 +104,12 @@ __global__ void __launch_bounds__(kActWarps * 32)
     for (; i < nvec; i += 32) scan8(__ldg(src + i), amax, bad);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) {
-      pdl_wait();  // a prepare before this kernel resets the status word
-      raise_status(status, SBL_STATUS_NONFINITE_X);
-    }
+    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) raise_status(status, SBL_STATUS_NONFINITE_X);
     const float ap = fmaxf(amax, 1e-5f);
     if (lane == 0) a_prime[row] = ap;
     uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
     for (int64_t j = lane; j < nvec; j += 32) dst[j] = quantise8(__ldg(src + j), ap);
   }
-  pdl_wait();
 }
 
 template <int R>

@@ -4,14 +4,17 @@
 // The weight stream is the whole cost at these token counts: 2 bits per
 // weight (one byte per group of four: the metadata nibble i0 | i1 << 2 in the
 // high half, the two kept codes in the low half, 01 = +1, 11 = -1).  Each
-// block owns a contiguous range of output rows; eight threads share a row and
-// each loads its 16-byte pieces of the row before anything else, so the
-// block's whole share of the weights is in flight from the start.  While those
-// loads land, the block quantises the t activation rows into shared memory
-// (the same arithmetic as the act-quant kernel; block 0 also writes them out
-// when the caller asked for them).  A group byte then expands through a
-// 256-entry table into its four int8 weights and dp4a multiplies them with
-// four activation codes of each token.
+// block owns a contiguous range of output rows.  Calls are launched with
+// programmatic dependent launch: a call starts while the kernel before it
+// still runs, prefetches its block's weight rows (and x) into L2 with one bulk
+// prefetch, lets the next call launch, and only then waits for its
+// predecessor, so in a chain of decode calls each weight stream overlaps the
+// call before it.  After the wait eight threads per row load the row's 16-byte
+// pieces (L2 hits), the block quantises the t activation rows into shared
+// memory (the same arithmetic as the act-quant kernel; block 0 also writes them
+// out when the caller asked for them), and a group byte expands through a
+// 256-entry table into its four int8 weights that dp4a multiplies with four
+// activation codes of each token.
 #include <mutex>
 
 #include "sbl_kernels.h"
@@ -58,13 +61,37 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
   uint32_t* xw = smem_w + kLutWords + 32;    // [TP][k/4] int8 codes as words
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kw = a.k / 4;                    // code words per token row
-  const int pieces = a.k / 64;               // 16-byte weight pieces per row
 
-  // Rows of this block, and the first batch of weight pieces (issued first).
+  // Rows of this block.  The kernel before this one in the stream may still
+  // be writing this call's inputs (a prepare writes the weights, the previous
+  // layer writes x), so they are only prefetched into L2 before the wait and
+  // read after it; the next call may launch at once and do the same, so the
+  // weight streams of consecutive calls overlap.
   const int rpb = (a.n_out + gridDim.x - 1) / gridDim.x;
   const int row_begin = blockIdx.x * rpb;
   const int row_end = min(a.n_out, row_begin + rpb);
   const int slot = tid / kRowThreads, sub = tid % kRowThreads;
+  const int pieces = a.k / 64;  // 16-byte weight pieces per row
+  if (tid == 0 && row_end > row_begin)
+    bulk_prefetch_l2(a.gemv + int64_t(row_begin) * pieces, static_cast<uint32_t>(row_end - row_begin) * pieces * 16u);
+  if (tid == 32 && blockIdx.x == 0) {
+    if (PREQUANT) bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
+    else bulk_prefetch_l2(a.x, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k) * 2u);
+  }
+  pdl_trigger();
+  // Expansion table: group byte -> four int8 weights, replicated so that
+  // lane l always reads bank l (the bytes a warp looks up are random).
+  {
+    const int i = tid >> 1, half = tid & 1;  // 256 entries x 2 threads, 16 copies each
+    const int c0 = (i & 1) ? ((i & 2) ? -1 : 1) : 0;  // 2-bit codes: 01 = +1, 11 = -1, 00 = 0
+    const int c1 = (i & 4) ? ((i & 8) ? -1 : 1) : 0;
+    const int i0 = (i >> 4) & 3, i1 = (i >> 6) & 3;
+    const uint32_t v = ((static_cast<uint32_t>(c0) & 0xFFu) << (8 * i0)) | ((static_cast<uint32_t>(c1) & 0xFFu) << (8 * i1));
+    uint4* dst = reinterpret_cast<uint4*>(lut + i * 32 + half * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(v, v, v, v);
+  }
+  pdl_wait();
   uint4 wbuf[kPieces];
   {
     const int row = row_begin + slot;
@@ -75,8 +102,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
     }
   }
 
-  // This thread's share of the activation rows (fused quantisation) and g,
-  // also requested before anything waits.
+  // This thread's share of the activation rows (fused quantisation) and g.
   constexpr int kXq = 4;  // 16-byte activation vectors kept in registers
   const int nvec = a.k / 8;
   const int wpr = (kGemvThreads / 32) / TP;  // warps per token row
@@ -92,18 +118,6 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
   }
   const float g = __ldg(a.g);
 
-  // Expansion table: group byte -> four int8 weights, replicated so that
-  // lane l always reads bank l (the bytes a warp looks up are random).
-  {
-    const int i = tid >> 1, half = tid & 1;  // 256 entries x 2 threads, 16 copies each
-    const int c0 = (i & 1) ? ((i & 2) ? -1 : 1) : 0;  // 2-bit codes: 01 = +1, 11 = -1, 00 = 0
-    const int c1 = (i & 4) ? ((i & 8) ? -1 : 1) : 0;
-    const int i0 = (i >> 4) & 3, i1 = (i >> 6) & 3;
-    const uint32_t v = ((static_cast<uint32_t>(c0) & 0xFFu) << (8 * i0)) | ((static_cast<uint32_t>(c1) & 0xFFu) << (8 * i1));
-    uint4* dst = reinterpret_cast<uint4*>(lut + i * 32 + half * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(v, v, v, v);
-  }
   const uint32_t* my_lut = lut + lane;
 
   if (!PREQUANT) {
@@ -157,10 +171,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
       }
     }
   } else {
-    // The act-quant kernel before this one (launched with programmatic
-    // serialisation, the weight loads above already in flight) wrote the
-    // codes and scales.
-    pdl_wait();
+    // The act-quant kernel before this one wrote the codes and scales.
     // One bulk copy brings all t rows of codes (t * k bytes, a multiple of 64).
     __shared__ uint64_t bar;
     if (tid == 0) {
@@ -254,10 +265,7 @@ static cudaError_t gemv_tp(const GemvArgs& a, int num_sms, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   // At most one block per SM, each owning a contiguous range of rows.
   int blocks = (a.n_out < num_sms) ? a.n_out : num_sms;
-  if (PREQUANT)
-    return launch_pdl(k_gemv<TP, PREQUANT>, dim3(blocks), dim3(kGemvThreads), smem, s, a);
-  k_gemv<TP, PREQUANT><<<blocks, kGemvThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_gemv<TP, PREQUANT>, dim3(blocks), dim3(kGemvThreads), smem, s, a);
 }
 
 bool gemv_fits(int64_t t, int64_t k) {
