@@ -64,6 +64,7 @@ def _load():
         "sbo_absmean_bits": (ctypes.c_uint32, [P, I64]),
         "sbo_clamped_scale": (F, [F]),
         "sbo_nm_mask": (None, [P, I64, I64, I, I, P]),
+        "sbo_nm_mask_from_codes": (None, [P, I64, I64, I, I, P]),
         "sbo_ternary": (None, [P, I64, F, P]),
         "sbo_apply_mask": (None, [P, P, I64, I64, I, P]),
         "sbo_pack24": (None, [P, P, I64, I64, P, P]),
@@ -75,6 +76,7 @@ def _load():
         "sbo_grad_x_at": (ctypes.c_double, [P, P, F, I64, I64, I64, I64]),
         "sbo_grad_w": (None, [P, P, I64, I64, I64, P]),
         "sbo_grad_w_at": (ctypes.c_double, [P, P, I64, I64, I64, I64, I64]),
+        "sbo_grad_w_masked": (None, [P, P, P, I64, I64, I64, I, P]),
         "sbo_round_bf16": (None, [P, I64, P]),
         "sbo_threads": (I, []),
     }
@@ -124,6 +126,15 @@ def nm_mask(w, n: int, m: int) -> np.ndarray:
     n_out, k = w.shape
     out = np.zeros((n_out, k // m), dtype=np.uint8)
     _load().sbo_nm_mask(_ptr(w), n_out, k, n, m, _ptr(out))
+    return out
+
+
+def nm_mask_from_codes(q: np.ndarray, n: int, m: int) -> np.ndarray:
+    """Ablation of A2 ([de] §4, [fr] §5): the mask from |q| instead of |w|."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    n_out, k = q.shape
+    out = np.zeros((n_out, k // m), dtype=np.uint8)
+    _load().sbo_nm_mask_from_codes(_ptr(q), n_out, k, n, m, _ptr(out))
     return out
 
 
@@ -231,6 +242,17 @@ def grad_w_at(dy, x, oi: int, ki: int) -> float:
     return float(_load().sbo_grad_w_at(_ptr(dy), _ptr(x), t, n_out, x.shape[1], oi, ki))
 
 
+def grad_w_masked(dy, x, mask: np.ndarray, m: int) -> np.ndarray:
+    """Ablation of A8 ([de] §4, [fr] §5): dW with the gradient of pruned weights blocked."""
+    dy, x = _u16(dy), _u16(x)
+    t, n_out = dy.shape
+    k = x.shape[1]
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    out = np.zeros((n_out, k), dtype=np.float64)
+    _load().sbo_grad_w_masked(_ptr(dy), _ptr(x), _ptr(mask), t, n_out, k, m, _ptr(out))
+    return out
+
+
 def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round fp64 values to bf16 (nearest, ties to even); returns uint16 bit patterns."""
     a = np.ascontiguousarray(a, dtype=np.float64)
@@ -239,20 +261,21 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
     return out
 
 
-def prepare(w, n: int, m: int):
-    """A1-A3 in the pages' order: returns dict(gamma, g, mask, q, weff)."""
+def prepare(w, n: int, m: int, mask_from_codes: bool = False):
+    """A1-A3 in the pages' order: returns dict(gamma, g, mask, q, weff).
+    mask_from_codes: the pages' ablation that builds the mask from |q|."""
     w = _u16(w)
     gamma = absmean_gamma(w)
     g = clamped_scale(gamma)
-    mask = nm_mask(w, n, m)
     q = ternary(w, g)
+    mask = nm_mask_from_codes(q, n, m) if mask_from_codes else nm_mask(w, n, m)
     weff = apply_mask(q, mask, m)
     return {"gamma": gamma, "g": g, "mask": mask, "q": q, "weff": weff}
 
 
-def forward(w, x, n: int, m: int):
+def forward(w, x, n: int, m: int, mask_from_codes: bool = False):
     """A1-A6: returns dict with the prepare outputs plus xq, a_prime, acc, y."""
-    p = prepare(w, n, m)
+    p = prepare(w, n, m, mask_from_codes)
     xq, ap = act_quant(x)
     acc = gemm_acc(xq, p["weff"])
     y = dequant(acc, ap, p["g"])

@@ -7,6 +7,7 @@
 #include "sbl_oracle.h"
 
 #include <algorithm>
+#include <cstdlib>
 #include <cmath>
 #include <cstring>
 #include <vector>
@@ -189,6 +190,24 @@ void sbo_nm_mask(const uint16_t* w, int64_t n_out, int64_t k, int n, int m,
 // A3 (ternarise).  w/g rounded half-to-even and clipped to [-1, 1] is 0 when
 // |w|/g <= 1/2 and sign(w) otherwise; 2|w| is exact in fp32, so the test
 // 2|w| > g decides it with no division rounding.
+void sbo_nm_mask_from_codes(const int8_t* q, int64_t n_out, int64_t k, int n, int m,
+                            uint8_t* mask) {
+  const int64_t groups = k / m;
+#pragma omp parallel for schedule(static)
+  for (int64_t row = 0; row < n_out; ++row) {
+    for (int64_t g = 0; g < groups; ++g) {
+      const int8_t* grp = q + row * k + g * m;
+      int order[8];
+      for (int j = 0; j < m; ++j) order[j] = j;
+      // stable: equal |q| keep index order, so ties go to the lowest index
+      std::stable_sort(order, order + m, [&](int a, int b) { return std::abs(int(grp[a])) > std::abs(int(grp[b])); });
+      uint8_t bits = 0;
+      for (int j = 0; j < n; ++j) bits |= uint8_t(1u << order[j]);
+      mask[row * groups + g] = bits;
+    }
+  }
+}
+
 void sbo_ternary(const uint16_t* w, int64_t numel, float g, int8_t* q) {
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < numel; ++i) {
@@ -332,6 +351,16 @@ void sbo_grad_w(const uint16_t* dy, const uint16_t* x, int64_t t,
       for (int64_t c = 0; c < k; ++c) out[c] += d * double(bf16_value(xr[c]));
     }
   }
+}
+
+void sbo_grad_w_masked(const uint16_t* dy, const uint16_t* x, const uint8_t* mask,
+                       int64_t t, int64_t n_out, int64_t k, int m, double* dw) {
+  sbo_grad_w(dy, x, t, n_out, k, dw);
+  const int64_t groups = k / m;
+#pragma omp parallel for schedule(static)
+  for (int64_t o = 0; o < n_out; ++o)
+    for (int64_t c = 0; c < k; ++c)
+      if (!((mask[o * groups + c / m] >> (c % m)) & 1u)) dw[o * k + c] = 0.0;
 }
 
 void sbo_round_bf16(const double* in, int64_t count, uint16_t* out) {

@@ -47,6 +47,14 @@ float sbo_clamped_scale(float gamma);
 void sbo_nm_mask(const uint16_t* w, int64_t n_out, int64_t k, int n, int m,
                  uint8_t* mask);
 
+/* Ablation of A2 named by the pages ([de] §4 "Ablationsstudien", [fr] §5):
+ * the mask built from the quantised ternary codes instead of the masters.
+ * For each group keep the n largest |q| (|q| in {0, 1}), ties to the lowest
+ * index, i.e. the first n nonzero codes, then the first zero ones.  Same
+ * output layout as sbo_nm_mask. */
+void sbo_nm_mask_from_codes(const int8_t* q, int64_t n_out, int64_t k, int n, int m,
+                            uint8_t* mask);
+
 /* A3 (ternarise): q = round-half-even(clip(w/g, -1, 1)), which is
  * sign(w) when 2|w| > g and 0 otherwise ([de] §1, [fr] §1 ternary set). */
 void sbo_ternary(const uint16_t* w, int64_t numel, float g, int8_t* q);
@@ -92,6 +100,12 @@ void sbo_grad_w(const uint16_t* dy, const uint16_t* x, int64_t t,
                 int64_t n_out, int64_t k, double* dw);
 double sbo_grad_w_at(const uint16_t* dy, const uint16_t* x, int64_t t,
                      int64_t n_out, int64_t k, int64_t oi, int64_t ki);
+
+/* Ablation of A8 named by the pages ([de] §4 "Ablationsstudien", [fr] §5):
+ * gradients blocked for masked weights, dW = (dY^T . X) * mask, fp64; the
+ * kept positions get exactly the dense gradient, pruned ones 0. */
+void sbo_grad_w_masked(const uint16_t* dy, const uint16_t* x, const uint8_t* mask,
+                       int64_t t, int64_t n_out, int64_t k, int m, double* dw);
 
 /* Round fp64 to bf16 (round to nearest, ties to even), bit patterns out. */
 void sbo_round_bf16(const double* in, int64_t count, uint16_t* out);

@@ -218,6 +218,39 @@ def test_mask_invariants_gaussian(n, m):
                     assert grp[i] > grp[j] or (grp[i] == grp[j] and i < j)
 
 
+def test_mask_from_codes_golden_cases():
+    for case in _golden("mask_from_codes_cases.json")["cases"]:
+        q = np.array(case["q"], dtype=np.int8).reshape(1, -1)
+        mask = oracle.nm_mask_from_codes(q, case["n"], case["m"])
+        assert int(mask[0, 0]) == case["mask"], case
+
+
+@pytest.mark.parametrize("n,m", [(1, 2), (2, 4), (3, 4), (6, 8), (4, 8), (3, 8)])
+def test_mask_from_codes_brute_force(n, m):
+    rng = np.random.default_rng(300 + 10 * n + m)
+    q = rng.choice(np.array([-1, 0, 1], dtype=np.int8), size=(7, 11 * m))
+    mask = oracle.nm_mask_from_codes(q, n, m)
+    for r in range(q.shape[0]):
+        for g in range(q.shape[1] // m):
+            want = _brute_force_mask([abs(int(v)) for v in q[r, g * m:(g + 1) * m]], n)
+            assert int(mask[r, g]) == want
+
+
+def test_mask_from_codes_differs_from_master_mask():
+    """The two masks coincide where the codes separate the magnitudes and
+    differ where a kept master magnitude quantises to 0 next to a nonzero one
+    that the master mask dropped; on Gaussian masters both must occur."""
+    w = synth.master_weights(64, 256, seed=8)
+    p_master = oracle.prepare(w, 2, 4)
+    p_codes = oracle.prepare(w, 2, 4, mask_from_codes=True)
+    assert np.array_equal(p_master["q"], p_codes["q"])
+    same = p_master["mask"] == p_codes["mask"]
+    assert same.any() and (~same).any()
+    # every code the master mask keeps nonzero is at least matched in count
+    nz_kept = lambda p: int(np.count_nonzero(p["weff"]))
+    assert nz_kept(p_codes) >= nz_kept(p_master)
+
+
 # ---------------------------------------------------------------------------
 # A3: ternary codes, quant-then-mask, packing
 # ---------------------------------------------------------------------------
@@ -401,6 +434,23 @@ def test_grad_w_equals_numpy_matmul_and_is_dense():
     assert math.isclose(oracle.grad_w_at(dy, x, 19, 35), ref[19, 35], rel_tol=1e-12, abs_tol=1e-12)
     # dense gradient flow: every master weight gets a gradient, including pruned ones
     assert np.count_nonzero(dw) == dw.size
+
+
+def test_grad_w_masked_blocks_exactly_the_pruned_positions():
+    dy = synth.upstream_grad(9, 16, seed=15)
+    x = synth.activations(9, 40, seed=16)
+    w = synth.master_weights(16, 40, seed=17)
+    for n, m in [(2, 4), (6, 8), (1, 2), (8, 8)]:
+        mask = oracle.nm_mask(synth.bits(w), n, m)
+        dw = oracle.grad_w_masked(dy, x, mask, m)
+        dense = _bf16_float(synth.bits(dy)).T @ _bf16_float(synth.bits(x))
+        keep = np.repeat(mask[:, :, None], m, axis=2) >> np.arange(m, dtype=np.uint8) & 1
+        keep = keep.reshape(16, 40).astype(bool)
+        assert np.allclose(dw[keep], dense[keep], rtol=1e-12, atol=1e-12)
+        assert (dw[~keep] == 0).all()
+        assert keep.sum() == 16 * 40 * n // m
+        if n == m:
+            assert np.array_equal(dw, oracle.grad_w(dy, x))
 
 
 def test_round_bf16_matches_rational_rounding():
