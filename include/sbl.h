@@ -68,14 +68,19 @@ typedef enum sbl_status {
 
 /* Flags of sbl_layer.flags (fixed at prepare time). */
 enum {
-  SBL_PACK_GEMV = 1u << 0 /* also write the 2-bit decode packing (2:4 only) */
+  SBL_PACK_GEMV = 1u << 0,      /* also write the 2-bit decode packing (2:4 only) */
+  SBL_MASK_FROM_QUANT = 1u << 1 /* ablation the pages report ([de] 4 "Ablationsstudien",
+                                   [fr] 5): build the N:M mask from the ternary codes
+                                   |q| instead of the masters (ties to the lowest index) */
 };
 
 /* Flags of sbl_backward's `flags` argument. */
 enum {
-  SBL_GRAD_F32 = 1u << 1, /* dx and dw are fp32 instead of bf16 */
-  SBL_NO_DX = 1u << 2,    /* skip dX (dx may be NULL) */
-  SBL_NO_DW = 1u << 3     /* skip dW (dw may be NULL) */
+  SBL_GRAD_F32 = 1u << 1,   /* dx and dw are fp32 instead of bf16 */
+  SBL_NO_DX = 1u << 2,      /* skip dX (dx may be NULL) */
+  SBL_NO_DW = 1u << 3,      /* skip dW (dw may be NULL) */
+  SBL_MASKED_GRAD = 1u << 4 /* ablation the pages report ([de] 4, [fr] 5): block the
+                               gradient of pruned weights, dw = (dy^T . x) * mask */
 };
 
 /* One Sparse-BitLinear layer: shapes, pattern and the caller-owned device

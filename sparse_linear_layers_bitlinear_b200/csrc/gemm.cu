@@ -168,7 +168,8 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
 // ---------------------------------------------------------------------------
 template <bool A_MN, bool B_MN, bool F32>
 static cudaError_t bf16_dispatch(const uint16_t* A, const uint16_t* B, int64_t M, int64_t N, int64_t K,
-                                 const float* alpha, void* out, uint32_t* status, int num_sms, cudaStream_t s) {
+                                 const float* alpha, void* out, uint32_t* status, int num_sms, cudaStream_t s,
+                                 const uint8_t* mask, int mask_m) {
   using Cfg = CfgPairBf16<A_MN, B_MN, F32>;
   CUtensorMap ta, tb;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -186,22 +187,24 @@ static cudaError_t bf16_dispatch(const uint16_t* A, const uint16_t* B, int64_t M
   p.out = out;
   p.ldo = N;
   p.status = status;
+  p.mask = mask;
+  p.mask_m = mask_m;
   return launch_pair<Cfg>(ta, tb, tb, p, p.M, p.N, num_sms, s);
 }
 
 cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t* A, const uint16_t* B, int64_t M,
                              int64_t N, int64_t K, const float* alpha, void* out, uint32_t* status, int num_sms,
-                             cudaStream_t s) {
+                             cudaStream_t s, const uint8_t* mask, int mask_m) {
   const int sel = (a_mn ? 4 : 0) | (b_mn ? 2 : 0) | (out_f32 ? 1 : 0);
   switch (sel) {
-    case 0: return bf16_dispatch<false, false, false>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 1: return bf16_dispatch<false, false, true>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 2: return bf16_dispatch<false, true, false>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 3: return bf16_dispatch<false, true, true>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 4: return bf16_dispatch<true, false, false>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 5: return bf16_dispatch<true, false, true>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    case 6: return bf16_dispatch<true, true, false>(A, B, M, N, K, alpha, out, status, num_sms, s);
-    default: return bf16_dispatch<true, true, true>(A, B, M, N, K, alpha, out, status, num_sms, s);
+    case 0: return bf16_dispatch<false, false, false>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 1: return bf16_dispatch<false, false, true>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 2: return bf16_dispatch<false, true, false>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 3: return bf16_dispatch<false, true, true>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 4: return bf16_dispatch<true, false, false>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 5: return bf16_dispatch<true, false, true>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    case 6: return bf16_dispatch<true, true, false>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
+    default: return bf16_dispatch<true, true, true>(A, B, M, N, K, alpha, out, status, num_sms, s, mask, mask_m);
   }
 }
 
@@ -252,8 +255,8 @@ const DualSchedule& dual_schedule(int tiles0, int kb0, int tiles1, int kb1, int 
 
 template <bool F32>
 cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16_t* x, int64_t t, int64_t n_out,
-                          int64_t k, const float* g, void* dx, void* dw, uint32_t* status, int num_sms,
-                          cudaStream_t s, bool* done) {
+                          int64_t k, const float* g, void* dx, void* dw, const uint8_t* dw_mask, int mask_m,
+                          uint32_t* status, int num_sms, cudaStream_t s, bool* done) {
   using Cfg = CfgPairDualBf16<F32>;
   *done = false;
   int max_clusters = 0;
@@ -290,6 +293,8 @@ cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16
   p.out[0] = dx;
   p.out[1] = dw;
   p.status = status;
+  p.mask1 = dw_mask;
+  p.mask_m = mask_m;
   std::copy(sch.off.begin(), sch.off.end(), p.sched_off);
   std::copy(sch.ids.begin(), sch.ids.end(), p.sched);
   k_gemm_pair<Cfg><<<2 * npairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
@@ -302,9 +307,10 @@ cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16
 
 cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const uint16_t* weff, const uint16_t* x,
                                       int64_t t, int64_t n_out, int64_t k, const float* g, void* dx, void* dw,
-                                      uint32_t* status, int num_sms, cudaStream_t s, bool* done) {
-  return out_f32 ? dual_dispatch<true>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done)
-                 : dual_dispatch<false>(dy, weff, x, t, n_out, k, g, dx, dw, status, num_sms, s, done);
+                                      const uint8_t* dw_mask, int mask_m, uint32_t* status, int num_sms,
+                                      cudaStream_t s, bool* done) {
+  return out_f32 ? dual_dispatch<true>(dy, weff, x, t, n_out, k, g, dx, dw, dw_mask, mask_m, status, num_sms, s, done)
+                 : dual_dispatch<false>(dy, weff, x, t, n_out, k, g, dx, dw, dw_mask, mask_m, status, num_sms, s, done);
 }
 
 // ---------------------------------------------------------------------------

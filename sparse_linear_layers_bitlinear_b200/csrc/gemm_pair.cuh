@@ -296,6 +296,8 @@ struct DualBf16Params {
   const float* alpha[2];    // device scalars or nullptr for 1
   void* out[2];
   uint32_t* status;
+  const uint8_t* mask1;     // optional keep bits for problem 1 (dW)
+  int mask_m;
   uint16_t sched_off[kDualMaxPairs + 1];  // pair p runs sched[sched_off[p] .. sched_off[p+1])
   uint16_t sched[kDualMaxTiles];
 };
@@ -364,6 +366,8 @@ struct CfgPairDualBf16 {
     q.out = p.out[prob];
     q.ldo = p.N;
     q.status = p.status;
+    q.mask = prob ? p.mask1 : nullptr;
+    q.mask_m = p.mask_m;
     CfgBf16<false, true, OUT_F32>::epilogue(q, t_acc, row, n0, lane, part, parts);
   }
 };

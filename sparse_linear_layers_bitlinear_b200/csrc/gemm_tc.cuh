@@ -198,7 +198,34 @@ struct Bf16Params {
   void* out;
   int64_t ldo;         // elements
   uint32_t* status;
+  const uint8_t* mask;  // optional N:M keep bits [M][N / mask_m]: zero out[r][c] where bit c % mask_m is clear
+  int mask_m;
 };
+
+// Keep bits of columns col0 .. col0 + 31 of row `row` (col0 a multiple of 32,
+// N a multiple of 64), one bit per column, from mask bytes of mask_m bits.
+__device__ __forceinline__ uint32_t keep_bits32(const uint8_t* mask, int mask_m, int row, int N, int col0) {
+  const uint8_t* src = mask + int64_t(row) * (N / mask_m) + col0 / mask_m;
+  uint32_t keep = 0;
+  if (mask_m == 8) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+    keep = w;  // four bytes of eight bits: byte i holds columns 8i .. 8i + 7
+  } else if (mask_m == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) keep |= ((w.x >> (8 * i)) & 0xFu) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) keep |= ((w.y >> (8 * i)) & 0xFu) << (16 + 4 * i);
+  } else {  // mask_m == 2
+    const uint4 w = *reinterpret_cast<const uint4*>(src);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) keep |= ((ws[j] >> (8 * i)) & 0x3u) << (8 * j + 2 * i);
+  }
+  return keep;
+}
 
 template <bool A_MN, bool B_MN, bool OUT_F32>
 struct CfgBf16 {
@@ -255,6 +282,11 @@ struct CfgBf16 {
       tmem_load_wait();
       const int col0 = n0 + c * 32;
       if (row >= p.M || col0 >= p.N) continue;  // after the warp-wide load: divergence is harmless
+      if (p.mask != nullptr) {
+        const uint32_t keep = keep_bits32(p.mask, p.mask_m, row, p.N, col0);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = ((keep >> e) & 1u) ? r[e] : 0u;
+      }
       if (OUT_F32) {
         float* dst = reinterpret_cast<float*>(p.out) + int64_t(row) * p.ldo + col0;
 #pragma unroll

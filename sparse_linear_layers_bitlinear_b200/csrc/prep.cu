@@ -661,17 +661,22 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       const bool active = i < v1;  // quads of lanes are all-or-nothing (v1 - v0 and upr are multiples of 8)
       const uint4 vv = active ? st[e] : make_uint4(0, 0, 0, 0);
       const uint32_t wd[4] = {vv.x, vv.y, vv.z, vv.w};
-      uint32_t mw[4];  // magnitudes, two per word
+      uint32_t mw[4], nz[4], key[4];  // magnitudes, code != 0 (0xFFFF per half), selection keys
 #pragma unroll
-      for (int q = 0; q < 4; ++q) mw[q] = wd[q] & 0x7FFF7FFFu;
+      for (int q = 0; q < 4; ++q) {
+        mw[q] = wd[q] & 0x7FFF7FFFu;
+        nz[q] = bf16x2_gt_mask(mw[q], thr2);  // code != 0 <=> |w| > g/2, a packed bf16 compare
+        // the mask is selected on |w|, or (ablation) on |q| as bf16 1.0 / 0
+        key[q] = a.out.mask_from_codes ? (nz[q] & 0x3F803F80u) : mw[q];
+      }
       uint32_t km[4];  // 0xFFFF per kept weight
       // Z: bits 0-3 / 8-11 kept pattern of group 0 / 1 (the mask section's
       // u16), bits 16-19 / 20-23 their 2:4 metadata nibbles; W: byte-permute
       // selector of the four kept high bytes.
       uint32_t Z = 0, W = 0;
       if (M == 4) {
-        const uint2 e0 = sel[outcomes4_index(mw[0], mw[1]) * 32 + lane];
-        const uint2 e1 = sel[outcomes4_index(mw[2], mw[3]) * 32 + lane];
+        const uint2 e0 = sel[outcomes4_index(key[0], key[1]) * 32 + lane];
+        const uint2 e1 = sel[outcomes4_index(key[2], key[3]) * 32 + lane];
         km[0] = prmt(e0.x, 0u, 0x9988u);
         km[1] = prmt(e0.x, 0u, 0xBBAAu);
         km[2] = prmt(e1.x, 0u, 0x9988u);
@@ -682,8 +687,8 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
         uint32_t mag[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          mag[2 * q] = mw[q] & 0xFFFFu;
-          mag[2 * q + 1] = mw[q] >> 16;
+          mag[2 * q] = key[q] & 0xFFFFu;
+          mag[2 * q + 1] = key[q] >> 16;
         }
         uint32_t kept = 0;
 #pragma unroll
@@ -696,11 +701,10 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
         }
       }
 
-      // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and
-      // code != 0 (code != 0 <=> |w| > g/2, a packed bf16 compare).
+      // W_eff in bf16, two weights per word: (sign | 0x3F80) where kept and code != 0.
       uint32_t weff[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) weff[q] = ((wd[q] | 0x3F803F80u) & 0xBF80BF80u) & bf16x2_gt_mask(mw[q], thr2) & km[q];
+      for (int q = 0; q < 4; ++q) weff[q] = ((wd[q] | 0x3F803F80u) & 0xBF80BF80u) & nz[q] & km[q];
       const uint32_t hb_lo = __byte_perm(weff[0], weff[1], 0x7531);  // high bytes of weights 0..3
       const uint32_t hb_hi = __byte_perm(weff[2], weff[3], 0x7531);  // weights 4..7
 
@@ -784,6 +788,7 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   a.slot_fast = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchSlotFast);
   a.slot_bins = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchSlotBins);
   a.gen = reinterpret_cast<uint64_t*>(blob + L.scratch + kScratchGen);
+  a.out.mask_from_codes = (flags & SBL_MASK_FROM_QUANT) ? 1 : 0;
   a.out.mask = blob + L.mask;
   a.out.codes = L.codes ? reinterpret_cast<int8_t*>(blob + L.codes) : nullptr;
   a.out.weff_bf16 = reinterpret_cast<uint16_t*>(blob + L.weff_bf16);

@@ -11,8 +11,8 @@ using namespace sbl;
 namespace {
 
 constexpr int64_t kMaxK = 131072;  // keeps |acc| <= 127 * k below 2^24: (float)acc is exact
-constexpr uint32_t kLayerFlags = SBL_PACK_GEMV;
-constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW;
+constexpr uint32_t kLayerFlags = SBL_PACK_GEMV | SBL_MASK_FROM_QUANT;
+constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW | SBL_MASKED_GRAD;
 
 struct DeviceInfo {
   bool checked = false;
@@ -189,6 +189,8 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
   if (t < 0 || t > (int64_t(1) << 30)) return SBL_ERR_SHAPE;
   const bool want_dx = !(flags & SBL_NO_DX), want_dw = !(flags & SBL_NO_DW);
   const bool f32 = (flags & SBL_GRAD_F32) != 0u;
+  // the blocked-gradient ablation multiplies dW by the mask section
+  const uint8_t* dw_mask = (flags & SBL_MASKED_GRAD) ? at<const uint8_t>(layer, L.mask) : nullptr;
   if ((want_dx && dx == nullptr) || (want_dw && dw == nullptr)) return SBL_ERR_INVALID_ARG;
   if (t > 0 && ((want_dx || want_dw) && dy == nullptr)) return SBL_ERR_INVALID_ARG;
   if (t > 0 && want_dw && x == nullptr) return SBL_ERR_INVALID_ARG;
@@ -207,7 +209,7 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
     bool done = false;
     const cudaError_t e = launch_bf16_backward_dual(
         f32, static_cast<const uint16_t*>(dy), at<const uint16_t>(layer, L.weff_bf16), static_cast<const uint16_t*>(x),
-        t, layer->n_out, layer->k, at<const float>(layer, L.g), dx, dw, status, sms, s, &done);
+        t, layer->n_out, layer->k, at<const float>(layer, L.g), dx, dw, dw_mask, layer->m, status, sms, s, &done);
     if (e != cudaSuccess) return SBL_ERR_CUDA;
     if (done) return SBL_OK;
   }
@@ -222,7 +224,7 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
     // dW[n_out, k] = dY^T . X:  A = dY stored [K=t][M=n_out], B = X stored [K=t][N=k].
     const cudaError_t e = launch_bf16_gemm(true, true, f32, static_cast<const uint16_t*>(dy),
                                            static_cast<const uint16_t*>(x), layer->n_out, layer->k, t, nullptr, dw,
-                                           status, sms, s);
+                                           status, sms, s, dw_mask, layer->m);
     if (e != cudaSuccess) return SBL_ERR_CUDA;
   }
   return SBL_OK;

@@ -30,6 +30,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 // Destinations of the pack pass (device pointers; optional ones may be null).
 struct PackOut {
+  int mask_from_codes;  // select on the ternary codes instead of the master magnitudes
   uint8_t* mask;
   int8_t* codes;
   uint16_t* weff_bf16;
@@ -67,15 +68,18 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const in
 
 // out[M][N] = alpha * A . B^T in bf16 x bf16 -> fp32 (tensor cores).
 //   a_mn: A stored [K][M] (else [M][K]);  b_mn: B stored [K][N] (else [N][K]).
+//   mask (optional): N:M keep bits [M][N/mask_m]; out is zeroed where a bit is clear.
 cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t* A, const uint16_t* B, int64_t M,
                              int64_t N, int64_t K, const float* alpha, void* out, uint32_t* status, int num_sms,
-                             cudaStream_t s);
+                             cudaStream_t s, const uint8_t* mask = nullptr, int mask_m = 0);
 
 // dX = g * dY . W_eff and dW = dY^T . X in one launch.  Sets *done = false
 // (and enqueues nothing) when the tile count exceeds the launch's schedule.
+// dw_mask (optional): the layer's mask section; dW is zeroed at pruned positions.
 cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const uint16_t* weff, const uint16_t* x,
                                       int64_t t, int64_t n_out, int64_t k, const float* g, void* dx, void* dw,
-                                      uint32_t* status, int num_sms, cudaStream_t s, bool* done);
+                                      const uint8_t* dw_mask, int mask_m, uint32_t* status, int num_sms,
+                                      cudaStream_t s, bool* done);
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 

@@ -33,10 +33,12 @@ STATUS_NAMES = {
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 # layer flags
 SBL_PACK_GEMV = 1 << 0
+SBL_MASK_FROM_QUANT = 1 << 1
 # backward flags
 SBL_GRAD_F32 = 1 << 1
 SBL_NO_DX = 1 << 2
 SBL_NO_DW = 1 << 3
+SBL_MASKED_GRAD = 1 << 4
 # device status bits
 SBL_STATUS_NONFINITE_W = 1 << 0
 SBL_STATUS_NONFINITE_X = 1 << 1

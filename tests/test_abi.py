@@ -70,6 +70,16 @@ def test_layout_sections_are_aligned_and_disjoint(lib):
         assert L.header <= L.gamma < L.header + 4096 and L.g == L.gamma + 4
 
 
+def test_ablation_flags_are_accepted_and_unknown_bits_rejected(lib):
+    base = sbl.prepared_bytes(264, 320, 2, 4, 0)
+    assert sbl.prepared_bytes(264, 320, 2, 4, sbl.SBL_MASK_FROM_QUANT) == base  # same sections
+    assert sbl.prepared_bytes(264, 320, 6, 8, sbl.SBL_MASK_FROM_QUANT) > 0
+    assert sbl.prepared_bytes(264, 320, 2, 4, sbl.SBL_MASK_FROM_QUANT | sbl.SBL_PACK_GEMV) > base
+    assert sbl.prepared_bytes(264, 320, 2, 4, 1 << 5) == 0
+    with pytest.raises(sbl.SblError):
+        sbl.prepared_layout(264, 320, 2, 4, 1 << 5)
+
+
 @pytest.mark.parametrize("args,code", [
     ((256, 256, 2, 3, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
     ((256, 256, 0, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),

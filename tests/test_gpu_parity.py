@@ -248,6 +248,74 @@ def test_gamma_and_codes_at_extreme_magnitudes(kind):
     _check_prepared(layer, w, n, m)
 
 
+@pytest.mark.parametrize("n_out,k,n,m,t", [(264, 320, 2, 4, 70), (136, 448, 6, 8, 33), (200, 128, 1, 2, 9),
+                                           (128, 384, 4, 8, 17)])
+def test_ablation_mask_from_codes(n_out, k, n, m, t):
+    """The pages' ablation that builds the mask from the ternary codes: the
+    prepared sections and the forward match the oracle's code-based mask."""
+    seed = 4 * n_out + k + n
+    w = synth.master_weights(n_out, k, seed)
+    x = synth.activations(t, k, seed + 1)
+    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_MASK_FROM_QUANT)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    ref = oracle.prepare(w, n, m, mask_from_codes=True)
+    gamma, g, status = bd.header_scalars(layer)
+    assert status == 0 and np.float32(g) == ref["g"]
+    assert np.array_equal(bd.mask(layer), ref["mask"])
+    assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"])
+    if (n, m) == (2, 4):
+        vals, meta = oracle.pack24(ref["weff"], ref["mask"])
+        assert np.array_equal(bd.sp_values(layer), vals)
+        assert np.array_equal(bd.sp_meta_canonical(layer)[0], meta)
+    else:
+        assert np.array_equal(bd.codes(layer), ref["weff"])
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), oracle.dequant(acc_ref, ap_ref, ref["g"]).view(np.uint32))
+
+
+@pytest.mark.parametrize("n_out,k,n,m,t", [(264, 320, 2, 4, 70), (136, 448, 6, 8, 33), (200, 128, 1, 2, 9),
+                                           (392, 832, 3, 8, 130)])
+@pytest.mark.parametrize("only_dw", [False, True])
+def test_ablation_masked_grad(n_out, k, n, m, t, only_dw):
+    """The pages' blocked-gradient ablation: dW is the dense dY^T X on kept
+    positions and exactly 0 on pruned ones; dX is unchanged."""
+    seed = 3 * n_out + k + m
+    w = synth.master_weights(n_out, k, seed)
+    x = synth.activations(t, k, seed + 1)
+    dy = synth.upstream_grad(t, n_out, seed + 2)
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, _dev(w))
+    ref = oracle.prepare(w, n, m)
+    dw_ref = oracle.grad_w_masked(dy, x, ref["mask"], m)
+    flags = sbl.SBL_MASKED_GRAD | (sbl.SBL_NO_DX if only_dw else 0)
+    dx = None if only_dw else torch.empty((t, k), dtype=torch.float32, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, dx, dw, flags | sbl.SBL_GRAD_F32)
+    torch.cuda.synchronize()
+    dw_gpu = dw.cpu().numpy()
+    _close(dw_gpu, dw_ref)
+    assert (dw_gpu[dw_ref == 0] == 0).all() and np.count_nonzero(dw_gpu) <= n_out * k * n // m
+    if not only_dw:
+        _close(dx.cpu().numpy(), oracle.grad_x(dy, ref["weff"], ref["g"]))
+    # bf16 outputs, the same launch shape (one dual launch, or dW alone)
+    dx16 = None if only_dw else torch.empty((t, k), dtype=torch.bfloat16, device="cuda")
+    dw16 = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, dx16, dw16, flags)
+    torch.cuda.synchronize()
+    _close(bd.bf16_to_f64(dw16), dw_ref, rtol=BF16_REL, atol=ATOL)
+    assert (bd.bf16_to_f64(dw16)[dw_ref == 0] == 0).all()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
 @pytest.mark.parametrize("fill", ["random", "ones", "zeros"])
 def test_prepare_on_uninitialised_blob_and_repeats(fill):
     """The prepare kernel's grid barrier keeps its state in the blob's scratch
