@@ -10,7 +10,7 @@
 // One cooperative launch, one CTA per SM.  Each CTA owns a contiguous range
 // of W (in 16-byte vectors of eight weights) and streams it twice through a
 // ring of shared-memory stages filled by bulk copies (one producer warp,
-// sixteen consumer warps):
+// twenty-four consumer warps):
 //   phase 1  from HBM: every |w| is added exactly (below); W stays in L2;
 //   barrier  every CTA publishes its partial sum and waits for the others
 //            (bounded wait on per-CTA arrival words);
@@ -27,12 +27,12 @@
 
 namespace sbl {
 
-constexpr int kPrepConsumers = 512;                    // 16 consumer warps
+constexpr int kPrepConsumers = 768;                    // 24 consumer warps
 constexpr int kPrepConsumerWarps = kPrepConsumers / 32;
 constexpr int kPrepThreads = kPrepConsumers + 32;      // + one producer warp
 constexpr int kVecsPerThread = 2;                      // 16-byte vectors per consumer per stage
 constexpr int kChunkVecs = kVecsPerThread * kPrepConsumers;  // 24 KB per stage
-constexpr int kPrepStages = 12;
+constexpr int kPrepStages = 8;
 constexpr size_t kPrepTailBytes = 4096;
 constexpr size_t kSelBytes = 64 * 32 * 8;  // 64 entries x 32 lane copies x 8 bytes
 constexpr size_t kPrepSmem = size_t(kPrepStages) * kChunkVecs * 16 + kSelBytes + kPrepTailBytes;
