@@ -544,36 +544,63 @@ def main():
     torch.cuda.synchronize(dev)
     phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
 
-    # End to end through the C ABI from pinned host buffers: H2D of the step's
-    # inputs, the step, D2H of its outputs, all inside the timed region.
+    # End to end through the C ABI from pinned host buffers: every step copies
+    # its inputs in (H2D), runs the step and copies its outputs back (D2H), all
+    # inside the timed region.  Three streams pipeline consecutive steps the
+    # way a training loop would: the inputs of step i+1 travel while step i
+    # computes and the outputs of step i-1 travel back; two device buffer sets
+    # alternate, and events keep each set's copies and compute in order.
     w_h = [s[0].cpu().pin_memory() for s in sets]
     x_h = [s[1].cpu().pin_memory() for s in sets]
     dy_h = [s[2].cpu().pin_memory() for s in sets]
-    y_h = torch.empty((T, N), dtype=torch.float32).pin_memory()
-    dx_h = torch.empty((T, K), dtype=torch.bfloat16).pin_memory()
-    dw_h = torch.empty((N, K), dtype=torch.bfloat16).pin_memory()
-    w_d, x_d, dy_d = (torch.empty_like(t) for t in sets[0])
+    outs_h = [(torch.empty((T, N), dtype=torch.float32).pin_memory(),
+               torch.empty((T, K), dtype=torch.bfloat16).pin_memory(),
+               torch.empty((N, K), dtype=torch.bfloat16).pin_memory()) for _ in range(2)]
+    ins_d = [tuple(torch.empty_like(t) for t in sets[0]) for _ in range(2)]
+    outs_d = [(y, dx, dw), (torch.empty_like(y), torch.empty_like(dx), torch.empty_like(dw))]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step(i):
-        r = i % ROTATE
-        w_d.copy_(w_h[r], non_blocking=True)
-        x_d.copy_(x_h[r], non_blocking=True)
-        dy_d.copy_(dy_h[r], non_blocking=True)
-        sbl.prepare_weights(layer, w_d)
-        sbl.forward(layer, x_d, T, y, workspace=ws)
-        sbl.backward(layer, x_d, dy_d, T, dx, dw, 0)
-        y_h.copy_(y, non_blocking=True)
-        dx_h.copy_(dx, non_blocking=True)
-        dw_h.copy_(dw, non_blocking=True)
+        b, r = i % 2, i % ROTATE
+        w_d, x_d, dy_d = ins_d[b]
+        y_d, dx_d, dw_d = outs_d[b]
+        s_in.wait_event(ev_comp[b])  # the step two back no longer reads this input set
+        with torch.cuda.stream(s_in):
+            w_d.copy_(w_h[r], non_blocking=True)
+            x_d.copy_(x_h[r], non_blocking=True)
+            dy_d.copy_(dy_h[r], non_blocking=True)
+        ev_in[b].record(s_in)
+        s_comp.wait_event(ev_in[b])
+        s_comp.wait_event(ev_out[b])  # the outputs of the step two back have left this set
+        sbl.prepare_weights(layer, w_d, stream=s_comp)
+        sbl.forward(layer, x_d, T, y_d, workspace=ws, stream=s_comp)
+        sbl.backward(layer, x_d, dy_d, T, dx_d, dw_d, 0, stream=s_comp)
+        ev_comp[b].record(s_comp)
+        s_out.wait_event(ev_comp[b])
+        with torch.cuda.stream(s_out):
+            for h_t, d_t in zip(outs_h[b], outs_d[b]):
+                h_t.copy_(d_t, non_blocking=True)
+        ev_out[b].record(s_out)
+
+    def join_streams():
+        for st in (s_in, s_comp, s_out):
+            stream.wait_stream(st)
 
     for i in range(3):
         e2e_step(i)
+    join_streams()
     torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    for st in (s_in, s_comp, s_out):
+        st.wait_stream(stream)  # nothing of the timed steps starts before e0
     for i in range(args.e2e_steps):
         e2e_step(i)
+    join_streams()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
