@@ -378,6 +378,56 @@ def bench_prefill68(dev, peaks, steps=20):
             "bwd_tflops": 2 * dense_ops / (ph[2] * 1e-3) / 1e12}
 
 
+def bench_nm_sweep(dev, peaks, steps=10):
+    """The N:M patterns the pages discuss, from dense ternary (8:8) down to
+    2:8, plus 2:4 and 1:4, on the FFN down projection (T=4096, K=6912,
+    N_out=2560): prepare + forward + dual-STE backward per step, CUDA events
+    around each phase.  2:4 runs the 2:4-sparse tensor-core GEMM, every other
+    pattern the dense int8 one over its W_eff codes."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    T, K, N = 4096, 6912, 2560
+    sets = [(synth.master_weights(N, K, 40 + 10 * r, device=dev), synth.activations(T, K, 41 + 10 * r, device=dev),
+             synth.upstream_grad(T, N, 42 + 10 * r, device=dev)) for r in range(ROTATE)]
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    dense_ops = 2.0 * T * K * N
+    out = []
+    for (n, m) in [(8, 8), (6, 8), (4, 8), (3, 8), (2, 8), (2, 4), (1, 4)]:
+        layer = sbl.Layer.allocate(N, K, n, m, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ph = [0.0, 0.0, 0.0]
+        for i in range(steps + 3):
+            w, x, dy = sets[i % ROTATE]
+            ev[0].record()
+            sbl.prepare_weights(layer, w)
+            ev[1].record()
+            sbl.forward(layer, x, T, y, workspace=ws)
+            ev[2].record()
+            sbl.backward(layer, x, dy, T, dx, dw, 0)
+            ev[3].record()
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                for j in range(3):
+                    ph[j] += ev[j].elapsed_time(ev[j + 1]) / steps
+        code, bits = sbl.read_status(layer)
+        assert code == sbl.SBL_OK, (code, bits)
+        peak = (4.0 if (n, m) == (2, 4) else 2.0) * peaks["bf16_tflops"]
+        out.append({"n": n, "m": m, "kept_fraction": n / m, "ms_per_step": sum(ph),
+                    "phase_ms": {"prepare": ph[0], "forward": ph[1], "backward": ph[2]},
+                    "fwd_dense_equiv_tops": dense_ops / (ph[1] * 1e-3) / 1e12,
+                    "fwd_kept_tops": dense_ops * n / m / (ph[1] * 1e-3) / 1e12,
+                    "fwd_frac_of_int8_peak": dense_ops / (ph[1] * 1e-3) / 1e12 / peak,
+                    "int8_peak": "2:4 sparse" if (n, m) == (2, 4) else "dense"})
+        del layer
+    return {"workload": "N:M sweep, FFN down projection T=4096, K=6912, N_out=2560, fwd + STE bwd",
+            "timing": f"CUDA events around each phase, mean of {steps} steps after 3", "points": out}
+
+
 def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     """One training step's linear layers: 30 x {q, k, v, o: 2560 x 2560;
     gate, up: 2560 -> 6912; down: 6912 -> 2560} at 8192 tokens.  Per step every
@@ -656,6 +706,7 @@ def main():
         line["decode_gemv"] = bench_decode(dev, peaks["hbm_gbs"])
         line["prefill_6of8"] = bench_prefill68(dev, peaks)
         line["train_step"] = [bench_train_step(dev, peaks, 2, 4), bench_train_step(dev, peaks, 4, 8)]
+        line["nm_sweep"] = bench_nm_sweep(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
     if rank == 0:

@@ -316,6 +316,29 @@ def test_ablation_masked_grad(n_out, k, n, m, t, only_dw):
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
 
 
+def test_dense_to_sparse_switch():
+    """The schedule the pages compare against sparse-from-scratch ([de] §4):
+    the same masters run dense ternary (N = M) first and then 2:4 and 6:8.
+    Each pattern is its own prepared layer; switching is preparing the masters
+    into the other one, and every stage matches the oracle."""
+    n_out, k, t = 264, 384, 40
+    w = synth.master_weights(n_out, k, 91)
+    x = synth.activations(t, k, 92)
+    xq_ref, ap_ref = oracle.act_quant(x)
+    for n, m in [(4, 4), (8, 8), (2, 4), (6, 8)]:
+        layer = sbl.Layer.allocate(n_out, k, n, m)
+        sbl.prepare_weights(layer, _dev(w))
+        ref = _check_prepared(layer, w, n, m)
+        y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+        acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+        ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+        sbl.forward(layer, _dev(x), t, y, acc_debug=acc, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(acc.cpu().numpy(), oracle.gemm_acc(xq_ref, ref["weff"]))
+        if n == m:  # dense ternary: nothing pruned
+            assert (bd.mask(layer) == (1 << m) - 1).all()
+
+
 @pytest.mark.parametrize("fill", ["random", "ones", "zeros"])
 def test_prepare_on_uninitialised_blob_and_repeats(fill):
     """The prepare kernel's grid barrier keeps its state in the blob's scratch
