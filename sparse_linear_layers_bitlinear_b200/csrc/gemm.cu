@@ -95,15 +95,21 @@ static cudaError_t pair_setup(int num_sms, int* max_clusters_out) {
   return cudaSuccess;
 }
 
+// pdl: launch with programmatic stream serialisation (the kernel's producer
+// waits for the predecessor before its first load).
 template <class Cfg>
 static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
-                               const typename Cfg::Params& p, int m_rows, int n_cols, int num_sms, cudaStream_t s) {
+                               const typename Cfg::Params& p, int m_rows, int n_cols, int num_sms, cudaStream_t s,
+                               bool pdl = false) {
   int max_clusters = 0;
   const cudaError_t err = pair_setup<Cfg>(num_sms, &max_clusters);
   if (err != cudaSuccess) return err;
   const int tiles = ((m_rows + 255) / 256) * ((n_cols + Cfg::BN - 1) / Cfg::BN);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
   if (pairs <= 0) return cudaSuccess;
+  if (pdl)
+    return launch_pdl(k_gemm_pair<Cfg>, dim3(2 * pairs), dim3(pair_threads<Cfg>()), pair_smem_bytes<Cfg>(), s, a, b,
+                      e, e, p);
   k_gemm_pair<Cfg><<<2 * pairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a, b, e, e, p);
   return cudaGetLastError();
 }
@@ -138,8 +144,8 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
         !encode_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 256, meta_bytes / 256, 256, 256, 16,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
-    return acc ? launch_pair<CfgPairSparse<true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s)
-               : launch_pair<CfgPairSparse<false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s);
+    return acc ? launch_pair<CfgPairSparse<true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true)
+               : launch_pair<CfgPairSparse<false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true);
   }
   // Dense int8 over W_eff codes.  Tile width: 256 tokens unless 192 leaves a
   // fuller last wave of pair tiles.
@@ -157,10 +163,10 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
       !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (narrow)
-    return acc ? launch_pair<CfgPairDense<true, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s)
-               : launch_pair<CfgPairDense<false, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s);
-  return acc ? launch_pair<CfgPairDense<true, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s)
-             : launch_pair<CfgPairDense<false, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s);
+    return acc ? launch_pair<CfgPairDense<true, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true)
+               : launch_pair<CfgPairDense<false, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true);
+  return acc ? launch_pair<CfgPairDense<true, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true)
+             : launch_pair<CfgPairDense<false, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true);
 }
 
 // ---------------------------------------------------------------------------

@@ -111,6 +111,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<Cfg>(),
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
+      // A forward launch may start while the activation quantiser before it
+      // still runs (programmatic dependent launch): wait for it before the
+      // first load.  A no-op for launches without a programmatic dependency.
+      pdl_wait();
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       const uint32_t leader_full0 = map_to_rank(&tail->full[0], 0);

@@ -166,7 +166,9 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
                             fused ? xscale_out : nullptr, status, sms, s);
     return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
   }
-  cudaError_t e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s);
+  // the forward GEMM is launched with programmatic dependent launch and waits
+  // for the quantiser's outputs itself, so the quantiser lets it launch early
+  cudaError_t e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true);
   if (e != cudaSuccess) return SBL_ERR_CUDA;
   if (is_24(layer->n, layer->m)) {
     e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
