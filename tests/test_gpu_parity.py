@@ -339,6 +339,70 @@ def test_dense_to_sparse_switch():
             assert (bd.mask(layer) == (1 << m) - 1).all()
 
 
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+def test_maximum_row_length(n, m):
+    """k at the library's limit (131072: |acc| <= 127 k stays exactly
+    representable in fp32): prepare, the long-row activation quantiser, the
+    forward GEMM over 512 k blocks and both backward products."""
+    n_out, k, t = 16, 131072, 5
+    w = synth.master_weights(n_out, k, 71)
+    x = synth.activations(t, k, 72)
+    dy = synth.upstream_grad(t, n_out, 73)
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    ref = _check_prepared(layer, w, n, m)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), oracle.dequant(acc_ref, ap_ref, ref["g"]).view(np.uint32))
+    dx = torch.empty((t, k), dtype=torch.float32, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, dx, dw, sbl.SBL_GRAD_F32)
+    torch.cuda.synchronize()
+    _close(dx.cpu().numpy(), oracle.grad_x(dy, ref["weff"], ref["g"]))
+    _close(dw.cpu().numpy(), oracle.grad_w(dy, x))
+    with pytest.raises(sbl.SblError):  # one step beyond the limit is refused before anything runs
+        sbl.Layer.allocate(n_out, k + 64, n, m)
+
+
+def test_degenerate_all_zero_inputs():
+    """All-zero masters give gamma = 0, so g = 1e-5 and every code 0; all-zero
+    activations give a' = 1e-5 and zero codes; all-zero upstream gradients
+    give zero gradients.  Every output is exactly 0 and no error is raised."""
+    n_out, k, t = 264, 320, 33
+    for n, m in [(2, 4), (6, 8)]:
+        w = torch.zeros((n_out, k), dtype=torch.bfloat16)
+        x = torch.zeros((t, k), dtype=torch.bfloat16)
+        dy = torch.zeros((t, n_out), dtype=torch.bfloat16)
+        layer = sbl.Layer.allocate(n_out, k, n, m)
+        sbl.prepare_weights(layer, _dev(w))
+        torch.cuda.synchronize()
+        ref = _check_prepared(layer, w, n, m)
+        gamma, g, _ = bd.header_scalars(layer)
+        assert gamma == 0.0 and np.float32(g) == np.float32(1e-5)
+        assert not ref["weff"].any()
+        assert (bd.mask(layer) == oracle.nm_mask(synth.bits(w), n, m)).all()  # all ties: lowest indices
+        y = torch.full((t, n_out), 7.0, dtype=torch.float32, device="cuda")
+        xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+        ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+        sbl.forward(layer, _dev(x), t, y, xq, ap)
+        dx = torch.full((t, k), 7.0, dtype=torch.float32, device="cuda")
+        dw = torch.full((n_out, k), 7.0, dtype=torch.float32, device="cuda")
+        sbl.backward(layer, _dev(x), _dev(dy), t, dx, dw, sbl.SBL_GRAD_F32)
+        torch.cuda.synchronize()
+        assert (y == 0).all() and (xq == 0).all() and (dx == 0).all() and (dw == 0).all()
+        assert np.array_equal(ap.cpu().numpy(), np.full(t, np.float32(1e-5)))
+        assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
 @pytest.mark.parametrize("fill", ["random", "ones", "zeros"])
 def test_prepare_on_uninitialised_blob_and_repeats(fill):
     """The prepare kernel's grid barrier keeps its state in the blob's scratch
