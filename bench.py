@@ -197,35 +197,78 @@ def replica_seed(rank: int, rotation: int, tensor: int) -> int:
 # CPU oracle baseline (bounded sample, extrapolated linearly in tokens)
 # ---------------------------------------------------------------------------
 def oracle_sample(wb, xb, dyb, n, m, tokens):
+    """Seconds for (prepare + act-quant over the whole batch, fwd + dX + dW over `tokens` tokens)."""
     import oracle
 
     t0 = time.perf_counter()
     p = oracle.prepare(wb, n, m)
     xq, ap = oracle.act_quant(xb)
-    t_fixed = time.perf_counter() - t0  # prepare + act-quant over the whole batch
+    t_fixed = time.perf_counter() - t0
     t1 = time.perf_counter()
     acc = oracle.gemm_acc(xq[:tokens], p["weff"])
     oracle.dequant(acc, ap[:tokens], p["g"])
     oracle.grad_x(dyb[:tokens], p["weff"], p["g"])
     oracle.grad_w(dyb[:tokens], xb[:tokens])
-    t_tok = (time.perf_counter() - t1) / tokens
-    return t_fixed, t_tok
+    return t_fixed, time.perf_counter() - t1
 
 
-def cpu_baseline(T, K, N, n, m, target_s=15.0):
+class OracleFit:
+    """Token-sampled oracle step time.
+
+    The token part is linear in tokens plus a token-independent share (the
+    n_out x k fp64 dW buffer is allocated and zeroed whatever the sample), so
+    it is fitted from two sample sizes: intercept + slope * tokens.  `tokens`
+    is sized so one sample takes about `target_s`.
+    """
+
+    def __init__(self, wb, xb, dyb, T, n, m, target_s):
+        self.args = (wb, xb, dyb, n, m)
+        self.T = T
+        lo = min(8, T)
+        _, v_lo = oracle_sample(*self.args, lo)
+        mid = min(64, T)
+        f_mid, v_mid = oracle_sample(*self.args, mid)
+        # size from the per-token cost at `mid` (intercept included): an upper
+        # bound on the slope, so the sample stays within its target
+        self.tokens = int(max(mid, min(T, (target_s - f_mid) / max(v_mid / mid, 1e-9))))
+        self.lo, self.v_lo = lo, v_lo
+        self.step_s = self.sample()
+
+    def sample(self):
+        """One timed sample; returns the extrapolated full-step seconds."""
+        f, v = oracle_sample(*self.args, self.tokens)
+        if self.tokens > self.lo:
+            slope = (v - self.v_lo) / (self.tokens - self.lo)
+            intercept = max(0.0, v - slope * self.tokens)
+        else:
+            slope, intercept = v / self.tokens, 0.0
+        return f + intercept + self.T * slope
+
+    def describe(self, step_s):
+        return (f"prepare and act-quant over the full batch, then fwd + dX + dW for {self.tokens} of {self.T} "
+                f"tokens; the token part fitted as intercept + slope x tokens from samples of {self.lo} and "
+                f"{self.tokens} tokens and extrapolated to {self.T} ({step_s:.1f} s per full step)")
+
+
+def cpu_baseline(T, K, N, n, m, target_s=12.0, target_1t_s=10.0):
+    """The oracle on all host cores, and on one thread beside it."""
     import oracle
     from sparse_linear_layers_bitlinear_b200 import synth
 
     wb = synth.bits(synth.master_weights(N, K, 0))
     xb = synth.bits(synth.activations(T, K, 1))
     dyb = synth.bits(synth.upstream_grad(T, N, 2))
-    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, 4)
-    tokens = int(max(4, min(T, (target_s - t_fixed) / max(t_tok, 1e-9))))
-    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, tokens)
-    step_s = t_fixed + T * t_tok
-    return {"value": T / step_s, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"prepare and act-quant over the full batch, then fwd + dX + dW for {tokens} of {T} tokens; "
-                      f"step time extrapolated linearly in tokens ({step_s:.1f} s per full step)"}
+    cores = oracle.threads()
+    fit = OracleFit(wb, xb, dyb, T, n, m, target_s)
+    oracle.set_threads(1)
+    try:
+        fit_1t = OracleFit(wb, xb, dyb, T, n, m, target_1t_s)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": T / fit.step_s, "unit": UNIT, "cores": cores, "nproc": os.cpu_count(), "kind": "oracle",
+            "sample": fit.describe(fit.step_s),
+            "single_thread": {"value": T / fit_1t.step_s, "unit": UNIT, "cores": 1,
+                              "sample": fit_1t.describe(fit_1t.step_s)}}
 
 
 def run_reference(args):
@@ -238,19 +281,14 @@ def run_reference(args):
     xb = synth.bits(synth.activations(T, K, 1))
     dyb = synth.bits(synth.upstream_grad(T, N, 2))
     # size each step's token sample so the whole run stays within ~2 minutes
-    t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, 2)
-    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
-    tokens = int(max(1, min(T, (per_step - t_fixed) / max(t_tok, 1e-9))))
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup + 2))
+    fit = OracleFit(wb, xb, dyb, T, n, m, per_step)
     for _ in range(args.warmup):
-        oracle_sample(wb, xb, dyb, n, m, tokens)
-    est = []
-    for _ in range(args.steps):
-        t_fixed, t_tok = oracle_sample(wb, xb, dyb, n, m, tokens)
-        est.append(t_fixed + T * t_tok)
+        fit.sample()
+    est = [fit.sample() for _ in range(args.steps)]
     step_s = statistics.mean(est)
     value = T / step_s
-    sample = (f"per step: prepare and act-quant over the full batch, fwd + dX + dW for {tokens} of {T} tokens; "
-              f"full-step time extrapolated linearly in tokens")
+    sample = "per step: " + fit.describe(step_s)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,

@@ -79,6 +79,7 @@ def _load():
         "sbo_grad_w_masked": (None, [P, P, P, I64, I64, I64, I, P]),
         "sbo_round_bf16": (None, [P, I64, P]),
         "sbo_threads": (I, []),
+        "sbo_set_threads": (None, [I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -106,6 +107,11 @@ def _u16(a) -> np.ndarray:
 
 def threads() -> int:
     return int(_load().sbo_threads())
+
+
+def set_threads(n: int) -> None:
+    """Set the OpenMP thread count for later oracle calls; results do not depend on it."""
+    _load().sbo_set_threads(int(n))
 
 
 def absmean_gamma(w) -> np.float32:

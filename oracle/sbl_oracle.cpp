@@ -124,6 +124,14 @@ int sbo_threads(void) {
 #endif
 }
 
+void sbo_set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
 // A1.  Exact sum over every master weight, masked ones included ([de] §2,
 // [fr] §2: quantisation happens before the mask), then one rounding.
 uint32_t sbo_absmean_bits(const uint16_t* w, int64_t numel) {

@@ -113,6 +113,11 @@ void sbo_round_bf16(const double* in, int64_t count, uint16_t* out);
 /* Number of OpenMP threads the oracle runs with. */
 int sbo_threads(void);
 
+/* Set the number of OpenMP threads for later calls from this host thread
+ * (values <= 0 are ignored).  Results do not depend on it: every sum is
+ * exact or taken in a fixed order per output. */
+void sbo_set_threads(int nthreads);
+
 #ifdef __cplusplus
 }
 #endif

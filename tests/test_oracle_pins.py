@@ -470,3 +470,32 @@ def test_round_bf16_matches_rational_rounding():
             assert gv == want, (v, gv, want)
     # ties go to even
     assert got[500] == 1.0 and got[501] == 1.0 + 2.0 ** -6 and got[502] == -1.0
+
+
+# ---------------------------------------------------------------------------
+# Thread count: every oracle sum is exact or runs in a fixed order per output,
+# so one thread and all threads give identical bits.
+# ---------------------------------------------------------------------------
+def test_results_do_not_depend_on_thread_count():
+    w = synth.master_weights(40, 96, seed=21)
+    x = synth.activations(7, 96, seed=22)
+    dy = synth.upstream_grad(7, 40, seed=23)
+
+    def run():
+        out = oracle.forward(w, x, 2, 4)
+        dx = oracle.grad_x(dy, out["weff"], out["g"])
+        dw = oracle.grad_w(dy, x)
+        return out, dx, dw
+
+    cores = oracle.threads()
+    many = run()
+    oracle.set_threads(1)
+    try:
+        assert oracle.threads() == 1 or cores == 1
+        one = run()
+    finally:
+        oracle.set_threads(cores)
+    assert oracle.threads() == cores
+    for key in ("g", "mask", "weff", "xq", "a_prime", "acc", "y"):
+        assert np.array_equal(np.asarray(many[0][key]), np.asarray(one[0][key])), key
+    assert np.array_equal(many[1], one[1]) and np.array_equal(many[2], one[2])
