@@ -212,6 +212,12 @@ enum {
 /* Library version string. */
 const char* sbl_version(void);
 
+/* Number of kernels this process has launched through the library so far
+ * (every successful launch submission, on any device and stream; memsets and
+ * copies are not counted).  A host-side counter for accounting: callers take
+ * the difference across a region.  Never fails. */
+uint64_t sbl_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

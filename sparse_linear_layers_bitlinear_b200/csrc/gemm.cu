@@ -59,7 +59,7 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, const t
   const int grid = tiles < num_sms ? tiles : num_sms;
   if (grid <= 0) return cudaSuccess;
   k_gemm_tc<Cfg><<<grid, kGemmThreads, smem, s>>>(a, b, p);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 // Pair kernels: grid = two CTAs per concurrently resident cluster, capped by
@@ -111,7 +111,7 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const
     return launch_pdl(k_gemm_pair<Cfg>, dim3(2 * pairs), dim3(pair_threads<Cfg>()), pair_smem_bytes<Cfg>(), s, a, b,
                       e, e, p);
   k_gemm_pair<Cfg><<<2 * pairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a, b, e, e, p);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 // ---------------------------------------------------------------------------
@@ -304,7 +304,7 @@ cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16
   std::copy(sch.off.begin(), sch.off.end(), p.sched_off);
   std::copy(sch.ids.begin(), sch.ids.end(), p.sched);
   k_gemm_pair<Cfg><<<2 * npairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
-  err = cudaGetLastError();
+  err = counted(cudaGetLastError());
   *done = err == cudaSuccess;
   return err;
 }
@@ -341,7 +341,7 @@ __global__ void k_selftest_wait(uint32_t* status, uint64_t limit_ns) {
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s) {
   k_selftest_wait<<<1, 32, 0, s>>>(status, limit_ns);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace sbl

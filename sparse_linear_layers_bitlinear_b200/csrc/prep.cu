@@ -768,7 +768,7 @@ static cudaError_t launch_prepare_m(const cudaLaunchConfig_t& cfg, const PrepArg
   static const cudaError_t attr_err =
       cudaFuncSetAttribute(k_prepare<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kPrepSmem));
   if (attr_err != cudaSuccess) return attr_err;
-  return cudaLaunchKernelEx(&cfg, k_prepare<M>, a);
+  return counted(cudaLaunchKernelEx(&cfg, k_prepare<M>, a));
 }
 
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,

@@ -1,5 +1,6 @@
 // C ABI of the Sparse-BitLinear library: argument checks, prepared-blob
 // layout and dispatch to the kernels.  See include/sbl.h for the contract.
+#include <atomic>
 #include <cstddef>
 #include <cstring>
 #include <mutex>
@@ -7,6 +8,13 @@
 #include "sbl_kernels.h"
 
 using namespace sbl;
+
+namespace sbl {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace sbl
 
 namespace {
 
@@ -70,6 +78,8 @@ T* at(const sbl_layer* layer, uint64_t off) {
 extern "C" {
 
 const char* sbl_version(void) { return "sbl 0.1 (sm_100a)"; }
+
+uint64_t sbl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t flags, sbl_blob_layout* out) {
   if (out == nullptr) return SBL_ERR_INVALID_ARG;

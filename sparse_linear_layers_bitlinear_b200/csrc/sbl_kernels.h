@@ -9,6 +9,13 @@
 
 namespace sbl {
 
+// Host-side count of submitted kernel launches (sbl_launch_count).
+void note_launch();
+inline cudaError_t counted(cudaError_t e) {
+  if (e == cudaSuccess) note_launch();
+  return e;
+}
+
 // Launch with programmatic stream serialisation: the kernel may start before
 // its predecessor on the stream completes and must call pdl_wait() before it
 // touches that predecessor's data, and before it completes.
@@ -25,7 +32,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  return counted(cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...));
 }
 
 // Destinations of the pack pass (device pointers; optional ones may be null).

@@ -84,6 +84,7 @@ SIGNATURES = {
     "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
     "sbl_version": (ctypes.c_char_p, []),
+    "sbl_launch_count": (ctypes.c_uint64, []),
 }
 
 _lib = None
@@ -218,6 +219,11 @@ def selftest_wait_timeout(status_dev, limit_ns: int, stream=None):
 
 def version() -> str:
     return lib().sbl_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process (sbl_launch_count)."""
+    return int(lib().sbl_launch_count())
 
 
 class SparseBitLinear:

@@ -104,6 +104,7 @@ def test_workspace_bytes(lib):
 
 def test_entry_points_validate_before_touching_the_device(lib):
     # These return before any CUDA call, so they run on a machine without a GPU.
+    launched_before = sbl.launch_count()
     layer = sbl.sbl_layer(256, 256, 2, 4, 0, 0x1000)
     assert lib.sbl_prepare_weights(None, ctypes.c_void_p(0x2000), None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_prepare_weights(ctypes.byref(layer), None, None) == sbl.SBL_ERR_INVALID_ARG
@@ -121,3 +122,5 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 0, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 1 << 7, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_selftest_wait_timeout(None, 1000, None) == sbl.SBL_ERR_INVALID_ARG
+    # rejected calls enqueue nothing, so they launch nothing
+    assert sbl.launch_count() == launched_before

@@ -440,3 +440,28 @@ def test_act_quant_row_lengths(k):
     xq_ref, ap_ref = oracle.act_quant(x)
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
     assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+
+
+def test_launch_count_per_step():
+    """The library's own launch counter: one prepare, two forward kernels
+    (act-quant, 2:4 GEMM) and one backward launch per training step."""
+    n_out, k, t = 512, 768, 320
+    w = synth.master_weights(n_out, k, 71, device="cuda")
+    x = synth.activations(t, k, 72, device="cuda")
+    dy = synth.upstream_grad(t, n_out, 73, device="cuda")
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, device="cuda")
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    dx = torch.empty((t, k), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
+    c0 = sbl.launch_count()
+    sbl.prepare_weights(layer, w)
+    c1 = sbl.launch_count()
+    sbl.forward(layer, x, t, y, workspace=ws)
+    c2 = sbl.launch_count()
+    sbl.backward(layer, x, dy, t, dx, dw, 0)
+    c3 = sbl.launch_count()
+    sbl.forward(layer, x, 0, y, workspace=ws)  # empty batch: nothing to launch
+    c4 = sbl.launch_count()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    assert (c1 - c0, c2 - c1, c3 - c2, c4 - c3) == (1, 2, 1, 0)
