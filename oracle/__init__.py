@@ -78,6 +78,7 @@ def _load():
         "sbo_grad_w_at": (ctypes.c_double, [P, P, I64, I64, I64, I64, I64]),
         "sbo_grad_w_masked": (None, [P, P, P, I64, I64, I64, I, P]),
         "sbo_round_bf16": (None, [P, I64, P]),
+        "sbo_dequant_act": (None, [P, P, I64, I64, P]),
         "sbo_threads": (I, []),
         "sbo_set_threads": (None, [I]),
     }
@@ -257,6 +258,22 @@ def grad_w_masked(dy, x, mask: np.ndarray, m: int) -> np.ndarray:
     out = np.zeros((n_out, k), dtype=np.float64)
     _load().sbo_grad_w_masked(_ptr(dy), _ptr(x), _ptr(mask), t, n_out, k, m, _ptr(out))
     return out
+
+
+def dequant_act(xq: np.ndarray, a_prime: np.ndarray) -> np.ndarray:
+    """dW operand of the detach-form STE: xhat = RN_bf16(xq * a' / 127), bf16 bits [t, k]."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    ap = np.ascontiguousarray(a_prime, dtype=np.float32)
+    t, k = xq.shape
+    out = np.zeros((t, k), dtype=np.uint16)
+    _load().sbo_dequant_act(_ptr(xq), _ptr(ap), t, k, _ptr(out))
+    return out
+
+
+def grad_w_quant_x(dy, x) -> np.ndarray:
+    """dW = dY^T . xhat, xhat the dequantised activations of x (SBL_DW_QUANT_X reading)."""
+    xq, ap = act_quant(x)
+    return grad_w(dy, dequant_act(xq, ap))
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:

@@ -371,6 +371,18 @@ void sbo_grad_w_masked(const uint16_t* dy, const uint16_t* x, const uint8_t* mas
       if (!((mask[o * groups + c / m] >> (c % m)) & 1u)) dw[o * k + c] = 0.0;
 }
 
+// Detach-form STE operand for dW: xhat = RN_bf16(xq * a' / 127), one
+// rounding of the exact value (see the header for why fp64 suffices).
+void sbo_dequant_act(const int8_t* xq, const float* a_prime, int64_t t, int64_t k, uint16_t* xhat) {
+#pragma omp parallel for schedule(static)
+  for (int64_t row = 0; row < t; ++row) {
+    for (int64_t c = 0; c < k; ++c) {
+      const double v = double(xq[row * k + c]) * double(a_prime[row]) / 127.0;
+      sbo_round_bf16(&v, 1, xhat + row * k + c);
+    }
+  }
+}
+
 void sbo_round_bf16(const double* in, int64_t count, uint16_t* out) {
   for (int64_t i = 0; i < count; ++i) {
     const double d = in[i];

@@ -107,6 +107,15 @@ double sbo_grad_w_at(const uint16_t* dy, const uint16_t* x, int64_t t,
 void sbo_grad_w_masked(const uint16_t* dy, const uint16_t* x, const uint8_t* mask,
                        int64_t t, int64_t n_out, int64_t k, int m, double* dw);
 
+/* Dequantised activations, the dW operand of the SBL_DW_QUANT_X reading of
+ * the STE for the quantiser ([ja] 2.2 "Dual STE": the standard STE for the
+ * quantisation function; detach form): xhat = RN_bf16(xq * a' / 127) taken
+ * exactly, bf16 bit patterns out.  The fp64 product is exact (8 x 24 bits);
+ * the fp64 quotient's one rounding cannot cross a bf16 rounding boundary:
+ * a non-dyadic quotient lies at least ~2^-32 relative from every 9-bit
+ * dyadic, and a dyadic one has at most 31 significant bits, so it is exact. */
+void sbo_dequant_act(const int8_t* xq, const float* a_prime, int64_t t, int64_t k, uint16_t* xhat);
+
 /* Round fp64 to bf16 (round to nearest, ties to even), bit patterns out. */
 void sbo_round_bf16(const double* in, int64_t count, uint16_t* out);
 

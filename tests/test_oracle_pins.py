@@ -499,3 +499,53 @@ def test_results_do_not_depend_on_thread_count():
     for key in ("g", "mask", "weff", "xq", "a_prime", "acc", "y"):
         assert np.array_equal(np.asarray(many[0][key]), np.asarray(one[0][key])), key
     assert np.array_equal(many[1], one[1]) and np.array_equal(many[2], one[2])
+
+
+# ---------------------------------------------------------------------------
+# Detach-form STE operand for dW (SBL_DW_QUANT_X): xhat = RN_bf16(xq a' / 127)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", [31, 32])
+def test_dequant_act_equals_exact_rational_rounding(seed):
+    x = synth.activations(6, 200, seed=seed)
+    xb = synth.bits(x).copy()
+    xb[0, :3] = [0x0000, 0x8000, 0x3F80]        # zeros and 1.0
+    xb[1, :] = 0                                 # all-zero row: a' = 1e-5
+    xb[2, 5] = 0x7F7F                            # near the bf16 maximum
+    xq, ap = oracle.act_quant(xb)
+    got = oracle.dequant_act(xq, ap)
+    for r in range(xq.shape[0]):
+        for c in range(xq.shape[1]):
+            want = _fraction_to_bf16_value(Fraction(int(xq[r, c])) * Fraction(float(ap[r])) / 127)
+            gv = float(_bf16_float(got[r, c:c + 1])[0])
+            assert gv == want, (r, c, int(xq[r, c]), float(ap[r]), gv, want)
+            if xq[r, c] == 0:
+                assert got[r, c] == 0  # +0, whatever the sign of x
+
+
+def test_dequant_act_invariants():
+    x = synth.activations(16, 256, seed=33)
+    xb = synth.bits(x)
+    xq, ap = oracle.act_quant(xb)
+    xhat = _bf16_float(oracle.dequant_act(xq, ap)).reshape(xq.shape)
+    xf = _bf16_float(xb).reshape(xq.shape)
+    for r in range(xq.shape[0]):
+        j = int(np.argmax(np.abs(xf[r])))
+        # the row's absmax element has code +-127 and comes back exactly
+        assert abs(int(xq[r, j])) == 127 and xhat[r, j] == xf[r, j]
+        # quantisation error: half a step a'/127, plus the bf16 rounding of xhat
+        err = np.abs(xhat[r] - xf[r])
+        bound = float(ap[r]) / 254.0 * (1 + 1e-6) + np.abs(xhat[r]) * 2.0 ** -8
+        assert np.all(err <= bound)
+        assert np.all(np.sign(xhat[r]) * np.sign(xf[r]) >= 0)
+
+
+def test_grad_w_quant_x_uses_the_dequantised_operand():
+    dy = synth.upstream_grad(9, 24, seed=34)
+    x = synth.activations(9, 64, seed=35)
+    dw_q = oracle.grad_w_quant_x(dy, x)
+    xq, ap = oracle.act_quant(x)
+    xhat = _bf16_float(oracle.dequant_act(xq, ap)).reshape(xq.shape)
+    ref = _bf16_float(synth.bits(dy)).reshape(9, 24).T @ xhat
+    assert np.allclose(dw_q, ref, rtol=1e-12, atol=1e-12)
+    # and it is not the raw-X gradient
+    assert not np.allclose(dw_q, oracle.grad_w(dy, x), rtol=1e-4, atol=0)
