@@ -79,8 +79,13 @@ enum {
   SBL_GRAD_F32 = 1u << 1,   /* dx and dw are fp32 instead of bf16 */
   SBL_NO_DX = 1u << 2,      /* skip dX (dx may be NULL) */
   SBL_NO_DW = 1u << 3,      /* skip dW (dw may be NULL) */
-  SBL_MASKED_GRAD = 1u << 4 /* ablation the pages report ([de] 4, [fr] 5): block the
+  SBL_MASKED_GRAD = 1u << 4, /* ablation the pages report ([de] 4, [fr] 5): block the
                                gradient of pruned weights, dw = (dy^T . x) * mask */
+  SBL_DW_QUANT_X = 1u << 5   /* reading of the standard STE for the quantiser ([ja] 2.2
+                               "Dual STE") in its detach form: dw = dy^T . xhat with
+                               xhat = RN_bf16(xq * a' / 127) (xq, a' as in sbl_forward),
+                               rounded once from the exact value; needs a workspace
+                               (sbl_backward_ws) */
 };
 
 /* One Sparse-BitLinear layer: shapes, pattern and the caller-owned device
@@ -186,6 +191,21 @@ sbl_status sbl_forward_noalloc(const sbl_layer* layer, const void* x, int64_t t,
  * cores.  SBL_NO_DX / SBL_NO_DW skip one of the two products. */
 sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
                         uint32_t flags, sbl_stream_t stream);
+
+/* Bytes of device workspace sbl_backward_ws needs for these flags: t*k*2
+ * (xhat, bf16 [t, k]) with SBL_DW_QUANT_X and dW wanted, else 0. */
+size_t sbl_backward_workspace_bytes(int64_t t, int64_t k, uint32_t flags);
+
+/* sbl_backward with a caller-owned device workspace of at least
+ * sbl_backward_workspace_bytes(t, layer->k, flags) bytes (16-byte aligned;
+ * NULL when that is 0).  With SBL_DW_QUANT_X the activations are quantised
+ * again from x (the same codes and a' as the forward pass) and written back
+ * as xhat into the workspace, which then holds xhat [t, k] when the call's
+ * work is done; dw = dy^T . xhat.  dX is unchanged.  Errors: as sbl_backward,
+ * plus SBL_ERR_INVALID_ARG when SBL_DW_QUANT_X needs a workspace and it is
+ * NULL.  sbl_backward(...) is sbl_backward_ws(..., NULL, stream). */
+sbl_status sbl_backward_ws(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
+                           uint32_t flags, void* workspace, sbl_stream_t stream);
 
 /* Synchronises `stream`, then maps the layer's device status word to a code:
  * SBL_OK, SBL_ERR_NONFINITE or SBL_ERR_TIMEOUT.  *bits_out (may be NULL)

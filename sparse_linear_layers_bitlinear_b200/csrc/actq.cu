@@ -12,6 +12,10 @@
 // kernel before it, and it waits for that kernel (which may have written x,
 // or reset the status word) before it reads anything.  With early_trigger it
 // then lets the next kernel (the decode GEMV) launch at once.
+//
+// DEQ = true is the same pass writing the dequantised activations
+// xhat = RN_bf16(xq * a' / 127) instead of the codes: the dW operand of the
+// detach-form STE (SBL_DW_QUANT_X).
 #include "sbl_kernels.h"
 
 #include "sbl_device.cuh"
@@ -22,9 +26,19 @@ namespace sbl {
 constexpr int kActThreads = 128;
 constexpr int kMaxR = 16;  // rows up to 16384 elements stay in registers
 
-template <int R>
+// Stores the quantised (or, with DEQ, dequantised) form of 8 elements.
+template <bool DEQ>
+__device__ __forceinline__ void store_quantised(void* out, int64_t row, int64_t nvec, int64_t i, const uint4 v,
+                                                float ap) {
+  if constexpr (DEQ)
+    reinterpret_cast<uint4*>(out)[row * nvec + i] = dequantise8(v, ap);
+  else
+    reinterpret_cast<uint2*>(out)[row * nvec + i] = quantise8(v, ap);
+}
+
+template <int R, bool DEQ>
 __global__ void __launch_bounds__(kActThreads)
-    k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
+    k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, void* __restrict__ out,
                      float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
   // x may be the output of the kernel before this one: bring this block's
   // rows towards L2 while that kernel runs, then wait for it.
@@ -68,14 +82,13 @@ __global__ void __launch_bounds__(kActThreads)
     __syncthreads();  // s_max is rewritten by the next row
     const float ap = fmaxf(amax, 1e-5f);
     if (tid == 0) {
-      a_prime[row] = ap;
+      if (!DEQ) a_prime[row] = ap;
       if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
-    uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = int64_t(r) * kActThreads + tid;
-      if (i < nvec) dst[i] = quantise8(v[r], ap);
+      if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], ap);
     }
   }
 }
@@ -83,8 +96,9 @@ __global__ void __launch_bounds__(kActThreads)
 // Long rows: one warp per row, absmax pass then a second (L1/L2) pass.
 constexpr int kActWarps = 8;
 
+template <bool DEQ>
 __global__ void __launch_bounds__(kActWarps * 32)
-    k_act_quant_long(const uint4* __restrict__ x, int64_t t, int64_t nvec, int8_t* __restrict__ xq,
+    k_act_quant_long(const uint4* __restrict__ x, int64_t t, int64_t nvec, void* __restrict__ out,
                      float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
   pdl_wait();  // x may be the output of the kernel before this one
   if (early_trigger) pdl_trigger();
@@ -106,42 +120,51 @@ __global__ void __launch_bounds__(kActWarps * 32)
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (__any_sync(0xffffffffu, bad != 0) && lane == 0) raise_status(status, SBL_STATUS_NONFINITE_X);
     const float ap = fmaxf(amax, 1e-5f);
-    if (lane == 0) a_prime[row] = ap;
-    uint2* dst = reinterpret_cast<uint2*>(xq + row * nvec * 8);
-    for (int64_t j = lane; j < nvec; j += 32) dst[j] = quantise8(__ldg(src + j), ap);
+    if (!DEQ && lane == 0) a_prime[row] = ap;
+    for (int64_t j = lane; j < nvec; j += 32) store_quantised<DEQ>(out, row, nvec, j, __ldg(src + j), ap);
   }
 }
 
-template <int R>
-static cudaError_t launch_rows(const uint4* x, int64_t t, int64_t nvec, int8_t* xq, float* ap, uint32_t* status,
+template <int R, bool DEQ>
+static cudaError_t launch_rows(const uint4* x, int64_t t, int64_t nvec, void* out, float* ap, uint32_t* status,
                                int num_sms, cudaStream_t s, int early) {
   int64_t blocks = t;
   const int64_t cap = int64_t(num_sms) * 64;
   if (blocks > cap) blocks = cap;
-  return launch_pdl(k_act_quant_rows<R>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t, nvec,
-                    xq, ap, status, early);
+  return launch_pdl(k_act_quant_rows<R, DEQ>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t,
+                    nvec, out, ap, status, early);
 }
 
-cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
-                             int num_sms, cudaStream_t s, bool early_trigger) {
-  const int early = early_trigger ? 1 : 0;
+template <bool DEQ>
+static cudaError_t launch_quant(const uint16_t* x, int64_t t, int64_t k, void* out, float* a_prime, uint32_t* status,
+                                int num_sms, cudaStream_t s, int early) {
   if (t <= 0) return cudaSuccess;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const int64_t nvec = k / 8;
   const int64_t r = (nvec + kActThreads - 1) / kActThreads;
-  if (r <= 1) return launch_rows<1>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 2) return launch_rows<2>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 3) return launch_rows<3>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 4) return launch_rows<4>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 6) return launch_rows<6>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 8) return launch_rows<8>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= 12) return launch_rows<12>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
-  if (r <= kMaxR) return launch_rows<kMaxR>(xv, t, nvec, xq, a_prime, status, num_sms, s, early);
+  if (r <= 1) return launch_rows<1, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 2) return launch_rows<2, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 3) return launch_rows<3, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 4) return launch_rows<4, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 6) return launch_rows<6, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 8) return launch_rows<8, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= 12) return launch_rows<12, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (r <= kMaxR) return launch_rows<kMaxR, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
   int64_t blocks = (t + kActWarps - 1) / kActWarps;
   const int64_t cap = int64_t(num_sms) * 16;
   if (blocks > cap) blocks = cap;
-  return launch_pdl(k_act_quant_long, dim3(static_cast<unsigned>(blocks)), dim3(kActWarps * 32), 0, s, xv, t, nvec, xq,
-                    a_prime, status, early);
+  return launch_pdl(k_act_quant_long<DEQ>, dim3(static_cast<unsigned>(blocks)), dim3(kActWarps * 32), 0, s, xv, t,
+                    nvec, out, a_prime, status, early);
+}
+
+cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
+                             int num_sms, cudaStream_t s, bool early_trigger) {
+  return launch_quant<false>(x, t, k, xq, a_prime, status, num_sms, s, early_trigger ? 1 : 0);
+}
+
+cudaError_t launch_act_dequant(const uint16_t* x, int64_t t, int64_t k, uint16_t* xhat, uint32_t* status, int num_sms,
+                               cudaStream_t s) {
+  return launch_quant<true>(x, t, k, xhat, nullptr, status, num_sms, s, 0);
 }
 
 }  // namespace sbl

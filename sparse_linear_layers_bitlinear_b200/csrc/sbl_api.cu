@@ -20,7 +20,7 @@ namespace {
 
 constexpr int64_t kMaxK = 131072;  // keeps |acc| <= 127 * k below 2^24: (float)acc is exact
 constexpr uint32_t kLayerFlags = SBL_PACK_GEMV | SBL_MASK_FROM_QUANT;
-constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW | SBL_MASKED_GRAD;
+constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW | SBL_MASKED_GRAD | SBL_DW_QUANT_X;
 
 struct DeviceInfo {
   bool checked = false;
@@ -192,14 +192,28 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
+size_t sbl_backward_workspace_bytes(int64_t t, int64_t k, uint32_t flags) {
+  if (t <= 0 || k <= 0 || (flags & SBL_NO_DW) || !(flags & SBL_DW_QUANT_X)) return 0;
+  return size_t(t) * size_t(k) * 2;
+}
+
 sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
                         uint32_t flags, sbl_stream_t stream) {
+  return sbl_backward_ws(layer, x, dy, t, dx, dw, flags, nullptr, stream);
+}
+
+sbl_status sbl_backward_ws(const sbl_layer* layer, const void* x, const void* dy, int64_t t, void* dx, void* dw,
+                           uint32_t flags, void* workspace, sbl_stream_t stream) {
   sbl_blob_layout L;
   sbl_status st = check_layer(layer, &L);
   if (st != SBL_OK) return st;
   if ((flags & ~kBackwardFlags) != 0u) return SBL_ERR_INVALID_ARG;
   if (t < 0 || t > (int64_t(1) << 30)) return SBL_ERR_SHAPE;
   const bool want_dx = !(flags & SBL_NO_DX), want_dw = !(flags & SBL_NO_DW);
+  // the detach-form STE takes dW against xhat, written into the workspace
+  const bool quant_x = want_dw && (flags & SBL_DW_QUANT_X) && t > 0;
+  if (quant_x && workspace == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return SBL_ERR_ALIGN;
   const bool f32 = (flags & SBL_GRAD_F32) != 0u;
   // the blocked-gradient ablation multiplies dW by the mask section
   const uint8_t* dw_mask = (flags & SBL_MASKED_GRAD) ? at<const uint8_t>(layer, L.mask) : nullptr;
@@ -217,10 +231,17 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
     return SBL_OK;
   }
   uint32_t* status = at<uint32_t>(layer, L.status);
+  const void* x_dw = x;  // the dW operand: x, or xhat with SBL_DW_QUANT_X
+  if (quant_x) {
+    uint16_t* xhat = static_cast<uint16_t*>(workspace);
+    if (launch_act_dequant(static_cast<const uint16_t*>(x), t, layer->k, xhat, status, sms, s) != cudaSuccess)
+      return SBL_ERR_CUDA;
+    x_dw = xhat;
+  }
   if (want_dx && want_dw) {
     bool done = false;
     const cudaError_t e = launch_bf16_backward_dual(
-        f32, static_cast<const uint16_t*>(dy), at<const uint16_t>(layer, L.weff_bf16), static_cast<const uint16_t*>(x),
+        f32, static_cast<const uint16_t*>(dy), at<const uint16_t>(layer, L.weff_bf16), static_cast<const uint16_t*>(x_dw),
         t, layer->n_out, layer->k, at<const float>(layer, L.g), dx, dw, dw_mask, layer->m, status, sms, s, &done);
     if (e != cudaSuccess) return SBL_ERR_CUDA;
     if (done) return SBL_OK;
@@ -233,9 +254,9 @@ sbl_status sbl_backward(const sbl_layer* layer, const void* x, const void* dy, i
     if (e != cudaSuccess) return SBL_ERR_CUDA;
   }
   if (want_dw) {
-    // dW[n_out, k] = dY^T . X:  A = dY stored [K=t][M=n_out], B = X stored [K=t][N=k].
+    // dW[n_out, k] = dY^T . X (or xhat):  A = dY stored [K=t][M=n_out], B = X stored [K=t][N=k].
     const cudaError_t e = launch_bf16_gemm(true, true, f32, static_cast<const uint16_t*>(dy),
-                                           static_cast<const uint16_t*>(x), layer->n_out, layer->k, t, nullptr, dw,
+                                           static_cast<const uint16_t*>(x_dw), layer->n_out, layer->k, t, nullptr, dw,
                                            status, sms, s, dw_mask, layer->m);
     if (e != cudaSuccess) return SBL_ERR_CUDA;
   }

@@ -55,6 +55,11 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
                              int num_sms, cudaStream_t s, bool early_trigger = false);
 
+// The dequantised activations xhat = RN_bf16(xq * a' / 127), bf16 [t][k]: the
+// act-quant pass writing xhat instead of the codes (SBL_DW_QUANT_X).
+cudaError_t launch_act_dequant(const uint16_t* x, int64_t t, int64_t k, uint16_t* xhat, uint32_t* status, int num_sms,
+                               cudaStream_t s);
+
 // Forward GEMM + dequant.  sparse: codes = 2:4 kept values [n_out][k/2] and
 // meta = tensor-core metadata; dense: codes = W_eff int8 [n_out][k].
 cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,

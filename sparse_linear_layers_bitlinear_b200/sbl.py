@@ -39,6 +39,7 @@ SBL_GRAD_F32 = 1 << 1
 SBL_NO_DX = 1 << 2
 SBL_NO_DW = 1 << 3
 SBL_MASKED_GRAD = 1 << 4
+SBL_DW_QUANT_X = 1 << 5
 # device status bits
 SBL_STATUS_NONFINITE_W = 1 << 0
 SBL_STATUS_NONFINITE_X = 1 << 1
@@ -78,6 +79,8 @@ SIGNATURES = {
     "sbl_prepare_weights": (_I32, [_LP, _P, _P]),
     "sbl_forward": (_I32, [_LP, _P, _I64, _P, _P, _P, _P, _P, _P]),
     "sbl_backward": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P]),
+    "sbl_backward_ws": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P, _P]),
+    "sbl_backward_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _U32]),
     "sbl_forward_noalloc": (_I32, [_LP, _P, _I64, _P, _P, _P]),
     "sbl_read_status": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "sbl_clear_status": (_I32, [_LP, _P]),
@@ -187,10 +190,19 @@ def forward_noalloc(layer: Layer, x, t: int, y, acc_debug=None, stream=None):
            "sbl_forward_noalloc")
 
 
-def backward(layer: Layer, x, dy, t: int, dx, dw, flags: int = 0, stream=None):
+def backward(layer: Layer, x, dy, t: int, dx, dw, flags: int = 0, stream=None, workspace=None):
+    """sbl_backward, or sbl_backward_ws when a workspace is given (SBL_DW_QUANT_X needs one)."""
     cl = layer.c()
-    _check(lib().sbl_backward(ctypes.byref(cl), _ptr(x), _ptr(dy), t, _ptr(dx), _ptr(dw), flags, _stream(stream)),
-           "sbl_backward")
+    if workspace is None:
+        _check(lib().sbl_backward(ctypes.byref(cl), _ptr(x), _ptr(dy), t, _ptr(dx), _ptr(dw), flags,
+                                  _stream(stream)), "sbl_backward")
+    else:
+        _check(lib().sbl_backward_ws(ctypes.byref(cl), _ptr(x), _ptr(dy), t, _ptr(dx), _ptr(dw), flags,
+                                     _ptr(workspace), _stream(stream)), "sbl_backward_ws")
+
+
+def backward_workspace_bytes(t: int, k: int, flags: int) -> int:
+    return int(lib().sbl_backward_workspace_bytes(t, k, flags))
 
 
 def read_status(layer: Layer, stream=None):

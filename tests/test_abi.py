@@ -80,6 +80,22 @@ def test_ablation_flags_are_accepted_and_unknown_bits_rejected(lib):
         sbl.prepared_layout(264, 320, 2, 4, 1 << 5)
 
 
+def test_backward_workspace_for_the_quantised_x_operand(lib):
+    q = sbl.SBL_DW_QUANT_X
+    assert sbl.backward_workspace_bytes(40, 256, 0) == 0
+    assert sbl.backward_workspace_bytes(40, 256, q) == 40 * 256 * 2
+    assert sbl.backward_workspace_bytes(40, 256, q | sbl.SBL_NO_DW) == 0  # no dW, no operand
+    assert sbl.backward_workspace_bytes(0, 256, q) == 0
+    # rejected before anything touches a device
+    layer = sbl.sbl_layer(256, 256, 2, 4, 0, 0x1000)
+    p = ctypes.c_void_p
+    args = (ctypes.byref(layer), p(0x2000), p(0x3000), 4, p(0x4000), p(0x5000))
+    assert lib.sbl_backward(*args, q, None) == sbl.SBL_ERR_INVALID_ARG          # needs a workspace
+    assert lib.sbl_backward_ws(*args, q, None, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_backward_ws(*args, q, p(0x6008), None) == sbl.SBL_ERR_ALIGN
+    assert lib.sbl_backward_ws(*args, q | (1 << 6), p(0x6000), None) == sbl.SBL_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("args,code", [
     ((256, 256, 2, 3, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
     ((256, 256, 0, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),

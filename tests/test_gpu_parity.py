@@ -465,3 +465,63 @@ def test_launch_count_per_step():
     c4 = sbl.launch_count()
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
     assert (c1 - c0, c2 - c1, c3 - c2, c4 - c3) == (1, 2, 1, 0)
+
+
+@pytest.mark.parametrize("n_out,k,n,m,t", [(264, 320, 2, 4, 70), (136, 448, 6, 8, 33), (392, 832, 3, 8, 130)])
+@pytest.mark.parametrize("only_dw", [False, True])
+def test_dw_quant_x(n_out, k, n, m, t, only_dw):
+    """The detach-form reading of the STE for the quantiser: dW is taken
+    against xhat = RN_bf16(xq a' / 127), which the call leaves in its
+    workspace (bit-exact against the oracle); dX is the same as without it."""
+    seed = 5 * n_out + k + m
+    w = synth.master_weights(n_out, k, seed)
+    x = synth.activations(t, k, seed + 1)
+    dy = synth.upstream_grad(t, n_out, seed + 2)
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, _dev(w))
+    ref = oracle.prepare(w, n, m)
+    xq_ref, ap_ref = oracle.act_quant(x)
+    xhat_ref = oracle.dequant_act(xq_ref, ap_ref)
+    dw_ref = oracle.grad_w_quant_x(dy, x)
+    flags = sbl.SBL_DW_QUANT_X | (sbl.SBL_NO_DX if only_dw else 0)
+    nbytes = sbl.backward_workspace_bytes(t, k, flags)
+    assert nbytes == t * k * 2
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sbl.SblError):
+        sbl.backward(layer, _dev(x), _dev(dy), t, None, None, flags)  # no workspace
+    for f32 in (True, False):
+        dt = torch.float32 if f32 else torch.bfloat16
+        dx = None if only_dw else torch.empty((t, k), dtype=dt, device="cuda")
+        dw = torch.empty((n_out, k), dtype=dt, device="cuda")
+        sbl.backward(layer, _dev(x), _dev(dy), t, dx, dw, flags | (sbl.SBL_GRAD_F32 if f32 else 0), workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(ws.cpu().numpy().view(np.uint16).reshape(t, k), xhat_ref)
+        if f32:
+            _close(dw.cpu().numpy(), dw_ref)
+        else:
+            _close(bd.bf16_to_f64(dw), dw_ref, rtol=BF16_REL, atol=ATOL)
+        if not only_dw:
+            dx_plain = torch.empty_like(dx)
+            dw_plain = torch.empty_like(dw)
+            sbl.backward(layer, _dev(x), _dev(dy), t, dx_plain, dw_plain, sbl.SBL_GRAD_F32 if f32 else 0)
+            torch.cuda.synchronize()
+            assert torch.equal(dx, dx_plain)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+@pytest.mark.parametrize("k", [64, 2560, 16448])
+def test_dequant_act_row_lengths(k):
+    """xhat for a register-resident row length and for the long-row kernel."""
+    n_out, t = 8, 5
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 52)))
+    x = synth.activations(t, k, 53)
+    dy = synth.upstream_grad(t, n_out, 54)
+    ws = torch.empty((sbl.backward_workspace_bytes(t, k, sbl.SBL_DW_QUANT_X),), dtype=torch.uint8, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, None, dw, sbl.SBL_DW_QUANT_X | sbl.SBL_NO_DX | sbl.SBL_GRAD_F32,
+                 workspace=ws)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(ws.cpu().numpy().view(np.uint16).reshape(t, k), oracle.dequant_act(xq_ref, ap_ref))
+    _close(dw.cpu().numpy(), oracle.grad_w_quant_x(dy, x))
