@@ -3,10 +3,14 @@
 // the BitNet b1.58 convention: a' = max(max_k |x|, 1e-5), and
 // xq = sign(x) * rne(fl32(127 |x|) / a') clamped to [-128, 127].
 //
-// One block of 128 threads per token row.  Each thread keeps its R 16-byte
-// vectors of the row in registers, so the row is read from memory once: the
-// block reduces the absmax, then every thread quantises what it holds.  Rows
-// longer than 128 * 8 * kMaxR elements take a two-pass, warp-per-row kernel.
+// Rows of up to 3072 elements: one warp per token row, the row in registers
+// (RW 16-byte vectors a lane), read from memory once.  The absmax is an
+// integer max over the bf16 magnitude bits (their order is the order of the
+// values, and a non-finite value shows as bits >= 0x7F80), two halves at a
+// time, then one warp reduction; no block barrier.  All rows of a
+// 4096-token batch are resident at once.  Longer rows: one block of 128
+// threads per row with R vectors a thread (up to 16384 elements), then a
+// two-pass, warp-per-row kernel.
 //
 // Launched with programmatic stream serialisation: its launch overlaps the
 // kernel before it, and it waits for that kernel (which may have written x,
@@ -29,21 +33,22 @@ constexpr int kMaxR = 16;  // rows up to 16384 elements stay in registers
 // Stores the quantised (or, with DEQ, dequantised) form of 8 elements.
 template <bool DEQ>
 __device__ __forceinline__ void store_quantised(void* out, int64_t row, int64_t nvec, int64_t i, const uint4 v,
-                                                float ap) {
+                                                const QScale& qs) {
   if constexpr (DEQ)
-    reinterpret_cast<uint4*>(out)[row * nvec + i] = dequantise8(v, ap);
+    reinterpret_cast<uint4*>(out)[row * nvec + i] = dequantise8(v, qs);
   else
-    reinterpret_cast<uint2*>(out)[row * nvec + i] = quantise8(v, ap);
+    reinterpret_cast<uint2*>(out)[row * nvec + i] = quantise8(v, qs);
 }
 
 template <int R, bool DEQ>
-__global__ void __launch_bounds__(kActThreads)
+__global__ void __launch_bounds__(kActThreads, 4)
     k_act_quant_rows(const uint4* __restrict__ x, int64_t t, int64_t nvec, void* __restrict__ out,
-                     float* __restrict__ a_prime, uint32_t* status, int early_trigger) {
-  // x may be the output of the kernel before this one: bring this block's
-  // rows towards L2 while that kernel runs, then wait for it.
-  if (threadIdx.x == 0)
-    for (int64_t row = blockIdx.x; row < t; row += gridDim.x)
+                     float* __restrict__ a_prime, uint32_t* status, int early_trigger, int pf_stride) {
+  // x may be the output of the kernel before this one: bring it towards L2
+  // while that kernel runs, then wait for it.  The first pf_stride blocks
+  // prefetch every row between them.
+  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < pf_stride)
+    for (int64_t row = blockIdx.x; row < t; row += pf_stride)
       bulk_prefetch_l2(x + row * nvec, static_cast<uint32_t>(nvec * 16));
   pdl_wait();
   if (early_trigger) pdl_trigger();
@@ -85,10 +90,11 @@ __global__ void __launch_bounds__(kActThreads)
       if (!DEQ) a_prime[row] = ap;
       if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
+    const QScale qs = make_qscale(ap);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = int64_t(r) * kActThreads + tid;
-      if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], ap);
+      if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
     }
   }
 }
@@ -121,8 +127,81 @@ __global__ void __launch_bounds__(kActWarps * 32)
     if (__any_sync(0xffffffffu, bad != 0) && lane == 0) raise_status(status, SBL_STATUS_NONFINITE_X);
     const float ap = fmaxf(amax, 1e-5f);
     if (!DEQ && lane == 0) a_prime[row] = ap;
-    for (int64_t j = lane; j < nvec; j += 32) store_quantised<DEQ>(out, row, nvec, j, __ldg(src + j), ap);
+    const QScale qs = make_qscale(ap);
+    for (int64_t j = lane; j < nvec; j += 32) store_quantised<DEQ>(out, row, nvec, j, __ldg(src + j), qs);
   }
+}
+
+constexpr int kWarpRowMax = 12;  // 16-byte vectors a lane: rows up to 3072 elements
+
+template <int RW, bool DEQ>
+__global__ void __launch_bounds__(kActThreads, DEQ ? 1 : 8)
+    k_act_quant_warp(const uint4* __restrict__ x, int64_t t, int64_t nvec, void* __restrict__ out,
+                     float* __restrict__ a_prime, uint32_t* status, int early_trigger, int pf_stride) {
+  // x may be the output of the kernel before this one: bring it towards L2
+  // while that kernel runs, then wait for it.
+  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < pf_stride)
+    for (int64_t row = blockIdx.x; row < t; row += pf_stride)
+      bulk_prefetch_l2(x + row * nvec, static_cast<uint32_t>(nvec * 16));
+  pdl_wait();
+  if (early_trigger) pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  constexpr int kWarps = kActThreads / 32;
+  for (int64_t row = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); row < t;
+       row += int64_t(gridDim.x) * kWarps) {
+    const uint4* src = x + row * nvec;
+    uint4 v[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      const int64_t i = int64_t(r) * 32 + lane;
+      v[r] = (i < nvec) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    }
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      m2 = __vmaxu2(m2, v[r].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].w & 0x7FFF7FFFu);
+    }
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    const float ap = fmaxf(__uint_as_float(m << 16), 1e-5f);
+    if (lane == 0) {
+      if (!DEQ) a_prime[row] = ap;
+      if (m >= 0x7F80u) raise_status(status, SBL_STATUS_NONFINITE_X);
+    }
+    const QScale qs = make_qscale(ap);
+    if (DEQ || qs.exact) {
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const int64_t i = int64_t(r) * 32 + lane;
+        if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
+      }
+    } else {
+      // An exact tie in any lane of a vector (lanes past the row hold zeros:
+      // never a tie) sends that vector through the exact path.
+      const float c127 = __fdiv_rn(127.0f, ap);
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const int64_t i = int64_t(r) * 32 + lane;
+        bool tie;
+        uint2 c = quantise8_fast(v[r], ap, c127, tie);
+        if (__any_sync(0xFFFFFFFFu, tie)) c = quantise8(v[r], qs);
+        if (i < nvec) reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
+      }
+    }
+  }
+}
+
+template <int RW, bool DEQ>
+static cudaError_t launch_warp_rows(const uint4* x, int64_t t, int64_t nvec, void* out, float* ap, uint32_t* status,
+                                    int num_sms, cudaStream_t s, int early) {
+  constexpr int kWarps = kActThreads / 32;
+  int64_t blocks = (t + kWarps - 1) / kWarps;
+  const int64_t cap = int64_t(num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(k_act_quant_warp<RW, DEQ>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t,
+                    nvec, out, ap, status, early, num_sms);
 }
 
 template <int R, bool DEQ>
@@ -132,7 +211,7 @@ static cudaError_t launch_rows(const uint4* x, int64_t t, int64_t nvec, void* ou
   const int64_t cap = int64_t(num_sms) * 64;
   if (blocks > cap) blocks = cap;
   return launch_pdl(k_act_quant_rows<R, DEQ>, dim3(static_cast<unsigned>(blocks)), dim3(kActThreads), 0, s, x, t,
-                    nvec, out, ap, status, early);
+                    nvec, out, ap, status, early, num_sms);
 }
 
 template <bool DEQ>
@@ -141,10 +220,14 @@ static cudaError_t launch_quant(const uint16_t* x, int64_t t, int64_t k, void* o
   if (t <= 0) return cudaSuccess;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const int64_t nvec = k / 8;
-  const int64_t r = (nvec + kActThreads - 1) / kActThreads;
-  if (r <= 1) return launch_rows<1, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
-  if (r <= 2) return launch_rows<2, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
-  if (r <= 3) return launch_rows<3, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  const int64_t rw = (nvec + 31) / 32;
+  if (rw <= 2) return launch_warp_rows<2, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (rw <= 4) return launch_warp_rows<4, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (rw <= 6) return launch_warp_rows<6, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (rw <= 8) return launch_warp_rows<8, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (rw <= 10) return launch_warp_rows<10, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  if (rw <= kWarpRowMax) return launch_warp_rows<kWarpRowMax, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
+  const int64_t r = (nvec + kActThreads - 1) / kActThreads;  // >= 4 here
   if (r <= 4) return launch_rows<4, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
   if (r <= 6) return launch_rows<6, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);
   if (r <= 8) return launch_rows<8, DEQ>(xv, t, nvec, out, a_prime, status, num_sms, s, early);

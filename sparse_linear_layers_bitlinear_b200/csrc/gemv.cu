@@ -153,19 +153,20 @@ __global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
           if (row_bad) raise_status(a.status, SBL_STATUS_NONFINITE_X);
         }
       }
+      const QScale qs = make_qscale(ap);
       uint2* dst = reinterpret_cast<uint2*>(xw + xrow * kw);
       uint2* gdst = (blockIdx.x == 0 && a.xq_out) ? reinterpret_cast<uint2*>(a.xq_out + int64_t(xrow) * a.k) : nullptr;
 #pragma unroll
       for (int q = 0; q < kXq; ++q) {
         const int i = (xsub + q * wpr) * 32 + lane;
         if (i < nvec) {
-          const uint2 c = quantise8(xbuf[q], ap);
+          const uint2 c = quantise8(xbuf[q], qs);
           dst[i] = c;
           if (gdst) gdst[i] = c;
         }
       }
       for (int i = (xsub + kXq * wpr) * 32 + lane; i < nvec; i += wpr * 32) {
-        const uint2 c = quantise8(__ldg(xsrc + i), ap);
+        const uint2 c = quantise8(__ldg(xsrc + i), qs);
         dst[i] = c;
         if (gdst) gdst[i] = c;
       }

@@ -424,7 +424,7 @@ def test_prepare_on_uninitialised_blob_and_repeats(fill):
         _check_prepared(layer, w, n, m)
 
 
-@pytest.mark.parametrize("k", [64, 1088, 2560, 4160, 6912, 12352, 16384, 16448])
+@pytest.mark.parametrize("k", [64, 768, 1088, 2048, 2560, 3072, 3136, 4160, 6912, 12352, 16384, 16448])
 def test_act_quant_row_lengths(k):
     """Activation codes and scales for row lengths that exercise every
     register-resident variant of the act-quant kernel and its long-row path."""
@@ -509,7 +509,7 @@ def test_dw_quant_x(n_out, k, n, m, t, only_dw):
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
 
 
-@pytest.mark.parametrize("k", [64, 2560, 16448])
+@pytest.mark.parametrize("k", [64, 1088, 2560, 3136, 16448])
 def test_dequant_act_row_lengths(k):
     """xhat for a register-resident row length and for the long-row kernel."""
     n_out, t = 8, 5
@@ -525,3 +525,60 @@ def test_dequant_act_row_lengths(k):
     xq_ref, ap_ref = oracle.act_quant(x)
     assert np.array_equal(ws.cpu().numpy().view(np.uint16).reshape(t, k), oracle.dequant_act(xq_ref, ap_ref))
     _close(dw.cpu().numpy(), oracle.grad_w_quant_x(dy, x))
+
+
+def _tie_rows(k):
+    """Rows whose quotients 127|x| / a' hit exact half-integers (ties go to the
+    even code), a row under the 1e-5 clamp, and a Gaussian row."""
+    rng = np.random.default_rng(61)
+    rows = np.zeros((4, k), dtype=np.float32)
+    halves = np.arange(0, 127) + 0.5                     # 0.5 .. 126.5, all bf16-exact
+    rows[0, :127] = halves * rng.choice([-1.0, 1.0], 127)
+    rows[0, 127] = 127.0                                 # a' = 127: quotient = |x|
+    odd = np.arange(1, 254, 2, dtype=np.float32)          # a' = 254: quotient = |x| / 2
+    rows[1, :odd.size] = odd * rng.choice([-1.0, 1.0], odd.size)
+    rows[1, odd.size] = -254.0
+    rows[2] = rng.uniform(-9e-6, 9e-6, size=k)            # every |x| < 1e-5: a' is the clamp
+    rows[3] = rng.normal(size=k)
+    bits = synth.bits(torch.from_numpy(rows).to(torch.bfloat16))
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("gemv", [False, True])
+def test_act_quant_exact_ties_and_clamp(gemv):
+    """The division-free quantiser against the oracle's IEEE division on exact
+    ties and on the clamped scale, in the act-quant kernel and in the GEMV."""
+    n_out, k = 64, 512
+    x = _tie_rows(k)
+    t = x.shape[0]
+    flags = sbl.SBL_PACK_GEMV if gemv else 0
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, flags)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 62)))
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    # the tie rows really are ties, and they went to the even code
+    assert np.array_equal(np.abs(xq_ref[0, :127].astype(int)), 2 * np.round(np.arange(127) / 2 + 0.25).astype(int))
+    assert (np.abs(xq_ref[1, :127].astype(int)) % 2 == 0).all()
+
+
+def test_act_quant_more_rows_than_resident_warps():
+    """More token rows than the warp-per-row kernel keeps resident, so warps
+    loop over rows."""
+    n_out, k, t = 8, 256, 10000
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 63)))
+    x = synth.activations(t, k, 64)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
