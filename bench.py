@@ -247,11 +247,11 @@ class OracleFit:
     def sample(self):
         """One timed sample; returns the extrapolated full-step seconds."""
         f, v = oracle_sample(*self.args, self.tokens)
-        if self.tokens > self.lo:
-            slope = (v - self.v_lo) / (self.tokens - self.lo)
-            intercept = max(0.0, v - slope * self.tokens)
-        else:
+        slope = (v - self.v_lo) / (self.tokens - self.lo) if self.tokens > self.lo else 0.0
+        if slope <= 0.0:  # timing noise on a small sample: no intercept, plain per-token cost
             slope, intercept = v / self.tokens, 0.0
+        else:
+            intercept = max(0.0, v - slope * self.tokens)
         return f + intercept + self.T * slope
 
     def describe(self, step_s):
