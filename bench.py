@@ -314,8 +314,9 @@ def run_reference(args):
 # Other workloads, reported beside the headline line
 # ---------------------------------------------------------------------------
 def bench_decode(dev, hbm_gbs, reps=10):
-    """Decode-shaped forward over the 2-bit weight packing: T in {1, 4, 16},
-    K = 2560, N_out in {2560, 6912}.  One replay = 64 forward calls in a CUDA
+    """Decode-shaped forward on layers with the 2-bit weight packing: T in
+    {1, 4, 16}, K = 2560, N_out in {2560, 6912}; the library sends each call
+    to the 2-bit GEMV or the 2:4 tensor-core GEMM, whichever is faster.  One replay = 64 forward calls in a CUDA
     graph over distinct weight blobs (more than 2 x L2 of weights in total),
     so every call streams its weights from HBM.  The per-call time includes the
     launch of each call inside the graph."""
@@ -355,14 +356,19 @@ def bench_decode(dev, hbm_gbs, reps=10):
             e1.record()
             torch.cuda.synchronize(dev)
             us = e0.elapsed_time(e1) / (64 * reps) * 1e3
-            by = N * K / 4 + 2 * T * K + 4 * T * N
-            out.append({"n_out": N, "k": K, "tokens": T, "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
+            gemv = sbl.forward_uses_gemv(layers[0], T)
+            # weight bytes of the path taken: 2-bit packing, or 2:4 values + metadata
+            wbytes = N * K / 4 if gemv else N * K / 2 + N * K / 8
+            by = wbytes + 2 * T * K + 4 * T * N
+            out.append({"n_out": N, "k": K, "tokens": T, "path": "gemv" if gemv else "2:4 tensor-core GEMM",
+                        "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
                         "gbs": by / (us * 1e-6) / 1e9, "hbm_frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
                         "bytes_per_call": by})
             del g
         del layers
         torch.cuda.empty_cache()
-    return {"workload": "decode 2:4 forward, 2-bit packed weights, K=2560",
+    return {"workload": "decode 2:4 forward on layers with the 2-bit packing, K=2560; each call takes the "
+                        "faster path for its size (`path`)",
             "timing": "CUDA graph of 64 calls over distinct weight blobs (> 2 x L2), per-call time incl. launch",
             "points": out}
 

@@ -152,9 +152,18 @@ sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl
  * then `workspace` (sbl_workspace_bytes(t, k) bytes) holds them.  acc_debug
  * (int32 [t, n_out]) may be NULL; when given, the raw accumulators are
  * written too.  t == 0 is a no-op.  2:4 layers run the 2:4-sparse int8
- * tensor-core GEMM; other patterns the dense int8 one over W_eff codes. */
+ * tensor-core GEMM; other patterns the dense int8 one over W_eff codes.  A
+ * layer prepared with SBL_PACK_GEMV takes the decode GEMV over its 2-bit
+ * packing instead for small calls (t <= 16 and t * n_out * k <= 8e7, where
+ * that GEMV is the faster of the two); the outputs are the same bits either
+ * way. */
 sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
                        float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
+
+/* 1 when sbl_forward on this layer with t tokens takes the decode GEMV over
+ * the 2-bit packing, 0 when it takes a tensor-core GEMM (or the arguments
+ * are invalid).  Host only, no device access. */
+int sbl_forward_uses_gemv(const sbl_layer* layer, int64_t t);
 
 /* Forward pass for callers that cannot allocate device memory.  The paper has
  * no counterpart: this is a deployment convenience, not a step of the method.

@@ -274,6 +274,15 @@ bool gemv_fits(int64_t t, int64_t k) {
   return t >= 1 && t <= 16 && (kLutWords + 32 + tp * (k / 4)) * 4 <= int64_t(kGemvMaxSmem);
 }
 
+// The GEMV's dot products run on the CUDA cores and grow with t * n_out * k,
+// while the 2:4 tensor-core GEMM costs about one round of tiles for a handful
+// of tokens (measured at k = 2560: ~12 us for t = 4..32 against 6.8-17.5 us
+// for the GEMV, which wins up to about 8e7 multiply-adds, e.g. t = 4 at
+// n_out = 6912 or t = 8 at n_out = 2560).
+constexpr int64_t kGemvMaxMacs = 80000000;
+
+bool gemv_preferred(int64_t t, int64_t n_out, int64_t k) { return t * n_out * k <= kGemvMaxMacs; }
+
 // Token counts up to kFusedMaxT quantise inside the GEMV (every block redoes
 // that small amount of work, which saves a launch); larger ones run the
 // act-quant kernel first.

@@ -79,6 +79,12 @@ extern "C" {
 
 const char* sbl_version(void) { return "sbl 0.1 (sm_100a)"; }
 
+int sbl_forward_uses_gemv(const sbl_layer* layer, int64_t t) {
+  sbl_blob_layout L;
+  if (check_layer(layer, &L) != SBL_OK || t <= 0) return 0;
+  return (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) ? 1 : 0;
+}
+
 uint64_t sbl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t flags, sbl_blob_layout* out) {
@@ -164,7 +170,7 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(layer, L.status);
   const float* g = at<const float>(layer, L.g);
-  if (L.gemv != 0 && gemv_fits(t, layer->k)) {
+  if (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) {
     // decode: the 2-bit weight stream
     const bool fused = gemv_fuses_act_quant(t);
     if (!fused &&

@@ -73,6 +73,7 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
 // with its early trigger and xq_in / ap_in are its outputs.  gemv_fits() says
 // whether the token rows fit the kernel's shared memory.
 bool gemv_fits(int64_t t, int64_t k);
+bool gemv_preferred(int64_t t, int64_t n_out, int64_t k);
 bool gemv_fuses_act_quant(int64_t t);
 cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const int8_t* xq_in, const float* ap_in,
                                 const float* g, int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out,

@@ -88,6 +88,7 @@ SIGNATURES = {
     "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
+    "sbl_forward_uses_gemv": (ctypes.c_int, [_LP, _I64]),
 }
 
 _lib = None
@@ -231,6 +232,12 @@ def selftest_wait_timeout(status_dev, limit_ns: int, stream=None):
 
 def version() -> str:
     return lib().sbl_version().decode()
+
+
+def forward_uses_gemv(layer: Layer, t: int) -> bool:
+    """Whether sbl_forward takes the 2-bit decode GEMV for t tokens on this layer."""
+    cl = layer.c()
+    return bool(lib().sbl_forward_uses_gemv(ctypes.byref(cl), t))
 
 
 def launch_count() -> int:

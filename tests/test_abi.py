@@ -26,6 +26,13 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(sbl_[a-z0-9_]+)\s*\(", text)))
 
 
+class _FakeBlob:
+    """Stands in for a device blob: only its (aligned) address is read."""
+
+    def data_ptr(self):
+        return 0x10000
+
+
 def test_header_declares_the_documented_entry_points():
     names = declared_functions()
     for required in ("sbl_prepare_weights", "sbl_forward", "sbl_backward", "sbl_prepared_bytes",
@@ -78,6 +85,20 @@ def test_ablation_flags_are_accepted_and_unknown_bits_rejected(lib):
     assert sbl.prepared_bytes(264, 320, 2, 4, 1 << 5) == 0
     with pytest.raises(sbl.SblError):
         sbl.prepared_layout(264, 320, 2, 4, 1 << 5)
+
+
+def test_forward_dispatch_query(lib):
+    def uses(n_out, k, n, m, flags, t):
+        return sbl.forward_uses_gemv(sbl.Layer(n_out, k, n, m, flags, _FakeBlob()), t)
+
+    g = sbl.SBL_PACK_GEMV
+    assert uses(6912, 2560, 2, 4, g, 1) and uses(6912, 2560, 2, 4, g, 4)
+    assert not uses(6912, 2560, 2, 4, g, 8) and not uses(6912, 2560, 2, 4, g, 16)  # tensor cores win
+    assert uses(2560, 2560, 2, 4, g, 8) and not uses(2560, 2560, 2, 4, g, 16)
+    assert not uses(256, 256, 2, 4, g, 17)      # beyond the GEMV's token count
+    assert not uses(6912, 2560, 2, 4, 0, 1)     # no 2-bit packing
+    assert not uses(6912, 2560, 2, 4, g, 0)
+    assert not uses(6912, 2560, 6, 8, g, 1)     # not a valid layer
 
 
 def test_backward_workspace_for_the_quantised_x_operand(lib):

@@ -582,3 +582,29 @@ def test_act_quant_more_rows_than_resident_warps():
     xq_ref, ap_ref = oracle.act_quant(x)
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
     assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("t", [4, 8, 16])
+def test_decode_dispatch_both_paths_bit_exact(t):
+    """A layer with the 2-bit packing at the decode sizes: small calls take the
+    GEMV, larger ones the 2:4 tensor-core GEMM; both give the oracle's bits."""
+    n_out, k = 6912, 2560
+    w = synth.master_weights(n_out, k, 81)
+    x = synth.activations(t, k, 82)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(w))
+    assert sbl.forward_uses_gemv(layer, t) == (t <= 4)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    c0 = sbl.launch_count()
+    sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
+    launched = sbl.launch_count() - c0
+    torch.cuda.synchronize()
+    ref = oracle.forward(w, x, 2, 4)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    assert launched == (1 if t <= 4 else 2)  # the fused GEMV, or act-quant + GEMM
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
