@@ -95,38 +95,54 @@ __device__ __forceinline__ bool in_window(const uint32_t (&mw)[4]) {
   return (bf16x2_lt_mask(mx, kHi2) & bf16x2_ge_mask_(mn, kLo2)) == 0xFFFFFFFFu;
 }
 
-__device__ __noinline__ void add_slow(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3,
-                                      unsigned long long* s_bins, uint32_t* s_flags) {
+// A vector with a magnitude outside the fast window: its in-window magnitudes
+// are returned as an fp64 sum for the caller's exact accumulator (so a stage
+// still adds at most 16 window terms there), the others go to the exact
+// 64-bit bins.  Flags: bit 0 a non-finite weight, bit 1 the bins are in use,
+// bit 2 a magnitude at or above the window (2^6); *s_tiny counts the non-zero
+// magnitudes below it (2^-30), whose total the scale's fast decision bounds.
+__device__ __noinline__ double add_slow(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3,
+                                        unsigned long long* s_bins, uint32_t* s_flags, uint32_t* s_tiny) {
   const uint32_t mw[4] = {m0, m1, m2, m3};
-  uint32_t bad = 0;
+  uint32_t fl = 0, tiny = 0;
+  double in_win = 0.0;
 #pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const uint32_t mag = (mw[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
-    const uint32_t e = mag >> 7;
-    if (e == 0xFFu) {
-      bad = 1u;
+    if (mag >= kWinLo && mag < kWinLo + kWinSpan) {
+      in_win += fp64_of_hi_word(mag << 13);
       continue;
     }
+    const uint32_t e = mag >> 7;
+    if (e == 0xFFu) {
+      fl |= 1u;
+      continue;
+    }
+    if (mag >= kWinLo) fl |= 4u;
+    else if (mag != 0u) ++tiny;
     const uint32_t s = max(e, 1u) - 1u;
     const uint32_t sig = mag - (s << 7);
     if (sig != 0u) atomicAdd(&s_bins[s >> 3], static_cast<unsigned long long>(sig << (s & 7u)));
   }
-  atomicOr(s_flags, 2u | bad);  // bit 1: the bins are in use; bit 0: a non-finite weight
+  atomicOr(s_flags, 2u | fl);
+  if (tiny) atomicAdd(s_tiny, tiny);
+  return in_win;
 }
 
 // Correct rounding without a division.  q approximates a positive value v
-// within 2^-51 relative.  If q is farther than that from the fp32 rounding
+// within 2^-51 relative, plus (when `extra` > 0) an unknown non-negative
+// addend below `extra`.  If q is farther than both from the fp32 rounding
 // midpoint on its side of RN_fp32(q), then v lies on the same side and
 // RN_fp32(v) = RN_fp32(q).  Returns false when q is too close to decide (an
 // exact or near tie) or too small (the fp32 subnormal range is left to the
 // exact path).
-__device__ __forceinline__ bool round_fp32_if_clear(double q, float* out) {
+__device__ __forceinline__ bool round_fp32_if_clear(double q, double extra, float* out) {
   if (!(q > 0x1p-120)) return false;
   const float f = __double2float_rn(q);
   const double fd = static_cast<double>(f);
   const double nb = (q >= fd) ? static_cast<double>(nextafterf(f, 3.0e38f)) : static_cast<double>(nextafterf(f, 0.0f));
   const double mid = 0.5 * (fd + nb);  // exact: both are fp32 values
-  if (fabs(q - mid) > q * 0x1p-48) {
+  if (fabs(q - mid) > q * 0x1p-48 + extra) {
     *out = f;
     return true;
   }
@@ -180,7 +196,7 @@ __device__ float exact_mean_fp32(const uint64_t* bins, uint64_t numel) {
     // division-free attempt: the top 64 bits of S (truncated) in fp64
     float r;
     const double ds = ldexp(static_cast<double>(get64(topS - 63)), topS - 63 - 133);
-    if (round_fp32_if_clear(ds / static_cast<double>(numel), &r)) return r;
+    if (round_fp32_if_clear(ds / static_cast<double>(numel), 0.0, &r)) return r;
   }
   const int low = topS - 127;  // bit of S that lands at bit 0 of N
   const unsigned __int128 N = (static_cast<unsigned __int128>(get64(low + 64)) << 64) | get64(low);
@@ -210,15 +226,20 @@ __device__ float exact_mean_fp32(const uint64_t* bins, uint64_t numel) {
 }
 
 
-// gamma = RN_fp32(S * 2^-37 / numel) for a sum S held as a 128-bit integer
-// (hi, lo), from an fp64 quotient (one rounding of S, one of the division).
-__device__ bool mean_fp32_fast(uint64_t lo, uint64_t hi, uint64_t numel, float* out) {
+// gamma = RN_fp32((S * 2^-37 + T) / numel) for a sum S held as a 128-bit
+// integer (hi, lo), from an fp64 quotient (one rounding of S, one of the
+// division), where T is the unknown total of `ntiny` magnitudes below 2^-30
+// (so 0 <= T < ntiny * 2^-30).  False when that does not decide the rounding.
+__device__ bool mean_fp32_fast(uint64_t lo, uint64_t hi, uint64_t numel, uint64_t ntiny, float* out) {
   const double s = __ull2double_rn(hi) * 0x1p64 + __ull2double_rn(lo);  // hi * 2^64 is exact
   if (s == 0.0) {
+    if (ntiny != 0) return false;  // the mean is the tiny magnitudes' alone
     *out = 0.0f;
     return true;
   }
-  return round_fp32_if_clear(__ddiv_rn(s, __ull2double_rn(numel)) * 0x1p-37, out);
+  const double dn = __ull2double_rn(numel);
+  const double slack = __ddiv_rn(static_cast<double>(ntiny) * 0x1p-30, dn) * (1.0 + 0x1p-40);
+  return round_fp32_if_clear(__ddiv_rn(s, dn) * 0x1p-37, slack, out);
 }
 
 // Keep-bits of one group of M magnitudes: position a is kept when fewer than
@@ -380,7 +401,8 @@ struct PrepTail {
   unsigned long long fold_bins[kExactBins];
   uint64_t warp_lo[kPrepConsumerWarps], warp_hi[kPrepConsumerWarps];
   uint64_t gen;
-  uint32_t flags;       // bit 0 non-finite, bit 1 slow bins in use (this CTA)
+  uint32_t flags;       // bit 0 non-finite, bit 1 slow bins in use, bit 2 a magnitude >= 2^6 (this CTA)
+  uint32_t ntiny;       // non-zero magnitudes below 2^-30 in this CTA's bins
   float g;
   int abort_flag;
 };
@@ -431,6 +453,7 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
     fence_mbar_init();
     tail->gen = ld_relaxed_u64(a.gen);
     tail->flags = 0u;
+    tail->ntiny = 0u;
     tail->abort_flag = 0;
     if (blk == 0) *status = 0u;  // a new prepare resets the status word
   }
@@ -484,7 +507,7 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
             acc[h2] += fp64_of_hi_word((wd[q] >> 3) & 0x0FFFE000u);
           }
         } else {
-          add_slow(mw[0], mw[1], mw[2], mw[3], tail->bins, &tail->flags);
+          acc[h2] += add_slow(mw[0], mw[1], mw[2], mw[3], tail->bins, &tail->flags, &tail->ntiny);
         }
       }
     }
@@ -525,7 +548,10 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       L += olo;
       H += ohi + ((L < olo) ? 1ull : 0ull);
     }
-    const uint32_t fl_own = tail->flags;
+    // flags in the low byte, the count of tiny magnitudes above it (a count
+    // too large to carry forces the exact path, as a huge magnitude does)
+    const uint32_t nt = tail->ntiny;
+    const uint32_t fl_own = (tail->flags | (nt > 0xFFFFFFu ? 4u : 0u)) | ((nt > 0xFFFFFFu ? 0u : nt) << 8);
     if (fl_own & 2u) {  // slow bins in use: publish them first
       for (int b = lane; b < kExactBins; b += 32) a.slot_bins[int64_t(blk) * kExactBins + b] = tail->bins[b];
       __threadfence();
@@ -540,12 +566,12 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       st_relaxed_u64(sf + 2, tag | (H & 0xFFFFFFFFull));
       st_release_u64(sf + 3, tag | fl_own);
     }
-    uint64_t s0 = 0, s1 = 0, s2 = 0;
+    uint64_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;  // s3: tiny magnitudes in all CTAs' bins
     uint32_t fl = 0, slow_r = 0;  // slow_r: bit r set when CTA lane + 32 r used its slow bins
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
       bool all = true;
-      s0 = s1 = s2 = 0;
+      s0 = s1 = s2 = s3 = 0;
       fl = slow_r = 0;
       auto take = [&](int c, int r) {
         const ulonglong2* sf = reinterpret_cast<const ulonglong2*>(a.slot_fast + int64_t(c) * 4);
@@ -554,7 +580,8 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
         s0 += p01.x & 0xFFFFFFFFull;
         s1 += p01.y & 0xFFFFFFFFull;
         s2 += p23.x & 0xFFFFFFFFull;
-        fl |= static_cast<uint32_t>(p23.y);
+        fl |= static_cast<uint32_t>(p23.y) & 0xFFu;
+        s3 += (p23.y >> 8) & 0xFFFFFFull;
         if (r < 32 && (p23.y & 2u)) slow_r |= 1u << r;
       };
 #pragma unroll
@@ -582,9 +609,26 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       s0 += __shfl_xor_sync(0xffffffffu, s0, off);
       s1 += __shfl_xor_sync(0xffffffffu, s1, off);
       s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      s3 += __shfl_xor_sync(0xffffffffu, s3, off);
       fl |= __shfl_xor_sync(0xffffffffu, fl, off);
     }
-    if (fl & 2u) {  // rare: fold the slow bins of the CTAs that used them, lanes over bins
+    // the 128-bit total: s0 + s1 * 2^32 + s2 * 2^64 (each below 2^42)
+    const uint64_t t1 = s1 << 32;
+    const uint64_t Lt = s0 + t1;
+    const uint64_t Ht = s2 + (s1 >> 32) + ((Lt < t1) ? 1ull : 0ull);
+    const uint64_t numel = uint64_t(a.n_out) * uint64_t(a.k);
+    // The fast sum decides gamma unless a weight is non-finite or at least
+    // 2^6, or the rounding is too close to call given the tiny magnitudes'
+    // bound; every lane computes the same decision.
+    float gamma = 0.0f;
+    bool decided = false;
+    if (fl & 1u) {
+      gamma = __int_as_float(0x7fc00000);
+      decided = true;
+    } else if (!(fl & 4u)) {
+      decided = mean_fp32_fast(Lt, Ht, numel, s3, &gamma);
+    }
+    if (!decided && (fl & 2u)) {  // rare: fold the slow bins of the CTAs that used them, lanes over bins
       for (int r = 0; 32 * r < G && r < 32; ++r) {
         uint32_t slow = __ballot_sync(0xffffffffu, (slow_r >> r) & 1u);
         while (slow) {
@@ -601,17 +645,7 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
     }
     if (lane == 0) {
       if (blk == 0) st_relaxed_u64(a.gen, gen0 + 1);
-      // the 128-bit total: s0 + s1 * 2^32 + s2 * 2^64 (each below 2^42)
-      const uint64_t t1 = s1 << 32;
-      const uint64_t Lt = s0 + t1;
-      const uint64_t Ht = s2 + (s1 >> 32) + ((Lt < t1) ? 1ull : 0ull);
-      const uint64_t numel = uint64_t(a.n_out) * uint64_t(a.k);
-      float gamma;
-      if (fl & 1u) {
-        gamma = __int_as_float(0x7fc00000);
-      } else if ((fl & 2u) || !mean_fp32_fast(Lt, Ht, numel, &gamma)) {
-        gamma = gamma_exact(tail->fold_bins, Lt, Ht, numel);
-      }
+      if (!decided) gamma = gamma_exact(tail->fold_bins, Lt, Ht, numel);
       const float g = (gamma > 1e-5f) ? gamma : 1e-5f;  // a NaN gamma gives 1e-5; the status word says why
       tail->g = g;
       if (blk == 0) {

@@ -608,3 +608,23 @@ def test_decode_dispatch_both_paths_bit_exact(t):
     assert np.array_equal(xq.cpu().numpy(), ref["xq"])
     assert launched == (1 if t <= 4 else 2)  # the fused GEMV, or act-quant + GEMM
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+@pytest.mark.parametrize("tiny", [2.0 ** -40, 0.0, -(2.0 ** -35)])
+def test_gamma_midpoint_decided_by_a_tiny_magnitude(tiny):
+    """8192 masters whose in-window magnitudes average exactly to the fp32
+    midpoint 1 + 2^-24: alone that ties to even (1.0), and one magnitude far
+    below the window (2^-40 or 2^-35) must round it up to 1 + 2^-23.  A scale
+    decided from the in-window sum without the tiny magnitudes would miss it."""
+    n_out, k = 32, 256
+    v = np.ones(n_out * k, dtype=np.float32)
+    v[0], v[1], v[2] = 3.0, 2.0 ** -11, tiny  # 8189 ones + 3 + 2^-11 + tiny
+    w = torch.from_numpy(v.reshape(n_out, k)).to(torch.bfloat16)
+    expect = 1.0 + 2.0 ** -23 if tiny != 0.0 else 1.0
+    assert float(oracle.absmean_gamma(w)) == expect
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(w))
+    gamma, g = sbl.read_scale(layer)
+    assert gamma == expect and g == expect
+    _check_prepared(layer, w, 2, 4)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
