@@ -8,7 +8,9 @@
 // integer max over the bf16 magnitude bits (their order is the order of the
 // values, and a non-finite value shows as bits >= 0x7F80), two halves at a
 // time, then one warp reduction; no block barrier.  All rows of a
-// 4096-token batch are resident at once.  Longer rows: one block of 128
+// 4096-token batch are resident at once.  Its codes come without a division
+// (quantise8_fast: the estimate's rounding plus an exact tie check, the IEEE
+// division only for tied vectors and clamped rows).  Longer rows: one block of 128
 // threads per row with R vectors a thread (up to 16384 elements), then a
 // two-pass, warp-per-row kernel.
 //
