@@ -482,6 +482,53 @@ def bench_nm_sweep(dev, peaks, steps=10):
             "timing": f"CUDA events around each phase, mean of {steps} steps after 3", "points": out}
 
 
+def bench_ablations(dev, steps=10):
+    """The pages' ablations and the STE reading variant as flags, on the
+    prefill 2:4 workload: the plain step, the mask from the ternary codes
+    (SBL_MASK_FROM_QUANT), the blocked gradient of pruned weights
+    (SBL_MASKED_GRAD), and dW against the dequantised activations
+    (SBL_DW_QUANT_X, which adds one quantise-and-dequantise pass).  CUDA events
+    around each phase."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    T, K, N, n, m = (WORKLOAD[k] for k in ("tokens", "k", "n_out", "n", "m"))
+    sets = [(synth.master_weights(N, K, 60 + 10 * r, device=dev), synth.activations(T, K, 61 + 10 * r, device=dev),
+             synth.upstream_grad(T, N, 62 + 10 * r, device=dev)) for r in range(ROTATE)]
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    bws = torch.empty(sbl.backward_workspace_bytes(T, K, sbl.SBL_DW_QUANT_X), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    out = []
+    for name, lflags, bflags in [("plain", 0, 0), ("mask_from_codes", sbl.SBL_MASK_FROM_QUANT, 0),
+                                 ("masked_grad", 0, sbl.SBL_MASKED_GRAD), ("dw_quant_x", 0, sbl.SBL_DW_QUANT_X)]:
+        layer = sbl.Layer.allocate(N, K, n, m, lflags, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ph = [0.0, 0.0, 0.0]
+        for i in range(steps + 3):
+            w, x, dy = sets[i % ROTATE]
+            ev[0].record()
+            sbl.prepare_weights(layer, w)
+            ev[1].record()
+            sbl.forward(layer, x, T, y, workspace=ws)
+            ev[2].record()
+            sbl.backward(layer, x, dy, T, dx, dw, bflags, workspace=bws if bflags else None)
+            ev[3].record()
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                for j in range(3):
+                    ph[j] += ev[j].elapsed_time(ev[j + 1]) / steps
+        code, bits = sbl.read_status(layer)
+        assert code == sbl.SBL_OK, (code, bits)
+        out.append({"variant": name, "layer_flags": lflags, "backward_flags": bflags, "ms_per_step": sum(ph),
+                    "phase_ms": {"prepare": ph[0], "forward": ph[1], "backward": ph[2]}})
+        del layer
+    return {"workload": WORKLOAD["name"], "timing": f"CUDA events around each phase, mean of {steps} steps after 3",
+            "points": out}
+
+
 def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     """One training step's linear layers: 30 x {q, k, v, o: 2560 x 2560;
     gate, up: 2560 -> 6912; down: 6912 -> 2560} at 8192 tokens.  Per step every
@@ -794,6 +841,7 @@ def main():
         line["prefill_6of8"] = bench_prefill68(dev, peaks)
         line["train_step"] = [bench_train_step(dev, peaks, 2, 4), bench_train_step(dev, peaks, 4, 8)]
         line["nm_sweep"] = bench_nm_sweep(dev, peaks)
+        line["ablations"] = bench_ablations(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
     if rank == 0:

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kActThreads, DEQ ? 1 : 8)
       if (m >= 0x7F80u) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
     const QScale qs = make_qscale(ap);
-    if (DEQ || qs.exact) {
+    if (qs.exact) {  // the clamp or a' >= 2^120: the IEEE division
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         const int64_t i = int64_t(r) * 32 + lane;
@@ -183,13 +183,19 @@ __global__ void __launch_bounds__(kActThreads, DEQ ? 1 : 8)
       // An exact tie in any lane of a vector (lanes past the row hold zeros:
       // never a tie) sends that vector through the exact path.
       const float c127 = __fdiv_rn(127.0f, ap);
+      const float a_over_127 = DEQ ? __fdiv_rn(ap, 127.0f) : 0.0f;
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         const int64_t i = int64_t(r) * 32 + lane;
         bool tie;
         uint2 c = quantise8_fast(v[r], ap, c127, tie);
         if (__any_sync(0xFFFFFFFFu, tie)) c = quantise8(v[r], qs);
-        if (i < nvec) reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
+        if (i < nvec) {
+          if constexpr (DEQ)
+            reinterpret_cast<uint4*>(out)[row * nvec + i] = dequant8_fast(c, a_over_127);
+          else
+            reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
+        }
       }
     }
   }

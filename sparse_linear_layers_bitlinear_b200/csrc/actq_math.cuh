@@ -4,6 +4,7 @@
 // clamped to [-128, 127].
 #pragma once
 
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace sbl {
@@ -23,14 +24,17 @@ __device__ __forceinline__ float bf16_abs_value(uint32_t bits16) { return __uint
 // within one of floor(Q), and the sign of the exact remainder
 // (i + 1/2) a' - t (an FMA of short significands) decides between i and
 // i + 1, a zero remainder being the tie that goes to the even code.  The
-// clamped a' = 1e-5 is not a bf16 value; those rows take the IEEE division.
+// clamped a' = 1e-5 is not a bf16 value, and from a' = 2^120 up the products
+// of that test can overflow fp32; those rows take the IEEE division.
 struct QScale {
   float ap;    // a'
   float inv;   // RN(1 / a')
-  bool exact;  // a' is the 1e-5 clamp
+  bool exact;  // a' is the 1e-5 clamp or at least 2^120 (or not finite)
 };
 
-__device__ __forceinline__ QScale make_qscale(float ap) { return QScale{ap, __frcp_rn(ap), ap == 1e-5f}; }
+__device__ __forceinline__ QScale make_qscale(float ap) {
+  return QScale{ap, __frcp_rn(ap), ap == 1e-5f || !(ap < 0x1p120f)};
+}
 
 // One magnitude code: rne(fl32(127 |x|) / a') clamped to 127.
 __device__ __forceinline__ int quant_code(float ax, const QScale& s) {
@@ -43,7 +47,7 @@ __device__ __forceinline__ int quant_code(float ax, const QScale& s) {
 }
 
 // The same codes with fewer instructions, for rows whose a' is a bf16 value
-// (not the clamp).  On signed values: n = rint(x * RN(127 / a')) (the
+// below 2^120 (QScale::exact false).  On signed values: n = rint(x * RN(127 / a')) (the
 // estimate cannot cross a rounding boundary, as above, and rint is odd-
 // symmetric), then the exact remainder r = 127 x - n a' (n a' and 127 x both
 // have at most 15 significant bits) flags an exact tie, |r| = a' / 2, where the
@@ -100,6 +104,31 @@ __device__ __forceinline__ uint32_t dequant_bf16(int code, float ap) {
   const int exp = static_cast<int>(top >> 7) - 1023 + 127;
   if (exp >= 255) return sign | 0x7F80u;      // rounds past the bf16 maximum
   return sign | (static_cast<uint32_t>(exp) << 7) | static_cast<uint32_t>(top & 0x7Fu);
+}
+
+// The same value with fp32 arithmetic, for a row whose a' is a bf16 value
+// below 2^120 (QScale::exact false), given c = RN(a' / 127): RN(code * c) is
+// within ~2^-23 (relative) of Q = code * a' / 127.  A Q that is not dyadic
+// lies at least 2^-16 (relative) from every bf16 rounding boundary (N 2^e /
+// 127 against a 9-bit dyadic, N = |code| * A < 2^15), so RN_bf16 of the
+// estimate is RN_bf16(Q); a dyadic Q (code = +-127, or A = 254) has at most 8
+// significant bits, is a bf16 value, and the estimate rounds back onto it.
+__device__ __forceinline__ uint32_t dequant_bf16_fast(int code, float a_over_127) {
+  const float v = __fmul_rn(static_cast<float>(code), a_over_127);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+}
+
+// 8 codes (two words) -> their dequantised values (bf16, one 16-byte vector).
+__device__ __forceinline__ uint4 dequant8_fast(const uint2 q, float a_over_127) {
+  const uint32_t codes[2] = {q.x, q.y};
+  uint32_t out[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const int c0 = static_cast<int8_t>((codes[h >> 1] >> (16 * (h & 1))) & 0xFFu);
+    const int c1 = static_cast<int8_t>((codes[h >> 1] >> (16 * (h & 1) + 8)) & 0xFFu);
+    out[h] = dequant_bf16_fast(c0, a_over_127) | (dequant_bf16_fast(c1, a_over_127) << 16);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // 8 bf16 values -> their 8 dequantised values (bf16, one 16-byte vector).

@@ -529,9 +529,10 @@ def test_dequant_act_row_lengths(k):
 
 def _tie_rows(k):
     """Rows whose quotients 127|x| / a' hit exact half-integers (ties go to the
-    even code), a row under the 1e-5 clamp, and a Gaussian row."""
+    even code), a row under the 1e-5 clamp, a Gaussian row, and ties next to
+    the bf16 maximum."""
     rng = np.random.default_rng(61)
-    rows = np.zeros((4, k), dtype=np.float32)
+    rows = np.zeros((5, k), dtype=np.float32)
     halves = np.arange(0, 127) + 0.5                     # 0.5 .. 126.5, all bf16-exact
     rows[0, :127] = halves * rng.choice([-1.0, 1.0], 127)
     rows[0, 127] = 127.0                                 # a' = 127: quotient = |x|
@@ -540,6 +541,10 @@ def _tie_rows(k):
     rows[1, odd.size] = -254.0
     rows[2] = rng.uniform(-9e-6, 9e-6, size=k)            # every |x| < 1e-5: a' is the clamp
     rows[3] = rng.normal(size=k)
+    # a' = 254 * 2^120 near the bf16 maximum: 127 |x| overflows fp32 for 253
+    # and 251 times 2^120, so by the fp32 definition their codes saturate at
+    # +-127 (the exact quotients would be the ties 126.5 and 125.5)
+    rows[4, :4] = [254.0 * 2.0 ** 120, 253.0 * 2.0 ** 120, -251.0 * 2.0 ** 120, 1.0]
     bits = synth.bits(torch.from_numpy(rows).to(torch.bfloat16))
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
 
@@ -565,6 +570,7 @@ def test_act_quant_exact_ties_and_clamp(gemv):
     # the tie rows really are ties, and they went to the even code
     assert np.array_equal(np.abs(xq_ref[0, :127].astype(int)), 2 * np.round(np.arange(127) / 2 + 0.25).astype(int))
     assert (np.abs(xq_ref[1, :127].astype(int)) % 2 == 0).all()
+    assert list(xq_ref[4, :3]) == [127, 127, -127]
 
 
 def test_act_quant_more_rows_than_resident_warps():
@@ -627,4 +633,27 @@ def test_gamma_midpoint_decided_by_a_tiny_magnitude(tiny):
     gamma, g = sbl.read_scale(layer)
     assert gamma == expect and g == expect
     _check_prepared(layer, w, 2, 4)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def test_dw_quant_x_operand_on_tie_clamp_and_huge_rows():
+    """xhat for rows with exact ties, the 1e-5 clamp, a Gaussian row and a row
+    whose a' is past 2^120 (fp64 path): bit-exact against the oracle."""
+    n_out, k = 64, 512
+    x = _tie_rows(k)
+    rows = x.float().numpy().copy()
+    rows[2, :] *= 1.0  # keep the clamp row
+    rows[3, :4] = [3.0e38, -1.5e38, 2.0e36, 1.0]  # a' past 2^120
+    x = torch.from_numpy(rows).to(torch.bfloat16)
+    t = x.shape[0]
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 66)))
+    dy = synth.upstream_grad(t, n_out, 67)
+    flags = sbl.SBL_DW_QUANT_X | sbl.SBL_NO_DX | sbl.SBL_GRAD_F32
+    ws = torch.empty((sbl.backward_workspace_bytes(t, k, flags),), dtype=torch.uint8, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, None, dw, flags, workspace=ws)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(ws.cpu().numpy().view(np.uint16).reshape(t, k), oracle.dequant_act(xq_ref, ap_ref))
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
