@@ -303,8 +303,11 @@ cudaError_t dual_dispatch(const uint16_t* dy, const uint16_t* weff, const uint16
   p.mask_m = mask_m;
   std::copy(sch.off.begin(), sch.off.end(), p.sched_off);
   std::copy(sch.ids.begin(), sch.ids.end(), p.sched);
-  k_gemm_pair<Cfg><<<2 * npairs, pair_threads<Cfg>(), pair_smem_bytes<Cfg>(), s>>>(a0, b0, a1, b1, p);
-  err = counted(cudaGetLastError());
+  // Programmatic dependent launch: the CTAs set up (barriers, tensor memory)
+  // as SMs free up under the kernel before; the producer waits for that
+  // kernel before its first load, and every output write follows the loads.
+  err = launch_pdl(k_gemm_pair<Cfg>, dim3(2 * npairs), dim3(pair_threads<Cfg>()), pair_smem_bytes<Cfg>(), s, a0, b0,
+                   a1, b1, p);
   *done = err == cudaSuccess;
   return err;
 }
