@@ -195,7 +195,7 @@ static cudaError_t bf16_dispatch(const uint16_t* A, const uint16_t* B, int64_t M
   p.status = status;
   p.mask = mask;
   p.mask_m = mask_m;
-  return launch_pair<Cfg>(ta, tb, tb, p, p.M, p.N, num_sms, s);
+  return launch_pair<Cfg>(ta, tb, tb, p, p.M, p.N, num_sms, s, true);  // producer waits before its first load
 }
 
 cudaError_t launch_bf16_gemm(bool a_mn, bool b_mn, bool out_f32, const uint16_t* A, const uint16_t* B, int64_t M,
