@@ -534,26 +534,35 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     gate, up: 2560 -> 6912; down: 6912 -> 2560} at 8192 tokens.  Per step every
     linear re-prepares its weights (mask and codes from its masters) and runs
     its forward; then every backward runs, last layer first.  Each linear has
-    its own masters, activations and upstream gradient; the whole step is one
-    CUDA graph."""
+    its own masters and upstream gradient; q, k and v share their input
+    activations, as do gate and up (as in a transformer block), and each such
+    group quantises them once (sbl_forward, then sbl_forward_quantized).  The
+    whole step is one CUDA graph."""
     import torch
 
     from sparse_linear_layers_bitlinear_b200 import sbl, synth
 
     H, F, T = 2560, 6912, tokens
     shapes = [("q", H, H), ("k", H, H), ("v", H, H), ("o", H, H), ("gate", F, H), ("up", F, H), ("down", H, F)]
+    lead = {"k": "q", "v": "q", "up": "gate"}  # linears that take the activations of another
     lin = []
     for l in range(layers):
+        by_name = {}
         for j, (name, n_out, k) in enumerate(shapes):
             seed = 1000 * l + 10 * j
-            lin.append(dict(
-                layer=sbl.Layer.allocate(n_out, k, n, m, device=dev),
-                w=synth.master_weights(n_out, k, seed, device=dev),
-                x=synth.activations(T, k, seed + 1, device=dev),
-                dy=synth.upstream_grad(T, n_out, seed + 2, device=dev), n_out=n_out, k=k))
+            d = dict(layer=sbl.Layer.allocate(n_out, k, n, m, device=dev),
+                     w=synth.master_weights(n_out, k, seed, device=dev),
+                     dy=synth.upstream_grad(T, n_out, seed + 2, device=dev), n_out=n_out, k=k, shared=name in lead)
+            if name in lead:
+                d["x"], d["xq"], d["ap"] = (by_name[lead[name]][key] for key in ("x", "xq", "ap"))
+            else:
+                d["x"] = synth.activations(T, k, seed + 1, device=dev)
+                d["xq"] = torch.empty((T, k), dtype=torch.int8, device=dev)
+                d["ap"] = torch.empty((T,), dtype=torch.float32, device=dev)
+            by_name[name] = d
+            lin.append(d)
     # outputs reuse one buffer per shape (their values are not read within the step)
     y = {n_out: torch.empty((T, n_out), dtype=torch.float32, device=dev) for n_out in (H, F)}
-    ws = {k: torch.empty(sbl.workspace_bytes(T, k), dtype=torch.uint8, device=dev) for k in (H, F)}
     dx = {k: torch.empty((T, k), dtype=torch.bfloat16, device=dev) for k in (H, F)}
     dw = {(o, k): torch.empty((o, k), dtype=torch.bfloat16, device=dev) for (_, o, k) in shapes}
     s = torch.cuda.Stream(dev)
@@ -561,7 +570,10 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     def step():
         for d in lin:
             sbl.prepare_weights(d["layer"], d["w"], stream=s)
-            sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], workspace=ws[d["k"]], stream=s)
+            if d["shared"]:
+                sbl.forward_quantized(d["layer"], d["xq"], d["ap"], T, y[d["n_out"]], stream=s)
+            else:
+                sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], d["xq"], d["ap"], stream=s)
         for d in reversed(lin):
             sbl.backward(d["layer"], d["x"], d["dy"], T, dx[d["k"]], dw[(d["n_out"], d["k"])], 0, stream=s)
 
@@ -587,10 +599,10 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     hbm, bf16 = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
     i8 = (4.0 if (n, m) == (2, 4) else 2.0) * bf16
     bound = 0.0
-    for (_, n_out, k) in shapes:
+    for (name, n_out, k) in shapes:
         ops = 2.0 * T * n_out * k
         prep_b = n_out * k * 2 + n_out * k * (0.625 if (n, m) == (2, 4) else 1.0)
-        fwd_b = T * k * 2 + T * k + T * n_out * 4
+        fwd_b = (0 if name in lead else T * k * 2) + T * k + T * n_out * 4  # shared inputs are quantised once
         bound += layers * (prep_b / hbm + max(ops / i8, fwd_b / hbm) + 2 * ops / bf16)
     del g
     del lin
@@ -695,6 +707,23 @@ def main():
     code, bits = sbl.read_status(layer)
     assert code == sbl.SBL_OK, (code, bits)
 
+    # The 2:4 forward GEMM alone, before the timed region (a kernel timed by
+    # itself, against the burst peak): the forward from codes
+    # (sbl_forward_quantized) on the activation codes of set 0, L2-resident as
+    # in a step, where the act-quant kernel writes them just before; events
+    # around each call.
+    xq_b = torch.empty((T, K), dtype=torch.int8, device=dev)
+    ap_b = torch.empty((T,), dtype=torch.float32, device=dev)
+    sbl.prepare_weights(layer, sets[0][0])
+    sbl.forward(layer, sets[0][1], T, y, xq_b, ap_b)
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    for e_a, e_b in gev:
+        e_a.record(stream)
+        sbl.forward_quantized(layer, xq_b, ap_b, T, y)
+        e_b.record(stream)
+    torch.cuda.synchronize(dev)
+    gemm_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in gev), world)
+
     # Timed region: the steps back to back.  Events sit only around the
     # backward launch; none between prepare and forward, where one would stop
     # the act-quant kernel from overlapping the weight pack as it does in a
@@ -713,6 +742,7 @@ def main():
         step(i, evs[i])
     torch.cuda.synchronize(dev)
     phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
+
 
     # End to end through the C ABI from pinned host buffers: every step copies
     # its inputs in (H2D), runs the step and copies its outputs back (D2H), all
@@ -818,6 +848,13 @@ def main():
         "phase_roofline_ms": bound_ms,
         "step_roofline_frac": sum(bound_ms.values()) / ms_step,
         "roofline": roof,
+        "fwd_gemm_roofline": {
+            "bound": "tensor", "achieved": A["fwd_gemm_ops"] / (gemm_ms * 1e-3) / 1e12, "peak": 4.0 * peaks["bf16_tflops"],
+            "unit": "TOPS (int8, dense-equivalent)", "frac": A["fwd_gemm_ops"] / (gemm_ms * 1e-3) / 1e12
+            / (4.0 * peaks["bf16_tflops"]), "traffic": ncu_traffic("fwd_gemm"), "launch_ms": gemm_ms,
+            "kernel": "k_gemm_pair<CfgPairSparse> (2:4 forward GEMM)",
+            "timing": "CUDA events around each of 20 sbl_forward_quantized calls, median",
+            "peak_note": f"2:4-sparse int8 = 4 x the {peaks['source']} bf16 burst figure (nominal ratio)"},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches,

@@ -160,6 +160,15 @@ sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl
 sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
                        float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
 
+/* Step 4 from activation codes the caller already holds: xq (int8 [t, k])
+ * and xscale (fp32 [t], the a'_i) exactly as sbl_forward writes them for some
+ * x, e.g. from an earlier call on the same activations.  Writes the same y
+ * (and acc_debug) as sbl_forward on that x, without quantising again, so
+ * layers that share an input (q, k and v; gate and up) quantise it once.
+ * Same dispatch as sbl_forward.  No workspace.  Errors: as sbl_forward. */
+sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const float* xscale, int64_t t, float* y,
+                                 int32_t* acc_debug, sbl_stream_t stream);
+
 /* 1 when sbl_forward on this layer with t tokens takes the decode GEMV over
  * the 2-bit packing, 0 when it takes a tensor-core GEMM (or the arguments
  * are invalid).  Host only, no device access. */

@@ -307,9 +307,12 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const in
   a.n_out = static_cast<int>(n_out);
   a.t = static_cast<int>(t);
   a.k = static_cast<int>(k);
-  if (t <= 1) return gemv_tp<1, false>(a, num_sms, s);
-  if (t <= 2) return gemv_tp<2, false>(a, num_sms, s);
-  if (t <= 4) return gemv_tp<4, false>(a, num_sms, s);
+  // codes from the caller (x == NULL) or from the act-quant kernel before
+  // this one, else quantised here
+  const bool pre = x == nullptr || !gemv_fuses_act_quant(t);
+  if (t <= 1) return pre ? gemv_tp<1, true>(a, num_sms, s) : gemv_tp<1, false>(a, num_sms, s);
+  if (t <= 2) return pre ? gemv_tp<2, true>(a, num_sms, s) : gemv_tp<2, false>(a, num_sms, s);
+  if (t <= 4) return pre ? gemv_tp<4, true>(a, num_sms, s) : gemv_tp<4, false>(a, num_sms, s);
   if (t <= 8) return gemv_tp<8, true>(a, num_sms, s);
   return gemv_tp<16, true>(a, num_sms, s);
 }

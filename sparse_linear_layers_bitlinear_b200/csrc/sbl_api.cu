@@ -198,6 +198,35 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
+sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const float* xscale, int64_t t, float* y,
+                                 int32_t* acc_debug, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (t < 0 || t > (int64_t(1) << 30)) return SBL_ERR_SHAPE;
+  if (t == 0) return SBL_OK;
+  if (xq == nullptr || xscale == nullptr || y == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(xscale) || !aligned16(y) || !aligned16(acc_debug)) return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(layer, L.status);
+  const float* g = at<const float>(layer, L.g);
+  cudaError_t e;
+  if (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) {
+    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), nullptr, xq, xscale, g, layer->n_out, t, layer->k, y,
+                            acc_debug, nullptr, nullptr, status, sms, s);
+  } else if (is_24(layer->n, layer->m)) {
+    e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
+                            static_cast<int>(meta_k_padded(layer->k) / 128), L.sp_meta_bytes, xq, xscale, g,
+                            layer->n_out, t, layer->k, y, acc_debug, status, sms, s);
+  } else {
+    e = launch_forward_gemm(false, at<const int8_t>(layer, L.codes), nullptr, 0, 0, xq, xscale, g, layer->n_out, t,
+                            layer->k, y, acc_debug, status, sms, s);
+  }
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
 size_t sbl_backward_workspace_bytes(int64_t t, int64_t k, uint32_t flags) {
   if (t <= 0 || k <= 0 || (flags & SBL_NO_DW) || !(flags & SBL_DW_QUANT_X)) return 0;
   return size_t(t) * size_t(k) * 2;

@@ -89,6 +89,7 @@ SIGNATURES = {
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
     "sbl_forward_uses_gemv": (ctypes.c_int, [_LP, _I64]),
+    "sbl_forward_quantized": (_I32, [_LP, _P, _P, _I64, _P, _P, _P]),
 }
 
 _lib = None
@@ -181,6 +182,13 @@ def forward(layer: Layer, x, t: int, y, xq_out=None, xscale_out=None, acc_debug=
     cl = layer.c()
     _check(lib().sbl_forward(ctypes.byref(cl), _ptr(x), t, _ptr(y), _ptr(xq_out), _ptr(xscale_out), _ptr(acc_debug),
                              _ptr(workspace), _stream(stream)), "sbl_forward")
+
+
+def forward_quantized(layer: Layer, xq, xscale, t: int, y, acc_debug=None, stream=None):
+    """sbl_forward_quantized: the forward from int8 codes and scales already at hand."""
+    cl = layer.c()
+    _check(lib().sbl_forward_quantized(ctypes.byref(cl), _ptr(xq), _ptr(xscale), t, _ptr(y), _ptr(acc_debug),
+                                       _stream(stream)), "sbl_forward_quantized")
 
 
 def forward_noalloc(layer: Layer, x, t: int, y, acc_debug=None, stream=None):

@@ -159,5 +159,12 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 0, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 1 << 7, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_selftest_wait_timeout(None, 1000, None) == sbl.SBL_ERR_INVALID_ARG
+    p = ctypes.c_void_p
+    assert lib.sbl_forward_quantized(ctypes.byref(layer), None, p(0x3000), 8, p(0x4000), None, None) == \
+        sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_forward_quantized(ctypes.byref(layer), p(0x2000), p(0x3008), 8, p(0x4000), None, None) == \
+        sbl.SBL_ERR_ALIGN
+    assert lib.sbl_forward_quantized(ctypes.byref(layer), None, None, 0, None, None, None) == sbl.SBL_OK
+    assert lib.sbl_forward_quantized(ctypes.byref(layer), None, None, -1, None, None, None) == sbl.SBL_ERR_SHAPE
     # rejected calls enqueue nothing, so they launch nothing
     assert sbl.launch_count() == launched_before

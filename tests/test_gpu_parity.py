@@ -657,3 +657,56 @@ def test_dw_quant_x_operand_on_tie_clamp_and_huge_rows():
     xq_ref, ap_ref = oracle.act_quant(x)
     assert np.array_equal(ws.cpu().numpy().view(np.uint16).reshape(t, k), oracle.dequant_act(xq_ref, ap_ref))
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def test_masked_grad_with_dequantised_operand():
+    """Both backward flags at once: dW = (dY^T . xhat) * mask, dX unchanged."""
+    n_out, k, t = 264, 320, 70
+    w = synth.master_weights(n_out, k, 95)
+    x = synth.activations(t, k, 96)
+    dy = synth.upstream_grad(t, n_out, 97)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(w))
+    ref = oracle.prepare(w, 2, 4)
+    xq_ref, ap_ref = oracle.act_quant(x)
+    dw_ref = oracle.grad_w_masked(dy, oracle.dequant_act(xq_ref, ap_ref), ref["mask"], 4)
+    flags = sbl.SBL_MASKED_GRAD | sbl.SBL_DW_QUANT_X | sbl.SBL_GRAD_F32
+    ws = torch.empty((sbl.backward_workspace_bytes(t, k, flags),), dtype=torch.uint8, device="cuda")
+    dx = torch.empty((t, k), dtype=torch.float32, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, dx, dw, flags, workspace=ws)
+    torch.cuda.synchronize()
+    _close(dw.cpu().numpy(), dw_ref)
+    assert (dw.cpu().numpy()[dw_ref == 0] == 0).all()
+    _close(dx.cpu().numpy(), oracle.grad_x(dy, ref["weff"], ref["g"]))
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+@pytest.mark.parametrize("n,m,flags,t", [(2, 4, 0, 300), (6, 8, 0, 300), (2, 4, sbl.SBL_PACK_GEMV, 3),
+                                          (2, 4, sbl.SBL_PACK_GEMV, 12)])
+def test_forward_from_codes_matches_forward(n, m, flags, t):
+    """sbl_forward_quantized on the codes and scales sbl_forward wrote for x
+    gives the same bits, on the 2:4 GEMM, the dense int8 GEMM and the GEMV
+    (fused-quantisation sizes included), and so does a second layer sharing x."""
+    n_out, k = 392, 512
+    x = synth.activations(t, k, 98)
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    for seed in (99, 100):  # two layers sharing the activations, like q and k
+        w = synth.master_weights(n_out, k, seed)
+        layer = sbl.Layer.allocate(n_out, k, n, m, flags)
+        sbl.prepare_weights(layer, _dev(w))
+        y0 = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+        y1 = torch.full((t, n_out), float("nan"), dtype=torch.float32, device="cuda")
+        acc1 = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+        if seed == 99:
+            sbl.forward(layer, _dev(x), t, y0, xq, ap)
+        else:
+            ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+            sbl.forward(layer, _dev(x), t, y0, workspace=ws)
+        sbl.forward_quantized(layer, xq, ap, t, y1, acc1)
+        torch.cuda.synchronize()
+        assert torch.equal(y0.view(torch.int32), y1.view(torch.int32))
+        ref = oracle.forward(w, x, n, m)
+        assert np.array_equal(acc1.cpu().numpy(), ref["acc"])
+        assert sbl.read_status(layer)[0] == sbl.SBL_OK
