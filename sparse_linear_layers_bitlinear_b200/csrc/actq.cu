@@ -93,10 +93,30 @@ __global__ void __launch_bounds__(kActThreads, 4)
       if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
     const QScale qs = make_qscale(ap);
+    if (qs.exact) {  // the clamp or a' >= 2^120: the IEEE division
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int64_t i = int64_t(r) * kActThreads + tid;
-      if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
+      for (int r = 0; r < R; ++r) {
+        const int64_t i = int64_t(r) * kActThreads + tid;
+        if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
+      }
+    } else {
+      // the division-free codes; a tie in any lane of a vector (threads past
+      // the row hold zeros: never a tie) sends it through the exact path
+      const float c127 = __fdiv_rn(127.0f, ap);
+      const float a_over_127 = DEQ ? __fdiv_rn(ap, 127.0f) : 0.0f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t i = int64_t(r) * kActThreads + tid;
+        bool tie;
+        uint2 c = quantise8_fast(v[r], ap, c127, tie);
+        if (__any_sync(0xFFFFFFFFu, tie)) c = quantise8(v[r], qs);
+        if (i < nvec) {
+          if constexpr (DEQ)
+            reinterpret_cast<uint4*>(out)[row * nvec + i] = dequant8_fast(c, a_over_127);
+          else
+            reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
+        }
+      }
     }
   }
 }
