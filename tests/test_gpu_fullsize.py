@@ -55,11 +55,16 @@ def test_fullsize_parity(name, n_out, k, n, m, t):
     ap = torch.empty((t,), dtype=torch.float32, device="cuda")
     acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
     sbl.forward(layer, x_d, t, y, xq, ap, acc)
+    # the launch the benchmark times: workspace, no accumulator output
+    y2 = torch.full((t, n_out), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, x_d, t, y2, workspace=ws)
     dx = torch.empty((t, k), dtype=torch.bfloat16, device="cuda")
     dw = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
     sbl.backward(layer, x_d, dy_d, t, dx, dw, 0)
     torch.cuda.synchronize()
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
 
     xq_ref, ap_ref = oracle.act_quant(x)
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
@@ -102,3 +107,58 @@ def test_decode_gemv_fullsize(t, n_out):
     ref = oracle.forward(w_d.cpu(), x_d.cpu(), 2, 4)
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (4, 8)])
+def test_fullsize_training_layer(n, m):
+    """One layer of the training-step workload at 8192 tokens: q, k, v, o
+    (2560 x 2560), gate, up (2560 -> 6912), down (6912 -> 2560), with q/k/v and
+    gate/up sharing their activations through sbl_forward_quantized as the
+    benchmark runs them.  Prepare outputs whole, products sampled."""
+    T, H, F = 8192, 2560, 6912
+    shapes = [("q", H, H), ("k", H, H), ("v", H, H), ("o", H, H), ("gate", F, H), ("up", F, H), ("down", H, F)]
+    lead = {"k": "q", "v": "q", "up": "gate"}
+    rng = np.random.default_rng(11)
+    acts = {}
+    for j, (name, n_out, k) in enumerate(shapes):
+        seed = 500 + 10 * j
+        w_d = synth.master_weights(n_out, k, seed, device="cuda")
+        dy_d = synth.upstream_grad(T, n_out, seed + 2, device="cuda")
+        layer = sbl.Layer.allocate(n_out, k, n, m)
+        sbl.prepare_weights(layer, w_d)
+        y = torch.empty((T, n_out), dtype=torch.float32, device="cuda")
+        if name in lead:
+            x_d, xq, ap, xq_ref, ap_ref = acts[lead[name]]
+            sbl.forward_quantized(layer, xq, ap, T, y)
+        else:
+            x_d = synth.activations(T, k, seed + 1, device="cuda")
+            xq = torch.empty((T, k), dtype=torch.int8, device="cuda")
+            ap = torch.empty((T,), dtype=torch.float32, device="cuda")
+            sbl.forward(layer, x_d, T, y, xq, ap)
+            xq_ref, ap_ref = oracle.act_quant(x_d.cpu())
+            acts[name] = (x_d, xq, ap, xq_ref, ap_ref)
+        dx = torch.empty((T, k), dtype=torch.bfloat16, device="cuda")
+        dw = torch.empty((n_out, k), dtype=torch.bfloat16, device="cuda")
+        sbl.backward(layer, x_d, dy_d, T, dx, dw, 0)
+        torch.cuda.synchronize()
+        assert sbl.read_status(layer)[0] == sbl.SBL_OK, name
+
+        w, x, dy = w_d.cpu(), x_d.cpu(), dy_d.cpu()
+        ref = oracle.prepare(w, n, m)
+        gamma, g, _ = bd.header_scalars(layer)
+        assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32), name
+        assert np.array_equal(bd.mask(layer), ref["mask"]), name
+        assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"]), name
+        if name not in lead:
+            assert np.array_equal(xq.cpu().numpy(), xq_ref), name
+        ti, oi = _samples(rng, T, n_out, 200)
+        accs = np.array([oracle.acc_at(xq_ref, ref["weff"], a, b) for a, b in zip(ti, oi)], dtype=np.int32)
+        y_ref = oracle.dequant(accs.reshape(-1, 1), ap_ref[ti], ref["g"]).ravel()
+        assert np.array_equal(y.cpu().numpy()[ti, oi].view(np.uint32), y_ref.view(np.uint32)), name
+        dx_h, dw_h = bd.bf16_to_f64(dx), bd.bf16_to_f64(dw)
+        ti, ki = _samples(rng, T, k, 100)
+        dxr = np.array([oracle.grad_x_at(dy, ref["weff"], ref["g"], a, b) for a, b in zip(ti, ki)])
+        assert (np.abs(dx_h[ti, ki] - dxr) <= 1e-2 + 2.0 ** -7 * np.abs(dxr)).all(), name
+        oi, ki = _samples(rng, n_out, k, 100)
+        dwr = np.array([oracle.grad_w_at(dy, x, a, b) for a, b in zip(oi, ki)])
+        assert (np.abs(dw_h[oi, ki] - dwr) <= 1e-2 + 2.0 ** -7 * np.abs(dwr)).all(), name
