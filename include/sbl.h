@@ -144,6 +144,34 @@ size_t sbl_workspace_bytes(int64_t t, int64_t k);
  * status word.  Raises SBL_ERR_NONFINITE (device) for NaN/Inf masters. */
 sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl_stream_t stream);
 
+/* Tensor parallelism by rows of W (each rank holds n_out / R rows; groups
+ * along k never split).  The scale gamma is the mean |w| over the WHOLE
+ * tensor, so the shards' exact sums are added first:
+ *   1. sbl_weight_abs_sum on each shard writes SBL_SUM_WORDS uint64 words;
+ *   2. the words of all shards are added word by word (an integer sum, e.g.
+ *      an all-reduce with SUM over uint64/int64; exact for up to 16 shards);
+ *   3. sbl_prepare_weights_from_sum prepares each shard with gamma from those
+ *      words over global_numel = (sum of all shards' rows) * k weights.
+ * Every shard then holds the gamma, mask and codes that sbl_prepare_weights
+ * gives the same rows of the whole tensor, bit for bit.  The forward needs no
+ * exchange (output columns are local); dX is the sum of the shards' dX. */
+#define SBL_SUM_WORDS 46
+
+/* Step 1 above: the exact sum of |w| over this shard's masters (bf16
+ * [layer->n_out, layer->k]) as SBL_SUM_WORDS words in sum_out (device, 16-byte
+ * aligned): three words of 32-bit pieces of the window sum, forty bins of
+ * magnitudes outside the window, and counts of non-finite, huge (>= 2^6) and
+ * tiny (< 2^-30) magnitudes.  Uses the layer's blob as scratch for its grid
+ * barrier and resets its status word (SBL_STATUS_NONFINITE_W is raised for
+ * NaN/Inf masters); the prepared sections are left as they were. */
+sbl_status sbl_weight_abs_sum(const sbl_layer* layer, const void* w_master, uint64_t* sum_out, sbl_stream_t stream);
+
+/* Step 3 above: sbl_prepare_weights for this shard with gamma taken from the
+ * summed words `global_sum` (device) over `global_numel` weights
+ * (>= layer->n_out * layer->k, else SBL_ERR_SHAPE). */
+sbl_status sbl_prepare_weights_from_sum(const sbl_layer* layer, const void* w_master, const uint64_t* global_sum,
+                                        int64_t global_numel, sbl_stream_t stream);
+
 /* Step 4.  x: bf16 [t, k] activations.  y: fp32 [t, n_out] output,
  *   y[i, o] = (float)acc[i, o] * ((g * a'_i) / 127),
  *   acc[i, o] = sum_k xq[i, k] * W_eff[o, k]   (int32),

@@ -382,9 +382,19 @@ __device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gmem_
       : "memory");
 }
 
+// What one launch does: the whole preparation; only the exact sum of |w| of
+// this (shard of the) matrix, written out as SBL_SUM_WORDS words; or the
+// preparation with the scale taken from given sum words (the word-wise sum
+// over all shards of a row-sharded matrix) instead of this matrix's own sum.
+enum PrepMode : int { kPrepFull = 0, kPrepSumOnly = 1, kPrepFromSum = 2 };
+
 struct PrepArgs {
   const uint4* w;
   int64_t n_out, k;
+  int mode;                 // PrepMode
+  uint64_t numel;           // weights the mean runs over (all shards' for kPrepFromSum)
+  uint64_t* sum_out;        // kPrepSumOnly: SBL_SUM_WORDS words, written by CTA 0
+  const uint64_t* sum_in;   // kPrepFromSum: SBL_SUM_WORDS words
   int n, m;
   uint32_t layer_flags;
   BlobHeader* h;
@@ -467,10 +477,13 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
     // does not depend on the scale, so refills need not wait for the barrier)
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
-      for (int J = 0; J < 2 * nch; ++J) {
+      // phase-1 chunks (J < nch) then phase-2 chunks; a launch streams only
+      // the phases its mode runs, ring slots counted from its first chunk
+      const int J0 = a.mode == kPrepFromSum ? nch : 0, J1 = a.mode == kPrepSumOnly ? nch : 2 * nch;
+      for (int J = J0; J < J1; ++J) {
         const int j = J < nch ? J : J - nch;
-        const int s = J % kPrepStages;
-        if (J >= kPrepStages && !mbar_wait(&tail->empty[s], ((J / kPrepStages) - 1) & 1, abort_flag, status)) break;
+        const int u = J - J0, s = u % kPrepStages;
+        if (u >= kPrepStages && !mbar_wait(&tail->empty[s], ((u / kPrepStages) - 1) & 1, abort_flag, status)) break;
         const int64_t c0 = v0 + int64_t(j) * kChunkVecs;
         const int64_t cnt = (v1 - c0 < kChunkVecs) ? v1 - c0 : kChunkVecs;
         const uint32_t bytes = static_cast<uint32_t>(cnt) * 16u;
@@ -483,7 +496,7 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
 
   // ---- consumers, phase 1: exact sum of |w| ----
   uint64_t lo = 0, hi = 0;
-  for (int j = 0; j < nch; ++j) {
+  for (int j = 0; j < (a.mode == kPrepFromSum ? 0 : nch); ++j) {
     const int s = j % kPrepStages;
     if (!mbar_wait(&tail->full[s], (j / kPrepStages) & 1, abort_flag, status)) break;
     const int64_t rem = v1 - v0 - int64_t(j) * kChunkVecs;
@@ -540,83 +553,101 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
   // summing the pieces as it goes, so the wait and the fold cost one pass.
   const uint64_t gen0 = tail->gen;
   if (warp == 0) {
-    uint64_t L = lane < kPrepConsumerWarps ? tail->warp_lo[lane] : 0ull;
-    uint64_t H = lane < kPrepConsumerWarps ? tail->warp_hi[lane] : 0ull;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint64_t olo = __shfl_xor_sync(0xffffffffu, L, off), ohi = __shfl_xor_sync(0xffffffffu, H, off);
-      L += olo;
-      H += ohi + ((L < olo) ? 1ull : 0ull);
-    }
-    // flags in the low byte, the count of tiny magnitudes above it (a count
-    // too large to carry forces the exact path, as a huge magnitude does)
-    const uint32_t nt = tail->ntiny;
-    const uint32_t fl_own = (tail->flags | (nt > 0xFFFFFFu ? 4u : 0u)) | ((nt > 0xFFFFFFu ? 0u : nt) << 8);
-    if (fl_own & 2u) {  // slow bins in use: publish them first
-      for (int b = lane; b < kExactBins; b += 32) a.slot_bins[int64_t(blk) * kExactBins + b] = tail->bins[b];
-      __threadfence();
-    }
-    __syncwarp();
-    const uint32_t tagv = static_cast<uint32_t>(gen0 + 1);
-    const uint64_t tag = uint64_t(tagv) << 32;
-    if (lane == 0) {  // H < 2^32: a CTA holds at most 2^40 weights below 2^6, i.e. below 2^83 units
-      uint64_t* sf = a.slot_fast + int64_t(blk) * 4;
-      st_relaxed_u64(sf + 0, tag | (L & 0xFFFFFFFFull));
-      st_relaxed_u64(sf + 1, tag | (L >> 32));
-      st_relaxed_u64(sf + 2, tag | (H & 0xFFFFFFFFull));
-      st_release_u64(sf + 3, tag | fl_own);
-    }
-    uint64_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;  // s3: tiny magnitudes in all CTAs' bins
+    uint64_t s0 = 0, s1 = 0, s2 = 0, s3 = 0;  // the sum in 32-bit pieces; s3: tiny magnitudes in the bins
     uint32_t fl = 0, slow_r = 0;  // slow_r: bit r set when CTA lane + 32 r used its slow bins
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-      bool all = true;
-      s0 = s1 = s2 = s3 = 0;
-      fl = slow_r = 0;
-      auto take = [&](int c, int r) {
-        const ulonglong2* sf = reinterpret_cast<const ulonglong2*>(a.slot_fast + int64_t(c) * 4);
-        const ulonglong2 p01 = ld_relaxed_v2u64(sf), p23 = ld_relaxed_v2u64(sf + 1);
-        all &= ((p01.x >> 32) == tagv) & ((p01.y >> 32) == tagv) & ((p23.x >> 32) == tagv) & ((p23.y >> 32) == tagv);
-        s0 += p01.x & 0xFFFFFFFFull;
-        s1 += p01.y & 0xFFFFFFFFull;
-        s2 += p23.x & 0xFFFFFFFFull;
-        fl |= static_cast<uint32_t>(p23.y) & 0xFFu;
-        s3 += (p23.y >> 8) & 0xFFFFFFull;
-        if (r < 32 && (p23.y & 2u)) slow_r |= 1u << r;
-      };
+    if (a.mode == kPrepFromSum) {
+      // The scale from given sum words (all shards' sums added word by
+      // word): every CTA reads them, so no grid barrier is needed.
+      s0 = a.sum_in[0];
+      s1 = a.sum_in[1];
+      s2 = a.sum_in[2];
+      for (int b = lane; b < kExactBins; b += 32) {
+        const uint64_t v = a.sum_in[3 + b];
+        tail->fold_bins[b] = v;
+        if (v != 0ull) fl = 2u;
+      }
+      fl = __ballot_sync(0xffffffffu, fl != 0u) ? 2u : 0u;
+      if (a.sum_in[3 + kExactBins] != 0ull) fl |= 1u;
+      if (a.sum_in[4 + kExactBins] != 0ull) fl |= 4u;
+      s3 = a.sum_in[5 + kExactBins];
+      __syncwarp();
+    } else {
+      uint64_t L = lane < kPrepConsumerWarps ? tail->warp_lo[lane] : 0ull;
+      uint64_t H = lane < kPrepConsumerWarps ? tail->warp_hi[lane] : 0ull;
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (lane + 32 * r < G) take(lane + 32 * r, r);
-      for (int c = lane + 256, r = 8; c < G; c += 32, ++r) take(c, r);
-      if (__all_sync(0xffffffffu, all)) break;
-      __nanosleep(128);
-      if ((it & 7u) == 7u) {
-        const uint64_t now = globaltimer_ns();
-        if (t0 == 0) {
-          t0 = now;
-        } else if (now - t0 > kWaitLimitNs) {
-          if (lane == 0) {
-            raise_status(status, SBL_STATUS_TIMEOUT);
-            st_relaxed_u64(a.gen, gen0 + 2);
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t olo = __shfl_xor_sync(0xffffffffu, L, off), ohi = __shfl_xor_sync(0xffffffffu, H, off);
+        L += olo;
+        H += ohi + ((L < olo) ? 1ull : 0ull);
+      }
+      // flags in the low byte, the count of tiny magnitudes above it (a count
+      // too large to carry forces the exact path, as a huge magnitude does)
+      const uint32_t nt = tail->ntiny;
+      const uint32_t fl_own = (tail->flags | (nt > 0xFFFFFFu ? 4u : 0u)) | ((nt > 0xFFFFFFu ? 0u : nt) << 8);
+      if (fl_own & 2u) {  // slow bins in use: publish them first
+        for (int b = lane; b < kExactBins; b += 32) a.slot_bins[int64_t(blk) * kExactBins + b] = tail->bins[b];
+        __threadfence();
+      }
+      __syncwarp();
+      const uint32_t tagv = static_cast<uint32_t>(gen0 + 1);
+      const uint64_t tag = uint64_t(tagv) << 32;
+      if (lane == 0) {  // H < 2^32: a CTA holds at most 2^40 weights below 2^6, i.e. below 2^83 units
+        uint64_t* sf = a.slot_fast + int64_t(blk) * 4;
+        st_relaxed_u64(sf + 0, tag | (L & 0xFFFFFFFFull));
+        st_relaxed_u64(sf + 1, tag | (L >> 32));
+        st_relaxed_u64(sf + 2, tag | (H & 0xFFFFFFFFull));
+        st_release_u64(sf + 3, tag | fl_own);
+      }
+      uint64_t t0 = 0;
+      for (uint32_t it = 0;; ++it) {
+        bool all = true;
+        s0 = s1 = s2 = s3 = 0;
+        fl = slow_r = 0;
+        auto take = [&](int c, int r) {
+          const ulonglong2* sf = reinterpret_cast<const ulonglong2*>(a.slot_fast + int64_t(c) * 4);
+          const ulonglong2 p01 = ld_relaxed_v2u64(sf), p23 = ld_relaxed_v2u64(sf + 1);
+          all &= ((p01.x >> 32) == tagv) & ((p01.y >> 32) == tagv) & ((p23.x >> 32) == tagv) & ((p23.y >> 32) == tagv);
+          s0 += p01.x & 0xFFFFFFFFull;
+          s1 += p01.y & 0xFFFFFFFFull;
+          s2 += p23.x & 0xFFFFFFFFull;
+          fl |= static_cast<uint32_t>(p23.y) & 0xFFu;
+          s3 += (p23.y >> 8) & 0xFFFFFFull;
+          if (r < 32 && (p23.y & 2u)) slow_r |= 1u << r;
+        };
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (lane + 32 * r < G) take(lane + 32 * r, r);
+        for (int c = lane + 256, r = 8; c < G; c += 32, ++r) take(c, r);
+        if (__all_sync(0xffffffffu, all)) break;
+        __nanosleep(128);
+        if ((it & 7u) == 7u) {
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > kWaitLimitNs) {
+            if (lane == 0) {
+              raise_status(status, SBL_STATUS_TIMEOUT);
+              st_relaxed_u64(a.gen, gen0 + 2);
+            }
+            break;
           }
-          break;
         }
       }
-    }
-    __threadfence();  // acquire: the slow bins behind the tags are visible from here on
+      __threadfence();  // acquire: the slow bins behind the tags are visible from here on
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      s0 += __shfl_xor_sync(0xffffffffu, s0, off);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, off);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, off);
-      s3 += __shfl_xor_sync(0xffffffffu, s3, off);
-      fl |= __shfl_xor_sync(0xffffffffu, fl, off);
+      for (int off = 16; off > 0; off >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+        s3 += __shfl_xor_sync(0xffffffffu, s3, off);
+        fl |= __shfl_xor_sync(0xffffffffu, fl, off);
+      }
     }
     // the 128-bit total: s0 + s1 * 2^32 + s2 * 2^64 (each below 2^42)
     const uint64_t t1 = s1 << 32;
     const uint64_t Lt = s0 + t1;
     const uint64_t Ht = s2 + (s1 >> 32) + ((Lt < t1) ? 1ull : 0ull);
-    const uint64_t numel = uint64_t(a.n_out) * uint64_t(a.k);
+    const uint64_t numel = a.numel;
     // The fast sum decides gamma unless a weight is non-finite or at least
     // 2^6, or the rounding is too close to call given the tiny magnitudes'
     // bound; every lane computes the same decision.
@@ -628,7 +659,9 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
     } else if (!(fl & 4u)) {
       decided = mean_fp32_fast(Lt, Ht, numel, s3, &gamma);
     }
-    if (!decided && (fl & 2u)) {  // rare: fold the slow bins of the CTAs that used them, lanes over bins
+    // Fold the slow bins of the CTAs that used them, lanes over bins: rarely
+    // needed for the scale; always for a sum-only launch, which writes them.
+    if (a.mode != kPrepFromSum && (fl & 2u) && (!decided || a.mode == kPrepSumOnly)) {
       for (int r = 0; 32 * r < G && r < 32; ++r) {
         uint32_t slow = __ballot_sync(0xffffffffu, (slow_r >> r) & 1u);
         while (slow) {
@@ -643,8 +676,24 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       }
       __syncwarp();
     }
-    if (lane == 0) {
-      if (blk == 0) st_relaxed_u64(a.gen, gen0 + 1);
+    if (a.mode == kPrepSumOnly) {
+      // the sum words: fast sum pieces, slow bins, then counts of non-finite
+      // and huge magnitudes (as 0/1) and of tiny ones; words of shards add up
+      if (blk == 0) {
+        for (int b = lane; b < kExactBins; b += 32) a.sum_out[3 + b] = tail->fold_bins[b];
+        if (lane == 0) {
+          a.sum_out[0] = s0;
+          a.sum_out[1] = s1;
+          a.sum_out[2] = s2;
+          a.sum_out[3 + kExactBins] = (fl & 1u) ? 1ull : 0ull;
+          a.sum_out[4 + kExactBins] = (fl & 4u) ? 1ull : 0ull;
+          a.sum_out[5 + kExactBins] = s3;
+          st_relaxed_u64(a.gen, gen0 + 1);
+          if (fl & 1u) raise_status(status, SBL_STATUS_NONFINITE_W);
+        }
+      }
+    } else if (lane == 0) {
+      if (blk == 0 && a.mode == kPrepFull) st_relaxed_u64(a.gen, gen0 + 1);
       if (!decided) gamma = gamma_exact(tail->fold_bins, Lt, Ht, numel);
       const float g = (gamma > 1e-5f) ? gamma : 1e-5f;  // a NaN gamma gives 1e-5; the status word says why
       tail->g = g;
@@ -664,6 +713,7 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
     }
   }
   consumers_sync();
+  if (a.mode == kPrepSumOnly) return;
   const float g = tail->g;
   // code != 0 <=> 2|w| > g <=> |w| > g/2 (exact) <=> the 15-bit magnitude
   // exceeds bits(g/2) >> 16, i.e. |w| > that bf16 value as a float compare.
@@ -684,8 +734,9 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
   }
   const int64_t meta_rb_bytes = int64_t(a.out.meta_kblocks) * 2048;  // one 128-row block of metadata
   const int step_rows = kChunkVecs / upr, step_cols = kChunkVecs % upr;  // one chunk, in (rows, vectors)
+  const int ring0 = a.mode == kPrepFromSum ? 0 : nch;  // ring slots used before phase 2
   for (int j = 0; j < nch; ++j) {
-    const int J = nch + j, s = J % kPrepStages;
+    const int J = ring0 + j, s = J % kPrepStages;
     if (!mbar_wait(&tail->full[s], (J / kPrepStages) & 1, abort_flag, status)) break;
     const uint4* st = ring + size_t(s) * kChunkVecs;
 #pragma unroll
@@ -805,9 +856,12 @@ static cudaError_t launch_prepare_m(const cudaLaunchConfig_t& cfg, const PrepArg
   return counted(cudaLaunchKernelEx(&cfg, k_prepare<M>, a));
 }
 
+static_assert(3 + kExactBins + 3 == SBL_SUM_WORDS, "sum words: fast pieces, bins, counts");
+
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
-                           uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s) {
-  if (L.sp_meta && (n_out % 256 != 0 || k % 256 != 0)) {
+                           uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s, int mode,
+                           uint64_t* sum_out, const uint64_t* sum_in, uint64_t numel) {
+  if (mode != kPrepSumOnly && L.sp_meta && (n_out % 256 != 0 || k % 256 != 0)) {
     cudaError_t e = cudaMemsetAsync(blob + L.sp_meta, 0x44, L.sp_meta_bytes, s);
     if (e != cudaSuccess) return e;
   }
@@ -815,6 +869,10 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   a.w = reinterpret_cast<const uint4*>(w);
   a.n_out = n_out;
   a.k = k;
+  a.mode = mode;
+  a.numel = numel;
+  a.sum_out = sum_out;
+  a.sum_in = sum_in;
   a.n = n;
   a.m = m;
   a.layer_flags = flags;

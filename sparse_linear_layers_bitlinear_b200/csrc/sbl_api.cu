@@ -142,7 +142,40 @@ sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl
   if ((st = current_device(&sms)) != SBL_OK) return st;
   const cudaError_t e =
       launch_prepare(static_cast<const uint16_t*>(w_master), layer->n_out, layer->k, layer->n, layer->m, layer->flags,
-                     static_cast<uint8_t*>(layer->prepared), L, sms, reinterpret_cast<cudaStream_t>(stream));
+                     static_cast<uint8_t*>(layer->prepared), L, sms, reinterpret_cast<cudaStream_t>(stream), 0,
+                     nullptr, nullptr, uint64_t(layer->n_out) * uint64_t(layer->k));
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_weight_abs_sum(const sbl_layer* layer, const void* w_master, uint64_t* sum_out, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (w_master == nullptr || sum_out == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(w_master) || !aligned16(sum_out)) return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  const cudaError_t e =
+      launch_prepare(static_cast<const uint16_t*>(w_master), layer->n_out, layer->k, layer->n, layer->m, layer->flags,
+                     static_cast<uint8_t*>(layer->prepared), L, sms, reinterpret_cast<cudaStream_t>(stream), 1, sum_out,
+                     nullptr, uint64_t(layer->n_out) * uint64_t(layer->k));
+  return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_prepare_weights_from_sum(const sbl_layer* layer, const void* w_master, const uint64_t* global_sum,
+                                        int64_t global_numel, sbl_stream_t stream) {
+  sbl_blob_layout L;
+  sbl_status st = check_layer(layer, &L);
+  if (st != SBL_OK) return st;
+  if (w_master == nullptr || global_sum == nullptr) return SBL_ERR_INVALID_ARG;
+  if (global_numel < layer->n_out * layer->k) return SBL_ERR_SHAPE;
+  if (!aligned16(w_master) || !aligned16(global_sum)) return SBL_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_device(&sms)) != SBL_OK) return st;
+  const cudaError_t e =
+      launch_prepare(static_cast<const uint16_t*>(w_master), layer->n_out, layer->k, layer->n, layer->m, layer->flags,
+                     static_cast<uint8_t*>(layer->prepared), L, sms, reinterpret_cast<cudaStream_t>(stream), 2, nullptr,
+                     global_sum, uint64_t(global_numel));
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 

@@ -47,8 +47,12 @@ struct PackOut {
   int meta_kblocks;
 };
 
+// mode 0: the whole preparation; 1: only the exact sum of |w| (SBL_SUM_WORDS
+// words to sum_out); 2: the preparation with the scale from sum_in (the sum
+// words of numel weights).
 cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags, uint8_t* blob,
-                           const sbl_blob_layout& L, int num_sms, cudaStream_t s);
+                           const sbl_blob_layout& L, int num_sms, cudaStream_t s, int mode = 0,
+                           uint64_t* sum_out = nullptr, const uint64_t* sum_in = nullptr, uint64_t numel = 0);
 
 // early_trigger: wait for the predecessor, then let the next kernel launch at
 // once (it must wait for this one before reading xq / a_prime).

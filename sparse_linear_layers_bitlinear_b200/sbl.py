@@ -89,6 +89,8 @@ SIGNATURES = {
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
     "sbl_forward_uses_gemv": (ctypes.c_int, [_LP, _I64]),
+    "sbl_weight_abs_sum": (_I32, [_LP, _P, _P, _P]),
+    "sbl_prepare_weights_from_sum": (_I32, [_LP, _P, _P, _I64, _P]),
     "sbl_forward_quantized": (_I32, [_LP, _P, _P, _I64, _P, _P, _P]),
 }
 
@@ -176,6 +178,46 @@ class Layer:
 def prepare_weights(layer: Layer, w_master, stream=None):
     cl = layer.c()
     _check(lib().sbl_prepare_weights(ctypes.byref(cl), _ptr(w_master), _stream(stream)), "sbl_prepare_weights")
+
+
+SBL_SUM_WORDS = 46
+
+
+def weight_abs_sum(layer: Layer, w_shard, sum_out, stream=None):
+    """sbl_weight_abs_sum: this shard's exact sum of |w| as SBL_SUM_WORDS words (int64 CUDA tensor)."""
+    cl = layer.c()
+    _check(lib().sbl_weight_abs_sum(ctypes.byref(cl), _ptr(w_shard), _ptr(sum_out), _stream(stream)),
+           "sbl_weight_abs_sum")
+
+
+def prepare_weights_from_sum(layer: Layer, w_shard, global_sum, global_numel: int, stream=None):
+    """sbl_prepare_weights_from_sum: prepare this shard with the scale of the summed words."""
+    cl = layer.c()
+    _check(lib().sbl_prepare_weights_from_sum(ctypes.byref(cl), _ptr(w_shard), _ptr(global_sum), global_numel,
+                                              _stream(stream)), "sbl_prepare_weights_from_sum")
+
+
+def allreduce_sum_words(words, group=None):
+    """Step 2 of the row-sharded scale: add every rank's sum words, word by
+    word (an exact integer all-reduce; the words are below 2^63)."""
+    import torch.distributed as dist
+
+    dist.all_reduce(words, op=dist.ReduceOp.SUM, group=group)
+    return words
+
+
+def prepare_weights_row_sharded(layer: Layer, w_shard, global_rows: int, group=None, stream=None):
+    """The three steps for this rank's row shard: its exact sum, the exact
+    all-reduce of the words, and the preparation with the whole tensor's scale."""
+    import torch
+
+    words = torch.empty(SBL_SUM_WORDS, dtype=torch.int64, device=w_shard.device)
+    weight_abs_sum(layer, w_shard, words, stream)
+    if stream is not None:
+        stream.synchronize()
+    allreduce_sum_words(words, group)
+    prepare_weights_from_sum(layer, w_shard, words, global_rows * layer.k, stream)
+    return words
 
 
 def forward(layer: Layer, x, t: int, y, xq_out=None, xscale_out=None, acc_debug=None, workspace=None, stream=None):

@@ -54,3 +54,38 @@ def test_two_gloo_ranks_agree_on_the_slowest_time_and_draw_distinct_inputs():
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(3.25, 1) == 3.25
     bench.barrier(1)
+
+
+def _sum_words_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from sparse_linear_layers_bitlinear_b200 import sbl
+
+        # words as a shard's sbl_weight_abs_sum writes them: 32-bit pieces,
+        # 64-bit bins below 2^60, counts
+        g = torch.Generator().manual_seed(100 + rank)
+        words = torch.randint(0, 2 ** 60, (sbl.SBL_SUM_WORDS,), generator=g, dtype=torch.int64)
+        words[:3] = torch.randint(0, 2 ** 32, (3,), generator=g, dtype=torch.int64)
+        mine = words.clone()
+        sbl.allreduce_sum_words(words)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, mine.tolist())
+        out[rank] = (words.tolist(), gathered)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_row_sharded_scale_words_add_exactly_across_two_gloo_ranks():
+    """Step 2 of the row-sharded scale: every rank ends with the word-by-word
+    integer sum of all ranks' sum words (no rounding anywhere)."""
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_sum_words_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    expect = [a + b for a, b in zip(*res[0][1])]
+    assert res[0][0] == res[1][0] == expect
+    assert all(v < 2 ** 63 for v in expect)

@@ -710,3 +710,57 @@ def test_forward_from_codes_matches_forward(n, m, flags, t):
         ref = oracle.forward(w, x, n, m)
         assert np.array_equal(acc1.cpu().numpy(), ref["acc"])
         assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def _row_sharded_prepare(w, n, m, shards):
+    """Row shards of w through the three steps (sum words, word-wise sum,
+    prepare from the sum); returns the shards' layers."""
+    n_out, k = w.shape
+    rows = n_out // shards
+    layers, words = [], []
+    for s in range(shards):
+        wd = _dev(w[s * rows:(s + 1) * rows].contiguous())
+        layer = sbl.Layer.allocate(rows, k, n, m)
+        out = torch.full((sbl.SBL_SUM_WORDS,), -1, dtype=torch.int64, device="cuda")
+        sbl.weight_abs_sum(layer, wd, out)
+        layers.append((layer, wd))
+        words.append(out)
+    total = torch.stack(words).sum(0)
+    for layer, wd in layers:
+        sbl.prepare_weights_from_sum(layer, wd, total, n_out * k)
+    torch.cuda.synchronize()
+    return [layer for layer, _ in layers]
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+@pytest.mark.parametrize("shards", [1, 2, 3])
+@pytest.mark.parametrize("case", ["gaussian", "huge_in_one_shard"])
+def test_row_sharded_prepare_matches_whole_tensor(n, m, shards, case):
+    """Every row shard holds the whole tensor's gamma, mask and codes."""
+    n_out, k = 384, 512
+    w = synth.master_weights(n_out, k, 120 + shards)
+    if case == "huge_in_one_shard":
+        w[n_out - 5, 7] = 96.0  # >= 2^6: the exact path, from the last shard's bins
+        w[3, 9] = 2.0 ** -40    # a tiny magnitude in the first shard
+    ref = oracle.prepare(w, n, m)
+    rows = n_out // shards
+    for s, layer in enumerate(_row_sharded_prepare(w, n, m, shards)):
+        gamma, g = sbl.read_scale(layer)
+        assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
+        assert np.float32(g) == ref["g"]
+        assert np.array_equal(bd.mask(layer), ref["mask"][s * rows:(s + 1) * rows])
+        assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"][s * rows:(s + 1) * rows])
+        assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def test_row_sharded_midpoint_decided_by_a_tiny_magnitude_in_another_shard():
+    """The midpoint construction (in-window mean exactly 1 + 2^-24) split in
+    two shards, the one tiny magnitude in the second: both shards must round
+    gamma up to 1 + 2^-23, as the whole tensor does."""
+    v = np.ones(32 * 256, dtype=np.float32)
+    v[0], v[1] = 3.0, 2.0 ** -11
+    v[16 * 256 + 5] = 2.0 ** -40  # in the second shard's rows
+    w = torch.from_numpy(v.reshape(32, 256)).to(torch.bfloat16)
+    assert float(oracle.absmean_gamma(w)) == 1.0 + 2.0 ** -23
+    for layer in _row_sharded_prepare(w, 2, 4, 2):
+        assert sbl.read_scale(layer) == (1.0 + 2.0 ** -23, 1.0 + 2.0 ** -23)
