@@ -135,7 +135,7 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
   CUtensorMap ta, tb, te;
   const bool acc = acc_out != nullptr;
   if (sparse) {
-    // A: compressed codes [n_out][k/2]; B: xq [t][k], 112-token halves; E:
+    // A: compressed codes [n_out][k/2]; B: xq [t][k], 120-token halves; E:
     // the metadata section viewed as rows of 256 bytes.
     if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k / 2, n_out, k / 2, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||

@@ -377,27 +377,38 @@ struct CfgPairDualBf16 {
 };
 
 // ---------------------------------------------------------------------------
-// 2:4 sparse int8 forward on pairs: tile 256 W rows x 224 tokens, 256 logical
+// 2:4 sparse int8 forward on pairs: tile 256 W rows x BN tokens, 256 logical
 // k per stage.  Each CTA holds its 128 rows of compressed codes (128 x 128
-// bytes), 112 tokens of xq (2 boxes of [112 rows][128 bytes]) and its rows'
-// metadata (2 blocks of 128 rows x 16 bytes, copied to tensor memory).
+// bytes), BN/2 tokens of xq (2 boxes of [BN/2 rows][128 bytes]) and its rows'
+// metadata (2 blocks of 128 rows x 16 bytes, copied to tensor memory).  A
+// stage costs about the same tensor-pipe time from 192 to 240 tokens (the
+// sparse MMA has a large fixed cost per instruction), so the tile is 240
+// tokens wide, the widest that tensor memory holds twice; it never needs more
+// tiles than 224 (the 30-layer training step: 88.1 -> 82.7 ms; the prefill
+// step unchanged within 0.2%).  Tensor memory at 240: accumulators at columns
+// 0 and 256, the two
+// metadata slots in the gap at 240-255 (at 224 tokens: accumulators at 0 and
+// 224, metadata after them at 448).
 // ---------------------------------------------------------------------------
-template <bool ACC_OUT>
+template <bool ACC_OUT, int BN_ = 240>
 struct CfgPairSparse {
   using Params = FwdParams;
   using Tiles = StripedTiles<CfgPairSparse>;
   static constexpr int MAPS = 3;
   static constexpr int EPI_WARPS = 8;  // the fp32 output is the heavy part of this epilogue
-  static constexpr int BN = 224, BK = 256, STAGES = 4;
+  static constexpr int BN = BN_, BK = 256, STAGES = 4;
   static constexpr int A_BYTES = 128 * BK / 2;      // 16 KB
-  static constexpr int B_BYTES = (BN / 2) * BK;     // 28 KB
+  static constexpr int B_BYTES = (BN / 2) * BK;     // 30 KB at 240 tokens
   static constexpr int E_BYTES = 2 * 2048;          // 4 KB
-  static constexpr int ACC_COLS = BN;
+  static constexpr int ACC_COLS = (BN + 31) / 32 * 32;  // accumulator stride, 32-column aligned
   static constexpr int TMEM_COLS = 512;
-  static constexpr int E_COL0 = 2 * BN;             // metadata after the two accumulators
   static constexpr int E_COLS = 8;                  // 2 blocks x 4 columns, two slots
+  static constexpr int E_COL0 = (ACC_COLS - BN >= 2 * E_COLS) ? BN : 2 * ACC_COLS;
   static constexpr uint32_t IDESC = idesc_i8(256, BN, true);
-  static_assert(E_COL0 + 2 * E_COLS <= TMEM_COLS, "tensor memory budget");
+  static_assert(BN % 16 == 0 && BN <= 256, "2-SM MMA tile width");
+  static_assert(ACC_COLS + BN <= TMEM_COLS && E_COL0 + 2 * E_COLS <= TMEM_COLS &&
+                    (E_COL0 >= 2 * ACC_COLS || E_COL0 + 2 * E_COLS <= ACC_COLS),
+                "tensor memory budget: two accumulators and two metadata slots, disjoint");
 
   __device__ static int rows_M(const Params& p) { return p.n_out; }
   __device__ static int cols_N(const Params& p) { return p.T; }
@@ -439,6 +450,16 @@ struct CfgPairSparse {
       tmem_load_wait();
       if (n0 + c * 32 >= p.T) continue;  // uniform across the warp
       fwd_epilogue_chunk<ACC_OUT>(p, r, row, n0 + c * 32, lane, g);
+    }
+    if constexpr (BN % 32 == 16) {  // the last 16 columns
+      constexpr int c = BN / 32;
+      if (c % parts == part) {
+        uint32_t r[16];
+        __syncwarp();
+        tmem_load_32x32b_x16(t_acc + c * 32, r);
+        tmem_load_wait();
+        if (n0 + c * 32 < p.T) fwd_epilogue_chunk<ACC_OUT, 16>(p, r, row, n0 + c * 32, lane, g);
+      }
     }
   }
 };

@@ -341,8 +341,9 @@ struct FwdParams {
 // (a TMEM lane) and holds its 32 int32 accumulators for tokens t0..t0+31;
 // lane j computes token t0+j's scale (g * a') / 127 and shares it with a
 // shuffle.  For each token the warp stores 32 consecutive floats of y.
-template <bool ACC_OUT>
-__device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uint32_t (&r)[32], int o, int t0,
+
+template <bool ACC_OUT, int NC = 32>
+__device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uint32_t (&r)[NC], int o, int t0,
                                                    int lane, float g) {
   const int tl = t0 + lane;
   const float f_mine = (tl < p.T) ? __fdiv_rn(__fmul_rn(g, p.a_prime[tl]), 127.0f) : 0.0f;
@@ -350,9 +351,9 @@ __device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uin
   const int64_t ld = p.n_out;
   float* yp = p.y + int64_t(t0) * ld + o;
   int32_t* ap = ACC_OUT ? p.acc_out + int64_t(t0) * ld + o : nullptr;
-  if (t0 + 32 <= p.T) {  // full chunk: no per-token bound
+  if (t0 + NC <= p.T) {  // full chunk: no per-token bound
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < NC; ++j) {
       const float f = __shfl_sync(0xffffffffu, f_mine, j);
       const int32_t a = static_cast<int32_t>(r[j]);
       if (row_ok) {
@@ -364,7 +365,7 @@ __device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uin
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < NC; ++j) {
       const float f = __shfl_sync(0xffffffffu, f_mine, j);
       const int32_t a = static_cast<int32_t>(r[j]);
       if (row_ok && t0 + j < p.T) {

@@ -764,3 +764,27 @@ def test_row_sharded_midpoint_decided_by_a_tiny_magnitude_in_another_shard():
     assert float(oracle.absmean_gamma(w)) == 1.0 + 2.0 ** -23
     for layer in _row_sharded_prepare(w, 2, 4, 2):
         assert sbl.read_scale(layer) == (1.0 + 2.0 ** -23, 1.0 + 2.0 ** -23)
+
+
+@pytest.mark.parametrize("t", [17000, 16000])
+def test_sparse_forward_many_token_tiles(t):
+    """256 weight rows at token counts on either side of one round of 240-token
+    pair tiles (71 and 67 tiles), with ragged last tiles: the oracle's bits,
+    with and without the accumulator output."""
+    n_out, k = 256, 128
+    w = synth.master_weights(n_out, k, 131)
+    x = synth.activations(t, k, 132)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(w))
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, acc_debug=acc, workspace=ws)
+    y2 = torch.empty_like(y)
+    sbl.forward(layer, _dev(x), t, y2, workspace=ws)  # the launch without accumulator output
+    torch.cuda.synchronize()
+    ref = oracle.forward(w, x, 2, 4)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
