@@ -8,9 +8,10 @@
 // integer max over the bf16 magnitude bits (their order is the order of the
 // values, and a non-finite value shows as bits >= 0x7F80), two halves at a
 // time, then one warp reduction; no block barrier.  All rows of a
-// 4096-token batch are resident at once.  Its codes come without a division
-// (quantise8_fast: the estimate's rounding plus an exact tie check, the IEEE
-// division only for tied vectors and clamped rows).  Longer rows: one block of 128
+// 4096-token batch are resident at once.  Its codes come without a division:
+// one fused multiply-add per element by RU(127 / a'), exact for every row
+// whose a' is a bf16 value (quantise8_fma), the IEEE division only for a row
+// under the 1e-5 clamp or with a' at or above 2^120.  Longer rows: one block of 128
 // threads per row with R vectors a thread (up to 16384 elements), then a
 // two-pass, warp-per-row kernel.
 //
@@ -40,6 +41,26 @@ __device__ __forceinline__ void store_quantised(void* out, int64_t row, int64_t 
     reinterpret_cast<uint4*>(out)[row * nvec + i] = dequantise8(v, qs);
   else
     reinterpret_cast<uint2*>(out)[row * nvec + i] = quantise8(v, qs);
+}
+
+// The codes of one row held in registers (v[r] is vector base + r * stride),
+// for a row whose a' is a bf16 value below 2^120: one fused multiply-add per
+// element (quantise8_fma).
+template <bool DEQ, int R>
+__device__ __forceinline__ void emit_codes(const uint4 (&v)[R], void* out, int64_t row, int64_t nvec, int base,
+                                           int stride, const QScale& qs) {
+  const float a_over_127 = DEQ ? __fdiv_rn(qs.ap, 127.0f) : 0.0f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = int64_t(r) * stride + base;
+    const uint2 c = quantise8_fma(v[r], qs.c);
+    if (i < nvec) {
+      if constexpr (DEQ)
+        reinterpret_cast<uint4*>(out)[row * nvec + i] = dequant8_fast(c, a_over_127);
+      else
+        reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
+    }
+  }
 }
 
 template <int R, bool DEQ>
@@ -99,24 +120,8 @@ __global__ void __launch_bounds__(kActThreads, 4)
         const int64_t i = int64_t(r) * kActThreads + tid;
         if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
       }
-    } else {
-      // the division-free codes; a tie in any lane of a vector (threads past
-      // the row hold zeros: never a tie) sends it through the exact path
-      const float c127 = __fdiv_rn(127.0f, ap);
-      const float a_over_127 = DEQ ? __fdiv_rn(ap, 127.0f) : 0.0f;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t i = int64_t(r) * kActThreads + tid;
-        bool tie;
-        uint2 c = quantise8_fast(v[r], ap, c127, tie);
-        if (__any_sync(0xFFFFFFFFu, tie)) c = quantise8(v[r], qs);
-        if (i < nvec) {
-          if constexpr (DEQ)
-            reinterpret_cast<uint4*>(out)[row * nvec + i] = dequant8_fast(c, a_over_127);
-          else
-            reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
-        }
-      }
+    } else {  // the division-free codes
+      emit_codes<DEQ>(v, out, row, nvec, tid, kActThreads, qs);
     }
   }
 }
@@ -199,24 +204,8 @@ __global__ void __launch_bounds__(kActThreads, DEQ ? 1 : 8)
         const int64_t i = int64_t(r) * 32 + lane;
         if (i < nvec) store_quantised<DEQ>(out, row, nvec, i, v[r], qs);
       }
-    } else {
-      // An exact tie in any lane of a vector (lanes past the row hold zeros:
-      // never a tie) sends that vector through the exact path.
-      const float c127 = __fdiv_rn(127.0f, ap);
-      const float a_over_127 = DEQ ? __fdiv_rn(ap, 127.0f) : 0.0f;
-#pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const int64_t i = int64_t(r) * 32 + lane;
-        bool tie;
-        uint2 c = quantise8_fast(v[r], ap, c127, tie);
-        if (__any_sync(0xFFFFFFFFu, tie)) c = quantise8(v[r], qs);
-        if (i < nvec) {
-          if constexpr (DEQ)
-            reinterpret_cast<uint4*>(out)[row * nvec + i] = dequant8_fast(c, a_over_127);
-          else
-            reinterpret_cast<uint2*>(out)[row * nvec + i] = c;
-        }
-      }
+    } else {  // the division-free codes
+      emit_codes<DEQ>(v, out, row, nvec, lane, 32, qs);
     }
   }
 }

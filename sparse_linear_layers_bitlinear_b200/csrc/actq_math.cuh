@@ -13,78 +13,68 @@ __device__ __forceinline__ float bf16_abs_value(uint32_t bits16) { return __uint
 
 // Per-row constants of the quantiser.
 //
-// The code is the integer nearest to the fp32 quotient fl32(t / a'), t =
-// 127 |x| (exact: 7-bit times 8-bit significands).  When a' is a row maximum
-// it is a bf16 value too, and that integer is found without a division:
-// writing t = T 2^e and a' = A 2^f (T < 2^15, A < 2^8 integers), a quotient
-// Q = t / a' that is not itself a half-integer h lies at least Q / T >= Q 2^-15
-// away from every h (the difference T 2^(e-f) - h A is a non-zero multiple of
-// min(2^(e-f), 1/2)), far more than the error of the estimate t * RN(1/a')
-// (~2^-23 relative) or of the fp32 rounding of Q.  So floor(estimate) is
-// within one of floor(Q), and the sign of the exact remainder
-// (i + 1/2) a' - t (an FMA of short significands) decides between i and
-// i + 1, a zero remainder being the tie that goes to the even code.  The
-// clamped a' = 1e-5 is not a bf16 value, and from a' = 2^120 up the products
-// of that test can overflow fp32; those rows take the IEEE division.
+// The code is rne(Q), Q = 127 |x| / a' (127 |x| is exact in fp32, and the
+// oracle's IEEE quotient rounds to the same integer).  When a' is a row
+// maximum it is a bf16 value too, and rne(Q) comes from one fused
+// multiply-add: the low byte of RN(x * c + 1.5 * 2^23), c = RU(127 / a')
+// rounded UP, whose ulp is 1 (quantise8_fma).  Why that is exact, writing
+// |x| = X 2^p and a' = A 2^q with X, A odd (at most 8 significant bits):
+//   - A quotient that is not a half-integer h lies at least 2^-16 (relative)
+//     from every h: Q - h is a non-zero multiple of 1 / (2A) when p >= q,
+//     of 2^(p-q) / (2A) otherwise, against Q <= 127.  The product x * c is
+//     Q (1 + d) with 0 <= d < 2^-23, so it rounds to the same integer.
+//   - A tie 127 X 2^(p-q+1) = (2n + 1) A needs 127 X = (2n + 1) A.  The prime
+//     127 then divides A (A = 127: a' is 254/128 times a power of two, so
+//     127 / a' is a power of two, c is exact, and the addition rounds the
+//     exact tie to even) or 2n + 1 = 127 (Q = 63.5 at |x| = a' / 2: d > 0
+//     unless a' is a power of two, so |x c| is just above 63.5 and rounds to
+//     the even 64; for a power of two c is exact and the tie rounds to even).
+// The clamped a' = 1e-5 is not a bf16 value, and from a' = 2^120 up the
+// reciprocal leaves the normal range; those rows take the IEEE division.
 struct QScale {
   float ap;    // a'
-  float inv;   // RN(1 / a')
+  float c;     // RU(127 / a'): the multiplier of quantise8_fma
   bool exact;  // a' is the 1e-5 clamp or at least 2^120 (or not finite)
 };
 
 __device__ __forceinline__ QScale make_qscale(float ap) {
-  return QScale{ap, __frcp_rn(ap), ap == 1e-5f || !(ap < 0x1p120f)};
+  return QScale{ap, __fdiv_ru(127.0f, ap), ap == 1e-5f || !(ap < 0x1p120f)};
 }
 
-// One magnitude code: rne(fl32(127 |x|) / a') clamped to 127.
-__device__ __forceinline__ int quant_code(float ax, const QScale& s) {
-  const float t = __fmul_rn(127.0f, ax);
-  if (s.exact) return min(__float2int_rn(__fdiv_rn(t, s.ap)), 127);  // nearest, ties to even
-  const int i0 = __float2int_rd(__fmul_rn(t, s.inv));
-  const float rem = __fmaf_rn(static_cast<float>(i0) + 0.5f, s.ap, -t);
-  const int q = i0 + ((rem < 0.0f || (rem == 0.0f && (i0 & 1))) ? 1 : 0);
-  return min(q, 127);
-}
-
-// The same codes with fewer instructions, for rows whose a' is a bf16 value
-// below 2^120 (QScale::exact false).  On signed values: n = rint(x * RN(127 / a')) (the
-// estimate cannot cross a rounding boundary, as above, and rint is odd-
-// symmetric), then the exact remainder r = 127 x - n a' (n a' and 127 x both
-// have at most 15 significant bits) flags an exact tie, |r| = a' / 2, where the
-// estimate may have rounded either way; `tie` reports one in any of the 8, and
-// the caller then takes quantise8 instead.  A code's byte is the low byte of
-// n + 1.5 * 2^23 (two's complement for |n| <= 127).
-__device__ __forceinline__ uint2 quantise8_fast(const uint4 v, float ap, float c127, bool& tie) {
+// 8 bf16 values -> 8 int8 codes (two words), for a row with QScale::exact
+// false.  A code's byte is the low byte of n + 1.5 * 2^23 (two's complement
+// for |n| <= 127).
+__device__ __forceinline__ uint2 quantise8_fma(const uint4 v, float c) {
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-  const float half = 0.5f * ap;
   uint32_t bytes[8];
-  bool any = false;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const uint32_t w = words[e >> 1];
     const float x = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
-    const float n = rintf(__fmul_rn(x, c127));
-    const float r = __fmaf_rn(127.0f, x, -__fmul_rn(n, ap));
-    any |= fabsf(r) == half;
-    bytes[e] = __float_as_uint(__fadd_rn(n, 12582912.0f));
+    bytes[e] = __float_as_uint(__fmaf_rn(x, c, 12582912.0f));
   }
-  tie = any;
   return make_uint2(__byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040), __byte_perm(bytes[2], bytes[3], 0x0040), 0x5410),
                     __byte_perm(__byte_perm(bytes[4], bytes[5], 0x0040), __byte_perm(bytes[6], bytes[7], 0x0040), 0x5410));
 }
 
-// 8 bf16 values -> 8 int8 codes (two words).
-__device__ __forceinline__ uint2 quantise8(const uint4 v, const QScale& s) {
+// 8 bf16 values -> 8 int8 codes by the IEEE division, for any a':
+// sign(x) * min(rne(fl32(127 |x|) / a'), 127).
+__device__ __forceinline__ uint2 quantise8_div(const uint4 v, float ap) {
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const uint32_t b = (words[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-    const int n = quant_code(bf16_abs_value(b), s);
+    const int n = min(__float2int_rn(__fdiv_rn(__fmul_rn(127.0f, bf16_abs_value(b)), ap)), 127);
     const int code = (b & 0x8000u) ? -n : n;
     packed[e >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (e & 3));
   }
   return make_uint2(packed[0], packed[1]);
+}
+
+// 8 codes by whichever form the row allows (uniform over a row).
+__device__ __forceinline__ uint2 quantise8(const uint4 v, const QScale& s) {
+  return s.exact ? quantise8_div(v, s.ap) : quantise8_fma(v, s.c);
 }
 
 // One code back to bf16: xhat = RN_bf16(code * a' / 127), rounded once from

@@ -529,10 +529,11 @@ def test_dequant_act_row_lengths(k):
 
 def _tie_rows(k):
     """Rows whose quotients 127|x| / a' hit exact half-integers (ties go to the
-    even code), a row under the 1e-5 clamp, a Gaussian row, and ties next to
-    the bf16 maximum."""
+    even code), a row under the 1e-5 clamp, a Gaussian row, ties next to the
+    bf16 maximum, and two rows whose a' has another significand than 254/128,
+    where the only tie is |x| = a'/2 (quotient 63.5, code 64)."""
     rng = np.random.default_rng(61)
-    rows = np.zeros((5, k), dtype=np.float32)
+    rows = np.zeros((7, k), dtype=np.float32)
     halves = np.arange(0, 127) + 0.5                     # 0.5 .. 126.5, all bf16-exact
     rows[0, :127] = halves * rng.choice([-1.0, 1.0], 127)
     rows[0, 127] = 127.0                                 # a' = 127: quotient = |x|
@@ -545,15 +546,28 @@ def _tie_rows(k):
     # and 251 times 2^120, so by the fp32 definition their codes saturate at
     # +-127 (the exact quotients would be the ties 126.5 and 125.5)
     rows[4, :4] = [254.0 * 2.0 ** 120, 253.0 * 2.0 ** 120, -251.0 * 2.0 ** 120, 1.0]
+    # a' = 3: ties at +-1.5, beside values one bf16 step either side of 1.5
+    # and a uniform fill
+    rows[5] = rng.uniform(-2.9, 2.9, size=k)
+    rows[5, 0] = 3.0
+    rows[5, 5:k:37] = 1.5
+    rows[5, 9:k:41] = -1.5
+    rows[5, 3], rows[5, 4] = 1.5078125, -1.4921875
+    # a' = 0.875 (a Gaussian row scaled under it): ties at +-0.4375
+    rows[6] = np.clip(rng.normal(scale=0.25, size=k), -0.87, 0.87)
+    rows[6, 1] = -0.875
+    rows[6, 2:k:29] = 0.4375
+    rows[6, 7:k:31] = -0.4375
     bits = synth.bits(torch.from_numpy(rows).to(torch.bfloat16))
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
 
 
-@pytest.mark.parametrize("gemv", [False, True])
-def test_act_quant_exact_ties_and_clamp(gemv):
+@pytest.mark.parametrize("gemv,k", [(False, 512), (True, 512), (False, 4096)])
+def test_act_quant_exact_ties_and_clamp(gemv, k):
     """The division-free quantiser against the oracle's IEEE division on exact
-    ties and on the clamped scale, in the act-quant kernel and in the GEMV."""
-    n_out, k = 64, 512
+    ties and on the clamped scale, in the act-quant kernels (one warp per row
+    at k = 512, one block per row at 4096) and in the GEMV."""
+    n_out = 64
     x = _tie_rows(k)
     t = x.shape[0]
     flags = sbl.SBL_PACK_GEMV if gemv else 0
@@ -571,6 +585,60 @@ def test_act_quant_exact_ties_and_clamp(gemv):
     assert np.array_equal(np.abs(xq_ref[0, :127].astype(int)), 2 * np.round(np.arange(127) / 2 + 0.25).astype(int))
     assert (np.abs(xq_ref[1, :127].astype(int)) % 2 == 0).all()
     assert list(xq_ref[4, :3]) == [127, 127, -127]
+    xb = x.float().numpy()
+    for r, half in ((5, 1.5), (6, 0.4375)):
+        tied = np.abs(xb[r]) == half
+        assert tied.sum() > 20
+        assert (np.abs(xq_ref[r][tied].astype(int)) == 64).all()
+
+
+def _bf16_grid_rows(k):
+    """One row per bf16 a' of two binades (256 rows): a' itself, then every
+    bf16 magnitude of the 11 binades at and below a''s (those above a' left
+    out), alternating signs, zero-filled: every quotient 127 |x| / a' down to
+    code 0, ties included (a' = 254/128 * 2^e and powers of two among them)."""
+    rows = np.zeros((256, k), dtype=np.float32)
+    for r in range(256):
+        e, mant = r // 128, r % 128
+        ap = (1.0 + mant / 128.0) * 2.0 ** (e - 1)
+        ex = np.arange(e - 11, e)[:, None]
+        xs = ((1.0 + np.arange(128)[None, :] / 128.0) * 2.0 ** (ex - 0.0)).ravel()
+        xs = xs[xs <= ap][: k - 1]
+        xs = xs * np.where(np.arange(xs.size) % 2 == 0, 1.0, -1.0)
+        rows[r, 0] = ap if r % 3 else -ap
+        rows[r, 1:1 + xs.size] = xs
+    return torch.from_numpy(rows).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("k", [1536, 4096])
+def test_act_quant_bf16_grid_bit_exact(k):
+    """The division-free codes against the oracle's IEEE division for every
+    bf16 value below a' in 11 binades, for all 256 bf16 a' of two binades, in
+    the warp-per-row kernel (k = 1536) and the block-per-row kernel (the same
+    values in 4096-wide rows), and the dequantised values xhat of both."""
+    n_out = 64
+    x = _bf16_grid_rows(k)
+    t = x.shape[0]
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 68)))
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    # the grid reaches the ties and the whole code range
+    assert (np.abs(xq_ref) == 64).sum() > 256 and (np.abs(xq_ref) == 127).sum() >= 256
+    # the dequantising form of the same kernels (the dW operand xhat)
+    dy = synth.upstream_grad(t, n_out, 69)
+    flags = sbl.SBL_DW_QUANT_X | sbl.SBL_NO_DX | sbl.SBL_GRAD_F32
+    ws = torch.empty((sbl.backward_workspace_bytes(t, k, flags),), dtype=torch.uint8, device="cuda")
+    dw = torch.empty((n_out, k), dtype=torch.float32, device="cuda")
+    sbl.backward(layer, _dev(x), _dev(dy), t, None, dw, flags, workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(ws.cpu().numpy().view(np.uint16)[: t * k].reshape(t, k), oracle.dequant_act(xq_ref, ap_ref))
 
 
 def test_act_quant_more_rows_than_resident_warps():
