@@ -147,17 +147,18 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
     return acc ? launch_pair<CfgPairSparse<true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true)
                : launch_pair<CfgPairSparse<false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true);
   }
-  // Dense int8 over W_eff codes.  Tile width: 256 tokens unless 192 leaves a
-  // fuller last wave of pair tiles.
+  // Dense int8 over W_eff codes.  Tile width: 192 tokens when that takes no
+  // more rounds of pair tiles than 256, else 256.  A round of 192-token tiles
+  // costs 0.91-0.98 of a round of 256-token ones (the mainloop also pays for
+  // re-reading W once per token block), so the count of rounds decides.
   int max_clusters = 0;
   cudaError_t err = pair_setup<CfgPairDense<false, 256>>(num_sms, &max_clusters);
   if (err != cudaSuccess) return err;
-  auto waste = [&](int bn) {
+  auto rounds = [&](int bn) {
     const int tiles = ((p.n_out + 255) / 256) * ((p.T + bn - 1) / bn);
-    const int rounds = (tiles + max_clusters - 1) / max_clusters;
-    return double(rounds) * bn;  // time ~ rounds x tile width
+    return (tiles + max_clusters - 1) / max_clusters;
   };
-  const bool narrow = waste(192) < waste(256);
+  const bool narrow = rounds(192) <= rounds(256);
   const int bn = narrow ? 192 : 256;
   if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k, n_out, k, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B))
