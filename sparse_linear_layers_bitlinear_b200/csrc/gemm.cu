@@ -44,24 +44,6 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
   return r == CUDA_SUCCESS;
 }
 
-template <class Cfg>
-static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, const typename Cfg::Params& p, int m_rows,
-                             int n_cols, int num_sms, cudaStream_t s) {
-  constexpr int smem = gemm_smem_bytes<Cfg>();
-  static_assert(smem <= 227 * 1024, "shared memory budget");
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm_tc<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  const int tiles = ((m_rows + Cfg::BM - 1) / Cfg::BM) * ((n_cols + Cfg::BN - 1) / Cfg::BN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  if (grid <= 0) return cudaSuccess;
-  k_gemm_tc<Cfg><<<grid, kGemmThreads, smem, s>>>(a, b, p);
-  return counted(cudaGetLastError());
-}
-
 // Pair kernels: grid = two CTAs per concurrently resident cluster, capped by
 // the tile count.
 template <class Cfg>

@@ -21,7 +21,7 @@
 // still signal.
 #pragma once
 
-#include "gemm_tc.cuh"
+#include "gemm_epilogue.cuh"
 
 namespace sbl {
 
@@ -226,7 +226,7 @@ constexpr int pair_smem_bytes() {
 
 // ---------------------------------------------------------------------------
 // bf16 backward on pairs: tile 256 (M) x 256 (N), K 64 per stage.  Each CTA
-// holds A 128 x 64 and B 128 x 64 (its half of N); output as CfgBf16.
+// holds A 128 x 64 and B 128 x 64 (its half of N); output by bf16_epilogue.
 // ---------------------------------------------------------------------------
 template <bool A_MN, bool B_MN, bool OUT_F32>
 struct CfgPairBf16 {
@@ -278,7 +278,7 @@ struct CfgPairBf16 {
 
   __device__ static void epilogue(const Params& p, int, uint32_t t_acc, int row, int n0, int lane, int part,
                                   int parts) {
-    CfgBf16<A_MN, B_MN, OUT_F32>::epilogue(p, t_acc, row, n0, lane, part, parts);
+    bf16_epilogue<OUT_F32>(p, t_acc, row, n0, part, parts);
   }
 };
 
@@ -372,7 +372,7 @@ struct CfgPairDualBf16 {
     q.status = p.status;
     q.mask = prob ? p.mask1 : nullptr;
     q.mask_m = p.mask_m;
-    CfgBf16<false, true, OUT_F32>::epilogue(q, t_acc, row, n0, lane, part, parts);
+    bf16_epilogue<OUT_F32>(q, t_acc, row, n0, part, parts);
   }
 };
 
