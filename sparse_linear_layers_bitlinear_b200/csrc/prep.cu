@@ -734,6 +734,14 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
   }
   const int64_t meta_rb_bytes = int64_t(a.out.meta_kblocks) * 2048;  // one 128-row block of metadata
   const int step_rows = kChunkVecs / upr, step_cols = kChunkVecs % upr;  // one chunk, in (rows, vectors)
+  // This CTA's part of every section, addressed by 32-bit vector offsets
+  // from v0 (u < v1 - v0 < 2^31), so a store address is one multiply-add.
+  const uint32_t nv = static_cast<uint32_t>(v1 - v0);
+  uint8_t* const mask_c = a.out.mask + v0 * (8 / M);
+  uint4* const weff_c = reinterpret_cast<uint4*>(a.out.weff_bf16) + v0;
+  uint2* const codes_c = a.out.codes != nullptr ? reinterpret_cast<uint2*>(a.out.codes) + v0 : nullptr;
+  uint32_t* const spv_c = a.out.sp_values != nullptr ? reinterpret_cast<uint32_t*>(a.out.sp_values) + v0 : nullptr;
+  uint16_t* const gemv_c = a.out.gemv != nullptr ? reinterpret_cast<uint16_t*>(a.out.gemv) + v0 : nullptr;
   const int ring0 = a.mode == kPrepFromSum ? 0 : nch;  // ring slots used before phase 2
   for (int j = 0; j < nch; ++j) {
     const int J = ring0 + j, s = J % kPrepStages;
@@ -742,8 +750,8 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
 #pragma unroll
     for (int h2 = 0; h2 < kVecsPerThread; ++h2) {
       const int e = tid + h2 * kPrepConsumers;
-      const int64_t i = v0 + int64_t(j) * kChunkVecs + e;
-      const bool active = i < v1;  // quads of lanes are all-or-nothing (v1 - v0 and upr are multiples of 8)
+      const uint32_t u = static_cast<uint32_t>(j) * kChunkVecs + e;  // vector v0 + u
+      const bool active = u < nv;
       const uint4 vv = active ? st[e] : make_uint4(0, 0, 0, 0);
       const uint32_t wd[4] = {vv.x, vv.y, vv.z, vv.w};
       uint32_t mw[4], nz[4], key[4];  // magnitudes, code != 0 (0xFFFF per half), selection keys
@@ -798,38 +806,31 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
       if (active) {
         if (M == 2) {
           const uint32_t kept = Z;
-          reinterpret_cast<uint32_t*>(a.out.mask)[i] =
+          reinterpret_cast<uint32_t*>(mask_c)[u] =
               (kept & 3u) | (((kept >> 2) & 3u) << 8) | (((kept >> 4) & 3u) << 16) | (((kept >> 6) & 3u) << 24);
         } else if (M == 4) {
-          reinterpret_cast<uint16_t*>(a.out.mask)[i] = static_cast<uint16_t>(Z);
+          reinterpret_cast<uint16_t*>(mask_c)[u] = static_cast<uint16_t>(Z);
         } else {
-          a.out.mask[i] = static_cast<uint8_t>(Z);
+          mask_c[u] = static_cast<uint8_t>(Z);
         }
-        reinterpret_cast<uint4*>(a.out.weff_bf16)[i] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
-        if (a.out.codes != nullptr)
-          reinterpret_cast<uint2*>(a.out.codes)[i] = make_uint2(codes_of_high_bytes(hb_lo), codes_of_high_bytes(hb_hi));
-      }
-      if (M == 4 && a.out.sp_values != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
-        const uint32_t vals = codes_of_high_bytes(__byte_perm(hb_lo, hb_hi, W));  // the kept codes, index order
-        // tensor-core metadata: [row_block][k_block][128 rows][16 bytes]; this
-        // lane's byte is byte (col % 16) of the row's 16 bytes in k block col / 16.
-        uint32_t word = (Z >> 16) << (8 * (lane & 3));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        if (active) {
-          reinterpret_cast<uint32_t*>(a.out.sp_values)[i] = vals;
-          if ((lane & 3) == 0) {
-            const int64_t r = row[h2];
-            const int c = col[h2];
-            *reinterpret_cast<uint32_t*>(a.out.sp_meta + (r >> 7) * meta_rb_bytes + (r & 127) * 16 + (c >> 4) * 2048 +
-                                         (c & 15)) = word;
-          }
-          if (a.out.gemv != nullptr) {
+        weff_c[u] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
+        if (codes_c != nullptr) codes_c[u] = make_uint2(codes_of_high_bytes(hb_lo), codes_of_high_bytes(hb_hi));
+        if (M == 4 && spv_c != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
+          const uint32_t vals = codes_of_high_bytes(__byte_perm(hb_lo, hb_hi, W));  // the kept codes, index order
+          spv_c[u] = vals;
+          // tensor-core metadata: [row_block][k_block][128 rows][16 bytes];
+          // this vector's byte (its two groups' nibbles) is byte col % 16 of
+          // the row's 16 bytes in k block col / 16.
+          const int64_t r = row[h2];
+          const int c = col[h2];
+          a.out.sp_meta[(r >> 7) * meta_rb_bytes + (r & 127) * 16 + (c >> 4) * 2048 + (c & 15)] =
+              static_cast<uint8_t>(Z >> 16);
+          if (gemv_c != nullptr) {
             // per group: the two kept 2-bit codes (01 = +1, 11 = -1) low, the metadata nibble high
             uint32_t t = vals & 0x03030303u;
             t |= t >> 6;
             const uint32_t nibs = ((Z >> 12) & 0xF0u) | ((Z >> 8) & 0xF000u);
-            reinterpret_cast<uint16_t*>(a.out.gemv)[i] = static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
+            gemv_c[u] = static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
           }
         }
       }
