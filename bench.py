@@ -38,7 +38,8 @@ WORKLOAD = dict(name="prefill 2:4 Sparse-BitLinear fwd+STE bwd, FFN up projectio
 ROTATE = 3  # distinct input sets cycled through the steps (3 x 112 MB > 126 MB L2)
 SUSTAINED_STEPS = 2000  # about 0.6 s of back-to-back steps: the power-capped regime
 
-# Algorithmic work of one step at this workload (Measurement).
+# Algorithmic work of one step at this workload: the minimum bytes each HBM-bound
+# kernel must move and the multiply-adds of each GEMM, the roofline numerators.
 def algorithmic(T, K, N):
     dense_ops = 2.0 * T * K * N                    # one GEMM, dense-equivalent multiply-adds x 2
     return {
