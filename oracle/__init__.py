@@ -12,7 +12,7 @@ operator it computes:
 
   A1 absmean scale            absmean_gamma / clamped_scale
   A2 N:M magnitude mask       nm_mask
-  A3 ternarise, mask, pack    ternary, apply_mask, pack24
+  A3 ternarise, mask, pack    ternary, apply_mask, pack24, pack_nm
   A4 per-token int8 absmax    act_quant
   A5 int32 product            gemm_acc, acc_at
   A6 dequant rescale          dequant
@@ -68,6 +68,7 @@ def _load():
         "sbo_ternary": (None, [P, I64, F, P]),
         "sbo_apply_mask": (None, [P, P, I64, I64, I, P]),
         "sbo_pack24": (None, [P, P, I64, I64, P, P]),
+        "sbo_pack_nm": (None, [P, P, I64, I64, I, I, P, P]),
         "sbo_act_quant": (None, [P, I64, I64, P, P]),
         "sbo_gemm_acc": (I, [P, P, I64, I64, I64, P]),
         "sbo_acc_at": (ctypes.c_int32, [P, P, I64]),
@@ -172,6 +173,20 @@ def pack24(weff: np.ndarray, mask: np.ndarray):
     meta = np.zeros((n_out, k // 8), dtype=np.uint8)
     _load().sbo_pack24(_ptr(weff), _ptr(mask), n_out, k, _ptr(vals), _ptr(meta))
     return vals, meta
+
+
+def pack_nm(weff: np.ndarray, mask: np.ndarray, n: int, m: int):
+    """Compressed-index decode pack of any N:M (blocks of 8 weights): returns
+    (masks8 [n_out, k/8] uint8, codes [n_out, k*n/(4m)] uint8), the kept
+    2-bit codes of each row in index order, least significant bit first."""
+    weff = np.ascontiguousarray(weff, dtype=np.int8)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    n_out, k = weff.shape
+    assert k % 64 == 0
+    masks8 = np.empty((n_out, k // 8), dtype=np.uint8)
+    codes = np.empty((n_out, k * n // (4 * m)), dtype=np.uint8)
+    _load().sbo_pack_nm(_ptr(weff), _ptr(mask), n_out, k, n, m, _ptr(masks8), _ptr(codes))
+    return masks8, codes
 
 
 def act_quant(x):

@@ -262,6 +262,37 @@ void sbo_pack24(const int8_t* weff, const uint8_t* mask, int64_t n_out,
   }
 }
 
+// Compressed-index packing for any N:M.  A block of 8 weights holds 8/m whole
+// groups; its mask byte is their masks side by side, and its kept codes are
+// appended to the row's bit stream in index order, two bits each.
+void sbo_pack_nm(const int8_t* weff, const uint8_t* mask, int64_t n_out,
+                 int64_t k, int n, int m, uint8_t* masks8, uint8_t* codes) {
+  const int64_t blocks = k / 8, groups = k / m;
+  const int64_t row_code_bytes = k * n / (4 * m);
+#pragma omp parallel for schedule(static)
+  for (int64_t row = 0; row < n_out; ++row) {
+    uint8_t* out = codes + row * row_code_bytes;
+    for (int64_t b = 0; b < row_code_bytes; ++b) out[b] = 0;
+    int64_t bit = 0;  // position in this row's code stream
+    for (int64_t blk = 0; blk < blocks; ++blk) {
+      uint32_t mbyte = 0;
+      for (int j = 0; j < 8; ++j) {
+        const int64_t col = blk * 8 + j;
+        const uint8_t gbits = mask[row * groups + col / m];
+        if ((gbits >> (col % m)) & 1u) mbyte |= 1u << j;
+      }
+      masks8[row * blocks + blk] = static_cast<uint8_t>(mbyte);
+      for (int j = 0; j < 8; ++j) {
+        if (!((mbyte >> j) & 1u)) continue;
+        const int8_t q = weff[row * k + blk * 8 + j];
+        const uint32_t code = q == 0 ? 0u : (q > 0 ? 1u : 3u);
+        out[bit / 8] = static_cast<uint8_t>(out[bit / 8] | (code << (bit % 8)));
+        bit += 2;
+      }
+    }
+  }
+}
+
 // A4.  Per-token absmax int8 quantisation (READING: the pages do not describe
 // activation quantisation; this is the BitNet b1.58 convention).
 void sbo_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq,

@@ -70,6 +70,18 @@ void sbo_apply_mask(const int8_t* q, const uint8_t* mask, int64_t n_out,
 void sbo_pack24(const int8_t* weff, const uint8_t* mask, int64_t n_out,
                 int64_t k, int8_t* vals, uint8_t* meta);
 
+/* Compressed-index packing of weff for any N:M (the "explicit N:M metadata"
+ * of [ja] §2.1 with the kept values beside it), the decode pack of every
+ * pattern other than 2:4.  READING of the layout: the row is cut into blocks
+ * of 8 consecutive weights (8/m whole groups each).  masks8[row, k/8] is the
+ * block's mask byte (bit j = position j kept; the groups' masks side by
+ * side), and the kept weights' 2-bit codes (01 = +1, 11 = -1, 00 = 0) follow
+ * in index order, 2*n8 bits per block with n8 = 8n/m, packed least
+ * significant bit first into one bit stream per row: codes[row, k*n/(4m)]
+ * bytes.  Requires k % 64 == 0. */
+void sbo_pack_nm(const int8_t* weff, const uint8_t* mask, int64_t n_out,
+                 int64_t k, int n, int m, uint8_t* masks8, uint8_t* codes);
+
 /* A4 (per-token int8 absmax; not on the pages, READING): a = max_k |x|,
  * a' = max(a, 1e-5f), xq = sign(x) * rne(fl32(127|x|) / a'), clamped to
  * [-128, 127]; a_prime[t] = a'.  All fp32 IEEE operations. */

@@ -328,6 +328,59 @@ def test_pack24_round_trip():
     assert np.array_equal(rebuilt, p["weff"])
 
 
+def test_pack_nm_golden_cases():
+    """Hand-worked bytes of the compressed-index pack (mask byte per block of
+    8, kept 2-bit codes in index order, least significant bit first)."""
+    for case in _golden("pack_nm_cases.json")["cases"]:
+        n, m, k = case["n"], case["m"], 64
+        weff = np.zeros((1, k), dtype=np.int8)
+        mask = np.full((1, k // m), case["rest_group_mask"], dtype=np.uint8)
+        for b, blk in enumerate(case["blocks"]):
+            weff[0, 8 * b:8 * b + 8] = blk["weff"]
+            mask[0, b * (8 // m):(b + 1) * (8 // m)] = blk["group_masks"]
+        masks8, codes = oracle.pack_nm(weff, mask, n, m)
+        assert list(masks8[0]) == case["masks8"], case["why"]
+        assert list(codes[0]) == case["codes"], case["why"]
+
+
+def _unpack_nm(masks8, codes, n, m, k):
+    """Decode the compressed-index pack back to dense codes, block by block."""
+    n_out = masks8.shape[0]
+    out = np.zeros((n_out, k), dtype=np.int8)
+    value = {0: 0, 1: 1, 3: -1}
+    for r in range(n_out):
+        stream = int.from_bytes(codes[r].tobytes(), "little")
+        pos = 0
+        for b in range(k // 8):
+            mb = int(masks8[r, b])
+            for j in range(8):
+                if mb >> j & 1:
+                    c = (stream >> pos) & 3
+                    assert c != 2, "code 10 is never written"
+                    out[r, 8 * b + j] = value[c]
+                    pos += 2
+        assert pos == 2 * (8 * n // m) * (k // 8)
+    return out
+
+
+@pytest.mark.parametrize("n,m", [(6, 8), (4, 8), (3, 8), (1, 8), (7, 8), (8, 8), (1, 4), (3, 4), (1, 2), (2, 4)])
+def test_pack_nm_round_trip_and_invariants(n, m):
+    """The pack decodes back to W_eff exactly; every block keeps 8n/m
+    positions, each group of m exactly n, and they are the mask's."""
+    k = 128
+    w = synth.master_weights(12, k, seed=40 + 8 * n + m)
+    p = oracle.prepare(w, n, m)
+    masks8, codes = oracle.pack_nm(p["weff"], p["mask"], n, m)
+    assert masks8.shape == (12, k // 8) and codes.shape == (12, k * n // (4 * m))
+    bits = np.unpackbits(masks8[..., None], axis=-1, bitorder="little").reshape(12, k)
+    assert (bits.reshape(12, -1, m).sum(-1) == n).all()
+    dense_mask = np.unpackbits(p["mask"][..., None], axis=-1, bitorder="little")[..., :m].reshape(12, k)
+    assert np.array_equal(bits, dense_mask)
+    assert np.array_equal(_unpack_nm(masks8, codes, n, m, k), p["weff"])
+    # the pack is no larger than 1 + 2n/m bits per weight (2.5 at 6:8)
+    assert masks8.nbytes + codes.nbytes == 12 * k * (1 + 2 * n / m) / 8
+
+
 # ---------------------------------------------------------------------------
 # A4: activation quantisation
 # ---------------------------------------------------------------------------
