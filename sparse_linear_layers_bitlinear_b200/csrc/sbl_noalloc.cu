@@ -35,10 +35,12 @@ std::mutex g_slots_mutex;
 
 // In host code `g_noalloc_scratch` names a host-side shadow, not device
 // memory, so its device address is looked up once per device, with that
-// device current, and cached.
+// device current, and cached by device ordinal (the cache is not told about a
+// cudaDeviceReset; see include/sbl.h).
 sbl_status scratch_on_current_device(uint8_t** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBL_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SBL_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SBL_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_slots_mutex);
   ScratchSlot& s = g_slots[dev];
   if (!s.ready) {
@@ -64,6 +66,12 @@ extern "C" sbl_status sbl_forward_noalloc(const sbl_layer* layer, const void* x,
   const uint64_t codes_bytes = sbl::align_up(uint64_t(t) * uint64_t(layer->k), 256);
   const uint64_t scale_bytes = sbl::align_up(uint64_t(t) * 4u, 256);
   if (codes_bytes + scale_bytes > SBL_NOALLOC_SCRATCH_BYTES) return SBL_ERR_SCRATCH;
+  // The argument checks of sbl_forward that need no device come first, so a
+  // rejected call never reaches the scratch set-up below.
+  if (layer->prepared == nullptr || x == nullptr || y == nullptr) return SBL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(layer->prepared) & 255u) != 0 || (reinterpret_cast<uintptr_t>(x) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(y) & 15u) != 0 || (reinterpret_cast<uintptr_t>(acc_debug) & 15u) != 0)
+    return SBL_ERR_ALIGN;
   uint8_t* scratch = nullptr;
   const sbl_status sst = scratch_on_current_device(&scratch);
   if (sst != SBL_OK) return sst;

@@ -40,6 +40,20 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     assert lib.sbl_forward_noalloc(None, dummy, 4, dummy, None, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_forward_noalloc(ctypes.byref(layer), None, 0, None, None, None) == sbl.SBL_OK
     assert t_max * k + 4 * t_max < sbl.NOALLOC_SCRATCH_BYTES
+    # bad pointers are rejected before the scratch lookup touches a device
+    assert lib.sbl_forward_noalloc(ctypes.byref(layer), None, 4, dummy, None, None) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_forward_noalloc(ctypes.byref(layer), ctypes.c_void_p(0x2008), 4, dummy, None, None) == \
+        sbl.SBL_ERR_ALIGN
+    assert lib.sbl_forward_noalloc(ctypes.byref(layer), dummy, 4, dummy, ctypes.c_void_p(0x3004), None) == \
+        sbl.SBL_ERR_ALIGN
+    unprepared = sbl.sbl_layer(256, k, 2, 4, 0, None)
+    assert lib.sbl_forward_noalloc(ctypes.byref(unprepared), dummy, 4, dummy, None, None) == sbl.SBL_ERR_INVALID_ARG
+    # the exact limit: k = 2048 and t = 8176 fill the 16 MiB to the byte
+    # (codes, then the scales from the next 256-byte boundary)
+    align256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    assert align256(8176 * 2048) + align256(8176 * 4) == sbl.NOALLOC_SCRATCH_BYTES
+    wide = sbl.sbl_layer(256, 2048, 2, 4, 0, 0x1000)
+    assert lib.sbl_forward_noalloc(ctypes.byref(wide), dummy, 8177, dummy, None, None) == sbl.SBL_ERR_SCRATCH
 
 
 @pytest.mark.gpu
@@ -65,3 +79,50 @@ def test_noalloc_forward_matches_forward_on_two_calls(n, m):
         assert torch.equal(acc, acc_ref)
         _close(y.cpu().numpy(), y_ref.cpu().numpy())
         assert torch.equal(y, y_ref)
+
+
+def _compare_with_forward(layer, t, seed):
+    """One sbl_forward_noalloc call against sbl_forward with a workspace on the
+    same inputs: accumulators and y bit for bit."""
+    k, n_out = layer.k, layer.n_out
+    x = synth.activations(t, k, seed, device="cuda")
+    y_ref = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc_ref = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, x, t, y_ref, acc_debug=acc_ref, workspace=ws)
+    y = torch.full((t, n_out), float("nan"), dtype=torch.float32, device="cuda")
+    acc = torch.zeros((t, n_out), dtype=torch.int32, device="cuda")
+    sbl.forward_noalloc(layer, x, t, y, acc)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    assert torch.equal(acc, acc_ref)
+    _close(y.cpu().numpy(), y_ref.cpu().numpy())
+    assert torch.equal(y, y_ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+def test_noalloc_through_the_decode_kernel_over_stale_scratch(n, m):
+    """A layer with the decode pack: a large call first fills the scratch,
+    then decode-sized calls (the kernel quantises t <= 8 itself and writes the
+    codes into the scratch; t = 16 runs the act-quant kernel into it first)."""
+    n_out, k = 392, 1024
+    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, synth.master_weights(n_out, k, 33, device="cuda"))
+    for i, t in enumerate((300, 1, 4, 16)):
+        assert sbl.forward_uses_gemv(layer, t) == (t <= 32)
+        _compare_with_forward(layer, t, 50 + i)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_its_exact_limit():
+    """t = 8176 at k = 2048: codes and scales fill the 16 MiB to the byte, so
+    the scales sit in its last 32 KB; one token more is refused."""
+    n_out, k, t = 256, 2048, 8176
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, synth.master_weights(n_out, k, 34, device="cuda"))
+    _compare_with_forward(layer, t, 60)
+    x = torch.zeros((t + 1, k), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((t + 1, n_out), dtype=torch.float32, device="cuda")
+    with pytest.raises(sbl.SblError):
+        sbl.forward_noalloc(layer, x, t + 1, y)
