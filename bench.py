@@ -282,6 +282,13 @@ def cpu_baseline(T, K, N, n, m, target_s=12.0, target_1t_s=10.0):
                               "sample": fit_1t.describe(fit_1t.step_s)}}
 
 
+def workload_config(world: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": WORKLOAD["name"], "tokens": WORKLOAD["tokens"], "k": WORKLOAD["k"], "n_out": WORKLOAD["n_out"],
+            "n": WORKLOAD["n"], "m": WORKLOAD["m"], "parallelism": f"replicas x{world}",
+            "l2": f"inputs rotate over {ROTATE} seeded sets (3 x 112 MB > 126 MB L2)"}
+
+
 def run_reference(args):
     """The oracle as the reference arm, timed on the host cores."""
     import oracle
@@ -296,15 +303,20 @@ def run_reference(args):
     fit = OracleFit(wb, xb, dyb, T, n, m, per_step)
     for _ in range(args.warmup):
         fit.sample()
+    t_run = time.perf_counter()
     est = [fit.sample() for _ in range(args.steps)]
+    sample_s = (time.perf_counter() - t_run) / max(1, args.steps)  # wall seconds of one timed sample
     step_s = statistics.mean(est)
     value = T / step_s
-    sample = "per step: " + fit.describe(step_s)
+    sample = ("per step: " + fit.describe(step_s) + "; ms_per_step is that extrapolated full step, "
+              "sample_s_per_step the measured seconds of the sample behind it")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i64/f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD["name"], "tokens": T, "k": K, "n_out": N, "n": n, "m": m},
+        "config": workload_config(args.gpus),
+        "extrapolated": True,
+        "sample_s_per_step": sample_s,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -315,62 +327,82 @@ def run_reference(args):
 # Other workloads, reported beside the headline line
 # ---------------------------------------------------------------------------
 def bench_decode(dev, hbm_gbs, reps=10):
-    """Decode-shaped forward on layers with the 2-bit weight packing: T in
-    {1, 4, 16}, K = 2560, N_out in {2560, 6912}; the library sends each call
-    to the 2-bit GEMV or the 2:4 tensor-core GEMM, whichever is faster.  One replay = 64 forward calls in a CUDA
-    graph over distinct weight blobs (more than 2 x L2 of weights in total),
-    so every call streams its weights from HBM.  The per-call time includes the
-    launch of each call inside the graph."""
+    """Decode-shaped forward: T in {1, 4, 16, 32}, K = 2560, N_out in {2560,
+    6912}, on layers prepared with the decode pack: 2:4 (2-bit codes and
+    metadata, 2 bits a weight) and 6:8 (the compressed-index pack, 2.5 bits a
+    weight).  One replay of a CUDA graph makes one call per distinct weight
+    blob, the blobs holding more than 2 x L2 of packed weights, so every call
+    streams its weights from HBM; the per-call time is the replay time over
+    the calls and includes each call's launch inside the graph.  `floor_us`
+    is the same chain of empty library launches (programmatic dependent
+    launch, as every call is launched): what a chain of dependent calls pays
+    before any work.  `hbm_frac` is the call's bytes (weights, bf16 x, fp32 y)
+    over the per-call time against the measured HBM copy rate."""
     import torch
 
     from sparse_linear_layers_bitlinear_b200 import sbl, synth
 
     K = 2560
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def per_call_us(body, calls, s):
+        with torch.cuda.stream(s):
+            for i in range(min(3, calls)):
+                body(i)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(calls):
+                body(i)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / (calls * reps) * 1e3
+
     out = []
-    for N in (2560, 6912):
-        nblob = max(8, int(2 * 126e6 / (N * K / 4)) + 1)
-        layers = []
-        for i in range(nblob):
-            L = sbl.Layer.allocate(N, K, 2, 4, sbl.SBL_PACK_GEMV, device=dev)
-            sbl.prepare_weights(L, synth.master_weights(N, K, 5000 + i, device=dev))
-            layers.append(L)
-        for T in (1, 4, 16):
-            x = synth.activations(T, K, 7, device=dev)
-            y = torch.empty((T, N), dtype=torch.float32, device=dev)
-            ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    floors = {}
+    for (n, m) in ((2, 4), (6, 8)):
+        for N in (2560, 6912):
+            wbytes = sbl.prepared_layout(N, K, n, m, sbl.SBL_PACK_GEMV).gemv_bytes
+            nblob = max(16, int(2.2 * 126e6 / wbytes) + 1)
+            layers = []
+            for i in range(nblob):
+                L = sbl.Layer.allocate(N, K, n, m, sbl.SBL_PACK_GEMV, device=dev)
+                sbl.prepare_weights(L, synth.master_weights(N, K, 5000 + i, device=dev))
+                layers.append(L)
             s = torch.cuda.Stream(dev)
-            with torch.cuda.stream(s):
-                for i in range(3):
-                    sbl.forward(layers[i % nblob], x, T, y, workspace=ws, stream=s)
-            torch.cuda.synchronize(dev)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
-                for i in range(64):
-                    sbl.forward(layers[i % nblob], x, T, y, workspace=ws, stream=s)
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(reps):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize(dev)
-            us = e0.elapsed_time(e1) / (64 * reps) * 1e3
-            gemv = sbl.forward_uses_gemv(layers[0], T)
-            # weight bytes of the path taken: 2-bit packing, or 2:4 values + metadata
-            wbytes = N * K / 4 if gemv else N * K / 2 + N * K / 8
-            by = wbytes + 2 * T * K + 4 * T * N
-            out.append({"n_out": N, "k": K, "tokens": T, "path": "gemv" if gemv else "2:4 tensor-core GEMM",
-                        "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
-                        "gbs": by / (us * 1e-6) / 1e9, "hbm_frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
-                        "bytes_per_call": by})
-            del g
-        del layers
-        torch.cuda.empty_cache()
-    return {"workload": "decode 2:4 forward on layers with the 2-bit packing, K=2560; each call takes the "
-                        "faster path for its size (`path`)",
-            "timing": "CUDA graph of 64 calls over distinct weight blobs (> 2 x L2), per-call time incl. launch",
+            if nblob not in floors:
+                floors[nblob] = per_call_us(lambda i: sbl.selftest_chain_floor(sms, stream=s), nblob, s)
+            for T in (1, 4, 16, 32):
+                x = synth.activations(T, K, 7, device=dev)
+                y = torch.empty((T, N), dtype=torch.float32, device=dev)
+                ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+                us = per_call_us(lambda i: sbl.forward(layers[i], x, T, y, workspace=ws, stream=s), nblob, s)
+                dec = sbl.forward_uses_gemv(layers[0], T)
+                # weight bytes of the path taken: the decode pack, or the GEMM's int8 operand
+                wb = wbytes if dec else (N * K * 0.625 if (n, m) == (2, 4) else N * K)
+                by = wb + 2 * T * K + 4 * T * N
+                floor = floors[nblob]
+                out.append({"pattern": f"{n}:{m}", "n_out": N, "k": K, "tokens": T,
+                            "path": "decode kernel" if dec else "tensor-core GEMM",
+                            "us_per_call": us, "floor_us": floor, "tokens_per_s": T / (us * 1e-6),
+                            "bytes_per_call": by, "gbs": by / (us * 1e-6) / 1e9,
+                            "hbm_frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+                            "over_floor_and_stream_us": us - floor - by / (hbm_gbs * 1e3),
+                            "calls_per_replay": nblob})
+            del layers
+            torch.cuda.empty_cache()
+    return {"workload": "decode forward on layers with the decode pack (2:4 at 2 bits a weight, 6:8 compressed "
+                        "index at 2.5), K=2560; each call takes the faster path for its size (`path`)",
+            "timing": "CUDA graph of one call per distinct weight blob (> 2 x L2 of packed weights), per-call "
+                      "time incl. launch; floor = the same chain of empty PDL launches",
             "points": out}
 
 
@@ -568,6 +600,21 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     dw = {(o, k): torch.empty((o, k), dtype=torch.bfloat16, device=dev) for (_, o, k) in shapes}
     s = torch.cuda.Stream(dev)
 
+    def prepare_phase():
+        for d in lin:
+            sbl.prepare_weights(d["layer"], d["w"], stream=s)
+
+    def forward_phase():
+        for d in lin:
+            if d["shared"]:
+                sbl.forward_quantized(d["layer"], d["xq"], d["ap"], T, y[d["n_out"]], stream=s)
+            else:
+                sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], d["xq"], d["ap"], stream=s)
+
+    def backward_phase():
+        for d in reversed(lin):
+            sbl.backward(d["layer"], d["x"], d["dy"], T, dx[d["k"]], dw[(d["n_out"], d["k"])], 0, stream=s)
+
     def step():
         for d in lin:
             sbl.prepare_weights(d["layer"], d["w"], stream=s)
@@ -575,8 +622,7 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
                 sbl.forward_quantized(d["layer"], d["xq"], d["ap"], T, y[d["n_out"]], stream=s)
             else:
                 sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], d["xq"], d["ap"], stream=s)
-        for d in reversed(lin):
-            sbl.backward(d["layer"], d["x"], d["dy"], T, dx[d["k"]], dw[(d["n_out"], d["k"])], 0, stream=s)
+        backward_phase()
 
     with torch.cuda.stream(s):
         step()
@@ -593,25 +639,57 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     e1.record()
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
+    del g
+    # The phases on their own: one graph per phase (all prepares; all
+    # act-quants and forwards; all backwards), replayed in step order.
+    graphs = []
+    for body in (prepare_phase, forward_phase, backward_phase):
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp, stream=s):
+            body()
+        graphs.append(gp)
+    for gp in graphs:
+        gp.replay()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    phase = [0.0, 0.0, 0.0]
+    for _ in range(steps):
+        with torch.cuda.stream(s):
+            for i, gp in enumerate(graphs):
+                ev[i].record(s)
+                gp.replay()
+            ev[3].record(s)
+        torch.cuda.synchronize(dev)
+        for i in range(3):
+            phase[i] += ev[i].elapsed_time(ev[i + 1]) / steps
+    del graphs
     for d in lin[:7]:
         code, bits = sbl.read_status(d["layer"])
         assert code == sbl.SBL_OK, (code, bits)
     # roofline of the step at the measured peaks
     hbm, bf16 = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
     i8 = (4.0 if (n, m) == (2, 4) else 2.0) * bf16
-    bound = 0.0
+    bound = {"prepare": 0.0, "forward": 0.0, "backward": 0.0}
     for (name, n_out, k) in shapes:
         ops = 2.0 * T * n_out * k
         prep_b = n_out * k * 2 + n_out * k * (0.625 if (n, m) == (2, 4) else 1.0)
         fwd_b = (0 if name in lead else T * k * 2) + T * k + T * n_out * 4  # shared inputs are quantised once
-        bound += layers * (prep_b / hbm + max(ops / i8, fwd_b / hbm) + 2 * ops / bf16)
-    del g
+        bound["prepare"] += layers * prep_b / hbm
+        bound["forward"] += layers * max(ops / i8, fwd_b / hbm)
+        bound["backward"] += layers * 2 * ops / bf16
+    total = sum(bound.values())
     del lin
     torch.cuda.empty_cache()
+    names = ("prepare", "forward", "backward")
     return {"workload": f"training step, {layers} layers x 7 linears, {n}:{m}", "tokens": T, "n": n, "m": m,
-            "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "roofline_ms": bound * 1e3,
-            "roofline_frac": bound * 1e3 / ms, "peak_note": "sustained bf16 peak (seconds-long step)",
-            "timing": f"one CUDA graph per step, {steps} replays after one warm-up"}
+            "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "roofline_ms": total * 1e3,
+            "roofline_frac": total * 1e3 / ms, "peak_note": "sustained bf16 peak (seconds-long step)",
+            "phase_ms": dict(zip(names, phase)),
+            "phase_roofline_ms": {k: v * 1e3 for k, v in bound.items()},
+            "phase_frac": {k: bound[k] * 1e3 / phase[i] for i, k in enumerate(names)},
+            "timing": f"one CUDA graph per step, {steps} replays after one warm-up; phase_ms: one graph per phase "
+                      f"(all 210 prepares; all act-quants and forwards; all backwards), replayed in step order, "
+                      f"events between them"}
 
 
 # ---------------------------------------------------------------------------
@@ -841,9 +919,7 @@ def main():
         "metric": METRIC, "value": tokens_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "i8xternary->i32 fwd, bf16->f32 bwd", "data": "synthetic",
-        "config": {"workload": WORKLOAD["name"], "tokens": T, "k": K, "n_out": N, "n": n, "m": m,
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotate over {ROTATE} seeded sets (3 x 112 MB > 126 MB L2)"},
+        "config": workload_config(world),
         "tops": A["step_ops"] * world / (ms_step * 1e-3) / 1e12,
         "phase_ms": dict(zip(names, phase_ms)),
         "phase_roofline_ms": bound_ms,

@@ -68,7 +68,9 @@ typedef enum sbl_status {
 
 /* Flags of sbl_layer.flags (fixed at prepare time). */
 enum {
-  SBL_PACK_GEMV = 1u << 0,      /* also write the 2-bit decode packing (2:4 only) */
+  SBL_PACK_GEMV = 1u << 0,      /* also write the decode pack that sbl_forward streams for
+                                   t <= 32 tokens (2:4: 2 bits a weight; other N:M: the
+                                   compressed-index pack, 1 + 2n/m bits a weight) */
   SBL_MASK_FROM_QUANT = 1u << 1 /* ablation the pages report ([de] 4 "Ablationsstudien",
                                    [fr] 5): build the N:M mask from the ternary codes
                                    |q| instead of the masters (ties to the lowest index) */
@@ -108,20 +110,35 @@ typedef struct sbl_blob_layout {
   uint64_t sp_values;   /* int8 [n_out, k/2]: the two kept codes of each group of 4 (2:4) */
   uint64_t sp_meta;     /* tensor-core metadata (2:4), sp_meta_bytes bytes; see below */
   uint64_t sp_meta_bytes;
-  uint64_t gemv;        /* uint8 [n_out, k/4]: 2-bit decode packing (SBL_PACK_GEMV) */
+  uint64_t gemv;        /* decode pack (SBL_PACK_GEMV), gemv_bytes bytes; see below */
   uint64_t gamma;       /* float: exact absmean, rounded to fp32 */
   uint64_t g;           /* float: max(gamma, 1e-5), the scale used everywhere */
   uint64_t status;      /* uint32 device status word */
   uint64_t scratch;     /* partial sums of the exact absmean (written and read by sbl_prepare_weights) */
+  uint64_t gemv_bytes;  /* size of the decode pack */
 } sbl_blob_layout;
 /* sp_meta layout: blocks of 128 rows x 128 k-positions, 2048 bytes each,
  * ordered [row_block][k_block]; inside a block, row r's 16 bytes hold 32
  * nibbles for its 32 groups of four in k order (group 2j in the low nibble
  * of byte j); a nibble is (i0 | i1 << 2) with i0 < i1 the kept positions.
  * Rows and k are padded up to multiples of 256 with nibble 0x4 over zero codes.
- * gemv layout: one byte per group of four: the metadata nibble in the high
- * half, the two kept codes in the low half (bits 1:0 the code at i0, bits 3:2
- * the code at i1; 00 = 0, 01 = +1, 11 = -1). */
+ * gemv layout, 2:4: one byte per group of four: the metadata nibble in the
+ * high half, the two kept codes in the low half (bits 1:0 the code at i0,
+ * bits 3:2 the code at i1; 00 = 0, 01 = +1, 11 = -1).  The bytes are cut into
+ * units of 16 rows x 128 k (rows padded to 16 and k to 128 with zero bytes),
+ * ordered [row tile][k unit], 512 bytes each: the 8 bytes of groups 8t..8t+7
+ * of the unit for row r sit at 16 * (4 * (r % 8) + t) + 8 * ((r % 16) / 8).
+ * gemv layout, any other N:M (compressed index: the explicit N:M metadata beside
+ * the kept values, [ja] 2.1): every block of 8 consecutive weights has a mask
+ * byte (bit j = position j kept) and its n8 = 8n/m kept codes in index order,
+ * 2 bits each (same code values).  The pack is cut into units of 16 rows x 128
+ * k (rows padded to 16 and k to 128 with zero bytes), ordered [row tile][k
+ * unit].  Unit bytes: a 256-byte mask block when n < m, then a code block of
+ * 32 x cb bytes, cb = 4 * ceil(2 n8 / 4).  The lane slot of a block is
+ * L = 4 * (row % 8) + (b / 4) % 4 for block b = (k % 128) / 8 of the unit:
+ * mask byte at L * 8 + 4 * ((row % 16) / 8) + b % 4; code field (2 n8 bits) at
+ * bit 8 * n8 * ((row % 16) / 8) + 2 n8 * (b % 4) of the slot's cb bytes,
+ * least significant bit first.  n = m (dense ternary) has no mask block. */
 
 /* Size and section offsets of the prepared blob.  Host only, no CUDA call.
  * Returns SBL_ERR_* on unsupported shapes/patterns (out is then untouched). */
@@ -220,9 +237,17 @@ int sbl_forward_uses_gemv(const sbl_layer* layer, int64_t t);
  * device code keeps those 16 MiB until the process exits.
  *
  * The first call with t > 0 on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls on a device share the one array and it keeps the
- * last call's contents, so calls that can overlap on the GPU (two streams,
+ * (cudaGetSymbolAddress) and caches it by device ordinal (devices 0-63; a
+ * higher ordinal returns SBL_ERR_DEVICE).  Under CUDA's lazy module loading
+ * that lookup is also when the library's device code is loaded on the device
+ * and the 16 MiB are committed, which can synchronise the device: make the
+ * first call once, outside any region that must not allocate or stall, and
+ * before any stream capture.  The cache does not see cudaDeviceReset: after a
+ * reset of a device, its cached address is stale and this entry point must
+ * not be called on that device again in the process.  All arguments that need
+ * no device are checked before the lookup.  All calls on a device share the
+ * one array and it keeps the last call's contents, so calls that can overlap
+ * on the GPU (two streams,
  * two host threads) race on it: serialise them.  Nothing in the array needs to
  * start at zero; each call writes everything it reads.  Errors: as
  * sbl_forward, plus SBL_ERR_SCRATCH. */
@@ -267,6 +292,15 @@ sbl_status sbl_read_scale(const sbl_layer* layer, sbl_stream_t stream, float* ga
  * complete, bounded by `limit_ns`; the kernel then records SBL_STATUS_TIMEOUT
  * in *status_dev (device uint32) and returns normally.  No fault, no hang. */
 sbl_status sbl_selftest_wait_timeout(uint32_t* status_dev, uint64_t limit_ns, sbl_stream_t stream);
+
+/* Measurement aid, no counterpart in the paper: launches one empty kernel of
+ * `blocks` blocks x 256 threads the way every kernel of the library is
+ * launched (programmatic dependent launch: it lets its successor launch,
+ * waits for its predecessor, and exits).  A chain of these in a CUDA graph
+ * gives the per-call floor that a chain of dependent library calls pays
+ * before any work.  Touches no memory.  Errors: SBL_ERR_INVALID_ARG for
+ * blocks outside 1..65535, SBL_ERR_DEVICE, SBL_ERR_CUDA. */
+sbl_status sbl_selftest_chain_floor(int32_t blocks, sbl_stream_t stream);
 
 /* Bits of the device status word. */
 enum {

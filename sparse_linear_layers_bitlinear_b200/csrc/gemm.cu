@@ -330,4 +330,18 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
   return counted(cudaGetLastError());
 }
 
+// ---------------------------------------------------------------------------
+// The floor of a chain of dependent launches: a kernel that lets its
+// successor launch, waits for its predecessor and exits, launched the way
+// every kernel of the library is (programmatic dependent launch).
+// ---------------------------------------------------------------------------
+__global__ void k_chain_floor() {
+  pdl_trigger();
+  pdl_wait();
+}
+
+cudaError_t launch_chain_floor(int blocks, cudaStream_t s) {
+  return launch_pdl(k_chain_floor, dim3(blocks), dim3(256), 0, s);
+}
+
 }  // namespace sbl

@@ -1,20 +1,51 @@
-// Decode-shaped forward (t <= 16 tokens) over the 2-bit weight packing, with
-// the per-token activation quantisation fused in.
+// Decode-shaped forward (t <= 32 tokens) over the 2-bit weight packs.
 //
-// The weight stream is the whole cost at these token counts: 2 bits per
-// weight (one byte per group of four: the metadata nibble i0 | i1 << 2 in the
-// high half, the two kept codes in the low half, 01 = +1, 11 = -1).  Each
-// block owns a contiguous range of output rows.  Calls are launched with
-// programmatic dependent launch: a call starts while the kernel before it
-// still runs, prefetches its block's weight rows (and x) into L2 with one bulk
-// prefetch, lets the next call launch, and only then waits for its
-// predecessor, so in a chain of decode calls each weight stream overlaps the
-// call before it.  After the wait eight threads per row load the row's 16-byte
-// pieces (L2 hits), the block quantises the t activation rows into shared
-// memory (the same arithmetic as the act-quant kernel; block 0 also writes them
-// out when the caller asked for them), and a group byte expands through a
-// 256-entry table into its four int8 weights that dp4a multiplies with four
-// activation codes of each token.
+// At these token counts the weight stream is the whole cost, so the weights
+// travel packed and are expanded to int8 in registers, straight into the
+// operand fragments of the warp-level int8 tensor-core instruction
+// (mma.sync m16n8k32: 16 weight rows x 8 tokens x 32 k per instruction).
+// That instruction takes its operands from registers, so the expansion never
+// goes through shared memory, and a block needs no tensor-memory allocation
+// or barrier round trip on a kernel whose whole budget is a few microseconds.
+//
+// Work: the rows are cut into tiles of 16, a tile's k into units of 128.  A
+// block owns whole tiles (so every sum closes inside the block) and its warps
+// split the block's (tile, unit) pairs evenly.  In a unit, lane (g, t) (g =
+// lane / 4, t = lane % 4) handles rows g and g + 8 and the 32 consecutive k
+// from 32t: k-step s of the unit covers its 8 weights 32t + 8s .. 32t + 8s + 7,
+// whose first four fill the fragment slots 4t..4t+3 and the last four the
+// slots 16 + 4t..16 + 4t + 3.  The activation fragments follow the same
+// permutation of k, so every product meets the right activation; a lane's
+// activation bytes for one k-step are 8 consecutive codes.
+//
+// Weight packs:
+//   2:4 (the 2-bit decode packing): one byte per group of four, the metadata
+//       nibble high and the two kept codes low, interleaved by unit and lane:
+//       a unit is 512 bytes, lane * 16 holding the 8 group bytes of row g
+//       (groups 8t..8t+7 of the unit) and then the 8 of row g + 8, so a lane
+//       reads one 16-byte piece per unit and a warp 512 contiguous bytes; a
+//       256-entry table expands a byte into the group's four int8 weights.
+//   any other N:M (compressed index): per block of 8 weights a mask byte and
+//       the n8 = 8n/m kept 2-bit codes in index order.  The section is
+//       interleaved by unit and lane so that a lane's mask bytes and code bits
+//       are contiguous: per unit a 256-byte mask block (lane * 8: row g's four
+//       blocks, then row g + 8's) and a code block (lane * cb bytes: row g's
+//       four fields of 2 n8 bits, then row g + 8's).  Expansion: a table turns
+//       each byte of codes into four int8 values in index order, and a second
+//       table turns the mask byte into the byte-permute selectors that scatter
+//       them onto the kept positions (pruned positions pick a zero byte).
+//       n = m (dense ternary) drops the mask block.
+//
+// Calls are launched with programmatic dependent launch: before the wait for
+// its predecessor a block builds its tables, clears its partial sums and
+// prefetches its weight bytes into L2 (the prefetch is safe even right after
+// a prepare: L2 is the coherence point, so a later write is never hidden),
+// and lets the next call launch; in a chain of decode calls the weight stream
+// of one call overlaps the call before it.  After the wait the block issues
+// its weight loads, quantises its token rows into shared memory (t <= 8) or
+// copies the codes the act-quant kernel wrote, and runs the products.  Partial
+// sums of warps sharing a tile are added in shared memory (exact integer
+// adds, any order); y = acc * ((g a') / 127) closes the block.
 #include <mutex>
 
 #include "sbl_kernels.h"
@@ -24,297 +55,540 @@
 
 namespace sbl {
 
-constexpr int kGemvThreads = 512;
-constexpr size_t kGemvMaxSmem = 200 * 1024;
-constexpr int kLutWords = 256 * 32;
-constexpr int kRowThreads = 8;                      // threads sharing one output row
-constexpr int kRowSlots = kGemvThreads / kRowThreads;  // rows in flight per block
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+// A table of 256 entries kept in kLutCopies copies, entry e of copy c at word
+// e * kLutCopies + c; lane l reads copy l % kLutCopies, so at most
+// 32 / kLutCopies lanes share a copy's banks.
+constexpr int kLutCopies = 16;
+constexpr int kLutWords = 256 * kLutCopies;
+constexpr int kDecBatch = 8;         // units whose weight bytes a lane holds at once
+constexpr size_t kDecMaxSmem = 227 * 1024;
+constexpr int kDecMaxT = 32;
+constexpr int kFusedMaxT = 8;  // token counts the kernel quantises itself
 
-struct GemvArgs {
-  const uint4* gemv;   // [n_out][k/64] 16-byte pieces
-  const uint4* x;      // bf16 [t][k/8] 16-byte vectors
+struct DecodeArgs {
+  const uint8_t* w;      // weight pack
+  const uint4* x;        // bf16 [t][k/8] (quantised here)
+  const int8_t* xq_in;   // int8 [t][k] from the act-quant kernel (else)
+  const float* ap_in;
   const float* g;
   float* y;
   int32_t* acc_out;
-  int8_t* xq_out;      // optional
-  float* ap_out;       // optional
-  const int8_t* xq_in; // codes written by the act-quant kernel (PREQUANT)
-  const float* ap_in;
+  int8_t* xq_out;        // optional, when quantised here
+  float* ap_out;
   uint32_t* status;
   int n_out, t, k;
+  int tiles, upr, tpb;   // 16-row tiles, 128-k units per row, tiles per block
+  int xs;                // shared-memory row stride of the codes (multiple of 128)
 };
 
-// 16-byte weight pieces each thread keeps in flight (fewer when many tokens'
-// accumulators need the registers).
-template <int TP>
-constexpr int gemv_pieces() {
-  return TP >= 8 ? 4 : 8;
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// The exact-division form of the quantiser, out of line: it runs only for a
+// row whose a' is the 1e-5 clamp or huge, and kept out of the fast path's
+// instruction stream.
+__device__ __noinline__ uint4 quantise16_div(uint4 v0, uint4 v1, float ap) {
+  const uint2 c0 = quantise8_div(v0, ap), c1 = quantise8_div(v1, ap);
+  return make_uint4(c0.x, c0.y, c1.x, c1.y);
 }
 
-template <int TP, bool PREQUANT>
-__global__ void __launch_bounds__(kGemvThreads) k_gemv(const GemvArgs a) {
-  constexpr int kPieces = gemv_pieces<TP>();
-  extern __shared__ __align__(16) uint32_t smem_w[];
-  uint32_t* lut = smem_w;                    // [256 entries][32 banks]: one copy per bank
-  float* s_scale = reinterpret_cast<float*>(smem_w + kLutWords);  // [TP] (g * a') / 127
-  float* s_red = s_scale + 16;               // [16 warps] reduction scratch
-  uint32_t* xw = smem_w + kLutWords + 32;    // [TP][k/4] int8 codes as words
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kw = a.k / 4;                    // code words per token row
+__device__ __forceinline__ uint4 quantise16(const uint4& v0, const uint4& v1, const QScale& qs) {
+  if (qs.exact) return quantise16_div(v0, v1, qs.ap);
+  const uint2 c0 = quantise8_fma(v0, qs.c), c1 = quantise8_fma(v1, qs.c);
+  return make_uint4(c0.x, c0.y, c1.x, c1.y);
+}
 
-  // Rows of this block.  The kernel before this one in the stream may still
-  // be writing this call's inputs (a prepare writes the weights, the previous
-  // layer writes x), so they are only prefetched into L2 before the wait and
-  // read after it; the next call may launch at once and do the same, so the
-  // weight streams of consecutive calls overlap.
-  const int rpb = (a.n_out + gridDim.x - 1) / gridDim.x;
-  const int row_begin = blockIdx.x * rpb;
-  const int row_end = min(a.n_out, row_begin + rpb);
-  const int slot = tid / kRowThreads, sub = tid % kRowThreads;
-  const int pieces = a.k / 64;  // 16-byte weight pieces per row
-  if (tid == 0 && row_end > row_begin)
-    bulk_prefetch_l2(a.gemv + int64_t(row_begin) * pieces, static_cast<uint32_t>(row_end - row_begin) * pieces * 16u);
-  if (tid == 32 && blockIdx.x == 0) {
-    if (PREQUANT) bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
-    else bulk_prefetch_l2(a.x, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k) * 2u);
+__device__ __forceinline__ void mma_s8_16x8x32(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  // a pure register operation: no volatile, so the compiler may interleave it
+  // with the table loads of the next k-step
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// int8 value of a 2-bit code: 01 = +1, 11 = -1, 00 (and the unused 10) = 0.
+__host__ __device__ constexpr uint32_t code_byte(uint32_t c) { return c == 1u ? 0x01u : c == 3u ? 0xFFu : 0u; }
+
+// Table entries.  kind 0: a 2:4 decode byte -> the group's four weights;
+// kind 1: a byte of four codes -> four int8 values in index order; kind 2: a
+// mask byte -> two byte-permute selectors (positions 0-3 in the low half,
+// 4-7 in the high half): a kept position picks its rank among the kept
+// values, a pruned one byte 7 (zero whenever fewer than 8 are kept).
+__device__ __forceinline__ uint32_t lut_entry(int kind, uint32_t b) {
+  if (kind == 0) {
+    const uint32_t i0 = (b >> 4) & 3u, i1 = (b >> 6) & 3u;
+    return (code_byte(b & 3u) << (8 * i0)) | (code_byte((b >> 2) & 3u) << (8 * i1));
+  }
+  if (kind == 1)
+    return code_byte(b & 3u) | (code_byte((b >> 2) & 3u) << 8) | (code_byte((b >> 4) & 3u) << 16) |
+           (code_byte((b >> 6) & 3u) << 24);
+  uint32_t sel = 0;
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t nib = ((b >> p) & 1u) ? static_cast<uint32_t>(__popc(b & ((1u << p) - 1u))) : 7u;
+    sel |= nib << (4 * p);
+  }
+  return sel;
+}
+
+__device__ __forceinline__ void fill_lut(uint32_t* lut, int kind, int tid) {
+  constexpr int kVecs = kLutCopies / 4;  // 16-byte stores per entry
+  for (int i = tid; i < 256 * kVecs; i += kDecThreads) {
+    const uint32_t v = lut_entry(kind, static_cast<uint32_t>(i / kVecs));
+    reinterpret_cast<uint4*>(lut)[i] = make_uint4(v, v, v, v);
+  }
+}
+
+// Compile-time facts of a weight pack.  FMT 0: 2:4 bytes; FMT 1..8: blocks of
+// 8 with FMT kept codes (8 = dense, no mask block).
+template <int FMT>
+struct Pack {
+  static constexpr bool k24 = FMT == 0;
+  static constexpr int n8 = FMT;
+  static constexpr bool has_mask = FMT >= 1 && FMT < 8;
+  static constexpr int cb = k24 ? 0 : (2 * FMT + 3) / 4 * 4;  // code bytes per lane and unit
+  static constexpr int cw = cb / 4;
+  static constexpr int unit_bytes = k24 ? 512 : (has_mask ? 256 : 0) + 32 * cb;
+  static constexpr int regs = k24 ? 4 : (has_mask ? 2 : 0) + cw;  // words a lane loads per unit
+};
+
+// One unit's weight words of this lane.
+template <int FMT>
+__device__ __forceinline__ void load_unit(const DecodeArgs& a, int tile, int u, int lane,
+                                          uint32_t (&r)[Pack<FMT>::regs]) {
+  using P = Pack<FMT>;
+  if constexpr (P::k24) {
+    // one 16-byte piece: 8 group bytes of row g, then 8 of row g + 8
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(a.w + (int64_t(tile) * a.upr + u) * P::unit_bytes) + lane);
+    r[0] = v.x;
+    r[1] = v.y;
+    r[2] = v.z;
+    r[3] = v.w;
+  } else {
+    const uint8_t* base = a.w + (int64_t(tile) * a.upr + u) * P::unit_bytes;
+    int o = 0;
+    if constexpr (P::has_mask) {
+      const uint2 mk = __ldcs(reinterpret_cast<const uint2*>(base + lane * 8));
+      r[0] = mk.x;
+      r[1] = mk.y;
+      o = 2;
+      base += 256;
+    }
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(base + lane * P::cb);
+    if constexpr (P::cw == 4) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(cw));
+      r[o] = v.x;
+      r[o + 1] = v.y;
+      r[o + 2] = v.z;
+      r[o + 3] = v.w;
+    } else if constexpr (P::cw == 2) {
+      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(cw));
+      r[o] = v.x;
+      r[o + 1] = v.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < P::cw; ++i) r[o + i] = __ldcs(cw + i);
+    }
+  }
+}
+
+// Bits [off, off + bits) of the lane's code words (off, bits compile-time
+// after unrolling; bits <= 16).
+template <int CW>
+__device__ __forceinline__ uint32_t code_field(const uint32_t* w, int off, int bits) {
+  const int wi = off >> 5, sh = off & 31;
+  uint32_t v = w[wi] >> sh;
+  if (sh + bits > 32) v |= w[wi + 1] << (32 - sh);
+  return bits == 32 ? v : (v & ((1u << bits) - 1u));
+}
+
+// Table entry (byte `pos` of w) in this lane's copy: the byte, shifted
+// straight into a byte offset (entries are 4 * kLutCopies bytes apart).
+__device__ __forceinline__ uint32_t lut_get(const uint8_t* lane_base, uint32_t w, int pos) {
+  constexpr int kShift = 2 + (kLutCopies == 16 ? 4 : kLutCopies == 32 ? 5 : 3);
+  static_assert(kLutCopies == 8 || kLutCopies == 16 || kLutCopies == 32, "table copies");
+  const int sh = 8 * pos - kShift;
+  const uint32_t off = (sh >= 0 ? (w >> sh) : (w << -sh)) & (0xFFu << kShift);
+  return *reinterpret_cast<const uint32_t*>(lane_base + off);
+}
+
+// The four A-fragment registers of k-step s: rows g (a0 low k slots, a2 high)
+// and g + 8 (a1, a3).  la / ls: this lane's copies of the tables.
+template <int FMT>
+__device__ __forceinline__ void decode_step(const uint32_t (&r)[Pack<FMT>::regs], int s, const uint8_t* la,
+                                            const uint8_t* ls, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) {
+  using P = Pack<FMT>;
+  if constexpr (P::k24) {
+    // bytes 2s, 2s + 1 of each row's 8: word s / 2, bytes 2 (s % 2) and + 1
+    const int b = 2 * (s & 1);
+    const uint32_t w0 = r[s >> 1], w1 = r[2 + (s >> 1)];
+    a0 = lut_get(la, w0, b);
+    a2 = lut_get(la, w0, b + 1);
+    a1 = lut_get(la, w1, b);
+    a3 = lut_get(la, w1, b + 1);
+  } else {
+    constexpr int o = P::has_mask ? 2 : 0;
+    uint32_t lo[2], hi[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t c = code_field<P::cw>(r + o, h * 8 * P::n8 + s * 2 * P::n8, 2 * P::n8);
+      const uint32_t A = lut_get(la, c, 0);
+      const uint32_t B = P::n8 > 4 ? lut_get(la, c, 1) : 0u;
+      if constexpr (P::has_mask) {
+        const uint32_t sel = lut_get(ls, r[h], s);
+        lo[h] = __byte_perm(A, B, sel & 0xFFFFu);
+        hi[h] = __byte_perm(A, B, sel >> 16);
+      } else {
+        lo[h] = A;
+        hi[h] = B;
+      }
+    }
+    a0 = lo[0];
+    a2 = hi[0];
+    a1 = lo[1];
+    a3 = hi[1];
+  }
+}
+
+// Byte offset of 16-code chunk j of token row n in shared memory: chunks are
+// XOR-swizzled inside each 128-byte line by the row, so the eight lanes of a
+// quarter warp (rows g, g + 1; four t) read eight distinct bank groups.
+__device__ __forceinline__ int xs_off(int n, int j, int xs) { return n * xs + ((j & ~7) | ((j & 7) ^ (n & 7))) * 16; }
+
+template <int FMT, int NT, bool FUSED>
+__global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
+  using P = Pack<FMT>;
+  constexpr int TP = 8 * NT;  // token columns
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t* lut_a = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* lut_s = lut_a + kLutWords;  // mask selectors (packs with a mask block)
+  uint8_t* xsm = smem + (P::has_mask ? 2 : 1) * kLutWords * 4;
+  int32_t* s_acc = reinterpret_cast<int32_t*>(xsm + TP * a.xs);  // [tpb][16][TP]
+  float* s_scale = reinterpret_cast<float*>(s_acc + a.tpb * 16 * TP);  // [32]
+  float* s_red = s_scale + kDecMaxT;                                    // [warps]
+  float* s_ap = s_red + kDecWarps;                                      // [8] a' (quantised here)
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile0 = blockIdx.x * a.tpb;
+  const int ntile = min(a.tpb, a.tiles - tile0);
+  const int units = ntile * a.upr;
+
+  // ---- before the wait: prefetch, tables, zeroed sums and padding ----
+  if (tid == 0) bulk_prefetch_l2(a.w + int64_t(tile0) * a.upr * P::unit_bytes, static_cast<uint32_t>(units) * P::unit_bytes);
+  if (tid == 32) {
+    if (FUSED) bulk_prefetch_l2(a.x, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k) * 2u);
+    else bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
   }
   pdl_trigger();
-  // Expansion table: group byte -> four int8 weights, replicated so that
-  // lane l always reads bank l (the bytes a warp looks up are random).
-  {
-    const int i = tid >> 1, half = tid & 1;  // 256 entries x 2 threads, 16 copies each
-    const int c0 = (i & 1) ? ((i & 2) ? -1 : 1) : 0;  // 2-bit codes: 01 = +1, 11 = -1, 00 = 0
-    const int c1 = (i & 4) ? ((i & 8) ? -1 : 1) : 0;
-    const int i0 = (i >> 4) & 3, i1 = (i >> 6) & 3;
-    const uint32_t v = ((static_cast<uint32_t>(c0) & 0xFFu) << (8 * i0)) | ((static_cast<uint32_t>(c1) & 0xFFu) << (8 * i1));
-    uint4* dst = reinterpret_cast<uint4*>(lut + i * 32 + half * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(v, v, v, v);
-  }
+  fill_lut(lut_a, P::k24 ? 0 : 1, tid);
+  if constexpr (P::has_mask) fill_lut(lut_s, 2, tid);
+  for (int i = tid; i < ntile * 16 * TP; i += kDecThreads) s_acc[i] = 0;
+  // Activation rows past t and columns past k are left as they are: a token
+  // column past t only feeds output columns that are never stored, and the
+  // weights past k are zero (guarded loads, zero-filled pack).
   pdl_wait();
-  uint4 wbuf[kPieces];
-  {
-    const int row = row_begin + slot;
+
+  const int nch = a.k / 16;  // 16-code chunks per token row
+  const int u_begin = (units * warp) / kDecWarps, u_end = (units * (warp + 1)) / kDecWarps;
+  // (tile, unit) of this warp's first unit; later ones follow by counting
+  const int tl_begin = u_begin / a.upr, un_begin = u_begin - tl_begin * a.upr;
+  uint32_t wr[kDecBatch][P::regs];
+  auto load_batch = [&](int ub, int tl, int un) {
 #pragma unroll
-    for (int q = 0; q < kPieces; ++q) {
-      const int j = sub + kRowThreads * q;
-      wbuf[q] = (row < row_end && j < pieces) ? __ldcs(a.gemv + int64_t(row) * pieces + j) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < kDecBatch; ++i) {
+      if (ub + i < u_end) load_unit<FMT>(a, tile0 + tl, un, lane, wr[i]);
+      if (++un == a.upr) {
+        un = 0;
+        ++tl;
+      }
     }
-  }
+  };
 
-  // This thread's share of the activation rows (fused quantisation) and g.
-  constexpr int kXq = 4;  // 16-byte activation vectors kept in registers
-  const int nvec = a.k / 8;
-  const int wpr = (kGemvThreads / 32) / TP;  // warps per token row
-  const int xrow = warp / wpr, xsub = warp % wpr;
-  const uint4* xsrc = a.x + int64_t(xrow) * nvec;
-  uint4 xbuf[kXq];
-  if (!PREQUANT) {
+  // ---- activation codes into shared memory ----
+  // The activation loads go out first (the rest of the block's path waits
+  // on them), then this warp's first batch of weight loads, which are needed
+  // only by the products.
+  if constexpr (FUSED) {
+    // Quantise the t <= 8 rows here: wpr warps per row, the row's absmax
+    // through the warps' maxima in shared memory.
+    const int tp2 = a.t <= 1 ? 1 : a.t <= 2 ? 2 : a.t <= 4 ? 4 : 8;
+    const int wpr = kDecWarps / tp2;
+    const int xrow = warp / wpr, xsub = warp % wpr;
+    const bool live = xrow < a.t;
+    const uint4* xsrc = a.x + int64_t(xrow) * (a.k / 8);
+    const bool scale_thread = live && xsub == 0 && lane == 0;
+    constexpr int kXc = 2;  // chunks kept in registers between the two passes
+    uint4 xr[kXc][2];
 #pragma unroll
-    for (int q = 0; q < kXq; ++q) {
-      const int i = (xsub + q * wpr) * 32 + lane;
-      xbuf[q] = (xrow < a.t && i < nvec) ? __ldg(xsrc + i) : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < kXc; ++q) {
+      const int j = (xsub + q * wpr) * 32 + lane;
+      if (live && j < nch) {
+        xr[q][0] = __ldg(xsrc + 2 * j);
+        xr[q][1] = __ldg(xsrc + 2 * j + 1);
+      } else {
+        xr[q][0] = xr[q][1] = make_uint4(0, 0, 0, 0);
+      }
     }
-  }
-  const float g = __ldg(a.g);
-
-  const uint32_t* my_lut = lut + lane;
-
-  if (!PREQUANT) {
-    // Activation quantisation of the t rows into shared memory: the warps
-    // split into t groups, one per row; two block barriers in all.
+    load_batch(u_begin, tl_begin, un_begin);
     float amax = 0.0f;
     uint32_t bad = 0;
-    if (xrow < a.t) {
 #pragma unroll
-      for (int q = 0; q < kXq; ++q) scan8(xbuf[q], amax, bad);
-      for (int i = (xsub + kXq * wpr) * 32 + lane; i < nvec; i += wpr * 32) scan8(__ldg(xsrc + i), amax, bad);
+    for (int q = 0; q < kXc; ++q) {
+      scan8(xr[q][0], amax, bad);
+      scan8(xr[q][1], amax, bad);
     }
+    if (live)
+      for (int j = (xsub + kXc * wpr) * 32 + lane; j < nch; j += wpr * 32) {
+        scan8(__ldg(xsrc + 2 * j), amax, bad);
+        scan8(__ldg(xsrc + 2 * j + 1), amax, bad);
+      }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       bad |= __shfl_xor_sync(0xffffffffu, bad, off);
     }
-    if (lane == 0) s_red[warp] = bad ? -1.0f : amax;  // amax >= 0, so -1 flags a non-finite row
+    if (lane == 0) s_red[warp] = bad ? -1.0f : amax;  // amax >= 0: -1 flags a non-finite row
     __syncthreads();
-    float m = 0.0f;
-    bool row_bad = false;
-    for (int w = 0; w < wpr; ++w) {
-      const float v = s_red[xrow * wpr + w];
-      row_bad |= v < 0.0f;
-      m = fmaxf(m, v);
-    }
-    const float ap = fmaxf(m, 1e-5f);
-    if (xrow < a.t) {
-      if (xsub == 0 && lane == 0) {
-        s_scale[xrow] = __fdiv_rn(__fmul_rn(g, ap), 127.0f);
+    if (live) {
+      float m = 0.0f;
+      bool row_bad = false;
+      for (int w = 0; w < wpr; ++w) {
+        const float v = s_red[xrow * wpr + w];
+        row_bad |= v < 0.0f;
+        m = fmaxf(m, v);
+      }
+      const float ap = fmaxf(m, 1e-5f);
+      const QScale qs = make_qscale(ap);
+      uint4* gdst = (blockIdx.x == 0 && a.xq_out) ? reinterpret_cast<uint4*>(a.xq_out + int64_t(xrow) * a.k) : nullptr;
+#pragma unroll
+      for (int q = 0; q < kXc; ++q) {
+        const int j = (xsub + q * wpr) * 32 + lane;
+        if (j < nch) {
+          const uint4 c = quantise16(xr[q][0], xr[q][1], qs);
+          *reinterpret_cast<uint4*>(xsm + xs_off(xrow, j, a.xs)) = c;
+          if (gdst) gdst[j] = c;
+        }
+      }
+      for (int j = (xsub + kXc * wpr) * 32 + lane; j < nch; j += wpr * 32) {
+        const uint4 c = quantise16(__ldg(xsrc + 2 * j), __ldg(xsrc + 2 * j + 1), qs);
+        *reinterpret_cast<uint4*>(xsm + xs_off(xrow, j, a.xs)) = c;
+        if (gdst) gdst[j] = c;
+      }
+      if (scale_thread) {
+        s_ap[xrow] = ap;  // the output scale is formed after the products
         if (blockIdx.x == 0) {
           if (a.ap_out) a.ap_out[xrow] = ap;
           if (row_bad) raise_status(a.status, SBL_STATUS_NONFINITE_X);
         }
       }
-      const QScale qs = make_qscale(ap);
-      uint2* dst = reinterpret_cast<uint2*>(xw + xrow * kw);
-      uint2* gdst = (blockIdx.x == 0 && a.xq_out) ? reinterpret_cast<uint2*>(a.xq_out + int64_t(xrow) * a.k) : nullptr;
-#pragma unroll
-      for (int q = 0; q < kXq; ++q) {
-        const int i = (xsub + q * wpr) * 32 + lane;
-        if (i < nvec) {
-          const uint2 c = quantise8(xbuf[q], qs);
-          dst[i] = c;
-          if (gdst) gdst[i] = c;
-        }
-      }
-      for (int i = (xsub + kXq * wpr) * 32 + lane; i < nvec; i += wpr * 32) {
-        const uint2 c = quantise8(__ldg(xsrc + i), qs);
-        dst[i] = c;
-        if (gdst) gdst[i] = c;
-      }
     }
   } else {
-    // The act-quant kernel before this one wrote the codes and scales.
-    // One bulk copy brings all t rows of codes (t * k bytes, a multiple of 64).
-    __shared__ uint64_t bar;
-    if (tid == 0) {
-      mbar_init(&bar, 1);
-      fence_mbar_init();
-      fence_proxy_async_smem();
-      const uint32_t bytes = static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k);
-      mbar_arrive_expect_tx(&bar, bytes);
-      bulk_load(xw, a.xq_in, bytes, &bar);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(&bar, 0)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          raise_status(a.status, SBL_STATUS_TIMEOUT);
-          break;
-        }
-      }
+    // codes and scales from the act-quant kernel (or the caller): copied into
+    // shared memory by asynchronous 16-byte copies, which hold no registers
+    const float g = tid < a.t ? __ldg(a.g) : 0.0f;
+    for (int i = tid; i < a.t * nch; i += kDecThreads) {
+      const int n = i / nch, j = i - n * nch;
+      cp_async16(xsm + xs_off(n, j, a.xs), reinterpret_cast<const uint4*>(a.xq_in + int64_t(n) * a.k) + j);
     }
-    if (tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(g, __ldcg(a.ap_in + tid)), 127.0f);
+    cp_async_commit();
+    const float apv = tid < a.t ? __ldcg(a.ap_in + tid) : 0.0f;
+    load_batch(u_begin, tl_begin, un_begin);
+    if (tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(g, apv), 127.0f);
+    cp_async_wait_all();
   }
-  for (int i = a.t * kw + tid; i < TP * kw; i += kGemvThreads) xw[i] = 0u;  // padding tokens
   __syncthreads();
 
-  // Dot products: eight threads per row, then a reduction inside the group.
-  for (int r0 = row_begin; r0 < row_end; r0 += kRowSlots) {
-    const int row = r0 + slot;
-    // a warp holds 4 rows; it skips the pass when all of them are past the end
-    if (r0 + (warp * 32) / kRowThreads >= row_end) continue;
-    int acc[TP];
+  // ---- products ----
+  const int gq = lane >> 2, tq = lane & 3;
+  const uint8_t* la = reinterpret_cast<const uint8_t*>(lut_a + (lane % kLutCopies));
+  const uint8_t* ls = reinterpret_cast<const uint8_t*>(lut_s + (lane % kLutCopies));
+  // this lane's activation chunks in unit 0 (token row gq + 8 nt, chunk
+  // 2 tq + p); unit un is 128 un bytes further
+  const uint8_t* bsrc[NT][2];
 #pragma unroll
-    for (int tt = 0; tt < TP; ++tt) acc[tt] = 0;
-    for (int j0 = 0; j0 < pieces; j0 += kRowThreads * kPieces) {
-      if (r0 != row_begin || j0 != 0) {  // the first batch was loaded up front
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int q = 0; q < kPieces; ++q) {
-          const int j = j0 + sub + kRowThreads * q;
-          wbuf[q] = (row < row_end && j < pieces) ? __ldcs(a.gemv + int64_t(row) * pieces + j) : make_uint4(0, 0, 0, 0);
+    for (int p = 0; p < 2; ++p) bsrc[nt][p] = xsm + xs_off(gq + 8 * nt, 2 * tq + p, a.xs);
+  // kSets independent MMA accumulators per token tile (k-step s adds into set
+  // s % kSets) keep consecutive MMAs from waiting on each other's results.
+  constexpr int kSets = NT == 1 ? 4 : NT == 2 ? 2 : 1;
+  int acc[kSets][NT][4];
+  int cur = -1;  // tile (local) the accumulators belong to
+  auto zero_acc = [&]() {
+#pragma unroll
+    for (int q = 0; q < kSets; ++q)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[q][nt][0] = acc[q][nt][1] = acc[q][nt][2] = acc[q][nt][3] = 0;
+  };
+  auto flush = [&](int t_local) {
+    int32_t* base = s_acc + t_local * 16 * TP;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      int v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        v[r] = acc[0][nt][r];
+#pragma unroll
+        for (int q = 1; q < kSets; ++q) v[r] += acc[q][nt][r];
+      }
+      const int col = nt * 8 + 2 * tq;
+      atomicAdd(base + gq * TP + col, v[0]);
+      atomicAdd(base + gq * TP + col + 1, v[1]);
+      atomicAdd(base + (gq + 8) * TP + col, v[2]);
+      atomicAdd(base + (gq + 8) * TP + col + 1, v[3]);
+    }
+  };
+  int tl = tl_begin, un = un_begin;  // (tile, unit) of unit ub + i
+  for (int ub = u_begin; ub < u_end; ub += kDecBatch) {
+    if (ub != u_begin) load_batch(ub, tl, un);
+#pragma unroll
+    for (int i = 0; i < kDecBatch; ++i) {
+      if (ub + i >= u_end) break;
+      if (tl != cur) {
+        if (cur >= 0) flush(cur);
+        cur = tl;
+        zero_acc();
+      }
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        uint4 bv[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) bv[nt] = *reinterpret_cast<const uint4*>(bsrc[nt][p] + 128 * un);
+#pragma unroll
+        for (int sp = 0; sp < 2; ++sp) {
+          uint32_t a0, a1, a2, a3;
+          decode_step<FMT>(wr[i], 2 * p + sp, la, ls, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_s8_16x8x32(acc[(2 * p + sp) % kSets][nt], a0, a1, a2, a3, sp ? bv[nt].z : bv[nt].x,
+                           sp ? bv[nt].w : bv[nt].y);
         }
       }
-#pragma unroll(TP >= 8 ? 1 : kPieces)
-      for (int q = 0; q < kPieces; ++q) {
-        const int j = j0 + sub + kRowThreads * q;
-        if (j >= pieces) break;
-        const uint32_t words[4] = {wbuf[q].x, wbuf[q].y, wbuf[q].z, wbuf[q].w};
-        // 16 groups = 64 weights = code words 16j .. 16j+15; the rotation by
-        // (sub >> 1) keeps the 16-byte shared loads of a row's threads on
-        // distinct banks.
-#pragma unroll
-        for (int i2 = 0; i2 < 4; ++i2) {
-          const int i = (i2 + (sub >> 1)) & 3;
-          const uint32_t wd = words[i];
-          const uint32_t w0 = my_lut[(wd & 0xFFu) << 5], w1 = my_lut[((wd >> 8) & 0xFFu) << 5];
-          const uint32_t w2 = my_lut[((wd >> 16) & 0xFFu) << 5], w3 = my_lut[(wd >> 24) << 5];
-#pragma unroll
-          for (int tt = 0; tt < TP; ++tt) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(xw + tt * kw + 16 * j + 4 * i);
-            int s = acc[tt];
-            s = __dp4a(static_cast<int>(w0), static_cast<int>(xv.x), s);
-            s = __dp4a(static_cast<int>(w1), static_cast<int>(xv.y), s);
-            s = __dp4a(static_cast<int>(w2), static_cast<int>(xv.z), s);
-            s = __dp4a(static_cast<int>(w3), static_cast<int>(xv.w), s);
-            acc[tt] = s;
-          }
-        }
+      if (++un == a.upr) {
+        un = 0;
+        ++tl;
       }
     }
-#pragma unroll
-    for (int tt = 0; tt < TP; ++tt) {
-#pragma unroll
-      for (int off = kRowThreads / 2; off > 0; off >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], off);
-    }
-    if (row < row_end) {
-#pragma unroll
-      for (int tt = 0; tt < TP; ++tt) {
-        if (tt % kRowThreads == sub && tt < a.t) {
-          a.y[int64_t(tt) * a.n_out + row] = __fmul_rn(static_cast<float>(acc[tt]), s_scale[tt]);
-          if (a.acc_out) a.acc_out[int64_t(tt) * a.n_out + row] = acc[tt];
-        }
-      }
+  }
+  if (cur >= 0) flush(cur);
+  if (FUSED && tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(__ldg(a.g), s_ap[tid]), 127.0f);
+  __syncthreads();
+
+  // ---- epilogue: y = acc * ((g a') / 127), consecutive rows per token ----
+  const int rows = min(ntile * 16, a.n_out - tile0 * 16);
+  for (int tok = 0; tok < a.t; ++tok) {
+    const float sc = s_scale[tok];
+    for (int r = tid; r < rows; r += kDecThreads) {
+      const int v = s_acc[(r >> 4) * 16 * TP + (r & 15) * TP + tok];
+      const int64_t o = int64_t(tok) * a.n_out + tile0 * 16 + r;
+      a.y[o] = __fmul_rn(static_cast<float>(v), sc);
+      if (a.acc_out) a.acc_out[o] = v;
     }
   }
 }
 
-template <int TP, bool PREQUANT>
-static cudaError_t gemv_tp(const GemvArgs& a, int num_sms, cudaStream_t s) {
-  const size_t smem = (kLutWords + 32 + size_t(TP) * size_t(a.k / 4)) * 4;
+namespace {
+
+int decode_nt(int64_t t) { return t <= 8 ? 1 : t <= 16 ? 2 : 4; }
+
+int decode_fmt(int n, int m) { return (n == 2 && m == 4) ? 0 : 8 * n / m; }
+
+size_t decode_smem(int fmt, int nt, int64_t k, int tpb) {
+  const bool sel = fmt >= 1 && fmt < 8;
+  const size_t xs = size_t((k + 127) / 128 * 128);
+  return size_t(sel ? 2 : 1) * kLutWords * 4 + size_t(8 * nt) * xs + size_t(tpb) * 16 * 8 * nt * 4 +
+         (kDecMaxT + kDecWarps + 8) * 4;
+}
+
+template <int FMT, int NT, bool FUSED>
+cudaError_t decode_launch(const DecodeArgs& a, int blocks, size_t smem, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(k_gemv<TP, PREQUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
+    err = cudaFuncSetAttribute(k_decode<FMT, NT, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kDecMaxSmem));
   });
   if (err != cudaSuccess) return err;
-  // At most one block per SM, each owning a contiguous range of rows.
-  int blocks = (a.n_out < num_sms) ? a.n_out : num_sms;
-  return launch_pdl(k_gemv<TP, PREQUANT>, dim3(blocks), dim3(kGemvThreads), smem, s, a);
+  return launch_pdl(k_decode<FMT, NT, FUSED>, dim3(blocks), dim3(kDecThreads), smem, s, a);
 }
 
-bool gemv_fits(int64_t t, int64_t k) {
-  const int64_t tp = t <= 1 ? 1 : t <= 2 ? 2 : t <= 4 ? 4 : t <= 8 ? 8 : 16;
-  return t >= 1 && t <= 16 && (kLutWords + 32 + tp * (k / 4)) * 4 <= int64_t(kGemvMaxSmem);
+template <int FMT>
+cudaError_t decode_fmt_launch(const DecodeArgs& a, bool fused, int nt, int blocks, size_t smem, cudaStream_t s) {
+  if (nt == 1) return fused ? decode_launch<FMT, 1, true>(a, blocks, smem, s) : decode_launch<FMT, 1, false>(a, blocks, smem, s);
+  if (nt == 2) return decode_launch<FMT, 2, false>(a, blocks, smem, s);
+  return decode_launch<FMT, 4, false>(a, blocks, smem, s);
 }
 
-// The GEMV's dot products run on the CUDA cores and grow with t * n_out * k,
-// while the 2:4 tensor-core GEMM costs about one round of tiles for a handful
-// of tokens (measured at k = 2560: ~12 us for t = 4..32 against 6.8-17.5 us
-// for the GEMV, which wins up to about 8e7 multiply-adds, e.g. t = 4 at
-// n_out = 6912 or t = 8 at n_out = 2560).
-constexpr int64_t kGemvMaxMacs = 80000000;
+}  // namespace
 
-bool gemv_preferred(int64_t t, int64_t n_out, int64_t k) { return t * n_out * k <= kGemvMaxMacs; }
+uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m) {
+  if (n == 2 && m == 4) return uint64_t((n_out + 15) / 16) * uint64_t((k + 127) / 128) * 512;
+  const int n8 = 8 * n / m;
+  const uint64_t cb = uint64_t(2 * n8 + 3) / 4 * 4;
+  const uint64_t unit = (n8 < 8 ? 256 : 0) + 32 * cb;
+  return uint64_t((n_out + 15) / 16) * uint64_t((k + 127) / 128) * unit;
+}
 
-// Token counts up to kFusedMaxT quantise inside the GEMV (every block redoes
-// that small amount of work, which saves a launch); larger ones run the
-// act-quant kernel first.
-constexpr int64_t kFusedMaxT = 4;
+bool gemv_fits(int64_t t, int64_t k, int n, int m) {
+  if (t < 1 || t > kDecMaxT) return false;
+  return decode_smem(decode_fmt(n, m), decode_nt(t), k, 1) <= kDecMaxSmem;
+}
+
+// The decode kernel streams the packed weights once for up to 32 tokens; the
+// tensor-core GEMMs pay a round of 240-token tiles for any token count.
+bool gemv_preferred(int64_t t, int64_t n_out, int64_t k) { return t <= kDecMaxT; }
 
 bool gemv_fuses_act_quant(int64_t t) { return t <= kFusedMaxT; }
 
-cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const int8_t* xq_in, const float* ap_in,
-                                const float* g, int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out,
-                                int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms, cudaStream_t s) {
-  GemvArgs a;
-  a.gemv = reinterpret_cast<const uint4*>(gemv);
+cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_t* x, const int8_t* xq_in,
+                                const float* ap_in, const float* g, int64_t n_out, int64_t t, int64_t k, float* y,
+                                int32_t* acc_out, int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms,
+                                cudaStream_t s) {
+  DecodeArgs a;
+  a.w = gemv;
   a.x = reinterpret_cast<const uint4*>(x);
+  a.xq_in = xq_in;
+  a.ap_in = ap_in;
   a.g = g;
   a.y = y;
   a.acc_out = acc_out;
   a.xq_out = xq_out;
   a.ap_out = ap_out;
-  a.xq_in = xq_in;
-  a.ap_in = ap_in;
   a.status = status;
   a.n_out = static_cast<int>(n_out);
   a.t = static_cast<int>(t);
   a.k = static_cast<int>(k);
-  // codes from the caller (x == NULL) or from the act-quant kernel before
-  // this one, else quantised here
-  const bool pre = x == nullptr || !gemv_fuses_act_quant(t);
-  if (t <= 1) return pre ? gemv_tp<1, true>(a, num_sms, s) : gemv_tp<1, false>(a, num_sms, s);
-  if (t <= 2) return pre ? gemv_tp<2, true>(a, num_sms, s) : gemv_tp<2, false>(a, num_sms, s);
-  if (t <= 4) return pre ? gemv_tp<4, true>(a, num_sms, s) : gemv_tp<4, false>(a, num_sms, s);
-  if (t <= 8) return gemv_tp<8, true>(a, num_sms, s);
-  return gemv_tp<16, true>(a, num_sms, s);
+  a.tiles = static_cast<int>((n_out + 15) / 16);
+  a.upr = static_cast<int>((k + 127) / 128);
+  a.xs = a.upr * 128;
+  const int fmt = decode_fmt(n, m), nt = decode_nt(t);
+  // codes from the caller (x == NULL), else quantised here for few tokens
+  const bool fused = x != nullptr && gemv_fuses_act_quant(t);
+  // Blocks: as many as fit two per SM; each takes an equal run of tiles.
+  const size_t smem1 = decode_smem(fmt, nt, k, 1);
+  const int per_sm = smem1 * 2 + 2048 <= 228 * 1024 ? 2 : 1;
+  int tpb = (a.tiles + num_sms * per_sm - 1) / (num_sms * per_sm);
+  while (decode_smem(fmt, nt, k, tpb) > kDecMaxSmem && tpb > 1) --tpb;
+  if (decode_smem(fmt, nt, k, tpb) > kDecMaxSmem) return cudaErrorInvalidValue;
+  a.tpb = tpb;
+  const int blocks = (a.tiles + tpb - 1) / tpb;
+  const size_t smem = decode_smem(fmt, nt, k, tpb);
+  switch (fmt) {
+    case 0: return decode_fmt_launch<0>(a, fused, nt, blocks, smem, s);
+    case 1: return decode_fmt_launch<1>(a, fused, nt, blocks, smem, s);
+    case 2: return decode_fmt_launch<2>(a, fused, nt, blocks, smem, s);
+    case 3: return decode_fmt_launch<3>(a, fused, nt, blocks, smem, s);
+    case 4: return decode_fmt_launch<4>(a, fused, nt, blocks, smem, s);
+    case 5: return decode_fmt_launch<5>(a, fused, nt, blocks, smem, s);
+    case 6: return decode_fmt_launch<6>(a, fused, nt, blocks, smem, s);
+    case 7: return decode_fmt_launch<7>(a, fused, nt, blocks, smem, s);
+    default: return decode_fmt_launch<8>(a, fused, nt, blocks, smem, s);
+  }
 }
 
 }  // namespace sbl

@@ -741,11 +741,12 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
   uint4* const weff_c = reinterpret_cast<uint4*>(a.out.weff_bf16) + v0;
   uint2* const codes_c = a.out.codes != nullptr ? reinterpret_cast<uint2*>(a.out.codes) + v0 : nullptr;
   uint32_t* const spv_c = a.out.sp_values != nullptr ? reinterpret_cast<uint32_t*>(a.out.sp_values) + v0 : nullptr;
-  uint16_t* const gemv_c = a.out.gemv != nullptr ? reinterpret_cast<uint16_t*>(a.out.gemv) + v0 : nullptr;
   const int ring0 = a.mode == kPrepFromSum ? 0 : nch;  // ring slots used before phase 2
   for (int j = 0; j < nch; ++j) {
     const int J = ring0 + j, s = J % kPrepStages;
-    if (!mbar_wait(&tail->full[s], (J / kPrepStages) & 1, abort_flag, status)) break;
+    // the whole warp leaves together (the decode pack's writer below uses
+    // warp shuffles)
+    if (!__all_sync(0xffffffffu, mbar_wait(&tail->full[s], (J / kPrepStages) & 1, abort_flag, status))) break;
     const uint4* st = ring + size_t(s) * kChunkVecs;
 #pragma unroll
     for (int h2 = 0; h2 < kVecsPerThread; ++h2) {
@@ -825,12 +826,64 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
           const int c = col[h2];
           a.out.sp_meta[(r >> 7) * meta_rb_bytes + (r & 127) * 16 + (c >> 4) * 2048 + (c & 15)] =
               static_cast<uint8_t>(Z >> 16);
-          if (gemv_c != nullptr) {
-            // per group: the two kept 2-bit codes (01 = +1, 11 = -1) low, the metadata nibble high
+          if (a.out.gemv != nullptr) {
+            // per group: the two kept 2-bit codes (01 = +1, 11 = -1) low, the
+            // metadata nibble high; the vector's two bytes go to its lane slot
+            // of the interleaved decode pack (16-row x 128-k units of 512
+            // bytes: lane (row % 8) * 4 + t holds 8 bytes of row r, then 8 of
+            // row r + 8, for the groups 8t..8t+7 of the unit)
             uint32_t t = vals & 0x03030303u;
             t |= t >> 6;
             const uint32_t nibs = ((Z >> 12) & 0xF0u) | ((Z >> 8) & 0xF000u);
-            gemv_c[u] = static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
+            const int lane_d = static_cast<int>(r & 7) * 4 + ((c >> 2) & 3);
+            uint8_t* unit = a.out.gemv + ((r >> 4) * a.out.gemv_upr + (c >> 4)) * int64_t(512);
+            *reinterpret_cast<uint16_t*>(unit + lane_d * 16 + ((r >> 3) & 1) * 8 + (c & 3) * 2) =
+                static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
+          }
+        }
+      }
+      if (M != 4 || n != 2) {
+        if (a.out.gemv != nullptr) {  // decode pack of every pattern other than 2:4 (uniform per launch)
+          // dense 2-bit codes of the 8 weights (01 = +1, 11 = -1), from the
+          // high bytes of W_eff (0x3F, 0xBF or 0)
+          const uint32_t t_lo = ((hb_lo >> 5) & 0x01010101u) | ((hb_lo >> 6) & 0x02020202u);
+          const uint32_t t_hi = ((hb_hi >> 5) & 0x01010101u) | ((hb_hi >> 6) & 0x02020202u);
+          const uint32_t d16 = ((t_lo | (t_lo >> 6) | (t_lo >> 12) | (t_lo >> 18)) & 0xFFu) |
+                               (((t_hi | (t_hi >> 6) | (t_hi >> 12) | (t_hi >> 18)) & 0xFFu) << 8);
+          // the block's mask byte and its kept codes in index order
+          const uint32_t mb = (M == 4) ? ((Z & 0xFu) | ((Z >> 4) & 0xF0u)) : (Z & 0xFFu);
+          uint32_t f = 0, pos = 0;
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            if ((mb >> p) & 1u) {
+              f |= ((d16 >> (2 * p)) & 3u) << pos;
+              pos += 2;
+            }
+          }
+          // Four consecutive blocks of a row (k-steps 0..3 of one lane of the
+          // decode kernel) sit in four consecutive lanes here; the first
+          // gathers their fields and mask bytes and writes them whole.
+          const int n8 = a.out.gemv_n8;
+          const uint32_t f1 = __shfl_down_sync(0xffffffffu, f, 1), f2 = __shfl_down_sync(0xffffffffu, f, 2),
+                         f3 = __shfl_down_sync(0xffffffffu, f, 3);
+          const uint32_t m1 = __shfl_down_sync(0xffffffffu, mb, 1), m2 = __shfl_down_sync(0xffffffffu, mb, 2),
+                         m3 = __shfl_down_sync(0xffffffffu, mb, 3);
+          if (active && (lane & 3) == 0) {
+            const uint64_t bits = uint64_t(f) | (uint64_t(f1) << (2 * n8)) | (uint64_t(f2) << (4 * n8)) |
+                                  (uint64_t(f3) << (6 * n8));
+            const int64_t r = row[h2];
+            const int c = col[h2];  // block of 8 within the row
+            const int gq = static_cast<int>(r & 7), hi = static_cast<int>((r >> 3) & 1);
+            const int lane_d = gq * 4 + ((c >> 2) & 3);
+            uint8_t* unit = a.out.gemv + ((r >> 4) * a.out.gemv_upr + (c >> 4)) * int64_t(a.out.gemv_unit_bytes);
+            uint8_t* code_dst = unit + lane_d * a.out.gemv_cb + hi * n8;
+            if (n8 < 8) {
+              *reinterpret_cast<uint32_t*>(unit + lane_d * 8 + hi * 4) = mb | (m1 << 8) | (m2 << 16) | (m3 << 24);
+              code_dst += 256;
+            }
+            for (int b = 0; b < n8; ++b) code_dst[b] = static_cast<uint8_t>(bits >> (8 * b));
+            if (hi == 1)  // the slot's bytes past both rows' fields (odd n8) are zero
+              for (int b = n8; b < a.out.gemv_cb - n8; ++b) code_dst[b] = 0;
           }
         }
       }
@@ -889,6 +942,16 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
   a.out.sp_meta = L.sp_meta ? blob + L.sp_meta : nullptr;
   a.out.gemv = L.gemv ? blob + L.gemv : nullptr;
   a.out.meta_kblocks = static_cast<int>(meta_k_padded(k) / 128);
+  a.out.gemv_n8 = 8 * n / m;
+  a.out.gemv_cb = (2 * a.out.gemv_n8 + 3) / 4 * 4;
+  a.out.gemv_unit_bytes = (a.out.gemv_n8 < 8 ? 256 : 0) + 32 * a.out.gemv_cb;
+  a.out.gemv_upr = static_cast<int>((k + 127) / 128);
+  if (mode != kPrepSumOnly && L.gemv && (n_out % 16 != 0 || k % 128 != 0)) {
+    // the interleaved pack covers whole 16-row, 128-k units: what no weight
+    // fills is zero
+    cudaError_t e = cudaMemsetAsync(blob + L.gemv, 0, L.gemv_bytes, s);
+    if (e != cudaSuccess) return e;
+  }
 
   // One CTA per SM (fewer for small matrices: at least one 16 KB stage of
   // weights per CTA), all resident at once for the grid barrier.

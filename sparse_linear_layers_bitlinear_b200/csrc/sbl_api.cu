@@ -54,7 +54,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 sbl_status check_shape(int64_t n_out, int64_t k, int n, int m, uint32_t flags) {
   if ((flags & ~kLayerFlags) != 0u) return SBL_ERR_INVALID_ARG;
   if (!(m == 2 || m == 4 || m == 8) || n < 1 || n > m) return SBL_ERR_UNSUPPORTED_NM;
-  if ((flags & SBL_PACK_GEMV) && !(n == 2 && m == 4)) return SBL_ERR_UNSUPPORTED_NM;
   if (n_out < 8 || n_out % 8 != 0 || k < 64 || k % 64 != 0) return SBL_ERR_SHAPE;
   if (k > kMaxK || n_out > (int64_t(1) << 30) || n_out * k > (int64_t(1) << 40)) return SBL_ERR_SHAPE;
   return SBL_OK;
@@ -66,6 +65,12 @@ sbl_status check_layer(const sbl_layer* layer, sbl_blob_layout* L) {
   if (layer == nullptr || layer->prepared == nullptr) return SBL_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(layer->prepared) & 255u) != 0) return SBL_ERR_ALIGN;
   return sbl_prepared_layout(layer->n_out, layer->k, layer->n, layer->m, layer->flags, L);
+}
+
+// The decode kernel takes the call when the layer has the decode pack and the
+// token rows fit its shared memory.
+bool uses_decode(const sbl_layer* layer, const sbl_blob_layout& L, int64_t t) {
+  return L.gemv != 0 && gemv_fits(t, layer->k, layer->n, layer->m) && gemv_preferred(t, layer->n_out, layer->k);
 }
 
 template <class T>
@@ -82,7 +87,7 @@ const char* sbl_version(void) { return "sbl 0.1 (sm_100a)"; }
 int sbl_forward_uses_gemv(const sbl_layer* layer, int64_t t) {
   sbl_blob_layout L;
   if (check_layer(layer, &L) != SBL_OK || t <= 0) return 0;
-  return (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) ? 1 : 0;
+  return uses_decode(layer, L, t) ? 1 : 0;
 }
 
 uint64_t sbl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
@@ -109,9 +114,12 @@ sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t 
     L.sp_values = take(uint64_t(n_out) * uint64_t(k / 2));
     L.sp_meta_bytes = uint64_t(meta_rows_padded(n_out)) * uint64_t(meta_k_padded(k) / 8);
     L.sp_meta = take(L.sp_meta_bytes);
-    if (flags & SBL_PACK_GEMV) L.gemv = take(uint64_t(n_out) * uint64_t(k / 4));
   } else {
     L.codes = take(uint64_t(n_out) * uint64_t(k));
+  }
+  if (flags & SBL_PACK_GEMV) {
+    L.gemv_bytes = decode_pack_bytes(n_out, k, n, m);
+    L.gemv = take(L.gemv_bytes);
   }
   L.total_bytes = off;
   L.gamma = L.header + offsetof(BlobHeader, gamma);
@@ -203,14 +211,15 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(layer, L.status);
   const float* g = at<const float>(layer, L.g);
-  if (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) {
-    // decode: the 2-bit weight stream
+  if (uses_decode(layer, L, t)) {
+    // decode: the packed weight stream
     const bool fused = gemv_fuses_act_quant(t);
     if (!fused &&
         launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true) != cudaSuccess)
       return SBL_ERR_CUDA;
     const cudaError_t e =
-        launch_forward_gemv(at<const uint8_t>(layer, L.gemv), static_cast<const uint16_t*>(x), xq, ap, g,
+        launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, static_cast<const uint16_t*>(x),
+                            fused ? nullptr : xq, ap, g,
                             layer->n_out, t, layer->k, y, acc_debug, fused ? xq_out : nullptr,
                             fused ? xscale_out : nullptr, status, sms, s);
     return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
@@ -246,8 +255,9 @@ sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const
   uint32_t* status = at<uint32_t>(layer, L.status);
   const float* g = at<const float>(layer, L.g);
   cudaError_t e;
-  if (L.gemv != 0 && gemv_fits(t, layer->k) && gemv_preferred(t, layer->n_out, layer->k)) {
-    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), nullptr, xq, xscale, g, layer->n_out, t, layer->k, y,
+  if (uses_decode(layer, L, t)) {
+    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, nullptr, xq, xscale, g,
+                            layer->n_out, t, layer->k, y,
                             acc_debug, nullptr, nullptr, status, sms, s);
   } else if (is_24(layer->n, layer->m)) {
     e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
@@ -374,6 +384,14 @@ sbl_status sbl_selftest_wait_timeout(uint32_t* status_dev, uint64_t limit_ns, sb
   return launch_selftest_wait(status_dev, limit_ns, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SBL_OK
              : SBL_ERR_CUDA;
+}
+
+sbl_status sbl_selftest_chain_floor(int32_t blocks, sbl_stream_t stream) {
+  if (blocks < 1 || blocks > 65535) return SBL_ERR_INVALID_ARG;
+  int sms = 0;
+  const sbl_status st = current_device(&sms);
+  if (st != SBL_OK) return st;
+  return launch_chain_floor(blocks, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
 }  // extern "C"

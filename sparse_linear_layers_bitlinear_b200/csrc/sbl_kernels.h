@@ -45,6 +45,9 @@ struct PackOut {
   uint8_t* sp_meta;
   uint8_t* gemv;
   int meta_kblocks;
+  // decode pack of patterns other than 2:4 (gemv != nullptr): kept codes per
+  // block of 8, code bytes per lane and unit, unit bytes, units per row
+  int gemv_n8, gemv_cb, gemv_unit_bytes, gemv_upr;
 };
 
 // mode 0: the whole preparation; 1: only the exact sum of |w| (SBL_SUM_WORDS
@@ -71,17 +74,21 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
                                 int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
                                 cudaStream_t s);
 
-// Decode forward for 1 <= t <= 16 over the 2-bit packing.  For t up to 4 the
-// kernel quantises the activations itself (xq_out / ap_out, when given,
-// receive the codes and scales); for larger t the act-quant kernel runs first
-// with its early trigger and xq_in / ap_in are its outputs.  gemv_fits() says
-// whether the token rows fit the kernel's shared memory.
-bool gemv_fits(int64_t t, int64_t k);
+// Decode forward for 1 <= t <= 32 tokens over the decode pack (2:4: one byte
+// per group of four; other N:M: the interleaved compressed-index pack, see
+// gemv.cu).  For t up to 8 the kernel quantises the activations itself
+// (xq_out / ap_out, when given, receive the codes and scales); otherwise, or
+// when x is NULL, xq_in / ap_in hold the codes (the act-quant kernel runs
+// first with its early trigger).  gemv_fits() says whether the token rows fit
+// the kernel's shared memory.
+uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m);
+bool gemv_fits(int64_t t, int64_t k, int n, int m);
 bool gemv_preferred(int64_t t, int64_t n_out, int64_t k);
 bool gemv_fuses_act_quant(int64_t t);
-cudaError_t launch_forward_gemv(const uint8_t* gemv, const uint16_t* x, const int8_t* xq_in, const float* ap_in,
-                                const float* g, int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out,
-                                int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms, cudaStream_t s);
+cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_t* x, const int8_t* xq_in,
+                                const float* ap_in, const float* g, int64_t n_out, int64_t t, int64_t k, float* y,
+                                int32_t* acc_out, int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms,
+                                cudaStream_t s);
 
 // out[M][N] = alpha * A . B^T in bf16 x bf16 -> fp32 (tensor cores).
 //   a_mn: A stored [K][M] (else [M][K]);  b_mn: B stored [K][N] (else [N][K]).
@@ -99,6 +106,7 @@ cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const ui
                                       cudaStream_t s, bool* done);
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
+cudaError_t launch_chain_floor(int blocks, cudaStream_t s);
 
 // cuTensorMapEncodeTiled, resolved through the runtime's driver entry point.
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,

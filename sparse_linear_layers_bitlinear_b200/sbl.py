@@ -66,7 +66,7 @@ class sbl_layer(ctypes.Structure):
 class sbl_blob_layout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_uint64) for name in (
         "total_bytes", "header", "mask", "codes", "weff_bf16", "sp_values", "sp_meta", "sp_meta_bytes",
-        "gemv", "gamma", "g", "status", "scratch")]
+        "gemv", "gamma", "g", "status", "scratch", "gemv_bytes")]
 
 
 # Every entry point of include/sbl.h with its ctypes signature.
@@ -86,6 +86,7 @@ SIGNATURES = {
     "sbl_clear_status": (_I32, [_LP, _P]),
     "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
+    "sbl_selftest_chain_floor": (_I32, [_I32, _P]),
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
     "sbl_forward_uses_gemv": (ctypes.c_int, [_LP, _I64]),
@@ -208,14 +209,24 @@ def allreduce_sum_words(words, group=None):
 
 def prepare_weights_row_sharded(layer: Layer, w_shard, global_rows: int, group=None, stream=None):
     """The three steps for this rank's row shard: its exact sum, the exact
-    all-reduce of the words, and the preparation with the whole tensor's scale."""
+    all-reduce of the words, and the preparation with the whole tensor's scale.
+
+    The all-reduce is ordered on torch's current stream (as every collective
+    is), so with an explicit ``stream`` the current stream first waits for the
+    sum on ``stream``, and ``stream`` then waits for the all-reduce before the
+    preparation reads the words.  No host synchronisation."""
     import torch
 
     words = torch.empty(SBL_SUM_WORDS, dtype=torch.int64, device=w_shard.device)
     weight_abs_sum(layer, w_shard, words, stream)
-    if stream is not None:
-        stream.synchronize()
+    cur = torch.cuda.current_stream(w_shard.device) if w_shard.is_cuda else None
+    side = stream is not None and cur is not None and stream != cur
+    if side:
+        cur.wait_stream(stream)
     allreduce_sum_words(words, group)
+    if side:
+        stream.wait_stream(cur)
+        words.record_stream(stream)
     prepare_weights_from_sum(layer, w_shard, words, global_rows * layer.k, stream)
     return words
 
@@ -278,6 +289,12 @@ def read_scale(layer: Layer, stream=None):
 
 def selftest_wait_timeout(status_dev, limit_ns: int, stream=None):
     _check(lib().sbl_selftest_wait_timeout(_ptr(status_dev), limit_ns, _stream(stream)), "sbl_selftest_wait_timeout")
+
+
+def selftest_chain_floor(blocks: int, stream=None):
+    """One empty kernel launched as the library launches its kernels (the
+    per-call floor of a chain of dependent calls)."""
+    _check(lib().sbl_selftest_chain_floor(blocks, _stream(stream)), "sbl_selftest_chain_floor")
 
 
 def version() -> str:

@@ -69,8 +69,18 @@ def sp_meta_canonical(layer):
 
 
 def gemv_bytes(layer):
+    """The interleaved 2:4 decode pack of a layer re-laid out as its canonical
+    [n_out, k/4] group bytes (units of 16 rows x 128 k: lane (row % 8) * 4 + t
+    holds 8 bytes of its row, then 8 of the row 8 below, for the groups
+    8t..8t+7 of the unit), plus every byte outside the matrix."""
     n_out, k = layer.n_out, layer.k
-    return section(layer, "gemv", n_out * k // 4).reshape(n_out, k // 4)
+    tiles, upr = (n_out + 15) // 16, (k + 127) // 128
+    L = layer.layout()
+    assert L.gemv_bytes == tiles * upr * 512
+    raw = section(layer, "gemv", int(L.gemv_bytes)).reshape(tiles, upr, 8, 4, 2, 8)  # tile, unit, g, t, hi, byte
+    full = raw.transpose(0, 4, 2, 1, 3, 5).reshape(tiles * 16, upr * 32)
+    pad = np.concatenate([full[n_out:].ravel(), full[:n_out, k // 4:].ravel()])
+    return full[:n_out, :k // 4], pad
 
 
 def decode_gemv(gb):
@@ -80,6 +90,48 @@ def decode_gemv(gb):
     c0 = to_code[gb & 3]
     c1 = to_code[(gb >> 2) & 3]
     return nib, c0, c1
+
+
+def nm_pack_fields(masks8, codes, n, m):
+    """The oracle's canonical compressed-index pack as (mask bytes [n_out, k/8],
+    code fields [n_out, k/8]): field b is the 2 n8 bits of block b's kept codes."""
+    n8 = 8 * n // m
+    n_out, blocks = masks8.shape
+    bits = np.unpackbits(codes, axis=1, bitorder="little").reshape(n_out, blocks, 2 * n8).astype(np.int64)
+    return masks8, (bits << np.arange(2 * n8, dtype=np.int64)).sum(-1)
+
+
+def gemv_nm_fields(layer):
+    """The interleaved decode pack of a non-2:4 layer re-laid out as (mask bytes
+    [n_out, k/8], code fields [n_out, k/8]), plus every byte that no weight
+    fills (rows padded to 16, k to 128) for a check that it is zero."""
+    n_out, k, n, m = layer.n_out, layer.k, layer.n, layer.m
+    n8 = 8 * n // m
+    cb = (2 * n8 + 3) // 4 * 4
+    has_mask = n8 < 8
+    ub = (256 if has_mask else 0) + 32 * cb
+    tiles, upr = (n_out + 15) // 16, (k + 127) // 128
+    L = layer.layout()
+    assert L.gemv_bytes == tiles * upr * ub
+    raw = section(layer, "gemv", int(L.gemv_bytes)).reshape(tiles, upr, ub)
+    rows, blocks = tiles * 16, upr * 16
+    masks = np.full((rows, blocks), 0xFF, dtype=np.uint8)
+    if has_mask:
+        # [tile][unit][g][t][hi][s] -> row tile*16 + hi*8 + g, block unit*16 + t*4 + s
+        mb = raw[:, :, :256].reshape(tiles, upr, 8, 4, 2, 4)
+        masks = mb.transpose(0, 4, 2, 1, 3, 5).reshape(rows, blocks)
+    cbytes = raw[:, :, 256 if has_mask else 0:].reshape(tiles, upr, 32, cb)
+    cbits = np.unpackbits(cbytes, axis=-1, bitorder="little").astype(np.int64)  # [..., 32, cb*8]
+    used = cbits[..., :16 * n8].reshape(tiles, upr, 8, 4, 2, 4, 2 * n8)  # g, t, hi, s, bit
+    spare = cbits[..., 16 * n8:]
+    fields = (used << np.arange(2 * n8, dtype=np.int64)).sum(-1)
+    fields = fields.transpose(0, 4, 2, 1, 3, 5).reshape(rows, blocks)
+    none = np.zeros(0, dtype=bool)
+    pad = np.concatenate([masks[n_out:].ravel() != 0 if has_mask else none,
+                          masks[:n_out, k // 8:].ravel() != 0 if has_mask else none,
+                          fields[n_out:].ravel() != 0, fields[:n_out, k // 8:].ravel() != 0,
+                          spare.ravel() != 0])
+    return masks[:n_out, :k // 8], fields[:n_out, :k // 8], pad
 
 
 def bf16_to_f64(t: torch.Tensor):

@@ -56,8 +56,10 @@ def test_version(lib):
 
 
 def test_layout_sections_are_aligned_and_disjoint(lib):
-    for (n_out, k, n, m, flags) in [(6912, 2560, 2, 4, 0), (2560, 6912, 6, 8, 0), (264, 320, 2, 4, sbl.SBL_PACK_GEMV),
-                                    (8, 64, 1, 2, 0)]:
+    g = sbl.SBL_PACK_GEMV
+    for (n_out, k, n, m, flags) in [(6912, 2560, 2, 4, 0), (2560, 6912, 6, 8, 0), (264, 320, 2, 4, g),
+                                    (8, 64, 1, 2, 0), (2560, 6912, 6, 8, g), (264, 320, 3, 8, g), (8, 64, 1, 2, g),
+                                    (136, 448, 8, 8, g)]:
         L = sbl.prepared_layout(n_out, k, n, m, flags)
         spans = [("header", L.header, 4096), ("scratch", L.scratch, 1024 * 40 * 8 + 1024 * 32 + 256), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
         if (n, m) == (2, 4):
@@ -65,10 +67,19 @@ def test_layout_sections_are_aligned_and_disjoint(lib):
             assert L.sp_meta_bytes == ((n_out + 255) // 256 * 256) * ((k + 255) // 256 * 256) // 8
             assert L.codes == 0
             if flags & sbl.SBL_PACK_GEMV:
-                spans.append(("gemv", L.gemv, n_out * k // 4))
+                assert L.gemv_bytes == ((n_out + 15) // 16) * ((k + 127) // 128) * 512  # interleaved units
         else:
             spans.append(("codes", L.codes, n_out * k))
             assert L.sp_values == 0 and L.sp_meta == 0
+            if flags & sbl.SBL_PACK_GEMV:
+                # units of 16 rows x 128 k: a 256-byte mask block (n < m) and 32 lanes' code bytes
+                n8 = 8 * n // m
+                unit = (256 if n8 < 8 else 0) + 32 * ((2 * n8 + 3) // 4 * 4)
+                assert L.gemv_bytes == ((n_out + 15) // 16) * ((k + 127) // 128) * unit
+        if flags & sbl.SBL_PACK_GEMV:
+            spans.append(("gemv", L.gemv, L.gemv_bytes))
+        else:
+            assert L.gemv == 0 and L.gemv_bytes == 0
         spans.sort(key=lambda s: s[1])
         for (_, off, size), (_, nxt, _) in zip(spans, spans[1:]):
             assert off % 256 == 0 and off + size <= nxt
@@ -92,13 +103,15 @@ def test_forward_dispatch_query(lib):
         return sbl.forward_uses_gemv(sbl.Layer(n_out, k, n, m, flags, _FakeBlob()), t)
 
     g = sbl.SBL_PACK_GEMV
-    assert uses(6912, 2560, 2, 4, g, 1) and uses(6912, 2560, 2, 4, g, 4)
-    assert not uses(6912, 2560, 2, 4, g, 8) and not uses(6912, 2560, 2, 4, g, 16)  # tensor cores win
-    assert uses(2560, 2560, 2, 4, g, 8) and not uses(2560, 2560, 2, 4, g, 16)
-    assert not uses(256, 256, 2, 4, g, 17)      # beyond the GEMV's token count
-    assert not uses(6912, 2560, 2, 4, 0, 1)     # no 2-bit packing
+    for t in (1, 4, 8, 16, 32):
+        assert uses(6912, 2560, 2, 4, g, t) and uses(2560, 2560, 2, 4, g, t)
+        assert uses(2560, 6912, 6, 8, g, t) == (t <= 16)  # 32 token rows of k = 6912 exceed shared memory
+        assert uses(2560, 2560, 4, 8, g, t) and uses(2560, 2560, 8, 8, g, t)
+    assert not uses(256, 256, 2, 4, g, 33)      # beyond the decode kernel's token count
+    assert not uses(6912, 2560, 2, 4, 0, 1)     # no decode pack
+    assert not uses(2560, 6912, 6, 8, 0, 1)
     assert not uses(6912, 2560, 2, 4, g, 0)
-    assert not uses(6912, 2560, 6, 8, g, 1)     # not a valid layer
+    assert not uses(6912, 2560, 6, 4, g, 1)     # not a valid layer
 
 
 def test_backward_workspace_for_the_quantised_x_operand(lib):
@@ -121,7 +134,7 @@ def test_backward_workspace_for_the_quantised_x_operand(lib):
     ((256, 256, 2, 3, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
     ((256, 256, 0, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
     ((256, 256, 5, 4, 0), sbl.SBL_ERR_UNSUPPORTED_NM),
-    ((256, 256, 6, 8, sbl.SBL_PACK_GEMV), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 256, 6, 4, sbl.SBL_PACK_GEMV), sbl.SBL_ERR_UNSUPPORTED_NM),
     ((256, 96, 2, 4, 0), sbl.SBL_ERR_SHAPE),
     ((250, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),
     ((0, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),

@@ -91,20 +91,25 @@ def test_fullsize_parity(name, n_out, k, n, m, t):
     assert (err <= 1e-2 + 2.0 ** -7 * np.abs(dwr)).all(), err.max()
 
 
-@pytest.mark.parametrize("t", [1, 4, 16])
+@pytest.mark.parametrize("t", [1, 4, 16, 32])
 @pytest.mark.parametrize("n_out", [2560, 6912])
-def test_decode_gemv_fullsize(t, n_out):
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+def test_decode_gemv_fullsize(t, n_out, n, m):
+    """The decode workload (k = 2560, n_out 2560 or 6912) through the decode
+    kernel, 2:4 on its 2-bit pack and 6:8 on the compressed-index pack: every
+    accumulator and output, bit for bit."""
     k = 2560
     w_d = synth.master_weights(n_out, k, 10, device="cuda")
     x_d = synth.activations(t, k, 11, device="cuda")
-    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
+    assert sbl.forward_uses_gemv(layer, t)
     sbl.prepare_weights(layer, w_d)
     y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
     acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
     ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
     sbl.forward(layer, x_d, t, y, acc_debug=acc, workspace=ws)
     torch.cuda.synchronize()
-    ref = oracle.forward(w_d.cpu(), x_d.cpu(), 2, 4)
+    ref = oracle.forward(w_d.cpu(), x_d.cpu(), n, m)
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
 

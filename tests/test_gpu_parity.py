@@ -48,12 +48,22 @@ def _check_prepared(layer, w, n, m):
         assert np.array_equal(canon, meta)
         assert (pad_rows == 0x44).all() and (pad_cols == 0x44).all()
         if layer.flags & sbl.SBL_PACK_GEMV:
-            nib, c0, c1 = bd.decode_gemv(bd.gemv_bytes(layer))
+            gb, pad = bd.gemv_bytes(layer)
+            assert not pad.any(), "bytes outside the matrix must be zero"
+            nib, c0, c1 = bd.decode_gemv(gb)
             mnib = np.stack([meta & 0xF, meta >> 4], axis=-1).reshape(meta.shape[0], -1)
             assert np.array_equal(nib, mnib)
             assert np.array_equal(c0, vals[:, 0::2]) and np.array_equal(c1, vals[:, 1::2])
     else:
         assert np.array_equal(bd.codes(layer), ref["weff"])
+        if layer.flags & sbl.SBL_PACK_GEMV:
+            masks8, codes = oracle.pack_nm(ref["weff"], ref["mask"], n, m)
+            want_m, want_f = bd.nm_pack_fields(masks8, codes, n, m)
+            got_m, got_f, pad = bd.gemv_nm_fields(layer)
+            if n < m:
+                assert np.array_equal(got_m, want_m)
+            assert np.array_equal(got_f, want_f)
+            assert not pad.any(), "bytes outside the matrix must be zero"
     return ref
 
 
@@ -123,7 +133,7 @@ def test_prepare_forward_backward_parity(n_out, k, n, m, t):
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
 
 
-@pytest.mark.parametrize("t", [1, 2, 3, 4, 5, 7, 8, 9, 16])
+@pytest.mark.parametrize("t", [1, 2, 3, 4, 5, 7, 8, 9, 16, 17, 24, 32])
 def test_gemv_path_parity(t):
     n_out, k = 392, 640
     w = synth.master_weights(n_out, k, 3)
@@ -658,16 +668,17 @@ def test_act_quant_more_rows_than_resident_warps():
     assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("t", [4, 8, 16])
+@pytest.mark.parametrize("t", [4, 8, 16, 33])
 def test_decode_dispatch_both_paths_bit_exact(t):
-    """A layer with the 2-bit packing at the decode sizes: small calls take the
-    GEMV, larger ones the 2:4 tensor-core GEMM; both give the oracle's bits."""
+    """A layer with the decode pack at the decode sizes: up to 32 tokens take
+    the decode kernel (quantising for itself up to 8), more the 2:4
+    tensor-core GEMM; both give the oracle's bits."""
     n_out, k = 6912, 2560
     w = synth.master_weights(n_out, k, 81)
     x = synth.activations(t, k, 82)
     layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
     sbl.prepare_weights(layer, _dev(w))
-    assert sbl.forward_uses_gemv(layer, t) == (t <= 4)
+    assert sbl.forward_uses_gemv(layer, t) == (t <= 32)
     y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
     acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
     xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
@@ -680,8 +691,91 @@ def test_decode_dispatch_both_paths_bit_exact(t):
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
     assert np.array_equal(xq.cpu().numpy(), ref["xq"])
-    assert launched == (1 if t <= 4 else 2)  # the fused GEMV, or act-quant + GEMM
+    assert launched == (1 if t <= 8 else 2)  # the decode kernel alone, or act-quant first
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+NM_PATTERNS = [(6, 8), (4, 8), (3, 8), (1, 8), (2, 8), (5, 8), (7, 8), (8, 8), (1, 4), (3, 4), (4, 4), (1, 2), (2, 2)]
+
+
+def _decode_check(n_out, k, n, m, t, seed, with_codes=True):
+    """Prepare with the decode pack (its bytes checked against the oracle's
+    pack), run sbl_forward at t tokens through the decode kernel and compare
+    the int32 accumulators and y bit for bit (and the codes and scales it
+    hands back)."""
+    w = synth.master_weights(n_out, k, seed)
+    x = synth.activations(t, k, seed + 1)
+    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(w))
+    torch.cuda.synchronize()
+    ref = _check_prepared(layer, w, n, m)
+    assert sbl.forward_uses_gemv(layer, t)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    if with_codes:
+        xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+        ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+        sbl.forward(layer, _dev(x), t, y, xq, ap, acc)
+    else:
+        ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+        sbl.forward(layer, _dev(x), t, y, acc_debug=acc, workspace=ws)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    xq_ref, ap_ref = oracle.act_quant(x)
+    if with_codes:
+        assert np.array_equal(xq.cpu().numpy(), xq_ref)
+        assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    acc_ref = oracle.gemm_acc(xq_ref, ref["weff"])
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    y_ref = oracle.dequant(acc_ref, ap_ref, ref["g"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), y_ref.view(np.uint32))
+    _close(y.cpu().numpy(), y_ref)
+    return layer
+
+
+@pytest.mark.parametrize("n,m", NM_PATTERNS)
+@pytest.mark.parametrize("t", [1, 3, 8, 9, 16, 32])
+def test_decode_compressed_index_patterns(n, m, t):
+    """Every N:M pattern through the compressed-index decode pack, on a shape
+    with a ragged last row tile (136 rows) and a half 128-k unit (k = 448)."""
+    _decode_check(136, 448, n, m, t, seed=700 + 16 * n + m + t)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (8, 8)])
+@pytest.mark.parametrize("t", [4, 20])
+def test_decode_blocks_of_several_tiles(n, m, t):
+    """11200 rows: three 16-row tiles per block and five units per tile, so a
+    warp's units straddle two tiles and their partial sums meet in shared
+    memory."""
+    _decode_check(11200, 640, n, m, t, seed=900 + n + t, with_codes=False)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
+@pytest.mark.parametrize("k,t", [(16384, 1), (16384, 8), (10240, 9)])
+def test_decode_long_rows(n, m, k, t):
+    """One tile of long rows: 128 (or 80) units over eight warps, each warp
+    loading its 16 (or 10) units in two batches; 9 token rows of k = 10240 is
+    about the most the kernel's shared memory holds."""
+    _decode_check(16, k, n, m, t, seed=950 + n + t)
+
+
+def test_decode_declines_rows_beyond_its_shared_memory():
+    """16 token rows of k = 16384 do not fit: the call takes the tensor-core
+    GEMM and still gives the oracle's bits."""
+    n_out, k, t = 256, 16384, 9
+    w = synth.master_weights(n_out, k, 960)
+    x = synth.activations(t, k, 961)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(w))
+    assert not sbl.forward_uses_gemv(layer, t)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, acc_debug=acc, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle.forward(w, x, 2, 4)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
 
 
 @pytest.mark.parametrize("tiny", [2.0 ** -40, 0.0, -(2.0 ** -35)])
@@ -832,6 +926,68 @@ def test_row_sharded_midpoint_decided_by_a_tiny_magnitude_in_another_shard():
     assert float(oracle.absmean_gamma(w)) == 1.0 + 2.0 ** -23
     for layer in _row_sharded_prepare(w, 2, 4, 2):
         assert sbl.read_scale(layer) == (1.0 + 2.0 ** -23, 1.0 + 2.0 ** -23)
+
+
+def test_row_sharded_helper_orders_the_exchange_on_a_side_stream(monkeypatch):
+    """sbl.prepare_weights_row_sharded with an explicit side stream: the
+    exchange of the sum words runs on torch's current stream, and the
+    preparation on the side stream must wait for it.  The stand-in exchange
+    adds the other shard's words after a long sleep on the current stream, so
+    a preparation that read the words early would decide gamma from this
+    shard alone."""
+    n_out, k = 384, 512
+    rows = n_out // 2
+    w = synth.master_weights(n_out, k, 77)
+    w[rows + 5, 3] = 96.0  # the other shard moves gamma well away from this shard's own
+    ref = oracle.prepare(w, 2, 4)
+    other = sbl.Layer.allocate(rows, k, 2, 4)
+    other_words = torch.empty(sbl.SBL_SUM_WORDS, dtype=torch.int64, device="cuda")
+    sbl.weight_abs_sum(other, _dev(w[rows:].contiguous()), other_words)
+    torch.cuda.synchronize()
+
+    def exchange(words, group=None):
+        torch.cuda._sleep(50_000_000)
+        words.add_(other_words)
+        return words
+
+    monkeypatch.setattr(sbl, "allreduce_sum_words", exchange)
+    side = torch.cuda.Stream()
+    layer = sbl.Layer.allocate(rows, k, 2, 4)
+    sbl.prepare_weights_row_sharded(layer, _dev(w[:rows].contiguous()), n_out, stream=side)
+    torch.cuda.synchronize()
+    gamma, g = sbl.read_scale(layer)
+    assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
+    assert np.array_equal(bd.mask(layer), ref["mask"][:rows])
+    assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"][:rows])
+
+
+def test_row_sharded_helper_over_a_one_rank_nccl_group():
+    """The helper end to end over a real NCCL process group of one rank, with
+    an explicit side stream: the whole tensor's gamma, mask and codes."""
+    import socket
+
+    import torch.distributed as dist
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        n_out, k = 256, 512
+        w = synth.master_weights(n_out, k, 78)
+        ref = oracle.prepare(w, 6, 8)
+        side = torch.cuda.Stream()
+        layer = sbl.Layer.allocate(n_out, k, 6, 8)
+        sbl.prepare_weights_row_sharded(layer, _dev(w), n_out, stream=side)
+        torch.cuda.synchronize()
+        gamma, g = sbl.read_scale(layer)
+        assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
+        assert np.array_equal(bd.mask(layer), ref["mask"])
+        assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"])
+        assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    finally:
+        dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("t", [17000, 16000])
