@@ -600,9 +600,20 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     dw = {(o, k): torch.empty((o, k), dtype=torch.bfloat16, device=dev) for (_, o, k) in shapes}
     s = torch.cuda.Stream(dev)
 
-    def prepare_phase():
+    # Grouped prepares per transformer block: q, k, v, o; gate, up; down
+    # (each group's masters fit L2, so the second read of every matrix hits).
+    groups = []
+    for l in range(layers):
+        blk = lin[7 * l:7 * l + 7]
+        groups += [blk[0:4], blk[4:6], blk[6:7]]
+
+    def prepare_phase_single():
         for d in lin:
             sbl.prepare_weights(d["layer"], d["w"], stream=s)
+
+    def prepare_phase():
+        for grp in groups:
+            sbl.prepare_weights_grouped([d["layer"] for d in grp], [d["w"] for d in grp], stream=s)
 
     def forward_phase():
         for d in lin:
@@ -616,12 +627,13 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
             sbl.backward(d["layer"], d["x"], d["dy"], T, dx[d["k"]], dw[(d["n_out"], d["k"])], 0, stream=s)
 
     def step():
-        for d in lin:
-            sbl.prepare_weights(d["layer"], d["w"], stream=s)
-            if d["shared"]:
-                sbl.forward_quantized(d["layer"], d["xq"], d["ap"], T, y[d["n_out"]], stream=s)
-            else:
-                sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], d["xq"], d["ap"], stream=s)
+        for grp in groups:
+            sbl.prepare_weights_grouped([d["layer"] for d in grp], [d["w"] for d in grp], stream=s)
+            for d in grp:
+                if d["shared"]:
+                    sbl.forward_quantized(d["layer"], d["xq"], d["ap"], T, y[d["n_out"]], stream=s)
+                else:
+                    sbl.forward(d["layer"], d["x"], T, y[d["n_out"]], d["xq"], d["ap"], stream=s)
         backward_phase()
 
     with torch.cuda.stream(s):
@@ -643,7 +655,7 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     # The phases on their own: one graph per phase (all prepares; all
     # act-quants and forwards; all backwards), replayed in step order.
     graphs = []
-    for body in (prepare_phase, forward_phase, backward_phase):
+    for body in (prepare_phase, forward_phase, backward_phase, prepare_phase_single):
         gp = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gp, stream=s):
             body()
@@ -651,16 +663,16 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     for gp in graphs:
         gp.replay()
     torch.cuda.synchronize(dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    phase = [0.0, 0.0, 0.0]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    phase = [0.0, 0.0, 0.0, 0.0]
     for _ in range(steps):
         with torch.cuda.stream(s):
             for i, gp in enumerate(graphs):
                 ev[i].record(s)
                 gp.replay()
-            ev[3].record(s)
+            ev[4].record(s)
         torch.cuda.synchronize(dev)
-        for i in range(3):
+        for i in range(4):
             phase[i] += ev[i].elapsed_time(ev[i + 1]) / steps
     del graphs
     for d in lin[:7]:
@@ -684,12 +696,81 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
     return {"workload": f"training step, {layers} layers x 7 linears, {n}:{m}", "tokens": T, "n": n, "m": m,
             "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "roofline_ms": total * 1e3,
             "roofline_frac": total * 1e3 / ms, "peak_note": "sustained bf16 peak (seconds-long step)",
-            "phase_ms": dict(zip(names, phase)),
+            "phase_ms": dict(zip(names, phase[:3])),
+            "prepare_one_launch_per_matrix_ms": phase[3],
+            "prepare_note": "the step prepares each transformer block's linears in three grouped launches "
+                            "(q, k, v, o; gate, up; down); prepare_one_launch_per_matrix_ms is the same phase "
+                            "with one launch per matrix",
             "phase_roofline_ms": {k: v * 1e3 for k, v in bound.items()},
             "phase_frac": {k: bound[k] * 1e3 / phase[i] for i, k in enumerate(names)},
             "timing": f"one CUDA graph per step, {steps} replays after one warm-up; phase_ms: one graph per phase "
-                      f"(all 210 prepares; all act-quants and forwards; all backwards), replayed in step order, "
-                      f"events between them"}
+                      f"(all 210 prepares in 90 grouped launches; all act-quants and forwards; all backwards), "
+                      f"replayed in step order, events between them"}
+
+
+# ---------------------------------------------------------------------------
+# Small fixed cases for a profiler (ncu): a few launches of one kernel family
+# ---------------------------------------------------------------------------
+def profile_decode():
+    """The decode kernel at K = 2560, N_out = 6912: 2:4 and 6:8 decode packs,
+    t = 1, 4 and 16 (t = 16 runs the act-quant kernel first), two calls each."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    dev = torch.device("cuda", 0)
+    K, N = 2560, 6912
+    for (n, m) in ((2, 4), (6, 8)):
+        L = sbl.Layer.allocate(N, K, n, m, sbl.SBL_PACK_GEMV, device=dev)
+        sbl.prepare_weights(L, synth.master_weights(N, K, 5000, device=dev))
+        for T in (1, 4, 16):
+            x = synth.activations(T, K, 7, device=dev)
+            y = torch.empty((T, N), dtype=torch.float32, device=dev)
+            ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+            for _ in range(2):
+                sbl.forward(L, x, T, y, workspace=ws)
+        torch.cuda.synchronize()
+
+
+def profile_prefill68():
+    """The 6:8 FFN down projection forward (T = 4096, K = 6912, N_out = 2560):
+    act-quant (rows of 6912) and the dense int8 pair GEMM, three times."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    dev = torch.device("cuda", 0)
+    T, K, N = 4096, 6912, 2560
+    L = sbl.Layer.allocate(N, K, 6, 8, device=dev)
+    sbl.prepare_weights(L, synth.master_weights(N, K, 0, device=dev))
+    x = synth.activations(T, K, 1, device=dev)
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        sbl.forward(L, x, T, y, workspace=ws)
+    torch.cuda.synchronize()
+
+
+def profile_grouped_prepare():
+    """One transformer block's seven linears (q, k, v, o 2560 x 2560; gate, up
+    2560 -> 6912; down 6912 -> 2560), 2:4, prepared in the three grouped
+    launches of the training step, twice."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    dev = torch.device("cuda", 0)
+    H, F = 2560, 6912
+    shapes = [(H, H)] * 4 + [(F, H)] * 2 + [(H, F)]
+    layers = [sbl.Layer.allocate(o, k, 2, 4, device=dev) for (o, k) in shapes]
+    ws = [synth.master_weights(o, k, 10 * j, device=dev) for j, (o, k) in enumerate(shapes)]
+    for _ in range(2):
+        for a, b in ((0, 4), (4, 6), (6, 7)):
+            sbl.prepare_weights_grouped(layers[a:b], ws[a:b])
+    torch.cuda.synchronize()
+
+
+PROFILE_CASES = {"decode": profile_decode, "prefill68": profile_prefill68, "grouped_prepare": profile_grouped_prepare}
 
 
 # ---------------------------------------------------------------------------
@@ -704,8 +785,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and 6:8 workloads")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run a few launches of one workload for a profiler and exit (no JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.profile_case:
+        PROFILE_CASES[args.profile_case]()
+        return
 
     world, rank, local = dist_setup()
     if args.impl == "reference":

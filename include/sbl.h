@@ -161,6 +161,20 @@ size_t sbl_workspace_bytes(int64_t t, int64_t k);
  * status word.  Raises SBL_ERR_NONFINITE (device) for NaN/Inf masters. */
 sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl_stream_t stream);
 
+/* Steps 1-3 for several layers in one launch (up to 8, all with the same m):
+ * the same preparation as one sbl_prepare_weights call per layer, bit for
+ * bit, with the device's SMs split among the matrices in proportion to their
+ * sizes; every matrix keeps its own exact scale and its own barrier in its
+ * own blob.  One launch pays the launch, the ramp of the weight stream and
+ * the barrier once for the group (the per-step recompute of a transformer
+ * block's linears, [ja] 2.1, [ko] 2.2).  The masters of a group should fit
+ * L2 together (about 100 MB), since each matrix is read twice.
+ * Errors: SBL_ERR_INVALID_ARG for count outside 1..8, a NULL pointer, two
+ * layers sharing a blob or more layers than SMs; SBL_ERR_UNSUPPORTED_NM for
+ * mixed m; otherwise as sbl_prepare_weights. */
+sbl_status sbl_prepare_weights_grouped(const sbl_layer* layers, const void* const* w_masters, int32_t count,
+                                       sbl_stream_t stream);
+
 /* Tensor parallelism by rows of W (each rank holds n_out / R rows; groups
  * along k never split).  The scale gamma is the mean |w| over the WHOLE
  * tensor, so the shards' exact sums are added first:
@@ -198,10 +212,12 @@ sbl_status sbl_prepare_weights_from_sum(const sbl_layer* layer, const void* w_ma
  * (int32 [t, n_out]) may be NULL; when given, the raw accumulators are
  * written too.  t == 0 is a no-op.  2:4 layers run the 2:4-sparse int8
  * tensor-core GEMM; other patterns the dense int8 one over W_eff codes.  A
- * layer prepared with SBL_PACK_GEMV takes the decode GEMV over its 2-bit
- * packing instead for small calls (t <= 16 and t * n_out * k <= 8e7, where
- * that GEMV is the faster of the two); the outputs are the same bits either
- * way. */
+ * layer prepared with SBL_PACK_GEMV takes the decode kernel over its decode
+ * pack instead for t <= 32 tokens, when that many token rows of k codes fit
+ * the kernel's shared memory (sbl_forward_uses_gemv says which path a call
+ * takes); for t <= 4 the decode kernel also quantises the activations
+ * itself, so the call is one launch.  The outputs are the same bits on every
+ * path. */
 sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
                        float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
 
@@ -214,8 +230,8 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
 sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const float* xscale, int64_t t, float* y,
                                  int32_t* acc_debug, sbl_stream_t stream);
 
-/* 1 when sbl_forward on this layer with t tokens takes the decode GEMV over
- * the 2-bit packing, 0 when it takes a tensor-core GEMM (or the arguments
+/* 1 when sbl_forward on this layer with t tokens takes the decode kernel
+ * over the decode pack, 0 when it takes a tensor-core GEMM (or the arguments
  * are invalid).  Host only, no device access. */
 int sbl_forward_uses_gemv(const sbl_layer* layer, int64_t t);
 

@@ -42,7 +42,7 @@
 // a prepare: L2 is the coherence point, so a later write is never hidden),
 // and lets the next call launch; in a chain of decode calls the weight stream
 // of one call overlaps the call before it.  After the wait the block issues
-// its weight loads, quantises its token rows into shared memory (t <= 8) or
+// its weight loads, quantises its token rows into shared memory (t <= 4) or
 // copies the codes the act-quant kernel wrote, and runs the products.  Partial
 // sums of warps sharing a tile are added in shared memory (exact integer
 // adds, any order); y = acc * ((g a') / 127) closes the block.
@@ -60,12 +60,12 @@ constexpr int kDecWarps = kDecThreads / 32;
 // A table of 256 entries kept in kLutCopies copies, entry e of copy c at word
 // e * kLutCopies + c; lane l reads copy l % kLutCopies, so at most
 // 32 / kLutCopies lanes share a copy's banks.
-constexpr int kLutCopies = 16;
+constexpr int kLutCopies = 32;
 constexpr int kLutWords = 256 * kLutCopies;
 constexpr int kDecBatch = 8;         // units whose weight bytes a lane holds at once
 constexpr size_t kDecMaxSmem = 227 * 1024;
 constexpr int kDecMaxT = 32;
-constexpr int kFusedMaxT = 8;  // token counts the kernel quantises itself
+constexpr int kFusedMaxT = 4;  // token counts the kernel quantises itself
 
 struct DecodeArgs {
   const uint8_t* w;      // weight pack
@@ -310,19 +310,23 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   };
 
   // ---- activation codes into shared memory ----
+  float g_early = 0.0f;
   // The activation loads go out first (the rest of the block's path waits
   // on them), then this warp's first batch of weight loads, which are needed
   // only by the products.
   if constexpr (FUSED) {
-    // Quantise the t <= 8 rows here: wpr warps per row, the row's absmax
+    // Quantise the t <= 4 rows here: wpr warps per row, the row's absmax
     // through the warps' maxima in shared memory.
-    const int tp2 = a.t <= 1 ? 1 : a.t <= 2 ? 2 : a.t <= 4 ? 4 : 8;
+    const int tp2 = a.t <= 1 ? 1 : a.t <= 2 ? 2 : 4;
     const int wpr = kDecWarps / tp2;
     const int xrow = warp / wpr, xsub = warp % wpr;
     const bool live = xrow < a.t;
     const uint4* xsrc = a.x + int64_t(xrow) * (a.k / 8);
     const bool scale_thread = live && xsub == 0 && lane == 0;
-    constexpr int kXc = 2;  // chunks kept in registers between the two passes
+    // the output scale (g a') / 127 is formed after the products by threads
+    // 0..t-1; their g load goes out now, off the critical path
+    g_early = tid < a.t ? __ldg(a.g) : 0.0f;
+    constexpr int kXc = 3;  // chunks kept in registers between the two passes
     uint4 xr[kXc][2];
 #pragma unroll
     for (int q = 0; q < kXc; ++q) {
@@ -355,12 +359,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     if (lane == 0) s_red[warp] = bad ? -1.0f : amax;  // amax >= 0: -1 flags a non-finite row
     __syncthreads();
     if (live) {
+      // the row's wpr partial maxima, read as two vectors
+      const float4 r0 = reinterpret_cast<const float4*>(s_red)[0], r1 = reinterpret_cast<const float4*>(s_red)[1];
+      const float part[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
       float m = 0.0f;
       bool row_bad = false;
-      for (int w = 0; w < wpr; ++w) {
-        const float v = s_red[xrow * wpr + w];
-        row_bad |= v < 0.0f;
-        m = fmaxf(m, v);
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        if (w / wpr == xrow) {
+          row_bad |= part[w] < 0.0f;
+          m = fmaxf(m, part[w]);
+        }
       }
       const float ap = fmaxf(m, 1e-5f);
       const QScale qs = make_qscale(ap);
@@ -458,7 +467,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       for (int p = 0; p < 2; ++p) {
         uint4 bv[NT];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) bv[nt] = *reinterpret_cast<const uint4*>(bsrc[nt][p] + 128 * un);
+        for (int nt = 0; nt < NT; ++nt)
+          bv[nt] = (gq + 8 * nt < a.t) ? *reinterpret_cast<const uint4*>(bsrc[nt][p] + 128 * un) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int sp = 0; sp < 2; ++sp) {
           uint32_t a0, a1, a2, a3;
@@ -476,17 +486,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     }
   }
   if (cur >= 0) flush(cur);
-  if (FUSED && tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(__ldg(a.g), s_ap[tid]), 127.0f);
+  if (FUSED && tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(g_early, s_ap[tid]), 127.0f);
   __syncthreads();
 
   // ---- epilogue: y = acc * ((g a') / 127), consecutive rows per token ----
   const int rows = min(ntile * 16, a.n_out - tile0 * 16);
-  for (int tok = 0; tok < a.t; ++tok) {
-    const float sc = s_scale[tok];
-    for (int r = tid; r < rows; r += kDecThreads) {
+  for (int idx = tid; idx < ntile * 16 * a.t; idx += kDecThreads) {
+    const int tok = idx / (ntile * 16), r = idx - tok * (ntile * 16);
+    if (r < rows) {
       const int v = s_acc[(r >> 4) * 16 * TP + (r & 15) * TP + tok];
       const int64_t o = int64_t(tok) * a.n_out + tile0 * 16 + r;
-      a.y[o] = __fmul_rn(static_cast<float>(v), sc);
+      a.y[o] = __fmul_rn(static_cast<float>(v), s_scale[tok]);
       if (a.acc_out) a.acc_out[o] = v;
     }
   }

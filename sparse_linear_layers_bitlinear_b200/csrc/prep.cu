@@ -430,14 +430,16 @@ __device__ __noinline__ float gamma_exact(const unsigned long long* slow_bins, u
   return exact_mean_fp32(bins, numel);
 }
 
+// The whole preparation of one matrix by CTA `blk` of the `G` CTAs that
+// work on it (a launch of one matrix, or one matrix's share of a grouped
+// launch).
 template <int M>
-__global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
+__device__ __forceinline__ void prepare_body(const PrepArgs& a, const int G, const int blk) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint4* ring = reinterpret_cast<uint4*>(smem);
   uint2* sel = reinterpret_cast<uint2*>(smem + size_t(kPrepStages) * kChunkVecs * 16);  // [64][32 lanes]
   PrepTail* tail = reinterpret_cast<PrepTail*>(smem + size_t(kPrepStages) * kChunkVecs * 16 + kSelBytes);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = static_cast<int>(gridDim.x), blk = static_cast<int>(blockIdx.x);
   uint32_t* status = &a.h->status;
   volatile int* abort_flag = &tail->abort_flag;
   // The successor only reads its own inputs before it waits for this kernel.
@@ -899,6 +901,28 @@ __global__ void __maxnreg__(72) k_prepare(const PrepArgs a) {
   }
 }
 
+template <int M>
+__global__ void __maxnreg__(72) k_prepare(const __grid_constant__ PrepArgs a) {
+  prepare_body<M>(a, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x));
+}
+
+// Several matrices of one launch: matrix i runs on CTAs
+// [cta_begin[i], cta_begin[i + 1]), with its own tagged barrier (in its own
+// blob) and its own exact scale.
+struct PrepGroup {
+  PrepArgs mats[kPrepMaxGroup];
+  int cta_begin[kPrepMaxGroup + 1];
+  int count;
+};
+
+template <int M>
+__global__ void __maxnreg__(72) k_prepare_group(const __grid_constant__ PrepGroup grp) {
+  const int b = static_cast<int>(blockIdx.x);
+  int i = 0;
+  while (i + 1 < grp.count && b >= grp.cta_begin[i + 1]) ++i;
+  prepare_body<M>(grp.mats[i], grp.cta_begin[i + 1] - grp.cta_begin[i], b - grp.cta_begin[i]);
+}
+
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
@@ -910,16 +934,25 @@ static cudaError_t launch_prepare_m(const cudaLaunchConfig_t& cfg, const PrepArg
   return counted(cudaLaunchKernelEx(&cfg, k_prepare<M>, a));
 }
 
+template <int M>
+static cudaError_t launch_prepare_group_m(const cudaLaunchConfig_t& cfg, const PrepGroup& grp) {
+  static const cudaError_t attr_err = cudaFuncSetAttribute(k_prepare_group<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                           static_cast<int>(kPrepSmem));
+  if (attr_err != cudaSuccess) return attr_err;
+  return counted(cudaLaunchKernelEx(&cfg, k_prepare_group<M>, grp));
+}
+
 static_assert(3 + kExactBins + 3 == SBL_SUM_WORDS, "sum words: fast pieces, bins, counts");
 
-cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
-                           uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s, int mode,
-                           uint64_t* sum_out, const uint64_t* sum_in, uint64_t numel) {
+// The arguments of one matrix's preparation, after the stream operations
+// that must precede it (padding of the metadata and decode-pack sections).
+static cudaError_t prep_args(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
+                             uint8_t* blob, const sbl_blob_layout& L, cudaStream_t s, int mode, uint64_t* sum_out,
+                             const uint64_t* sum_in, uint64_t numel, PrepArgs& a) {
   if (mode != kPrepSumOnly && L.sp_meta && (n_out % 256 != 0 || k % 256 != 0)) {
     cudaError_t e = cudaMemsetAsync(blob + L.sp_meta, 0x44, L.sp_meta_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  PrepArgs a;
   a.w = reinterpret_cast<const uint4*>(w);
   a.n_out = n_out;
   a.k = k;
@@ -952,29 +985,79 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
     cudaError_t e = cudaMemsetAsync(blob + L.gemv, 0, L.gemv_bytes, s);
     if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
+}
 
-  // One CTA per SM (fewer for small matrices: at least one 16 KB stage of
-  // weights per CTA), all resident at once for the grid barrier.
-  const int64_t nvec = n_out * k / 8;
-  int64_t grid = (nvec + kChunkVecs - 1) / kChunkVecs;
-  if (grid > num_sms) grid = num_sms;
-  if (grid > kPrepSlots) grid = kPrepSlots;
-  if (grid < 1) grid = 1;
-
+static cudaLaunchConfig_t prep_config(int64_t grid, cudaStream_t s, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kPrepThreads);
   cfg.dynamicSmemBytes = kPrepSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cfg;
+}
+
+// CTAs that a matrix of nvec 16-byte vectors can use: at least one stage of
+// weights each.
+static int64_t prep_max_ctas(int64_t nvec) {
+  const int64_t c = (nvec + kChunkVecs - 1) / kChunkVecs;
+  return c < 1 ? 1 : c > kPrepSlots ? kPrepSlots : c;
+}
+
+cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, int m, uint32_t flags,
+                           uint8_t* blob, const sbl_blob_layout& L, int num_sms, cudaStream_t s, int mode,
+                           uint64_t* sum_out, const uint64_t* sum_in, uint64_t numel) {
+  PrepArgs a;
+  cudaError_t e = prep_args(w, n_out, k, n, m, flags, blob, L, s, mode, sum_out, sum_in, numel, a);
+  if (e != cudaSuccess) return e;
+  // One CTA per SM (fewer for small matrices), all resident at once for the
+  // grid barrier.
+  int64_t grid = prep_max_ctas(n_out * k / 8);
+  if (grid > num_sms) grid = num_sms;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = prep_config(grid, s, attr);
   switch (m) {
     case 2: return launch_prepare_m<2>(cfg, a);
     case 4: return launch_prepare_m<4>(cfg, a);
     default: return launch_prepare_m<8>(cfg, a);
+  }
+}
+
+cudaError_t launch_prepare_group(const PrepMatrix* mats, int count, int num_sms, cudaStream_t s) {
+  if (count < 1 || count > kPrepMaxGroup || count > num_sms) return cudaErrorInvalidValue;
+  PrepGroup grp;
+  grp.count = count;
+  int64_t nvec[kPrepMaxGroup], total = 0;
+  for (int i = 0; i < count; ++i) {
+    const PrepMatrix& q = mats[i];
+    if (q.m != mats[0].m) return cudaErrorInvalidValue;
+    cudaError_t e = prep_args(q.w, q.n_out, q.k, q.n, q.m, q.flags, q.blob, *q.layout, s, 0, nullptr, nullptr,
+                              uint64_t(q.n_out) * uint64_t(q.k), grp.mats[i]);
+    if (e != cudaSuccess) return e;
+    nvec[i] = q.n_out * q.k / 8;
+    total += nvec[i];
+  }
+  // The SMs split in proportion to the matrices' sizes, at least one CTA each.
+  int ctas[kPrepMaxGroup], used = 0;
+  for (int i = 0; i < count; ++i) {
+    int64_t c = (nvec[i] * (num_sms - count)) / total + 1;
+    const int64_t cap = prep_max_ctas(nvec[i]);
+    ctas[i] = static_cast<int>(c < cap ? c : cap);
+    used += ctas[i];
+  }
+  grp.cta_begin[0] = 0;
+  for (int i = 0; i < count; ++i) grp.cta_begin[i + 1] = grp.cta_begin[i] + ctas[i];
+  for (int i = count + 1; i <= kPrepMaxGroup; ++i) grp.cta_begin[i] = grp.cta_begin[count];
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = prep_config(used, s, attr);
+  switch (mats[0].m) {
+    case 2: return launch_prepare_group_m<2>(cfg, grp);
+    case 4: return launch_prepare_group_m<4>(cfg, grp);
+    default: return launch_prepare_group_m<8>(cfg, grp);
   }
 }
 

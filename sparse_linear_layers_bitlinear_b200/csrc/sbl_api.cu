@@ -155,6 +155,30 @@ sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
+sbl_status sbl_prepare_weights_grouped(const sbl_layer* layers, const void* const* w_masters, int32_t count,
+                                       sbl_stream_t stream) {
+  if (layers == nullptr || w_masters == nullptr || count < 1 || count > kPrepMaxGroup) return SBL_ERR_INVALID_ARG;
+  sbl_blob_layout L[kPrepMaxGroup];
+  PrepMatrix mats[kPrepMaxGroup];
+  for (int i = 0; i < count; ++i) {
+    const sbl_status st = check_layer(&layers[i], &L[i]);
+    if (st != SBL_OK) return st;
+    if (layers[i].m != layers[0].m) return SBL_ERR_UNSUPPORTED_NM;
+    if (w_masters[i] == nullptr) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(w_masters[i])) return SBL_ERR_ALIGN;
+    for (int j = 0; j < i; ++j)
+      if (layers[j].prepared == layers[i].prepared) return SBL_ERR_INVALID_ARG;  // one blob, two matrices
+    mats[i] = PrepMatrix{static_cast<const uint16_t*>(w_masters[i]), layers[i].n_out, layers[i].k, layers[i].n,
+                         layers[i].m, layers[i].flags, static_cast<uint8_t*>(layers[i].prepared), &L[i]};
+  }
+  int sms = 0;
+  const sbl_status st = current_device(&sms);
+  if (st != SBL_OK) return st;
+  if (count > sms) return SBL_ERR_INVALID_ARG;
+  return launch_prepare_group(mats, count, sms, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SBL_OK
+                                                                                                       : SBL_ERR_CUDA;
+}
+
 sbl_status sbl_weight_abs_sum(const sbl_layer* layer, const void* w_master, uint64_t* sum_out, sbl_stream_t stream) {
   sbl_blob_layout L;
   sbl_status st = check_layer(layer, &L);

@@ -57,6 +57,19 @@ cudaError_t launch_prepare(const uint16_t* w, int64_t n_out, int64_t k, int n, i
                            const sbl_blob_layout& L, int num_sms, cudaStream_t s, int mode = 0,
                            uint64_t* sum_out = nullptr, const uint64_t* sum_in = nullptr, uint64_t numel = 0);
 
+// One matrix of a grouped preparation (launch_prepare_group): every matrix
+// of a group has the same m.
+constexpr int kPrepMaxGroup = 8;
+struct PrepMatrix {
+  const uint16_t* w;
+  int64_t n_out, k;
+  int n, m;
+  uint32_t flags;
+  uint8_t* blob;
+  const sbl_blob_layout* layout;
+};
+cudaError_t launch_prepare_group(const PrepMatrix* mats, int count, int num_sms, cudaStream_t s);
+
 // early_trigger: wait for the predecessor, then let the next kernel launch at
 // once (it must wait for this one before reading xq / a_prime).
 cudaError_t launch_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq, float* a_prime, uint32_t* status,
@@ -76,7 +89,7 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
 
 // Decode forward for 1 <= t <= 32 tokens over the decode pack (2:4: one byte
 // per group of four; other N:M: the interleaved compressed-index pack, see
-// gemv.cu).  For t up to 8 the kernel quantises the activations itself
+// gemv.cu).  For t up to 4 the kernel quantises the activations itself
 // (xq_out / ap_out, when given, receive the codes and scales); otherwise, or
 // when x is NULL, xq_in / ap_in hold the codes (the act-quant kernel runs
 // first with its early trigger).  gemv_fits() says whether the token rows fit

@@ -77,6 +77,7 @@ SIGNATURES = {
     "sbl_prepared_bytes": (ctypes.c_size_t, [_I64, _I64, _I32, _I32, _U32]),
     "sbl_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
     "sbl_prepare_weights": (_I32, [_LP, _P, _P]),
+    "sbl_prepare_weights_grouped": (_I32, [_LP, ctypes.POINTER(_P), _I32, _P]),
     "sbl_forward": (_I32, [_LP, _P, _I64, _P, _P, _P, _P, _P, _P]),
     "sbl_backward": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P]),
     "sbl_backward_ws": (_I32, [_LP, _P, _P, _I64, _P, _P, _U32, _P, _P]),
@@ -179,6 +180,14 @@ class Layer:
 def prepare_weights(layer: Layer, w_master, stream=None):
     cl = layer.c()
     _check(lib().sbl_prepare_weights(ctypes.byref(cl), _ptr(w_master), _stream(stream)), "sbl_prepare_weights")
+
+
+def prepare_weights_grouped(layers, w_masters, stream=None):
+    """sbl_prepare_weights_grouped: several layers (same m) prepared in one launch."""
+    count = len(layers)
+    arr = (sbl_layer * count)(*[L.c() for L in layers])
+    ws = (_P * count)(*[_ptr(w) for w in w_masters])
+    _check(lib().sbl_prepare_weights_grouped(arr, ws, count, _stream(stream)), "sbl_prepare_weights_grouped")
 
 
 SBL_SUM_WORDS = 46

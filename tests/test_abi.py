@@ -181,3 +181,25 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.sbl_forward_quantized(ctypes.byref(layer), None, None, -1, None, None, None) == sbl.SBL_ERR_SHAPE
     # rejected calls enqueue nothing, so they launch nothing
     assert sbl.launch_count() == launched_before
+
+
+def test_grouped_prepare_validates_before_touching_the_device(lib):
+    launched = sbl.launch_count()
+    p = ctypes.c_void_p
+    L = lambda n, m, blob: sbl.sbl_layer(256, 256, n, m, 0, blob)  # noqa: E731
+
+    def call(layers, masters, count=None):
+        arr = (sbl.sbl_layer * len(layers))(*layers)
+        ws = (ctypes.c_void_p * len(masters))(*masters)
+        return lib.sbl_prepare_weights_grouped(arr, ws, len(layers) if count is None else count, None)
+
+    two = [L(2, 4, 0x1000), L(1, 4, 0x2000)]
+    assert call(two, [0x10000, 0x20000], count=0) == sbl.SBL_ERR_INVALID_ARG
+    assert call(two, [0x10000, 0x20000], count=9) == sbl.SBL_ERR_INVALID_ARG
+    assert lib.sbl_prepare_weights_grouped(None, None, 1, None) == sbl.SBL_ERR_INVALID_ARG
+    assert call([L(2, 4, 0x1000), L(6, 8, 0x2000)], [0x10000, 0x20000]) == sbl.SBL_ERR_UNSUPPORTED_NM
+    assert call([L(2, 4, 0x1000), L(1, 4, 0x1000)], [0x10000, 0x20000]) == sbl.SBL_ERR_INVALID_ARG  # one blob
+    assert call(two, [0x10000, None]) == sbl.SBL_ERR_INVALID_ARG
+    assert call(two, [0x10000, 0x20008]) == sbl.SBL_ERR_ALIGN
+    assert call([L(2, 4, 0x1000), L(1, 4, 0x2010)], [0x10000, 0x20000]) == sbl.SBL_ERR_ALIGN  # blob alignment
+    assert sbl.launch_count() == launched

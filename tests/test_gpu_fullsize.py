@@ -70,8 +70,19 @@ def test_fullsize_parity(name, n_out, k, n, m, t):
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
     assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
 
-    rng = np.random.default_rng(7)
+    # Every accumulator and output: the oracle's codes times its W_eff in
+    # float64 (a library matmul; the integer sums stay below 2^24, so fp64
+    # holds them exactly), so every output tile of the GEMM's schedule is
+    # checked, ragged last tiles included.
+    acc_full = (xq_ref.astype(np.float64) @ ref["weff"].astype(np.float64).T)
+    assert np.abs(acc_full).max() < 2 ** 31
+    acc_full = acc_full.astype(np.int32)
     acc_h, y_h = acc.cpu().numpy(), y.cpu().numpy()
+    assert np.array_equal(acc_h, acc_full)
+    y_full = oracle.dequant(acc_full, ap_ref, ref["g"])
+    assert np.array_equal(y_h.view(np.uint32), y_full.view(np.uint32))
+
+    rng = np.random.default_rng(7)
     ti, oi = _samples(rng, t, n_out, 1500)
     accs = np.array([oracle.acc_at(xq_ref, ref["weff"], a, b) for a, b in zip(ti, oi)], dtype=np.int32)
     assert np.array_equal(acc_h[ti, oi], accs)
@@ -89,6 +100,43 @@ def test_fullsize_parity(name, n_out, k, n, m, t):
     dwr = np.array([oracle.grad_w_at(dy, x, a, b) for a, b in zip(oi, ki)])
     err = np.abs(dw_h[oi, ki] - dwr)
     assert (err <= 1e-2 + 2.0 ** -7 * np.abs(dwr)).all(), err.max()
+
+
+@pytest.mark.parametrize("name,n_out,k,n,m,t", WORKLOADS)
+@pytest.mark.parametrize("f32", [False, True])
+def test_fullsize_gradients_whole_arrays(name, n_out, k, n, m, t, f32):
+    """dX and dW of both prefill workloads, every element, in bf16 and in
+    fp32 mode (SBL_GRAD_F32), against float64 products of the oracle's W_eff
+    and scale (the oracle's gradient definitions, by a library matmul), plus
+    sampled elements from the oracle itself."""
+    w_d = synth.master_weights(n_out, k, 0, device="cuda")
+    x_d = synth.activations(t, k, 1, device="cuda")
+    dy_d = synth.upstream_grad(t, n_out, 2, device="cuda")
+    layer = sbl.Layer.allocate(n_out, k, n, m)
+    sbl.prepare_weights(layer, w_d)
+    dt = torch.float32 if f32 else torch.bfloat16
+    dx = torch.empty((t, k), dtype=dt, device="cuda")
+    dw = torch.empty((n_out, k), dtype=dt, device="cuda")
+    sbl.backward(layer, x_d, dy_d, t, dx, dw, sbl.SBL_GRAD_F32 if f32 else 0)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    ref = oracle.prepare(w_d.cpu(), n, m)
+    dy64 = dy_d.cpu().double().numpy()
+    x64 = x_d.cpu().double().numpy()
+    dx_ref = (dy64 @ ref["weff"].astype(np.float64)) * np.float64(ref["g"])
+    dw_ref = dy64.T @ x64
+    rel = 1e-3 if f32 else 2.0 ** -7
+    for got, want in ((dx, dx_ref), (dw, dw_ref)):
+        g64 = got.double().cpu().numpy()
+        err = np.abs(g64 - want)
+        assert (err <= 1e-2 + rel * np.abs(want)).all(), err.max()
+    rng = np.random.default_rng(17)
+    ti, ki = _samples(rng, t, k, 200)
+    dxr = np.array([oracle.grad_x_at(dy_d.cpu(), ref["weff"], ref["g"], a, b) for a, b in zip(ti, ki)])
+    assert np.allclose(dx_ref[ti, ki], dxr, rtol=1e-12, atol=1e-12)
+    oi, ki = _samples(rng, n_out, k, 200)
+    dwr = np.array([oracle.grad_w_at(dy_d.cpu(), x_d.cpu(), a, b) for a, b in zip(oi, ki)])
+    assert np.allclose(dw_ref[oi, ki], dwr, rtol=1e-12, atol=1e-12)
 
 
 @pytest.mark.parametrize("t", [1, 4, 16, 32])
@@ -115,7 +163,8 @@ def test_decode_gemv_fullsize(t, n_out, n, m):
 
 
 @pytest.mark.parametrize("n,m", [(2, 4), (4, 8)])
-def test_fullsize_training_layer(n, m):
+@pytest.mark.parametrize("layer_index", [0, 29])
+def test_fullsize_training_layer(n, m, layer_index):
     """One layer of the training-step workload at 8192 tokens: q, k, v, o
     (2560 x 2560), gate, up (2560 -> 6912), down (6912 -> 2560), with q/k/v and
     gate/up sharing their activations through sbl_forward_quantized as the
@@ -126,7 +175,7 @@ def test_fullsize_training_layer(n, m):
     rng = np.random.default_rng(11)
     acts = {}
     for j, (name, n_out, k) in enumerate(shapes):
-        seed = 500 + 10 * j
+        seed = 1000 * layer_index + 10 * j  # the benchmark's seeds for this layer
         w_d = synth.master_weights(n_out, k, seed, device="cuda")
         dy_d = synth.upstream_grad(T, n_out, seed + 2, device="cuda")
         layer = sbl.Layer.allocate(n_out, k, n, m)
@@ -167,3 +216,26 @@ def test_fullsize_training_layer(n, m):
         oi, ki = _samples(rng, n_out, k, 100)
         dwr = np.array([oracle.grad_w_at(dy, x, a, b) for a, b in zip(oi, ki)])
         assert (np.abs(dw_h[oi, ki] - dwr) <= 1e-2 + 2.0 ** -7 * np.abs(dwr)).all(), name
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (4, 8)])
+def test_training_step_prepares_all_210_matrices(n, m):
+    """Every matrix of the 30-layer training step, drawn with the benchmark's
+    seeds (layer l, projection j: seed 1000 l + 10 j): gamma, mask and W_eff
+    of all 210 prepares, whole arrays."""
+    H, F = 2560, 6912
+    shapes = [(H, H), (H, H), (H, H), (H, H), (F, H), (F, H), (H, F)]
+    layers = {(o, k): sbl.Layer.allocate(o, k, n, m) for (o, k) in set(shapes)}
+    for l in range(30):
+        for j, (n_out, k) in enumerate(shapes):
+            w_d = synth.master_weights(n_out, k, 1000 * l + 10 * j, device="cuda")
+            layer = layers[(n_out, k)]
+            sbl.prepare_weights(layer, w_d)
+            torch.cuda.synchronize()
+            assert sbl.read_status(layer)[0] == sbl.SBL_OK
+            ref = oracle.prepare(w_d.cpu(), n, m)
+            gamma, _, _ = bd.header_scalars(layer)
+            where = f"layer {l} projection {j}"
+            assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32), where
+            assert np.array_equal(bd.mask(layer), ref["mask"]), where
+            assert np.array_equal(bd.weff_from_bf16(layer), ref["weff"]), where

@@ -671,7 +671,7 @@ def test_act_quant_more_rows_than_resident_warps():
 @pytest.mark.parametrize("t", [4, 8, 16, 33])
 def test_decode_dispatch_both_paths_bit_exact(t):
     """A layer with the decode pack at the decode sizes: up to 32 tokens take
-    the decode kernel (quantising for itself up to 8), more the 2:4
+    the decode kernel (quantising for itself up to 4), more the 2:4
     tensor-core GEMM; both give the oracle's bits."""
     n_out, k = 6912, 2560
     w = synth.master_weights(n_out, k, 81)
@@ -691,7 +691,7 @@ def test_decode_dispatch_both_paths_bit_exact(t):
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
     assert np.array_equal(xq.cpu().numpy(), ref["xq"])
-    assert launched == (1 if t <= 8 else 2)  # the decode kernel alone, or act-quant first
+    assert launched == (1 if t <= 4 else 2)  # the decode kernel alone, or act-quant first
     assert sbl.read_status(layer)[0] == sbl.SBL_OK
 
 
@@ -926,6 +926,50 @@ def test_row_sharded_midpoint_decided_by_a_tiny_magnitude_in_another_shard():
     assert float(oracle.absmean_gamma(w)) == 1.0 + 2.0 ** -23
     for layer in _row_sharded_prepare(w, 2, 4, 2):
         assert sbl.read_scale(layer) == (1.0 + 2.0 ** -23, 1.0 + 2.0 ** -23)
+
+
+GROUPS = [
+    # (n_out, k, n, flags) per matrix; every group shares m
+    (4, [(264, 320, 2, sbl.SBL_PACK_GEMV), (520, 192, 1, 0), (64, 64, 3, sbl.SBL_MASK_FROM_QUANT),
+         (2560, 2560, 2, 0), (8, 64, 2, 0)]),
+    (8, [(136, 448, 6, sbl.SBL_PACK_GEMV), (392, 832, 3, 0), (384, 512, 8, 0), (128, 384, 4, sbl.SBL_PACK_GEMV)]),
+    (4, [(2560, 2560, 2, 0)] * 4 + [(6912, 2560, 2, 0)] * 2 + [(2560, 6912, 2, 0)]),  # a transformer block's linears
+]
+
+
+@pytest.mark.parametrize("m,mats", GROUPS)
+def test_grouped_prepare_matches_one_call_per_layer(m, mats):
+    """sbl_prepare_weights_grouped: every matrix's sections equal those of its
+    own sbl_prepare_weights call and the oracle's, bit for bit."""
+    layers, solo, ws = [], [], []
+    for i, (n_out, k, n, flags) in enumerate(mats):
+        w = synth.master_weights(n_out, k, 300 + i)
+        if i == 1:
+            w[3, 5] = 96.0  # one matrix with a magnitude outside the fast window
+        ws.append(_dev(w))
+        layers.append(sbl.Layer.allocate(n_out, k, n, m, flags))
+        solo.append(sbl.Layer.allocate(n_out, k, n, m, flags))
+        sbl.prepare_weights(solo[-1], ws[-1])
+    sbl.prepare_weights_grouped(layers, ws)
+    torch.cuda.synchronize()
+    for i, (n_out, k, n, flags) in enumerate(mats):
+        L = layers[i].layout()
+        assert sbl.read_status(layers[i])[0] == sbl.SBL_OK
+        assert sbl.read_scale(layers[i]) == sbl.read_scale(solo[i])
+        # every section the prepare writes, padding included (the gaps between
+        # sections are never written)
+        spans = [(L.mask, n_out * k // m), (L.weff_bf16, 2 * n_out * k), (L.sp_values, n_out * k // 2),
+                 (L.sp_meta, L.sp_meta_bytes), (L.codes, n_out * k), (L.gemv, L.gemv_bytes)]
+        for off, size in spans:
+            if off:
+                assert torch.equal(layers[i].blob[off:off + size], solo[i].blob[off:off + size]), (i, off)
+        from_codes = bool(flags & sbl.SBL_MASK_FROM_QUANT)
+        if n_out * k <= 400 * 1024 and not from_codes:
+            _check_prepared(layers[i], ws[i].cpu(), n, m)
+        else:
+            ref = oracle.prepare(ws[i].cpu(), n, m, mask_from_codes=from_codes)
+            assert np.array_equal(bd.mask(layers[i]), ref["mask"])
+            assert np.array_equal(bd.weff_from_bf16(layers[i]), ref["weff"])
 
 
 def test_row_sharded_helper_orders_the_exchange_on_a_side_stream(monkeypatch):

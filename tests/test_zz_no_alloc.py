@@ -104,7 +104,7 @@ def _compare_with_forward(layer, t, seed):
 @pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
 def test_noalloc_through_the_decode_kernel_over_stale_scratch(n, m):
     """A layer with the decode pack: a large call first fills the scratch,
-    then decode-sized calls (the kernel quantises t <= 8 itself and writes the
+    then decode-sized calls (the kernel quantises t <= 4 itself and writes the
     codes into the scratch; t = 16 runs the act-quant kernel into it first)."""
     n_out, k = 392, 1024
     layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
