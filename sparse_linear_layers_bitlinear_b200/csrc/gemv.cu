@@ -57,11 +57,12 @@ namespace sbl {
 
 constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
-// A table of 256 entries kept in kLutCopies copies, entry e of copy c at word
-// e * kLutCopies + c; lane l reads copy l % kLutCopies, so at most
-// 32 / kLutCopies lanes share a copy's banks.
-constexpr int kLutCopies = 32;
-constexpr int kLutWords = 256 * kLutCopies;
+// A table of 256 entries kept in C copies, entry e of copy c at word
+// e * C + c; lane l reads copy l % C, so at most 32 / C lanes share a copy's
+// banks.  16 copies measured best: 32 doubled the table fill before the wait
+// (which competes with the call before) for no gain in the products.
+constexpr int kLutCopiesReg = 16;
+constexpr int lut_words(int copies) { return 256 * copies; }
 constexpr int kDecBatch = 8;         // units whose weight bytes a lane holds at once
 constexpr size_t kDecMaxSmem = 227 * 1024;
 constexpr int kDecMaxT = 32;
@@ -136,8 +137,9 @@ __device__ __forceinline__ uint32_t lut_entry(int kind, uint32_t b) {
   return sel;
 }
 
+template <int C>
 __device__ __forceinline__ void fill_lut(uint32_t* lut, int kind, int tid) {
-  constexpr int kVecs = kLutCopies / 4;  // 16-byte stores per entry
+  constexpr int kVecs = C / 4;  // 16-byte stores per entry
   for (int i = tid; i < 256 * kVecs; i += kDecThreads) {
     const uint32_t v = lut_entry(kind, static_cast<uint32_t>(i / kVecs));
     reinterpret_cast<uint4*>(lut)[i] = make_uint4(v, v, v, v);
@@ -208,10 +210,11 @@ __device__ __forceinline__ uint32_t code_field(const uint32_t* w, int off, int b
 }
 
 // Table entry (byte `pos` of w) in this lane's copy: the byte, shifted
-// straight into a byte offset (entries are 4 * kLutCopies bytes apart).
+// straight into a byte offset (entries are 4 * C bytes apart).
+template <int C>
 __device__ __forceinline__ uint32_t lut_get(const uint8_t* lane_base, uint32_t w, int pos) {
-  constexpr int kShift = 2 + (kLutCopies == 16 ? 4 : kLutCopies == 32 ? 5 : 3);
-  static_assert(kLutCopies == 8 || kLutCopies == 16 || kLutCopies == 32, "table copies");
+  constexpr int kShift = 2 + (C == 16 ? 4 : C == 32 ? 5 : 3);
+  static_assert(C == 8 || C == 16 || C == 32, "table copies");
   const int sh = 8 * pos - kShift;
   const uint32_t off = (sh >= 0 ? (w >> sh) : (w << -sh)) & (0xFFu << kShift);
   return *reinterpret_cast<const uint32_t*>(lane_base + off);
@@ -219,7 +222,7 @@ __device__ __forceinline__ uint32_t lut_get(const uint8_t* lane_base, uint32_t w
 
 // The four A-fragment registers of k-step s: rows g (a0 low k slots, a2 high)
 // and g + 8 (a1, a3).  la / ls: this lane's copies of the tables.
-template <int FMT>
+template <int FMT, int C>
 __device__ __forceinline__ void decode_step(const uint32_t (&r)[Pack<FMT>::regs], int s, const uint8_t* la,
                                             const uint8_t* ls, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) {
   using P = Pack<FMT>;
@@ -227,20 +230,20 @@ __device__ __forceinline__ void decode_step(const uint32_t (&r)[Pack<FMT>::regs]
     // bytes 2s, 2s + 1 of each row's 8: word s / 2, bytes 2 (s % 2) and + 1
     const int b = 2 * (s & 1);
     const uint32_t w0 = r[s >> 1], w1 = r[2 + (s >> 1)];
-    a0 = lut_get(la, w0, b);
-    a2 = lut_get(la, w0, b + 1);
-    a1 = lut_get(la, w1, b);
-    a3 = lut_get(la, w1, b + 1);
+    a0 = lut_get<C>(la, w0, b);
+    a2 = lut_get<C>(la, w0, b + 1);
+    a1 = lut_get<C>(la, w1, b);
+    a3 = lut_get<C>(la, w1, b + 1);
   } else {
     constexpr int o = P::has_mask ? 2 : 0;
     uint32_t lo[2], hi[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const uint32_t c = code_field<P::cw>(r + o, h * 8 * P::n8 + s * 2 * P::n8, 2 * P::n8);
-      const uint32_t A = lut_get(la, c, 0);
-      const uint32_t B = P::n8 > 4 ? lut_get(la, c, 1) : 0u;
+      const uint32_t A = lut_get<C>(la, c, 0);
+      const uint32_t B = P::n8 > 4 ? lut_get<C>(la, c, 1) : 0u;
       if constexpr (P::has_mask) {
-        const uint32_t sel = lut_get(ls, r[h], s);
+        const uint32_t sel = lut_get<C>(ls, r[h], s);
         lo[h] = __byte_perm(A, B, sel & 0xFFFFu);
         hi[h] = __byte_perm(A, B, sel >> 16);
       } else {
@@ -260,71 +263,32 @@ __device__ __forceinline__ void decode_step(const uint32_t (&r)[Pack<FMT>::regs]
 // quarter warp (rows g, g + 1; four t) read eight distinct bank groups.
 __device__ __forceinline__ int xs_off(int n, int j, int xs) { return n * xs + ((j & ~7) | ((j & 7) ^ (n & 7))) * 16; }
 
-template <int FMT, int NT, bool FUSED>
-__global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
-  using P = Pack<FMT>;
-  constexpr int TP = 8 * NT;  // token columns
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* lut_a = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* lut_s = lut_a + kLutWords;  // mask selectors (packs with a mask block)
-  uint8_t* xsm = smem + (P::has_mask ? 2 : 1) * kLutWords * 4;
-  int32_t* s_acc = reinterpret_cast<int32_t*>(xsm + TP * a.xs);  // [tpb][16][TP]
-  float* s_scale = reinterpret_cast<float*>(s_acc + a.tpb * 16 * TP);  // [32]
-  float* s_red = s_scale + kDecMaxT;                                    // [warps]
-  float* s_ap = s_red + kDecWarps;                                      // [8] a' (quantised here)
+// Shared-memory scalars of both kernels.
+struct DecScalars {
+  float scale[kDecMaxT];  // (g a') / 127 per token
+  float red[kDecWarps];   // per-warp partial maxima of |x|
+  float ap[8];            // a' of the rows quantised here
+};
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile0 = blockIdx.x * a.tpb;
-  const int ntile = min(a.tpb, a.tiles - tile0);
-  const int units = ntile * a.upr;
-
-  // ---- before the wait: prefetch, tables, zeroed sums and padding ----
-  if (tid == 0) bulk_prefetch_l2(a.w + int64_t(tile0) * a.upr * P::unit_bytes, static_cast<uint32_t>(units) * P::unit_bytes);
-  if (tid == 32) {
-    if (FUSED) bulk_prefetch_l2(a.x, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k) * 2u);
-    else bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
-  }
-  pdl_trigger();
-  fill_lut(lut_a, P::k24 ? 0 : 1, tid);
-  if constexpr (P::has_mask) fill_lut(lut_s, 2, tid);
-  for (int i = tid; i < ntile * 16 * TP; i += kDecThreads) s_acc[i] = 0;
-  // Activation rows past t and columns past k are left as they are: a token
-  // column past t only feeds output columns that are never stored, and the
-  // weights past k are zero (guarded loads, zero-filled pack).
-  pdl_wait();
-
+// The activation codes of the t token rows into shared memory, by all warps.
+// With FUSED the t <= 4 rows are quantised here: wpr warps per row, the row's
+// absmax through the warps' maxima in shared memory; otherwise the codes of
+// the act-quant kernel (or the caller) arrive by asynchronous 16-byte copies.
+// `issued` runs once the activation loads are out (the weight loads go out
+// there).  g_early: g in threads 0..t-1 (the output scale is
+// formed after the products, off the critical path).
+template <bool FUSED, class Issued>
+__device__ __forceinline__ void stage_activations(const DecodeArgs& a, uint8_t* xsm, DecScalars* sc, float& g_early,
+                                                  int tid, int warp, int lane, Issued issued) {
+  constexpr int XW = kDecWarps;
   const int nch = a.k / 16;  // 16-code chunks per token row
-  const int u_begin = (units * warp) / kDecWarps, u_end = (units * (warp + 1)) / kDecWarps;
-  // (tile, unit) of this warp's first unit; later ones follow by counting
-  const int tl_begin = u_begin / a.upr, un_begin = u_begin - tl_begin * a.upr;
-  uint32_t wr[kDecBatch][P::regs];
-  auto load_batch = [&](int ub, int tl, int un) {
-#pragma unroll
-    for (int i = 0; i < kDecBatch; ++i) {
-      if (ub + i < u_end) load_unit<FMT>(a, tile0 + tl, un, lane, wr[i]);
-      if (++un == a.upr) {
-        un = 0;
-        ++tl;
-      }
-    }
-  };
-
-  // ---- activation codes into shared memory ----
-  float g_early = 0.0f;
-  // The activation loads go out first (the rest of the block's path waits
-  // on them), then this warp's first batch of weight loads, which are needed
-  // only by the products.
   if constexpr (FUSED) {
-    // Quantise the t <= 4 rows here: wpr warps per row, the row's absmax
-    // through the warps' maxima in shared memory.
     const int tp2 = a.t <= 1 ? 1 : a.t <= 2 ? 2 : 4;
-    const int wpr = kDecWarps / tp2;
+    const int wpr = XW / tp2;
     const int xrow = warp / wpr, xsub = warp % wpr;
     const bool live = xrow < a.t;
     const uint4* xsrc = a.x + int64_t(xrow) * (a.k / 8);
     const bool scale_thread = live && xsub == 0 && lane == 0;
-    // the output scale (g a') / 127 is formed after the products by threads
-    // 0..t-1; their g load goes out now, off the critical path
     g_early = tid < a.t ? __ldg(a.g) : 0.0f;
     constexpr int kXc = 3;  // chunks kept in registers between the two passes
     uint4 xr[kXc][2];
@@ -338,7 +302,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         xr[q][0] = xr[q][1] = make_uint4(0, 0, 0, 0);
       }
     }
-    load_batch(u_begin, tl_begin, un_begin);
+    issued();
     float amax = 0.0f;
     uint32_t bad = 0;
 #pragma unroll
@@ -356,16 +320,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       bad |= __shfl_xor_sync(0xffffffffu, bad, off);
     }
-    if (lane == 0) s_red[warp] = bad ? -1.0f : amax;  // amax >= 0: -1 flags a non-finite row
+    if (lane == 0) sc->red[warp] = bad ? -1.0f : amax;  // amax >= 0: -1 flags a non-finite row
     __syncthreads();
     if (live) {
-      // the row's wpr partial maxima, read as two vectors
-      const float4 r0 = reinterpret_cast<const float4*>(s_red)[0], r1 = reinterpret_cast<const float4*>(s_red)[1];
+      // the row's wpr partial maxima, read as vectors
+      const float4 r0 = reinterpret_cast<const float4*>(sc->red)[0];
+      const float4 r1 = reinterpret_cast<const float4*>(sc->red)[1];
       const float part[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
       float m = 0.0f;
       bool row_bad = false;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
+      for (int w = 0; w < XW; ++w) {
         if (w / wpr == xrow) {
           row_bad |= part[w] < 0.0f;
           m = fmaxf(m, part[w]);
@@ -389,7 +354,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
         if (gdst) gdst[j] = c;
       }
       if (scale_thread) {
-        s_ap[xrow] = ap;  // the output scale is formed after the products
+        sc->ap[xrow] = ap;  // the output scale is formed after the products
         if (blockIdx.x == 0) {
           if (a.ap_out) a.ap_out[xrow] = ap;
           if (row_bad) raise_status(a.status, SBL_STATUS_NONFINITE_X);
@@ -397,25 +362,128 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    // codes and scales from the act-quant kernel (or the caller): copied into
-    // shared memory by asynchronous 16-byte copies, which hold no registers
     const float g = tid < a.t ? __ldg(a.g) : 0.0f;
-    for (int i = tid; i < a.t * nch; i += kDecThreads) {
+    for (int i = tid; i < a.t * nch; i += XW * 32) {
       const int n = i / nch, j = i - n * nch;
       cp_async16(xsm + xs_off(n, j, a.xs), reinterpret_cast<const uint4*>(a.xq_in + int64_t(n) * a.k) + j);
     }
     cp_async_commit();
     const float apv = tid < a.t ? __ldcg(a.ap_in + tid) : 0.0f;
-    load_batch(u_begin, tl_begin, un_begin);
-    if (tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(g, apv), 127.0f);
+    issued();
+    if (tid < a.t) sc->scale[tid] = __fdiv_rn(__fmul_rn(g, apv), 127.0f);
     cp_async_wait_all();
   }
+}
+
+// MMA accumulators of one warp: kSets independent sets per token tile (k-step
+// s adds into set s % kSets), so consecutive MMAs do not wait on each other;
+// flush() adds the sets into the tile's sums in shared memory.
+template <int NT>
+struct DecAcc {
+  static constexpr int kSets = NT == 1 ? 4 : NT == 2 ? 2 : 1;
+  int v[kSets][NT][4];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int q = 0; q < kSets; ++q)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) v[q][nt][0] = v[q][nt][1] = v[q][nt][2] = v[q][nt][3] = 0;
+  }
+  __device__ __forceinline__ void flush(int32_t* tile_sums, int gq, int tq) {
+    constexpr int TP = 8 * NT;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      int r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        r[i] = v[0][nt][i];
+#pragma unroll
+        for (int q = 1; q < kSets; ++q) r[i] += v[q][nt][i];
+      }
+      const int col = nt * 8 + 2 * tq;
+      atomicAdd(tile_sums + gq * TP + col, r[0]);
+      atomicAdd(tile_sums + gq * TP + col + 1, r[1]);
+      atomicAdd(tile_sums + (gq + 8) * TP + col, r[2]);
+      atomicAdd(tile_sums + (gq + 8) * TP + col + 1, r[3]);
+    }
+  }
+};
+
+// The block's outputs from its tiles' sums: y = acc * ((g a') / 127) (and the
+// raw sums), consecutive rows per token.
+template <int NT>
+__device__ __forceinline__ void write_outputs(const DecodeArgs& a, const int32_t* s_acc, const DecScalars* sc,
+                                              int tile0, int ntile, int tid) {
+  constexpr int TP = 8 * NT;
+  const int rows = min(ntile * 16, a.n_out - tile0 * 16);
+  for (int idx = tid; idx < ntile * 16 * a.t; idx += kDecThreads) {
+    const int tok = idx / (ntile * 16), r = idx - tok * (ntile * 16);
+    if (r < rows) {
+      const int v = s_acc[(r >> 4) * 16 * TP + (r & 15) * TP + tok];
+      const int64_t o = int64_t(tok) * a.n_out + tile0 * 16 + r;
+      a.y[o] = __fmul_rn(static_cast<float>(v), sc->scale[tok]);
+      if (a.acc_out) a.acc_out[o] = v;
+    }
+  }
+}
+
+// Every warp stages activations, then expands its own units' weights into MMA
+// fragments on the fly (table lookups between the MMAs).
+template <int FMT, int NT, bool FUSED>
+__global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
+  using P = Pack<FMT>;
+  constexpr int C = kLutCopiesReg;
+  constexpr int TP = 8 * NT;  // token columns
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t* lut_a = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* lut_s = lut_a + lut_words(C);  // mask selectors (packs with a mask block)
+  uint8_t* xsm = smem + (P::has_mask ? 2 : 1) * lut_words(C) * 4;
+  int32_t* s_acc = reinterpret_cast<int32_t*>(xsm + a.t * a.xs);  // [tpb][16][TP]
+  DecScalars* sc = reinterpret_cast<DecScalars*>(s_acc + a.tpb * 16 * TP);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile0 = blockIdx.x * a.tpb;
+  const int ntile = min(a.tpb, a.tiles - tile0);
+  const int units = ntile * a.upr;
+
+  // ---- before the wait: prefetch, tables, zeroed sums ----
+  if (tid == 0) bulk_prefetch_l2(a.w + int64_t(tile0) * a.upr * P::unit_bytes, static_cast<uint32_t>(units) * P::unit_bytes);
+  if (tid == 32) {
+    if (FUSED) bulk_prefetch_l2(a.x, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k) * 2u);
+    else bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
+  }
+  pdl_trigger();
+  fill_lut<C>(lut_a, P::k24 ? 0 : 1, tid);
+  if constexpr (P::has_mask) fill_lut<C>(lut_s, 2, tid);
+  for (int i = tid; i < ntile * 16 * TP; i += kDecThreads) s_acc[i] = 0;
+  // Activation columns past k are left as they are: the weights there are
+  // zero (zero-filled pack).  Token rows past t are neither stored nor read.
+  pdl_wait();
+
+  const int u_begin = (units * warp) / kDecWarps, u_end = (units * (warp + 1)) / kDecWarps;
+  // (tile, unit) of this warp's first unit; later ones follow by counting
+  const int tl_begin = u_begin / a.upr, un_begin = u_begin - tl_begin * a.upr;
+  uint32_t wr[kDecBatch][P::regs];
+  auto load_batch = [&](int ub, int tl, int un) {
+#pragma unroll
+    for (int i = 0; i < kDecBatch; ++i) {
+      if (ub + i < u_end) load_unit<FMT>(a, tile0 + tl, un, lane, wr[i]);
+      if (++un == a.upr) {
+        un = 0;
+        ++tl;
+      }
+    }
+  };
+  float g_early = 0.0f;
+  // the activation loads go out first (the rest of the block's path waits on
+  // them), then this warp's first batch of weight loads
+  stage_activations<FUSED>(a, xsm, sc, g_early, tid, warp, lane,
+                                      [&]() { load_batch(u_begin, tl_begin, un_begin); });
   __syncthreads();
 
   // ---- products ----
   const int gq = lane >> 2, tq = lane & 3;
-  const uint8_t* la = reinterpret_cast<const uint8_t*>(lut_a + (lane % kLutCopies));
-  const uint8_t* ls = reinterpret_cast<const uint8_t*>(lut_s + (lane % kLutCopies));
+  const uint8_t* la = reinterpret_cast<const uint8_t*>(lut_a + (lane % C));
+  const uint8_t* ls = reinterpret_cast<const uint8_t*>(lut_s + (lane % C));
   // this lane's activation chunks in unit 0 (token row gq + 8 nt, chunk
   // 2 tq + p); unit un is 128 un bytes further
   const uint8_t* bsrc[NT][2];
@@ -423,35 +491,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int p = 0; p < 2; ++p) bsrc[nt][p] = xsm + xs_off(gq + 8 * nt, 2 * tq + p, a.xs);
-  // kSets independent MMA accumulators per token tile (k-step s adds into set
-  // s % kSets) keep consecutive MMAs from waiting on each other's results.
-  constexpr int kSets = NT == 1 ? 4 : NT == 2 ? 2 : 1;
-  int acc[kSets][NT][4];
-  int cur = -1;  // tile (local) the accumulators belong to
-  auto zero_acc = [&]() {
-#pragma unroll
-    for (int q = 0; q < kSets; ++q)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) acc[q][nt][0] = acc[q][nt][1] = acc[q][nt][2] = acc[q][nt][3] = 0;
-  };
-  auto flush = [&](int t_local) {
-    int32_t* base = s_acc + t_local * 16 * TP;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      int v[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        v[r] = acc[0][nt][r];
-#pragma unroll
-        for (int q = 1; q < kSets; ++q) v[r] += acc[q][nt][r];
-      }
-      const int col = nt * 8 + 2 * tq;
-      atomicAdd(base + gq * TP + col, v[0]);
-      atomicAdd(base + gq * TP + col + 1, v[1]);
-      atomicAdd(base + (gq + 8) * TP + col, v[2]);
-      atomicAdd(base + (gq + 8) * TP + col + 1, v[3]);
-    }
-  };
+  DecAcc<NT> acc;
+  int cur = -1;                      // tile (local) the accumulators belong to
   int tl = tl_begin, un = un_begin;  // (tile, unit) of unit ub + i
   for (int ub = u_begin; ub < u_end; ub += kDecBatch) {
     if (ub != u_begin) load_batch(ub, tl, un);
@@ -459,9 +500,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     for (int i = 0; i < kDecBatch; ++i) {
       if (ub + i >= u_end) break;
       if (tl != cur) {
-        if (cur >= 0) flush(cur);
+        if (cur >= 0) acc.flush(s_acc + cur * 16 * TP, gq, tq);
         cur = tl;
-        zero_acc();
+        acc.zero();
       }
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
@@ -472,10 +513,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
 #pragma unroll
         for (int sp = 0; sp < 2; ++sp) {
           uint32_t a0, a1, a2, a3;
-          decode_step<FMT>(wr[i], 2 * p + sp, la, ls, a0, a1, a2, a3);
+          decode_step<FMT, C>(wr[i], 2 * p + sp, la, ls, a0, a1, a2, a3);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-            mma_s8_16x8x32(acc[(2 * p + sp) % kSets][nt], a0, a1, a2, a3, sp ? bv[nt].z : bv[nt].x,
+            mma_s8_16x8x32(acc.v[(2 * p + sp) % DecAcc<NT>::kSets][nt], a0, a1, a2, a3, sp ? bv[nt].z : bv[nt].x,
                            sp ? bv[nt].w : bv[nt].y);
         }
       }
@@ -485,21 +526,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
       }
     }
   }
-  if (cur >= 0) flush(cur);
-  if (FUSED && tid < a.t) s_scale[tid] = __fdiv_rn(__fmul_rn(g_early, s_ap[tid]), 127.0f);
+  if (cur >= 0) acc.flush(s_acc + cur * 16 * TP, gq, tq);
+  if (FUSED && tid < a.t) sc->scale[tid] = __fdiv_rn(__fmul_rn(g_early, sc->ap[tid]), 127.0f);
   __syncthreads();
-
-  // ---- epilogue: y = acc * ((g a') / 127), consecutive rows per token ----
-  const int rows = min(ntile * 16, a.n_out - tile0 * 16);
-  for (int idx = tid; idx < ntile * 16 * a.t; idx += kDecThreads) {
-    const int tok = idx / (ntile * 16), r = idx - tok * (ntile * 16);
-    if (r < rows) {
-      const int v = s_acc[(r >> 4) * 16 * TP + (r & 15) * TP + tok];
-      const int64_t o = int64_t(tok) * a.n_out + tile0 * 16 + r;
-      a.y[o] = __fmul_rn(static_cast<float>(v), s_scale[tok]);
-      if (a.acc_out) a.acc_out[o] = v;
-    }
-  }
+  write_outputs<NT>(a, s_acc, sc, tile0, ntile, tid);
 }
 
 namespace {
@@ -508,11 +538,12 @@ int decode_nt(int64_t t) { return t <= 8 ? 1 : t <= 16 ? 2 : 4; }
 
 int decode_fmt(int n, int m) { return (n == 2 && m == 4) ? 0 : 8 * n / m; }
 
-size_t decode_smem(int fmt, int nt, int64_t k, int tpb) {
-  const bool sel = fmt >= 1 && fmt < 8;
+bool fmt_has_mask(int fmt) { return fmt >= 1 && fmt < 8; }
+
+size_t decode_smem(int fmt, int nt, int64_t t, int64_t k, int tpb) {
   const size_t xs = size_t((k + 127) / 128 * 128);
-  return size_t(sel ? 2 : 1) * kLutWords * 4 + size_t(8 * nt) * xs + size_t(tpb) * 16 * 8 * nt * 4 +
-         (kDecMaxT + kDecWarps + 8) * 4;
+  return size_t(fmt_has_mask(fmt) ? 2 : 1) * lut_words(kLutCopiesReg) * 4 + size_t(t) * xs +
+         size_t(tpb) * 16 * 8 * nt * 4 + sizeof(DecScalars);
 }
 
 template <int FMT, int NT, bool FUSED>
@@ -529,7 +560,8 @@ cudaError_t decode_launch(const DecodeArgs& a, int blocks, size_t smem, cudaStre
 
 template <int FMT>
 cudaError_t decode_fmt_launch(const DecodeArgs& a, bool fused, int nt, int blocks, size_t smem, cudaStream_t s) {
-  if (nt == 1) return fused ? decode_launch<FMT, 1, true>(a, blocks, smem, s) : decode_launch<FMT, 1, false>(a, blocks, smem, s);
+  if (nt == 1)
+    return fused ? decode_launch<FMT, 1, true>(a, blocks, smem, s) : decode_launch<FMT, 1, false>(a, blocks, smem, s);
   if (nt == 2) return decode_launch<FMT, 2, false>(a, blocks, smem, s);
   return decode_launch<FMT, 4, false>(a, blocks, smem, s);
 }
@@ -546,10 +578,10 @@ uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m) {
 
 bool gemv_fits(int64_t t, int64_t k, int n, int m) {
   if (t < 1 || t > kDecMaxT) return false;
-  return decode_smem(decode_fmt(n, m), decode_nt(t), k, 1) <= kDecMaxSmem;
+  return decode_smem(decode_fmt(n, m), decode_nt(t), t, k, 1) <= kDecMaxSmem;
 }
 
-// The decode kernel streams the packed weights once for up to 32 tokens; the
+// The decode kernels stream the packed weights once for up to 32 tokens; the
 // tensor-core GEMMs pay a round of 240-token tiles for any token count.
 bool gemv_preferred(int64_t t, int64_t n_out, int64_t k) { return t <= kDecMaxT; }
 
@@ -579,15 +611,15 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_
   const int fmt = decode_fmt(n, m), nt = decode_nt(t);
   // codes from the caller (x == NULL), else quantised here for few tokens
   const bool fused = x != nullptr && gemv_fuses_act_quant(t);
-  // Blocks: as many as fit two per SM; each takes an equal run of tiles.
-  const size_t smem1 = decode_smem(fmt, nt, k, 1);
+  // As many blocks as fit two per SM; each takes an equal run of tiles.
+  const size_t smem1 = decode_smem(fmt, nt, t, k, 1);
   const int per_sm = smem1 * 2 + 2048 <= 228 * 1024 ? 2 : 1;
   int tpb = (a.tiles + num_sms * per_sm - 1) / (num_sms * per_sm);
-  while (decode_smem(fmt, nt, k, tpb) > kDecMaxSmem && tpb > 1) --tpb;
-  if (decode_smem(fmt, nt, k, tpb) > kDecMaxSmem) return cudaErrorInvalidValue;
+  while (decode_smem(fmt, nt, t, k, tpb) > kDecMaxSmem && tpb > 1) --tpb;
+  const size_t smem = decode_smem(fmt, nt, t, k, tpb);
+  if (smem > kDecMaxSmem) return cudaErrorInvalidValue;
   a.tpb = tpb;
   const int blocks = (a.tiles + tpb - 1) / tpb;
-  const size_t smem = decode_smem(fmt, nt, k, tpb);
   switch (fmt) {
     case 0: return decode_fmt_launch<0>(a, fused, nt, blocks, smem, s);
     case 1: return decode_fmt_launch<1>(a, fused, nt, blocks, smem, s);

@@ -760,9 +760,10 @@ def test_decode_long_rows(n, m, k, t):
 
 
 def test_decode_declines_rows_beyond_its_shared_memory():
-    """16 token rows of k = 16384 do not fit: the call takes the tensor-core
-    GEMM and still gives the oracle's bits."""
-    n_out, k, t = 256, 16384, 9
+    """17 token rows of k = 16384 (278 KB of codes) do not fit the decode
+    kernel's shared memory: the call takes the tensor-core GEMM and still
+    gives the oracle's bits."""
+    n_out, k, t = 256, 16384, 17
     w = synth.master_weights(n_out, k, 960)
     x = synth.activations(t, k, 961)
     layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
