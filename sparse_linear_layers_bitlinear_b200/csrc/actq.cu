@@ -75,8 +75,7 @@ __global__ void __launch_bounds__(kActThreads, 4)
       bulk_prefetch_l2(x + row * nvec, static_cast<uint32_t>(nvec * 16));
   pdl_wait();
   if (early_trigger) pdl_trigger();
-  __shared__ float s_max[kActThreads / 32];
-  __shared__ uint32_t s_bad[kActThreads / 32];
+  __shared__ uint32_t s_max[kActThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int64_t row = blockIdx.x; row < t; row += gridDim.x) {
     const uint4* src = x + row * nvec;
@@ -86,32 +85,27 @@ __global__ void __launch_bounds__(kActThreads, 4)
       const int64_t i = int64_t(r) * kActThreads + tid;
       v[r] = (i < nvec) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
     }
-    float amax = 0.0f;
-    uint32_t bad = 0;
+    // the absmax as an integer max over the magnitude bits, two halves at a
+    // time (as in the warp-per-row kernel)
+    uint32_t m2 = 0;
 #pragma unroll
-    for (int r = 0; r < R; ++r) scan8(v[r], amax, bad);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      bad |= __shfl_xor_sync(0xffffffffu, bad, off);
+    for (int r = 0; r < R; ++r) {
+      m2 = __vmaxu2(m2, v[r].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[r].w & 0x7FFF7FFFu);
     }
-    if (lane == 0) {
-      s_max[warp] = amax;
-      s_bad[warp] = bad;
-    }
+    const uint32_t mw = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    if (lane == 0) s_max[warp] = mw;
     __syncthreads();
-    amax = s_max[0];
-    bad = s_bad[0];
+    uint32_t m = s_max[0];
 #pragma unroll
-    for (int w = 1; w < kActThreads / 32; ++w) {
-      amax = fmaxf(amax, s_max[w]);
-      bad |= s_bad[w];
-    }
+    for (int w = 1; w < kActThreads / 32; ++w) m = max(m, s_max[w]);
     __syncthreads();  // s_max is rewritten by the next row
-    const float ap = fmaxf(amax, 1e-5f);
+    const float ap = fmaxf(__uint_as_float(m << 16), 1e-5f);
     if (tid == 0) {
       if (!DEQ) a_prime[row] = ap;
-      if (bad) raise_status(status, SBL_STATUS_NONFINITE_X);
+      if (m >= 0x7F80u) raise_status(status, SBL_STATUS_NONFINITE_X);
     }
     const QScale qs = make_qscale(ap);
     if (qs.exact) {  // the clamp or a' >= 2^120: the IEEE division

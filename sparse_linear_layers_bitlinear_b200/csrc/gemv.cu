@@ -266,7 +266,7 @@ __device__ __forceinline__ int xs_off(int n, int j, int xs) { return n * xs + ((
 // Shared-memory scalars of both kernels.
 struct DecScalars {
   float scale[kDecMaxT];  // (g a') / 127 per token
-  float red[kDecWarps];   // per-warp partial maxima of |x|
+  uint32_t red[kDecWarps];  // per-warp partial maxima of the bf16 magnitude bits of x
   float ap[8];            // a' of the rows quantised here
 };
 
@@ -303,40 +303,39 @@ __device__ __forceinline__ void stage_activations(const DecodeArgs& a, uint8_t* 
       }
     }
     issued();
-    float amax = 0.0f;
-    uint32_t bad = 0;
+    // the absmax as an integer max over the magnitude bits (their order is
+    // the order of the values; a non-finite value shows as bits >= 0x7F80),
+    // two halves at a time
+    auto vmax16 = [](uint32_t m2, const uint4& v0, const uint4& v1) {
+      m2 = __vmaxu2(m2, v0.x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v0.y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v0.z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v0.w & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v1.x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v1.y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v1.z & 0x7FFF7FFFu);
+      return __vmaxu2(m2, v1.w & 0x7FFF7FFFu);
+    };
+    uint32_t m2 = 0;
 #pragma unroll
-    for (int q = 0; q < kXc; ++q) {
-      scan8(xr[q][0], amax, bad);
-      scan8(xr[q][1], amax, bad);
-    }
+    for (int q = 0; q < kXc; ++q) m2 = vmax16(m2, xr[q][0], xr[q][1]);
     if (live)
-      for (int j = (xsub + kXc * wpr) * 32 + lane; j < nch; j += wpr * 32) {
-        scan8(__ldg(xsrc + 2 * j), amax, bad);
-        scan8(__ldg(xsrc + 2 * j + 1), amax, bad);
-      }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      bad |= __shfl_xor_sync(0xffffffffu, bad, off);
-    }
-    if (lane == 0) sc->red[warp] = bad ? -1.0f : amax;  // amax >= 0: -1 flags a non-finite row
+      for (int j = (xsub + kXc * wpr) * 32 + lane; j < nch; j += wpr * 32)
+        m2 = vmax16(m2, __ldg(xsrc + 2 * j), __ldg(xsrc + 2 * j + 1));
+    const uint32_t mw = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    if (lane == 0) sc->red[warp] = mw;
     __syncthreads();
     if (live) {
       // the row's wpr partial maxima, read as vectors
-      const float4 r0 = reinterpret_cast<const float4*>(sc->red)[0];
-      const float4 r1 = reinterpret_cast<const float4*>(sc->red)[1];
-      const float part[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-      float m = 0.0f;
-      bool row_bad = false;
+      const uint4 r0 = reinterpret_cast<const uint4*>(sc->red)[0];
+      const uint4 r1 = reinterpret_cast<const uint4*>(sc->red)[1];
+      const uint32_t part[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      uint32_t m = 0;
 #pragma unroll
-      for (int w = 0; w < XW; ++w) {
-        if (w / wpr == xrow) {
-          row_bad |= part[w] < 0.0f;
-          m = fmaxf(m, part[w]);
-        }
-      }
-      const float ap = fmaxf(m, 1e-5f);
+      for (int w = 0; w < XW; ++w)
+        if (w / wpr == xrow) m = max(m, part[w]);
+      const bool row_bad = m >= 0x7F80u;
+      const float ap = fmaxf(__uint_as_float(m << 16), 1e-5f);
       const QScale qs = make_qscale(ap);
       uint4* gdst = (blockIdx.x == 0 && a.xq_out) ? reinterpret_cast<uint4*>(a.xq_out + int64_t(xrow) * a.k) : nullptr;
 #pragma unroll
