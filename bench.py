@@ -204,6 +204,18 @@ def replica_seed(rank: int, rotation: int, tensor: int) -> int:
     return 1000 * rank + 10 * rotation + tensor
 
 
+def exchange_dw(dw, world: int) -> None:
+    """The one exchange of data-parallel training: every rank's dW summed over
+    the ranks (in place; NCCL over NVLink on the GPU, gloo on the host).  The
+    masters are the same on every rank, so the summed gradient updates them
+    alike; the optimizer step that would scale and apply it is not part of
+    the operator."""
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(dw, op=dist.ReduceOp.SUM)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample, extrapolated linearly in tokens)
 # ---------------------------------------------------------------------------
@@ -285,7 +297,8 @@ def cpu_baseline(T, K, N, n, m, target_s=12.0, target_1t_s=10.0):
 def workload_config(world: int) -> dict:
     """The `config` object of both arms' JSON lines."""
     return {"workload": WORKLOAD["name"], "tokens": WORKLOAD["tokens"], "k": WORKLOAD["k"], "n_out": WORKLOAD["n_out"],
-            "n": WORKLOAD["n"], "m": WORKLOAD["m"], "parallelism": f"replicas x{world}",
+            "n": WORKLOAD["n"], "m": WORKLOAD["m"],
+            "parallelism": f"data parallel x{world}" + (" (dW all-reduce each step)" if world > 1 else ""),
             "l2": f"inputs rotate over {ROTATE} seeded sets (3 x 112 MB > 126 MB L2)"}
 
 
@@ -813,10 +826,11 @@ def main():
     A = algorithmic(T, K, N)
     peaks = load_peaks()
 
-    # Inputs: ROTATE seeded sets, different per rank (independent batches).
+    # Inputs: ROTATE seeded sets; the masters are the same on every rank (data
+    # parallel), the activations and upstream gradients are each rank's own batch.
     sets = []
     for r in range(ROTATE):
-        sets.append((synth.master_weights(N, K, replica_seed(rank, r, 0), device=dev),
+        sets.append((synth.master_weights(N, K, replica_seed(0, r, 0), device=dev),
                      synth.activations(T, K, replica_seed(rank, r, 1), device=dev),
                      synth.upstream_grad(T, N, replica_seed(rank, r, 2), device=dev)))
     layer = sbl.Layer.allocate(N, K, n, m, device=dev)
@@ -841,6 +855,7 @@ def main():
         sbl.backward(layer, x, dy, T, dx, dw, 0)  # dX and dW in one launch
         if bwd is not None:
             bwd[1].record(stream)
+        exchange_dw(dw, world)  # the data-parallel gradient exchange (none on one GPU)
         if ev is not None:
             ev[3].record(stream)
 
@@ -943,6 +958,8 @@ def main():
         sbl.prepare_weights(layer, w_d, stream=s_comp)
         sbl.forward(layer, x_d, T, y_d, workspace=ws, stream=s_comp)
         sbl.backward(layer, x_d, dy_d, T, dx_d, dw_d, 0, stream=s_comp)
+        with torch.cuda.stream(s_comp):
+            exchange_dw(dw_d, world)  # ordered after the backward on the compute stream
         ev_comp[b].record(s_comp)
         s_out.wait_event(ev_comp[b])
         with torch.cuda.stream(s_out):

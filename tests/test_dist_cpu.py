@@ -1,7 +1,8 @@
 """Multi-rank plumbing of bench.py on CPU: two gloo ranks on 127.0.0.1.
 
-bench.py runs one independent replica per GPU (no collective on the data
-path): each rank draws its own inputs, the ranks meet at a barrier around the
+bench.py runs data parallel, one rank per GPU: the masters are the same on
+every rank, each rank draws its own batch, every step ends with the sum of dW
+over the ranks (the gradient exchange), the ranks meet at a barrier around the
 timed region, and the reported time is the slowest rank's.  These tests run
 that host logic with world size 2 and no GPU.
 """
@@ -33,7 +34,10 @@ def _worker(rank, world, port, out):
         seeds = [bench.replica_seed(rank, r, j) for r in range(bench.ROTATE) for j in range(3)]
         gathered = [None] * world
         dist.all_gather_object(gathered, seeds)
-        out[rank] = (mx, gathered)
+        # the gradient exchange: each rank's dW summed in place
+        dw = torch.full((4, 8), float(rank + 1))
+        bench.exchange_dw(dw, world)
+        out[rank] = (mx, gathered, dw.tolist())
         bench.barrier(world)
     finally:
         dist.destroy_process_group()
@@ -49,6 +53,7 @@ def test_two_gloo_ranks_agree_on_the_slowest_time_and_draw_distinct_inputs():
     assert res[0][0] == res[1][0] == 2.5
     seeds0, seeds1 = res[0][1]
     assert len(set(seeds0)) == len(seeds0) and not set(seeds0) & set(seeds1)
+    assert res[0][2] == res[1][2] == [[3.0] * 8] * 4  # 1 + 2 on both ranks
 
 
 def test_single_rank_needs_no_process_group():

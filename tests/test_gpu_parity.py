@@ -741,6 +741,56 @@ def test_decode_compressed_index_patterns(n, m, t):
     _decode_check(136, 448, n, m, t, seed=700 + 16 * n + m + t)
 
 
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (1, 4), (8, 8)])
+@pytest.mark.parametrize("t", [1, 5, 32])
+def test_decode_smallest_layer(n, m, t):
+    """The smallest layer the library takes (8 rows, k = 64): half a row tile
+    and half a k unit, every other lane's weights padding."""
+    _decode_check(8, 64, n, m, t, seed=760 + 8 * n + m + t)
+
+
+@pytest.mark.parametrize("t,k", [(1, 2560), (3, 2560), (9, 2560), (2, 6912)])
+def test_decode_nonfinite_activations_raise_status(t, k):
+    """A non-finite activation in a decode call, quantised in the decode
+    kernel (t <= 4) or by the act-quant kernel first, sets the status bit;
+    clearing it restores SBL_OK on the next clean call."""
+    n_out = 64
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 64)))
+    assert sbl.forward_uses_gemv(layer, t)
+    x = synth.activations(t, k, 65)
+    x[t - 1, k // 3] = float("nan") if t % 2 else float("inf")
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, workspace=ws)
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_ERR_NONFINITE and bits & sbl.SBL_STATUS_NONFINITE_X
+    sbl.clear_status(layer)
+    sbl.forward(layer, _dev(synth.activations(t, k, 66)), t, y, workspace=ws)
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+
+
+def test_act_quant_long_rows_flag_nonfinite():
+    """Rows of 6912 (one block per row, the integer absmax): an Inf, a NaN and
+    a finite row; the codes of the finite rows match the oracle and the status
+    word records the non-finite input."""
+    n_out, k, t = 64, 6912, 4
+    layer = sbl.Layer.allocate(n_out, k, 6, 8)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 67)))
+    x = synth.activations(t, k, 68)
+    x[1, 100] = float("inf")
+    x[2, 6911] = float("nan")
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, xq, ap)
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_ERR_NONFINITE and bits & sbl.SBL_STATUS_NONFINITE_X
+    xq_ref, ap_ref = oracle.act_quant(x[[0, 3]])
+    assert np.array_equal(xq.cpu().numpy()[[0, 3]], xq_ref)
+    assert np.array_equal(ap.cpu().numpy()[[0, 3]].view(np.uint32), ap_ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (8, 8)])
 @pytest.mark.parametrize("t", [4, 20])
 def test_decode_blocks_of_several_tiles(n, m, t):
