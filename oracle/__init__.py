@@ -12,7 +12,7 @@ operator it computes:
 
   A1 absmean scale            absmean_gamma / clamped_scale
   A2 N:M magnitude mask       nm_mask
-  A3 ternarise, mask, pack    ternary, apply_mask, pack24, pack_nm
+  A3 ternarise, mask, pack    ternary, apply_mask, pack24, pack_nm, pack24_code6
   A4 per-token int8 absmax    act_quant
   A5 int32 product            gemm_acc, acc_at
   A6 dequant rescale          dequant
@@ -69,6 +69,7 @@ def _load():
         "sbo_apply_mask": (None, [P, P, I64, I64, I, P]),
         "sbo_pack24": (None, [P, P, I64, I64, P, P]),
         "sbo_pack_nm": (None, [P, P, I64, I64, I, I, P, P]),
+        "sbo_pack24_code6": (None, [P, P, I64, I64, P]),
         "sbo_act_quant": (None, [P, I64, I64, P, P]),
         "sbo_gemm_acc": (I, [P, P, I64, I64, I64, P]),
         "sbo_acc_at": (ctypes.c_int32, [P, P, I64]),
@@ -187,6 +188,20 @@ def pack_nm(weff: np.ndarray, mask: np.ndarray, n: int, m: int):
     codes = np.empty((n_out, k * n // (4 * m)), dtype=np.uint8)
     _load().sbo_pack_nm(_ptr(weff), _ptr(mask), n_out, k, n, m, _ptr(masks8), _ptr(codes))
     return masks8, codes
+
+
+def pack24_code6(weff: np.ndarray, mask: np.ndarray):
+    """The 6-bit 2:4 group code (54 states, 1.5 bits a weight): uint8
+    [n_out, 3k/16], one least-significant-bit-first stream of 6-bit states per
+    row, state = 9 p + 3 d(c_i0) + d(c_i1) (p: rank of the kept pair, d: code
+    mod 3)."""
+    weff = np.ascontiguousarray(weff, dtype=np.int8)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    n_out, k = weff.shape
+    assert k % 16 == 0
+    out = np.empty((n_out, k * 6 // 32), dtype=np.uint8)
+    _load().sbo_pack24_code6(_ptr(weff), _ptr(mask), n_out, k, _ptr(out))
+    return out
 
 
 def act_quant(x):

@@ -293,6 +293,40 @@ void sbo_pack_nm(const int8_t* weff, const uint8_t* mask, int64_t n_out,
   }
 }
 
+// The denser 2:4 decode code: a group of four has C(4,2) = 6 choices of its
+// two kept positions and 3 x 3 ternary values for them, 54 states, so 6 bits
+// hold it (1.5 bits a weight).  READING of the numbering, which the pages do
+// not give: the position pairs in lexicographic order (0,1) (0,2) (0,3)
+// (1,2) (1,3) (2,3) are p = 0..5, a code c in {-1, 0, +1} is the digit
+// c mod 3 (0, 1, 2 for 0, +1, -1), and the state is 9 p + 3 d(c_i0) + d(c_i1),
+// so the all-zero group under positions (0,1) is state 0.  States go least
+// significant bit first into one bit stream per row, 6 bits each.
+void sbo_pack24_code6(const int8_t* weff, const uint8_t* mask, int64_t n_out,
+                      int64_t k, uint8_t* out) {
+  const int64_t groups = k / 4, row_bytes = k * 6 / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t row = 0; row < n_out; ++row) {
+    uint8_t* dst = out + row * row_bytes;
+    for (int64_t b = 0; b < row_bytes; ++b) dst[b] = 0;
+    for (int64_t g = 0; g < groups; ++g) {
+      const uint8_t bits = mask[row * groups + g];
+      int idx[2], found = 0;
+      for (int j = 0; j < 4 && found < 2; ++j)
+        if ((bits >> j) & 1u) idx[found++] = j;
+      int pair = 0, rank = 0;  // rank of (idx[0], idx[1]) among the six pairs
+      for (int a = 0; a < 4; ++a)
+        for (int b = a + 1; b < 4; ++b, ++rank)
+          if (a == idx[0] && b == idx[1]) pair = rank;
+      const int c0 = weff[row * k + 4 * g + idx[0]], c1 = weff[row * k + 4 * g + idx[1]];
+      const uint32_t state = uint32_t(9 * pair + 3 * ((c0 + 3) % 3) + (c1 + 3) % 3);
+      for (int bit = 0; bit < 6; ++bit) {
+        const int64_t pos = g * 6 + bit;
+        if ((state >> bit) & 1u) dst[pos / 8] = static_cast<uint8_t>(dst[pos / 8] | (1u << (pos % 8)));
+      }
+    }
+  }
+}
+
 // A4.  Per-token absmax int8 quantisation (READING: the pages do not describe
 // activation quantisation; this is the BitNet b1.58 convention).
 void sbo_act_quant(const uint16_t* x, int64_t t, int64_t k, int8_t* xq,

@@ -82,6 +82,16 @@ void sbo_pack24(const int8_t* weff, const uint8_t* mask, int64_t n_out,
 void sbo_pack_nm(const int8_t* weff, const uint8_t* mask, int64_t n_out,
                  int64_t k, int n, int m, uint8_t* masks8, uint8_t* codes);
 
+/* The denser 2:4 decode code (6 bits a group of four, 1.5 bits a weight):
+ * C(4,2) = 6 kept-position pairs x 3^2 ternary values = 54 states.  READING
+ * of the numbering (the pages give none): pairs (0,1) (0,2) (0,3) (1,2)
+ * (1,3) (2,3) are p = 0..5, a code c is the digit c mod 3 (0 -> 0, +1 -> 1,
+ * -1 -> 2), state = 9 p + 3 d(c_i0) + d(c_i1); states packed least
+ * significant bit first, one stream per row: out[row, 3k/16] bytes.
+ * Requires a 2:4 mask (two positions of every group kept). */
+void sbo_pack24_code6(const int8_t* weff, const uint8_t* mask, int64_t n_out,
+                      int64_t k, uint8_t* out);
+
 /* A4 (per-token int8 absmax; not on the pages, READING): a = max_k |x|,
  * a' = max(a, 1e-5f), xq = sign(x) * rne(fl32(127|x|) / a'), clamped to
  * [-128, 127]; a_prime[t] = a'.  All fp32 IEEE operations. */

@@ -381,6 +381,71 @@ def test_pack_nm_round_trip_and_invariants(n, m):
     assert masks8.nbytes + codes.nbytes == 12 * k * (1 + 2 * n / m) / 8
 
 
+def test_pack24_code6_golden_cases():
+    """Hand-worked bytes of the 6-bit 2:4 group code."""
+    for case in _golden("pack24_code6_cases.json")["cases"]:
+        weff = np.array([case["weff"]], dtype=np.int8)
+        mask = np.array([case["group_masks"]], dtype=np.uint8)
+        assert list(oracle.pack24_code6(weff, mask)[0]) == case["bytes"], case["why"]
+
+
+_PAIRS = [(a, b) for a in range(4) for b in range(a + 1, 4)]
+
+
+def _unpack_code6(packed, k):
+    """Decode the 6-bit group code by division: (weff [n_out, k], group masks)."""
+    n_out = packed.shape[0]
+    weff = np.zeros((n_out, k), dtype=np.int8)
+    masks = np.zeros((n_out, k // 4), dtype=np.uint8)
+    value = {0: 0, 1: 1, 2: -1}
+    for r in range(n_out):
+        stream = int.from_bytes(packed[r].tobytes(), "little")
+        for gi in range(k // 4):
+            state = (stream >> (6 * gi)) & 63
+            assert state < 54
+            p, rest = divmod(state, 9)
+            d0, d1 = divmod(rest, 3)
+            i0, i1 = _PAIRS[p]
+            weff[r, 4 * gi + i0], weff[r, 4 * gi + i1] = value[d0], value[d1]
+            masks[r, gi] = (1 << i0) | (1 << i1)
+    return weff, masks
+
+
+def test_pack24_code6_is_a_bijection_onto_54_states():
+    """Every (kept pair, code, code) of a group gets its own state below 54,
+    and the all-zero group under the pair (0, 1) is state 0 (so zero bytes
+    decode to zero weights)."""
+    combos = [(pair, c0, c1) for pair in _PAIRS for c0 in (-1, 0, 1) for c1 in (-1, 0, 1)]
+    k = 4 * 56  # 54 groups, padded to a multiple of 16 with zero groups under (0, 1)
+    weff = np.zeros((1, k), dtype=np.int8)
+    mask = np.full((1, k // 4), 3, dtype=np.uint8)
+    for gi, ((i0, i1), c0, c1) in enumerate(combos):
+        weff[0, 4 * gi + i0], weff[0, 4 * gi + i1] = c0, c1
+        mask[0, gi] = (1 << i0) | (1 << i1)
+    packed = oracle.pack24_code6(weff, mask)
+    stream = int.from_bytes(packed[0].tobytes(), "little")
+    states = [(stream >> (6 * gi)) & 63 for gi in range(k // 4)]
+    assert sorted(states[:54]) == list(range(54))
+    assert states[54:] == [0, 0]
+    assert states[combos.index(((0, 1), 0, 0))] == 0
+    back, masks = _unpack_code6(packed, k)
+    assert np.array_equal(back, weff) and np.array_equal(masks, mask)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_pack24_code6_round_trip(seed):
+    """On prepared 2:4 weights the code decodes back to W_eff and the mask,
+    at 1.5 bits a weight."""
+    k = 256
+    w = synth.master_weights(10, k, seed=70 + seed)
+    p = oracle.prepare(w, 2, 4)
+    packed = oracle.pack24_code6(p["weff"], p["mask"])
+    assert packed.shape == (10, 3 * k // 16)
+    back, masks = _unpack_code6(packed, k)
+    assert np.array_equal(back, p["weff"])
+    assert np.array_equal(masks, p["mask"])
+
+
 # ---------------------------------------------------------------------------
 # A4: activation quantisation
 # ---------------------------------------------------------------------------
