@@ -419,7 +419,45 @@ def bench_decode(dev, hbm_gbs, reps=10):
             "points": out}
 
 
-def bench_prefill68(dev, peaks, steps=20):
+MMA_KINDS = {0: "2:4 int8 forward stage (256 x 240 x 256 logical k, with its metadata copy)",
+             1: "dense int8 forward stage (256 x 256 x 128)",
+             2: "bf16 backward stage (256 x 256 x 64)"}
+
+
+def bench_mma_ceiling(dev, peaks, stages=2048, reps=5):
+    """The rate each GEMM stage's MMA instructions reach with resident
+    operands (sbl_selftest_mma_rate): one launch over every CTA pair, CUDA
+    events around it, median of `reps` after 3 warm-up launches.  Returns per
+    kind the rate in dense-equivalent TOPS beside its nominal peak (4x / 2x /
+    1x the measured bf16 figure for 2:4 int8 / dense int8 / bf16)."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl
+
+    pairs = torch.cuda.get_device_properties(dev).multi_processor_count // 2
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ratio = {0: 4.0, 1: 2.0, 2: 1.0}
+    out = {}
+    for kind, what in MMA_KINDS.items():
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for _ in range(3):
+            macs = sbl.selftest_mma_rate(kind, stages, pairs, status)
+        for a, b in evs:
+            a.record()
+            sbl.selftest_mma_rate(kind, stages, pairs, status)
+            b.record()
+        torch.cuda.synchronize(dev)
+        assert int(status.item()) == 0, ("mma rate self test timed out", kind)
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        tops = 2.0 * macs * stages * pairs / (ms * 1e-3) / 1e12
+        nominal = ratio[kind] * peaks["bf16_tflops"]
+        out[{0: "sparse_i8", 1: "dense_i8", 2: "bf16"}[kind]] = {
+            "what": what, "tops": tops, "nominal_tops": nominal, "frac_of_nominal": tops / nominal,
+            "launch_ms": ms, "pairs": pairs, "stages_per_pair": stages}
+    return out
+
+
+def bench_prefill68(dev, peaks, ceiling=None, steps=20):
     """The 6:8 FFN down projection: T=4096, K=6912, N_out=2560, prepare +
     forward (dense int8 over W_eff codes) + dual-STE backward per step."""
     import torch
@@ -466,15 +504,31 @@ def bench_prefill68(dev, peaks, steps=20):
         torch.cuda.synchronize(dev)
         for j in range(3):
             ph[j] += ev[j].elapsed_time(ev[j + 1]) / 5
+    # the dense int8 GEMM alone, from the codes of set 0 (events around each call)
+    xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    ap = torch.empty((T,), dtype=torch.float32, device=dev)
+    sbl.prepare_weights(layer, sets[0][0])
+    sbl.forward(layer, sets[0][1], T, y, xq, ap)
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a, b in gev:
+        a.record()
+        sbl.forward_quantized(layer, xq, ap, T, y)
+        b.record()
+    torch.cuda.synchronize(dev)
+    gemm_ms = statistics.median(a.elapsed_time(b) for a, b in gev)
     code, bits = sbl.read_status(layer)
     assert code == sbl.SBL_OK, (code, bits)
     dense_ops = 2.0 * T * K * N
     i8_dense = 2.0 * peaks["bf16_tflops"] * 1e12
+    gemm_tops = dense_ops / (gemm_ms * 1e-3) / 1e12
+    ceil = ceiling["dense_i8"]["tops"] if ceiling else None
     return {"workload": "prefill 6:8 Sparse-BitLinear fwd+STE bwd, FFN down projection", "tokens": T, "k": K,
             "n_out": N, "n": 6, "m": 8, "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3),
             "phase_ms": {"prepare": ph[0], "forward": ph[1], "backward": ph[2]},
             "fwd_dense_int8_tops": dense_ops / (ph[1] * 1e-3) / 1e12,
             "fwd_frac_of_dense_int8_peak": dense_ops / (ph[1] * 1e-3) / i8_dense,
+            "gemm_ms": gemm_ms, "gemm_tops": gemm_tops, "gemm_frac_of_dense_int8_peak": gemm_tops * 1e12 / i8_dense,
+            "gemm_frac_of_measured_ceiling": gemm_tops / ceil if ceil else None,
             "bwd_tflops": 2 * dense_ops / (ph[2] * 1e-3) / 1e12}
 
 
@@ -905,6 +959,8 @@ def main():
         e_b.record(stream)
     torch.cuda.synchronize(dev)
     gemm_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in gev), world)
+    # The rates the GEMMs' MMA instructions reach with resident operands.
+    ceiling = bench_mma_ceiling(dev, peaks)
 
     # Timed region: the steps back to back.  Events sit only around the
     # backward launch of every fifth step.
@@ -1034,7 +1090,10 @@ def main():
             / (4.0 * peaks["bf16_tflops"]), "traffic": ncu_traffic("fwd_gemm"), "launch_ms": gemm_ms,
             "kernel": "k_gemm_pair<CfgPairSparse> (2:4 forward GEMM)",
             "timing": "CUDA events around each of 20 sbl_forward_quantized calls, median",
-            "peak_note": f"2:4-sparse int8 = 4 x the {peaks['source']} bf16 burst figure (nominal ratio)"},
+            "peak_note": f"2:4-sparse int8 = 4 x the {peaks['source']} bf16 burst figure (nominal ratio)",
+            "measured_ceiling_tops": ceiling["sparse_i8"]["tops"],
+            "frac_of_measured_ceiling": A["fwd_gemm_ops"] / (gemm_ms * 1e-3) / 1e12 / ceiling["sparse_i8"]["tops"]},
+        "mma_ceiling": ceiling,
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches,
@@ -1055,7 +1114,7 @@ def main():
             if peaks.get("bf16_tflops_sustained") else None,
             "clocks": s_clocks.summary()}
         line["decode_gemv"] = bench_decode(dev, peaks["hbm_gbs"])
-        line["prefill_6of8"] = bench_prefill68(dev, peaks)
+        line["prefill_6of8"] = bench_prefill68(dev, peaks, ceiling)
         line["train_step"] = [bench_train_step(dev, peaks, 2, 4), bench_train_step(dev, peaks, 4, 8)]
         line["nm_sweep"] = bench_nm_sweep(dev, peaks)
         line["ablations"] = bench_ablations(dev)

@@ -318,6 +318,27 @@ sbl_status sbl_selftest_wait_timeout(uint32_t* status_dev, uint64_t limit_ns, sb
  * blocks outside 1..65535, SBL_ERR_DEVICE, SBL_ERR_CUDA. */
 sbl_status sbl_selftest_chain_floor(int32_t blocks, sbl_stream_t stream);
 
+/* Measurement aid, no counterpart in the paper: the tensor-core rate of one
+ * of the library's GEMM stages with its operands resident in shared memory.
+ * `pairs` CTA pairs each issue `stages` stages of the chosen GEMM's
+ * instructions back to back, with no copies, waits or epilogues between them:
+ *   kind 0  the 2:4 sparse int8 forward (tile 256 x 240 tokens, 256 logical
+ *           k a stage, with the stage's metadata copy into tensor memory),
+ *   kind 1  the dense int8 forward of the other N:M patterns (256 x 256,
+ *           128 k a stage),
+ *   kind 2  the bf16 backward (256 x 256, 64 k a stage).
+ * The operands are synthetic (ternary and int8 codes, valid 2:4 metadata,
+ * finite bf16 values) and no result leaves the kernel, so the launch's
+ * duration on `stream` gives the ceiling that the GEMM's MMA instructions
+ * allow.  *macs_per_stage_out (may be NULL) receives the multiply-adds of one
+ * pair's stage (logical k for 2:4).  A tensor pipe that does not drain within
+ * the library's wait limit records SBL_STATUS_TIMEOUT in *status_dev (device
+ * uint32).  Errors: SBL_ERR_INVALID_ARG for a NULL status_dev, kind outside
+ * 0..2, stages outside 1..2^20 or pairs outside 1..SMs/2; SBL_ERR_DEVICE;
+ * SBL_ERR_CUDA. */
+sbl_status sbl_selftest_mma_rate(int32_t kind, int32_t stages, int32_t pairs, uint32_t* status_dev,
+                                 int64_t* macs_per_stage_out, sbl_stream_t stream);
+
 /* Bits of the device status word. */
 enum {
   SBL_STATUS_NONFINITE_W = 1u << 0,

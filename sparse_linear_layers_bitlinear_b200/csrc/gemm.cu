@@ -306,6 +306,129 @@ cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const ui
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-pipe rate with resident operands.  One CTA pair issues a GEMM
+// configuration's per-stage instructions (the MMAs, and for 2:4 the copy of
+// the stage's metadata into tensor memory) back to back over its shared-
+// memory stages, which are filled once: ternary codes for the weights, int8
+// activations, valid 2:4 metadata (kept positions 0 and 1), finite bf16
+// values for the backward.  No copies, waits or epilogues come in between,
+// so the launch time over `pairs` pairs gives the rate those instructions
+// reach on their own: the ceiling of the GEMM that issues them.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t rate_hash(uint32_t x) {
+  x ^= x >> 16;
+  x *= 0x7FEB352Du;
+  x ^= x >> 15;
+  x *= 0x846CA68Bu;
+  x ^= x >> 16;
+  return x;
+}
+
+template <class Cfg, bool INT8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_mma_rate(int stages, uint32_t* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smA = smem;
+  uint8_t* smB = smA + Cfg::STAGES * Cfg::A_BYTES;
+  uint8_t* smE = smB + Cfg::STAGES * Cfg::B_BYTES;
+  PairSmemTail* tail = reinterpret_cast<PairSmemTail*>(smE + Cfg::STAGES * Cfg::E_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool leader = cluster_rank() == 0;
+
+  constexpr int nA = Cfg::STAGES * Cfg::A_BYTES / 4, nB = Cfg::STAGES * Cfg::B_BYTES / 4;
+  constexpr int nE = Cfg::STAGES * Cfg::E_BYTES / 4;
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem);
+  for (int i = threadIdx.x; i < nA + nB + nE; i += blockDim.x) {
+    const uint32_t h = rate_hash(static_cast<uint32_t>(i) * 2654435761u + blockIdx.x);
+    uint32_t v;
+    if (i >= nA + nB) {
+      v = 0x44444444u;  // metadata nibbles i0 = 0, i1 = 1
+    } else if (!INT8) {
+      v = (h & 0x807F807Fu) | 0x3C003C00u;  // two bf16 of magnitude in [2^-7, 2^-6)
+    } else if (i < nA) {
+      // four ternary codes: byte value h_b mod 3 -> 0, +1, -1
+      v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t r = ((h >> (8 * b)) & 0xFFu) % 3u;
+        v |= (r == 0u ? 0u : (r == 1u ? 0x01u : 0xFFu)) << (8 * b);
+      }
+    } else {
+      v = h;  // int8 activation codes
+    }
+    words[i] = v;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&tail->drain, 1);
+    fence_mbar_init();
+  }
+  fence_proxy_async_smem();  // the operands written above are read by the tensor pipe
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) tmem_alloc_pair(&tail->tmem_base, Cfg::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+
+  if (warp == 1 && leader && lane == 0) {
+    typename Cfg::Params p{};
+    for (int i = 0; i < stages; ++i) {
+      const uint32_t s = static_cast<uint32_t>(i % Cfg::STAGES);
+      Cfg::mma_stage(p, 0, tmem_base, tmem_base + Cfg::E_COL0 + (s & 1u) * Cfg::E_COLS, smA + s * Cfg::A_BYTES,
+                     smB + s * Cfg::B_BYTES, smE + s * Cfg::E_BYTES, i == 0);
+    }
+    mma_commit_pair(&tail->drain);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&tail->drain, 0)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        raise_status(status, SBL_STATUS_TIMEOUT);
+        break;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's MMAs no longer read the partner's operands
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+template <class Cfg, bool INT8>
+static cudaError_t mma_rate_launch(int stages, int pairs, uint32_t* status, cudaStream_t s) {
+  constexpr int smem = pair_smem_bytes<Cfg>();
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_mma_rate<Cfg, INT8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  k_mma_rate<Cfg, INT8><<<2 * pairs, 128, smem, s>>>(stages, status);
+  return counted(cudaGetLastError());
+}
+
+int64_t mma_rate_macs_per_stage(int kind) {
+  switch (kind) {
+    case 0: return int64_t(256) * CfgPairSparse<false>::BN * CfgPairSparse<false>::BK;  // logical k
+    case 1: return int64_t(256) * CfgPairDense<false, 256>::BN * CfgPairDense<false, 256>::BK;
+    case 2: return int64_t(256) * CfgPairDualBf16<false>::BN * CfgPairDualBf16<false>::BK;
+    default: return 0;
+  }
+}
+
+cudaError_t launch_mma_rate(int kind, int stages, int pairs, uint32_t* status, cudaStream_t s) {
+  switch (kind) {
+    case 0: return mma_rate_launch<CfgPairSparse<false>, true>(stages, pairs, status, s);
+    case 1: return mma_rate_launch<CfgPairDense<false, 256>, true>(stages, pairs, status, s);
+    case 2: return mma_rate_launch<CfgPairDualBf16<false>, false>(stages, pairs, status, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Bounded-wait self test: waits on an mbarrier that nothing arrives on.
 // ---------------------------------------------------------------------------
 __global__ void k_selftest_wait(uint32_t* status, uint64_t limit_ns) {

@@ -418,4 +418,18 @@ sbl_status sbl_selftest_chain_floor(int32_t blocks, sbl_stream_t stream) {
   return launch_chain_floor(blocks, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
+sbl_status sbl_selftest_mma_rate(int32_t kind, int32_t stages, int32_t pairs, uint32_t* status_dev,
+                                 int64_t* macs_per_stage_out, sbl_stream_t stream) {
+  if (status_dev == nullptr || kind < 0 || kind > 2 || stages < 1 || stages > (1 << 20) || pairs < 1)
+    return SBL_ERR_INVALID_ARG;
+  int sms = 0;
+  const sbl_status st = current_device(&sms);
+  if (st != SBL_OK) return st;
+  if (pairs > sms / 2) return SBL_ERR_INVALID_ARG;
+  if (macs_per_stage_out) *macs_per_stage_out = mma_rate_macs_per_stage(kind);
+  return launch_mma_rate(kind, stages, pairs, status_dev, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SBL_OK
+             : SBL_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -120,6 +120,10 @@ cudaError_t launch_bf16_backward_dual(bool out_f32, const uint16_t* dy, const ui
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_chain_floor(int blocks, cudaStream_t s);
+// Resident-operand tensor-pipe rate of a GEMM stage (kind 0: 2:4 int8
+// forward, 1: dense int8 forward, 2: bf16 backward).
+cudaError_t launch_mma_rate(int kind, int stages, int pairs, uint32_t* status, cudaStream_t s);
+int64_t mma_rate_macs_per_stage(int kind);
 
 // cuTensorMapEncodeTiled, resolved through the runtime's driver entry point.
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,

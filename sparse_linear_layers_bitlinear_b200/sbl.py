@@ -88,6 +88,7 @@ SIGNATURES = {
     "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
     "sbl_selftest_chain_floor": (_I32, [_I32, _P]),
+    "sbl_selftest_mma_rate": (_I32, [_I32, _I32, _I32, _P, ctypes.POINTER(ctypes.c_int64), _P]),
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
     "sbl_forward_uses_gemv": (ctypes.c_int, [_LP, _I64]),
@@ -306,12 +307,22 @@ def selftest_chain_floor(blocks: int, stream=None):
     _check(lib().sbl_selftest_chain_floor(blocks, _stream(stream)), "sbl_selftest_chain_floor")
 
 
+def selftest_mma_rate(kind: int, stages: int, pairs: int, status, stream=None) -> int:
+    """Resident-operand tensor-pipe rate launch of a GEMM stage (kind 0: 2:4
+    int8 forward, 1: dense int8 forward, 2: bf16 backward); returns the
+    multiply-adds of one pair's stage.  `status` is a device uint32 tensor."""
+    macs = ctypes.c_int64(0)
+    _check(lib().sbl_selftest_mma_rate(kind, stages, pairs, _ptr(status), ctypes.byref(macs), _stream(stream)),
+           "sbl_selftest_mma_rate")
+    return int(macs.value)
+
+
 def version() -> str:
     return lib().sbl_version().decode()
 
 
 def forward_uses_gemv(layer: Layer, t: int) -> bool:
-    """Whether sbl_forward takes the 2-bit decode GEMV for t tokens on this layer."""
+    """Whether sbl_forward takes the decode kernel over the packed weights for t tokens on this layer."""
     cl = layer.c()
     return bool(lib().sbl_forward_uses_gemv(ctypes.byref(cl), t))
 

@@ -172,6 +172,10 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 0, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 1 << 7, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_selftest_wait_timeout(None, 1000, None) == sbl.SBL_ERR_INVALID_ARG
+    st = ctypes.c_void_p(0x5000)
+    for kind, stages, pairs, status in ((3, 16, 1, st), (-1, 16, 1, st), (0, 0, 1, st), (0, (1 << 20) + 1, 1, st),
+                                        (0, 16, 0, st), (0, 16, 1, None)):
+        assert lib.sbl_selftest_mma_rate(kind, stages, pairs, status, None, None) == sbl.SBL_ERR_INVALID_ARG
     p = ctypes.c_void_p
     assert lib.sbl_forward_quantized(ctypes.byref(layer), None, p(0x3000), 8, p(0x4000), None, None) == \
         sbl.SBL_ERR_INVALID_ARG

@@ -217,6 +217,18 @@ def test_bounded_wait_reports_timeout():
     assert float(torch.ones(4, device="cuda").sum()) == 4.0
 
 
+@pytest.mark.parametrize("kind,macs", [(0, 256 * 240 * 256), (1, 256 * 256 * 128), (2, 256 * 256 * 64)])
+def test_mma_rate_selftest_runs_and_drains(kind, macs):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    assert sbl.selftest_mma_rate(kind, 64, pairs, status) == macs
+    assert sbl.selftest_mma_rate(kind, 1, 1, status) == macs
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    with pytest.raises(sbl.SblError):
+        sbl.selftest_mma_rate(kind, 64, pairs + 1, status)
+
+
 def test_gamma_scale_readback():
     w = synth.master_weights(128, 256, 5)
     layer = sbl.Layer.allocate(128, 256, 6, 8)
