@@ -342,8 +342,8 @@ def run_reference(args):
 def bench_decode(dev, hbm_gbs, reps=10):
     """Decode-shaped forward: T in {1, 4, 16, 32}, K = 2560, N_out in {2560,
     6912}, on layers prepared with the decode pack: 2:4 (2-bit codes and
-    metadata, 2 bits a weight) and 6:8 (the compressed-index pack, 2.5 bits a
-    weight).  One replay of a CUDA graph makes one call per distinct weight
+    metadata, 2 bits a weight, or the 6-bit group code, 1.5 bits a weight) and
+    6:8 (the compressed-index pack, 2.5 bits a weight).  One replay of a CUDA graph makes one call per distinct weight
     blob, the blobs holding more than 2 x L2 of packed weights, so every call
     streams its weights from HBM; the per-call time is the replay time over
     the calls and includes each call's launch inside the graph.  `floor_us`
@@ -381,13 +381,14 @@ def bench_decode(dev, hbm_gbs, reps=10):
 
     out = []
     floors = {}
-    for (n, m) in ((2, 4), (6, 8)):
+    g6 = sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT
+    for (n, m, flags) in ((2, 4, sbl.SBL_PACK_GEMV), (2, 4, g6), (6, 8, sbl.SBL_PACK_GEMV)):
         for N in (2560, 6912):
-            wbytes = sbl.prepared_layout(N, K, n, m, sbl.SBL_PACK_GEMV).gemv_bytes
+            wbytes = sbl.prepared_layout(N, K, n, m, flags).gemv_bytes
             nblob = max(16, int(2.2 * 126e6 / wbytes) + 1)
             layers = []
             for i in range(nblob):
-                L = sbl.Layer.allocate(N, K, n, m, sbl.SBL_PACK_GEMV, device=dev)
+                L = sbl.Layer.allocate(N, K, n, m, flags, device=dev)
                 sbl.prepare_weights(L, synth.master_weights(N, K, 5000 + i, device=dev))
                 layers.append(L)
             s = torch.cuda.Stream(dev)
@@ -403,7 +404,9 @@ def bench_decode(dev, hbm_gbs, reps=10):
                 wb = wbytes if dec else (N * K * 0.625 if (n, m) == (2, 4) else N * K)
                 by = wb + 2 * T * K + 4 * T * N
                 floor = floors[nblob]
-                out.append({"pattern": f"{n}:{m}", "n_out": N, "k": K, "tokens": T,
+                out.append({"pattern": f"{n}:{m}", "pack": "6-bit group code" if flags & sbl.SBL_PACK_GEMV_6BIT
+                            else ("2-bit codes + metadata" if (n, m) == (2, 4) else "compressed index"),
+                            "n_out": N, "k": K, "tokens": T,
                             "path": "decode kernel" if dec else "tensor-core GEMM",
                             "us_per_call": us, "floor_us": floor, "tokens_per_s": T / (us * 1e-6),
                             "bytes_per_call": by, "gbs": by / (us * 1e-6) / 1e9,
@@ -412,8 +415,9 @@ def bench_decode(dev, hbm_gbs, reps=10):
                             "calls_per_replay": nblob})
             del layers
             torch.cuda.empty_cache()
-    return {"workload": "decode forward on layers with the decode pack (2:4 at 2 bits a weight, 6:8 compressed "
-                        "index at 2.5), K=2560; each call takes the faster path for its size (`path`)",
+    return {"workload": "decode forward on layers with the decode pack (2:4 at 2 bits a weight or its 6-bit group "
+                        "code at 1.5, 6:8 compressed index at 2.5), K=2560; each call takes the faster path for its "
+                        "size (`path`)",
             "timing": "CUDA graph of one call per distinct weight blob (> 2 x L2 of packed weights), per-call "
                       "time incl. launch; floor = the same chain of empty PDL launches",
             "points": out}
@@ -779,16 +783,18 @@ def bench_train_step(dev, peaks, n, m, layers=30, tokens=8192, steps=3):
 # Small fixed cases for a profiler (ncu): a few launches of one kernel family
 # ---------------------------------------------------------------------------
 def profile_decode():
-    """The decode kernel at K = 2560, N_out = 6912: 2:4 and 6:8 decode packs,
-    t = 1, 4 and 16 (t = 16 runs the act-quant kernel first), two calls each."""
+    """The decode kernel at K = 2560, N_out = 6912: the 2:4 decode packs (a
+    byte or 6 bits a group) and the 6:8 one, t = 1, 4 and 16 (t = 16 runs the
+    act-quant kernel first), two calls each."""
     import torch
 
     from sparse_linear_layers_bitlinear_b200 import sbl, synth
 
     dev = torch.device("cuda", 0)
     K, N = 2560, 6912
-    for (n, m) in ((2, 4), (6, 8)):
-        L = sbl.Layer.allocate(N, K, n, m, sbl.SBL_PACK_GEMV, device=dev)
+    g6 = sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT
+    for (n, m, flags) in ((2, 4, sbl.SBL_PACK_GEMV), (2, 4, g6), (6, 8, sbl.SBL_PACK_GEMV)):
+        L = sbl.Layer.allocate(N, K, n, m, flags, device=dev)
         sbl.prepare_weights(L, synth.master_weights(N, K, 5000, device=dev))
         for T in (1, 4, 16):
             x = synth.activations(T, K, 7, device=dev)

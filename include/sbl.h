@@ -71,9 +71,24 @@ enum {
   SBL_PACK_GEMV = 1u << 0,      /* also write the decode pack that sbl_forward streams for
                                    t <= 32 tokens (2:4: 2 bits a weight; other N:M: the
                                    compressed-index pack, 1 + 2n/m bits a weight) */
-  SBL_MASK_FROM_QUANT = 1u << 1 /* ablation the pages report ([de] 4 "Ablationsstudien",
+  SBL_MASK_FROM_QUANT = 1u << 1, /* ablation the pages report ([de] 4 "Ablationsstudien",
                                    [fr] 5): build the N:M mask from the ternary codes
                                    |q| instead of the masters (ties to the lowest index) */
+  SBL_PACK_GEMV_6BIT = 1u << 2, /* with SBL_PACK_GEMV on a 2:4 layer: the decode pack holds
+                                   each group of four as one of its 54 states in 6 bits
+                                   (1.5 bits a weight) instead of a byte; any other
+                                   pattern: SBL_ERR_UNSUPPORTED_NM; without SBL_PACK_GEMV:
+                                   SBL_ERR_INVALID_ARG */
+  SBL_FUSE_ACT_QUANT = 1u << 3  /* sbl_forward on the tensor-core GEMM path quantises the
+                                   activations inside the GEMM launch (the epilogue warps
+                                   of every CTA quantise token rows while the first tiles
+                                   load, each tile's loads wait for its rows' count)
+                                   instead of a separate kernel before it; taken when
+                                   k <= 3072 and the call passes a workspace (it holds the
+                                   counters), else the two-launch path.  Same bits.  The
+                                   launch's CTAs must all be resident at once, which they
+                                   are on an otherwise idle GPU; a stall shows as
+                                   SBL_ERR_TIMEOUT.  No effect on the blob's layout */
 };
 
 /* Flags of sbl_backward's `flags` argument. */
@@ -128,6 +143,14 @@ typedef struct sbl_blob_layout {
  * units of 16 rows x 128 k (rows padded to 16 and k to 128 with zero bytes),
  * ordered [row tile][k unit], 512 bytes each: the 8 bytes of groups 8t..8t+7
  * of the unit for row r sit at 16 * (4 * (r % 8) + t) + 8 * ((r % 16) / 8).
+ * gemv layout, 2:4 with SBL_PACK_GEMV_6BIT: group state 9 p + 3 d0 + d1 < 54,
+ * p = 0..5 the kept pair (i0, i1) in the order (0,1) (0,2) (0,3) (1,2) (1,3)
+ * (2,3), d0 / d1 the codes at i0 / i1 as digits mod 3 (0 -> 0, +1 -> 1,
+ * -1 -> 2); so state 0 is an all-zero group.  Units of 16 rows x 128 k as
+ * above, 384 bytes each: slot s = 4 * (r % 8) + t holds 96 bits, the 8
+ * states of groups 8t..8t+7 of row r (bits 6j..6j+5 for group 8t+j), then
+ * those of row r + 8 (from bit 48), least significant bit first; word j
+ * (bits 32j..32j+31) of slot s sits at byte 128 * j + 4 * s of the unit.
  * gemv layout, any other N:M (compressed index: the explicit N:M metadata beside
  * the kept values, [ja] 2.1): every block of 8 consecutive weights has a mask
  * byte (bit j = position j kept) and its n8 = 8n/m kept codes in index order,
@@ -148,8 +171,9 @@ sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t 
 /* Total bytes of the prepared blob, 0 for unsupported arguments. */
 size_t sbl_prepared_bytes(int64_t n_out, int64_t k, int n, int m, uint32_t flags);
 
-/* Bytes of scratch that sbl_forward needs when xq_out / xscale_out are NULL:
- * t*k int8 codes plus t fp32 scales (256-byte aligned pieces). */
+/* Bytes of scratch that sbl_forward needs when xq_out / xscale_out are NULL
+ * (or for SBL_FUSE_ACT_QUANT): t*k int8 codes, t fp32 scales, then one uint32
+ * counter per 16 tokens, each piece starting on a 256-byte boundary. */
 size_t sbl_workspace_bytes(int64_t t, int64_t k);
 
 /* Steps 1-3 ([de] 2, [ja] 2.1, [ko] 2.1-2.2).  Reads the bf16 masters

@@ -99,10 +99,22 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const
 // ---------------------------------------------------------------------------
 // Forward int8 GEMM
 // ---------------------------------------------------------------------------
+// The forward configuration for (accumulators out, tile width, in-launch
+// quantisation), launched by programmatic dependent launch.
+template <template <bool, int, bool> class Cfg, int BN>
+static cudaError_t launch_fwd(bool acc, bool qx, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
+                              const FwdParams& p, int num_sms, cudaStream_t s) {
+  if (qx)
+    return acc ? launch_pair<Cfg<true, BN, true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true)
+               : launch_pair<Cfg<false, BN, true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true);
+  return acc ? launch_pair<Cfg<true, BN, false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true)
+             : launch_pair<Cfg<false, BN, false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true);
+}
+
 cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,
                                 uint64_t meta_bytes, const int8_t* xq, const float* a_prime, const float* g,
                                 int64_t n_out, int64_t t, int64_t k, float* y, int32_t* acc_out, uint32_t* status,
-                                int num_sms, cudaStream_t s) {
+                                int num_sms, cudaStream_t s, const uint16_t* x_quantise, uint32_t* ready) {
   FwdParams p;
   p.n_out = static_cast<int>(n_out);
   p.T = static_cast<int>(t);
@@ -114,6 +126,18 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
   p.meta = meta;
   p.meta_kblocks = meta_kblocks;
   p.status = status;
+  // In-launch quantisation: the codes and a' go to xq / a_prime, counted per
+  // token tile on `ready` (zeroed here, ahead of the launch).
+  const bool qx = x_quantise != nullptr;
+  p.x = reinterpret_cast<const uint4*>(x_quantise);
+  p.xq = const_cast<int8_t*>(xq);
+  p.ap_out = const_cast<float*>(a_prime);
+  p.ready = ready;
+  if (qx) {
+    if (k > int64_t(kQxMaxRW) * 256 || ready == nullptr) return cudaErrorInvalidValue;
+    const cudaError_t e = cudaMemsetAsync(ready, 0, size_t(forward_tile_counters(t)) * 4, s);
+    if (e != cudaSuccess) return e;
+  }
   CUtensorMap ta, tb, te;
   const bool acc = acc_out != nullptr;
   if (sparse) {
@@ -126,8 +150,7 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
         !encode_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 256, meta_bytes / 256, 256, 256, 16,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
-    return acc ? launch_pair<CfgPairSparse<true>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true)
-               : launch_pair<CfgPairSparse<false>>(ta, tb, te, p, p.n_out, p.T, num_sms, s, true);
+    return launch_fwd<CfgPairSparse, 240>(acc, qx, ta, tb, te, p, num_sms, s);
   }
   // Dense int8 over W_eff codes.  Tile width: 192 tokens when that takes no
   // more rounds of pair tiles than 256, else 256.  A round of 192-token tiles
@@ -145,12 +168,13 @@ cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t*
   if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, k, n_out, k, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, k, t, k, 128, bn / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (narrow)
-    return acc ? launch_pair<CfgPairDense<true, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true)
-               : launch_pair<CfgPairDense<false, 192>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true);
-  return acc ? launch_pair<CfgPairDense<true, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true)
-             : launch_pair<CfgPairDense<false, 256>>(ta, tb, tb, p, p.n_out, p.T, num_sms, s, true);
+  if (narrow) return launch_fwd<CfgPairDense, 192>(acc, qx, ta, tb, tb, p, num_sms, s);
+  return launch_fwd<CfgPairDense, 256>(acc, qx, ta, tb, tb, p, num_sms, s);
 }
+
+// Token-tile counters the in-launch quantisation needs: one per 16 tokens
+// covers every tile width (192, 240, 256).
+int64_t forward_tile_counters(int64_t t) { return (t + 15) / 16; }
 
 // ---------------------------------------------------------------------------
 // Backward bf16 GEMM

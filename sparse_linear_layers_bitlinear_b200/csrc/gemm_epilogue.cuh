@@ -4,6 +4,7 @@
 // 32*(w%4) .. +31, i.e. one output row per thread, in 32-column chunks.
 #pragma once
 
+#include "actq_math.cuh"
 #include "sbl_device.cuh"
 
 namespace sbl {
@@ -116,7 +117,52 @@ struct FwdParams {
   const uint8_t* meta;   // sparse: tensor-core metadata section
   int meta_kblocks;      // 128-wide k blocks per row block in the metadata section
   uint32_t* status;
+  // Configurations that quantise the activations in the same launch (QX):
+  const uint4* x;        // bf16 [T][K] as 16-byte vectors
+  int8_t* xq;            // the codes (the B operand's tensor map covers them)
+  float* ap_out;         // a' per token (the array a_prime points to)
+  uint32_t* ready;       // per BN-token tile: rows quantised so far, zero at launch
 };
+
+// Rows of up to kQxMaxRW * 32 * 8 elements are quantised by one warp, the row
+// held in registers.
+constexpr int kQxMaxRW = 12;  // 16-byte vectors a lane: K <= 3072
+
+// One token row quantised by one warp: a' = max(max_k |x|, 1e-5) through an
+// integer max over the bf16 magnitude bits, then the codes by one fused
+// multiply-add each (or the IEEE division for a row under the clamp or at
+// 2^120 and above), as the act-quant kernel computes them.
+__device__ __forceinline__ void quantise_row_warp(const FwdParams& p, int row, int lane) {
+  const int nvec = p.K / 8;
+  const uint4* src = p.x + int64_t(row) * nvec;
+  uint4 v[kQxMaxRW];
+#pragma unroll
+  for (int r = 0; r < kQxMaxRW; ++r) {
+    const int i = r * 32 + lane;
+    v[r] = (i < nvec) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+  }
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int r = 0; r < kQxMaxRW; ++r) {
+    m2 = __vmaxu2(m2, v[r].x & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v[r].y & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v[r].z & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v[r].w & 0x7FFF7FFFu);
+  }
+  const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+  const float ap = fmaxf(__uint_as_float(m << 16), 1e-5f);
+  if (lane == 0) {
+    p.ap_out[row] = ap;
+    if (m >= 0x7F80u) raise_status(p.status, SBL_STATUS_NONFINITE_X);
+  }
+  const QScale qs = make_qscale(ap);
+  uint2* dst = reinterpret_cast<uint2*>(p.xq + int64_t(row) * p.K);
+#pragma unroll
+  for (int r = 0; r < kQxMaxRW; ++r) {
+    const int i = r * 32 + lane;
+    if (i < nvec) dst[i] = qs.exact ? quantise8_div(v[r], qs.ap) : quantise8_fma(v[r], qs.c);
+  }
+}
 
 // One 32-token chunk of the forward epilogue.  The thread owns output row o
 // (a TMEM lane) and holds its 32 int32 accumulators for tokens t0..t0+31;
@@ -127,7 +173,9 @@ template <bool ACC_OUT, int NC = 32>
 __device__ __forceinline__ void fwd_epilogue_chunk(const FwdParams& p, const uint32_t (&r)[NC], int o, int t0,
                                                    int lane, float g) {
   const int tl = t0 + lane;
-  const float f_mine = (tl < p.T) ? __fdiv_rn(__fmul_rn(g, p.a_prime[tl]), 127.0f) : 0.0f;
+  // a' through L2: in a launch that quantises the activations itself, other
+  // CTAs wrote it during this launch
+  const float f_mine = (tl < p.T) ? __fdiv_rn(__fmul_rn(g, __ldcg(p.a_prime + tl)), 127.0f) : 0.0f;
   const bool row_ok = o < p.n_out;
   const int64_t ld = p.n_out;
   float* yp = p.y + int64_t(t0) * ld + o;

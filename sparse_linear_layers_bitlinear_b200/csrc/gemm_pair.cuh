@@ -122,6 +122,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<Cfg>(),
         const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
         const int m0 = t.mb * 256 + 128 * int(rank);
         const int n0 = t.nb * Cfg::BN + int(rank) * (Cfg::BN / 2);
+        if constexpr (Cfg::QUANT_X) {
+          // the tile's token rows are quantised by the epilogue warps of the
+          // whole grid: wait for their count, then read the codes by TMA
+          if (!wait_count(p.ready + t.nb, Cfg::tile_rows(p, t.nb), abort_flag, status)) break;
+          fence_proxy_async_global();
+        }
         for (int kb = 0; kb < t.kblocks; ++kb) {
           if (!mbar_wait(&tail->empty[stage], phase ^ 1u, abort_flag, status)) {
             ok = false;
@@ -190,6 +196,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<Cfg>(),
     const int quarter = warp & 3;
     const int part = (warp - 2) >> 2, parts = Cfg::EPI_WARPS / 4;
     const uint32_t leader_acc_empty0 = map_to_rank(&tail->acc_empty[0], 0);
+    if constexpr (Cfg::QUANT_X) {
+      // Before the first accumulator is ready, the epilogue warps of the grid
+      // quantise the token rows, warp by warp in row order (so the first
+      // tiles' rows come first), each row counted on its tile once written.
+      pdl_wait();  // x may come from the kernel before
+      const int nw = int(gridDim.x) * Cfg::EPI_WARPS;
+      for (int row = int(blockIdx.x) * Cfg::EPI_WARPS + (warp - 2); row < p.T; row += nw) {
+        quantise_row_warp(p, row, lane);
+        fence_proxy_async_global();  // the codes are read by TMA
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.ready + row / Cfg::BN, 1u);
+      }
+    }
     for (int i = 0; i < ntiles; ++i) {
       const PairTile t = Cfg::Tiles::at(p, pair, npairs, i);
       const uint32_t ab = uint32_t(i) & 1u;
@@ -198,6 +218,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<Cfg>(),
       if (lane == 0) ready = mbar_wait(&tail->acc_full[ab], aphase, abort_flag, status);
       ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
       if (!ready) break;
+      if constexpr (Cfg::QUANT_X) {
+        // the tile's a' were written by other CTAs: acquire their count
+        // (complete by now: the producer waited for it before the loads)
+        if (!__all_sync(0xffffffffu, wait_count(p.ready + t.nb, Cfg::tile_rows(p, t.nb), abort_flag, status))) break;
+      }
       tc_fence_after();
       const int m0 = t.mb * 256 + 128 * int(rank);
       const int n0 = t.nb * Cfg::BN;
@@ -232,6 +257,7 @@ template <bool A_MN, bool B_MN, bool OUT_F32>
 struct CfgPairBf16 {
   using Params = Bf16Params;
   using Tiles = StripedTiles<CfgPairBf16>;
+  static constexpr bool QUANT_X = false;
   static constexpr int MAPS = 2;
   static constexpr int EPI_WARPS = 4;
   static constexpr int BN = 256, BK = 64, STAGES = 6;
@@ -309,6 +335,7 @@ struct DualBf16Params {
 template <bool OUT_F32>
 struct CfgPairDualBf16 {
   using Params = DualBf16Params;
+  static constexpr bool QUANT_X = false;
   static constexpr int MAPS = 4;
   static constexpr int EPI_WARPS = 4;
   static constexpr int BN = 256, BK = 64, STAGES = 6;
@@ -390,10 +417,11 @@ struct CfgPairDualBf16 {
 // metadata slots in the gap at 240-255 (at 224 tokens: accumulators at 0 and
 // 224, metadata after them at 448).
 // ---------------------------------------------------------------------------
-template <bool ACC_OUT, int BN_ = 240>
+template <bool ACC_OUT, int BN_ = 240, bool QX = false>
 struct CfgPairSparse {
   using Params = FwdParams;
   using Tiles = StripedTiles<CfgPairSparse>;
+  static constexpr bool QUANT_X = QX;  // quantise the activations in the same launch
   static constexpr int MAPS = 3;
   static constexpr int EPI_WARPS = 8;  // the fp32 output is the heavy part of this epilogue
   static constexpr int BN = BN_, BK = 256, STAGES = 4;
@@ -413,6 +441,7 @@ struct CfgPairSparse {
   __device__ static int rows_M(const Params& p) { return p.n_out; }
   __device__ static int cols_N(const Params& p) { return p.T; }
   __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
+  __device__ static uint32_t tile_rows(const Params& p, int nb) { return static_cast<uint32_t>(min(BN, p.T - nb * BN)); }
 
   __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tE,
                                     const CUtensorMap*, const Params& p, int, uint8_t* sA, uint8_t* sB, uint8_t* sE,
@@ -469,10 +498,11 @@ struct CfgPairSparse {
 // rows x BN tokens, 128 k per stage.  Each CTA holds 128 rows of W_eff codes
 // (128 x 128 bytes) and BN/2 tokens of xq.
 // ---------------------------------------------------------------------------
-template <bool ACC_OUT, int BN_>
+template <bool ACC_OUT, int BN_, bool QX = false>
 struct CfgPairDense {
   using Params = FwdParams;
   using Tiles = StripedTiles<CfgPairDense>;
+  static constexpr bool QUANT_X = QX;  // quantise the activations in the same launch
   static constexpr int MAPS = 2;
   static constexpr int EPI_WARPS = 8;
   static constexpr int BN = BN_, BK = 128;
@@ -489,6 +519,7 @@ struct CfgPairDense {
   __device__ static int rows_M(const Params& p) { return p.n_out; }
   __device__ static int cols_N(const Params& p) { return p.T; }
   __device__ static int k_blocks(const Params& p) { return (p.K + BK - 1) / BK; }
+  __device__ static uint32_t tile_rows(const Params& p, int nb) { return static_cast<uint32_t>(min(BN, p.T - nb * BN)); }
 
   __device__ static void load_stage(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap*,
                                     const CUtensorMap*, const Params&, int, uint8_t* sA, uint8_t* sB, uint8_t*, int m0,

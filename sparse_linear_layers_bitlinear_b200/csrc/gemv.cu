@@ -1,4 +1,4 @@
-// Decode-shaped forward (t <= 32 tokens) over the 2-bit weight packs.
+// Decode-shaped forward (t <= 32 tokens) over the packed weights.
 //
 // At these token counts the weight stream is the whole cost, so the weights
 // travel packed and are expanded to int8 in registers, straight into the
@@ -25,6 +25,13 @@
 //       (groups 8t..8t+7 of the unit) and then the 8 of row g + 8, so a lane
 //       reads one 16-byte piece per unit and a warp 512 contiguous bytes; a
 //       256-entry table expands a byte into the group's four int8 weights.
+//   2:4, 6-bit group code (1.5 bits a weight): a group's kept pair p (0..5,
+//       lexicographic) and its two codes as digits mod 3 form the state
+//       9 p + 3 d0 + d1 < 54.  A lane's 16 states of a unit (row g groups
+//       8t..8t+7, then row g + 8) are 96 bits, least significant first, held
+//       as three words; word j of every lane forms the unit's j-th 128-byte
+//       plane, so each of a lane's three loads is one coalesced 128-byte row
+//       for the warp (a unit is 384 bytes).  A 64-entry table expands a state.
 //   any other N:M (compressed index): per block of 8 weights a mask byte and
 //       the n8 = 8n/m kept 2-bit codes in index order.  The section is
 //       interleaved by unit and lane so that a lane's mask bytes and code bits
@@ -62,7 +69,7 @@ constexpr int kDecWarps = kDecThreads / 32;
 // banks.  16 copies measured best: 32 doubled the table fill before the wait
 // (which competes with the call before) for no gain in the products.
 constexpr int kLutCopiesReg = 16;
-constexpr int lut_words(int copies) { return 256 * copies; }
+constexpr int lut_words(int copies, int entries = 256) { return entries * copies; }
 constexpr int kDecBatch = 8;         // units whose weight bytes a lane holds at once
 constexpr size_t kDecMaxSmem = 227 * 1024;
 constexpr int kDecMaxT = 32;
@@ -120,8 +127,17 @@ __host__ __device__ constexpr uint32_t code_byte(uint32_t c) { return c == 1u ? 
 // kind 1: a byte of four codes -> four int8 values in index order; kind 2: a
 // mask byte -> two byte-permute selectors (positions 0-3 in the low half,
 // 4-7 in the high half): a kept position picks its rank among the kept
-// values, a pruned one byte 7 (zero whenever fewer than 8 are kept).
+// values, a pruned one byte 7 (zero whenever fewer than 8 are kept); kind 3:
+// a 6-bit group state -> the group's four weights (states 54..63 unused).
 __device__ __forceinline__ uint32_t lut_entry(int kind, uint32_t b) {
+  if (kind == 3) {
+    if (b >= 54u) return 0u;
+    const uint32_t p = b / 9u, d0 = (b / 3u) % 3u, d1 = b % 3u;
+    const uint32_t i0 = p < 3u ? 0u : (p < 5u ? 1u : 2u);
+    const uint32_t i1 = p < 3u ? p + 1u : (p < 5u ? p - 1u : 3u);
+    auto digit = [](uint32_t d) { return d == 1u ? 0x01u : d == 2u ? 0xFFu : 0u; };
+    return (digit(d0) << (8 * i0)) | (digit(d1) << (8 * i1));
+  }
   if (kind == 0) {
     const uint32_t i0 = (b >> 4) & 3u, i1 = (b >> 6) & 3u;
     return (code_byte(b & 3u) << (8 * i0)) | (code_byte((b >> 2) & 3u) << (8 * i1));
@@ -138,25 +154,29 @@ __device__ __forceinline__ uint32_t lut_entry(int kind, uint32_t b) {
 }
 
 template <int C>
-__device__ __forceinline__ void fill_lut(uint32_t* lut, int kind, int tid) {
+__device__ __forceinline__ void fill_lut(uint32_t* lut, int kind, int tid, int entries = 256) {
   constexpr int kVecs = C / 4;  // 16-byte stores per entry
-  for (int i = tid; i < 256 * kVecs; i += kDecThreads) {
+  for (int i = tid; i < entries * kVecs; i += kDecThreads) {
     const uint32_t v = lut_entry(kind, static_cast<uint32_t>(i / kVecs));
     reinterpret_cast<uint4*>(lut)[i] = make_uint4(v, v, v, v);
   }
 }
 
 // Compile-time facts of a weight pack.  FMT 0: 2:4 bytes; FMT 1..8: blocks of
-// 8 with FMT kept codes (8 = dense, no mask block).
+// 8 with FMT kept codes (8 = dense, no mask block); FMT 9: 2:4 6-bit states.
+constexpr int kFmtCode6 = 9;
 template <int FMT>
 struct Pack {
   static constexpr bool k24 = FMT == 0;
+  static constexpr bool c6 = FMT == kFmtCode6;
   static constexpr int n8 = FMT;
   static constexpr bool has_mask = FMT >= 1 && FMT < 8;
-  static constexpr int cb = k24 ? 0 : (2 * FMT + 3) / 4 * 4;  // code bytes per lane and unit
+  static constexpr int cb = (k24 || c6) ? 0 : (2 * FMT + 3) / 4 * 4;  // code bytes per lane and unit
   static constexpr int cw = cb / 4;
-  static constexpr int unit_bytes = k24 ? 512 : (has_mask ? 256 : 0) + 32 * cb;
-  static constexpr int regs = k24 ? 4 : (has_mask ? 2 : 0) + cw;  // words a lane loads per unit
+  static constexpr int unit_bytes = k24 ? 512 : c6 ? 384 : (has_mask ? 256 : 0) + 32 * cb;
+  static constexpr int regs = k24 ? 4 : c6 ? 3 : (has_mask ? 2 : 0) + cw;  // words a lane loads per unit
+  static constexpr int lut_entries = c6 ? 64 : 256;
+  static constexpr int lut_kind = k24 ? 0 : c6 ? 3 : 1;
 };
 
 // One unit's weight words of this lane.
@@ -171,6 +191,11 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, int tile, int u, 
     r[1] = v.y;
     r[2] = v.z;
     r[3] = v.w;
+  } else if constexpr (P::c6) {
+    // word j of the lane's 96 state bits from plane j of the unit
+    const uint32_t* base = reinterpret_cast<const uint32_t*>(a.w + (int64_t(tile) * a.upr + u) * P::unit_bytes);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) r[j] = __ldcs(base + 32 * j + lane);
   } else {
     const uint8_t* base = a.w + (int64_t(tile) * a.upr + u) * P::unit_bytes;
     int o = 0;
@@ -220,6 +245,17 @@ __device__ __forceinline__ uint32_t lut_get(const uint8_t* lane_base, uint32_t w
   return *reinterpret_cast<const uint32_t*>(lane_base + off);
 }
 
+// Table entry of the 6-bit state at bit `off` of the lane's words (off
+// compile-time after unrolling), shifted straight into a byte offset.
+template <int C>
+__device__ __forceinline__ uint32_t lut_get6(const uint8_t* lane_base, const uint32_t* w, int off) {
+  constexpr int kShift = 2 + (C == 16 ? 4 : C == 32 ? 5 : 3);
+  const int wi = off >> 5, sh = (off & 31) - kShift;
+  uint32_t v = sh >= 0 ? (w[wi] >> sh) : (w[wi] << -sh);
+  if ((off & 31) + 6 > 32) v |= w[wi + 1] << (32 - sh);
+  return *reinterpret_cast<const uint32_t*>(lane_base + (v & (0x3Fu << kShift)));
+}
+
 // The four A-fragment registers of k-step s: rows g (a0 low k slots, a2 high)
 // and g + 8 (a1, a3).  la / ls: this lane's copies of the tables.
 template <int FMT, int C>
@@ -234,6 +270,13 @@ __device__ __forceinline__ void decode_step(const uint32_t (&r)[Pack<FMT>::regs]
     a2 = lut_get<C>(la, w0, b + 1);
     a1 = lut_get<C>(la, w1, b);
     a3 = lut_get<C>(la, w1, b + 1);
+  } else if constexpr (P::c6) {
+    // groups 2s, 2s + 1 of each row: states at 12 s, 12 s + 6 (row g) and
+    // 48 bits further (row g + 8)
+    a0 = lut_get6<C>(la, r, 12 * s);
+    a2 = lut_get6<C>(la, r, 12 * s + 6);
+    a1 = lut_get6<C>(la, r, 48 + 12 * s);
+    a3 = lut_get6<C>(la, r, 54 + 12 * s);
   } else {
     constexpr int o = P::has_mask ? 2 : 0;
     uint32_t lo[2], hi[2];
@@ -435,7 +478,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t* lut_a = reinterpret_cast<uint32_t*>(smem);
   uint32_t* lut_s = lut_a + lut_words(C);  // mask selectors (packs with a mask block)
-  uint8_t* xsm = smem + (P::has_mask ? 2 : 1) * lut_words(C) * 4;
+  uint8_t* xsm = smem + (P::has_mask ? 2 * lut_words(C) : lut_words(C, P::lut_entries)) * 4;
   int32_t* s_acc = reinterpret_cast<int32_t*>(xsm + a.t * a.xs);  // [tpb][16][TP]
   DecScalars* sc = reinterpret_cast<DecScalars*>(s_acc + a.tpb * 16 * TP);
 
@@ -451,7 +494,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     else bulk_prefetch_l2(a.xq_in, static_cast<uint32_t>(a.t) * static_cast<uint32_t>(a.k));
   }
   pdl_trigger();
-  fill_lut<C>(lut_a, P::k24 ? 0 : 1, tid);
+  fill_lut<C>(lut_a, P::lut_kind, tid, P::lut_entries);
   if constexpr (P::has_mask) fill_lut<C>(lut_s, 2, tid);
   for (int i = tid; i < ntile * 16 * TP; i += kDecThreads) s_acc[i] = 0;
   // Activation columns past k are left as they are: the weights there are
@@ -535,14 +578,18 @@ namespace {
 
 int decode_nt(int64_t t) { return t <= 8 ? 1 : t <= 16 ? 2 : 4; }
 
-int decode_fmt(int n, int m) { return (n == 2 && m == 4) ? 0 : 8 * n / m; }
+int decode_fmt(int n, int m, bool code6) {
+  return (n == 2 && m == 4) ? (code6 ? kFmtCode6 : 0) : 8 * n / m;
+}
 
-bool fmt_has_mask(int fmt) { return fmt >= 1 && fmt < 8; }
+size_t decode_lut_bytes(int fmt) {
+  const bool has_mask = fmt >= 1 && fmt < 8;
+  return size_t(has_mask ? 2 * lut_words(kLutCopiesReg) : lut_words(kLutCopiesReg, fmt == kFmtCode6 ? 64 : 256)) * 4;
+}
 
 size_t decode_smem(int fmt, int nt, int64_t t, int64_t k, int tpb) {
   const size_t xs = size_t((k + 127) / 128 * 128);
-  return size_t(fmt_has_mask(fmt) ? 2 : 1) * lut_words(kLutCopiesReg) * 4 + size_t(t) * xs +
-         size_t(tpb) * 16 * 8 * nt * 4 + sizeof(DecScalars);
+  return decode_lut_bytes(fmt) + size_t(t) * xs + size_t(tpb) * 16 * 8 * nt * 4 + sizeof(DecScalars);
 }
 
 template <int FMT, int NT, bool FUSED>
@@ -567,17 +614,17 @@ cudaError_t decode_fmt_launch(const DecodeArgs& a, bool fused, int nt, int block
 
 }  // namespace
 
-uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m) {
-  if (n == 2 && m == 4) return uint64_t((n_out + 15) / 16) * uint64_t((k + 127) / 128) * 512;
+uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m, bool code6) {
+  if (n == 2 && m == 4) return uint64_t((n_out + 15) / 16) * uint64_t((k + 127) / 128) * (code6 ? 384 : 512);
   const int n8 = 8 * n / m;
   const uint64_t cb = uint64_t(2 * n8 + 3) / 4 * 4;
   const uint64_t unit = (n8 < 8 ? 256 : 0) + 32 * cb;
   return uint64_t((n_out + 15) / 16) * uint64_t((k + 127) / 128) * unit;
 }
 
-bool gemv_fits(int64_t t, int64_t k, int n, int m) {
+bool gemv_fits(int64_t t, int64_t k, int n, int m, bool code6) {
   if (t < 1 || t > kDecMaxT) return false;
-  return decode_smem(decode_fmt(n, m), decode_nt(t), t, k, 1) <= kDecMaxSmem;
+  return decode_smem(decode_fmt(n, m, code6), decode_nt(t), t, k, 1) <= kDecMaxSmem;
 }
 
 // The decode kernels stream the packed weights once for up to 32 tokens; the
@@ -586,7 +633,7 @@ bool gemv_preferred(int64_t t, int64_t n_out, int64_t k) { return t <= kDecMaxT;
 
 bool gemv_fuses_act_quant(int64_t t) { return t <= kFusedMaxT; }
 
-cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_t* x, const int8_t* xq_in,
+cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, bool code6, const uint16_t* x, const int8_t* xq_in,
                                 const float* ap_in, const float* g, int64_t n_out, int64_t t, int64_t k, float* y,
                                 int32_t* acc_out, int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms,
                                 cudaStream_t s) {
@@ -607,7 +654,7 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_
   a.tiles = static_cast<int>((n_out + 15) / 16);
   a.upr = static_cast<int>((k + 127) / 128);
   a.xs = a.upr * 128;
-  const int fmt = decode_fmt(n, m), nt = decode_nt(t);
+  const int fmt = decode_fmt(n, m, code6), nt = decode_nt(t);
   // codes from the caller (x == NULL), else quantised here for few tokens
   const bool fused = x != nullptr && gemv_fuses_act_quant(t);
   // As many blocks as fit two per SM; each takes an equal run of tiles.
@@ -628,6 +675,7 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_
     case 5: return decode_fmt_launch<5>(a, fused, nt, blocks, smem, s);
     case 6: return decode_fmt_launch<6>(a, fused, nt, blocks, smem, s);
     case 7: return decode_fmt_launch<7>(a, fused, nt, blocks, smem, s);
+    case kFmtCode6: return decode_fmt_launch<kFmtCode6>(a, fused, nt, blocks, smem, s);
     default: return decode_fmt_launch<8>(a, fused, nt, blocks, smem, s);
   }
 }

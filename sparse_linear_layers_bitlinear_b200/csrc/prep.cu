@@ -828,7 +828,7 @@ __device__ __forceinline__ void prepare_body(const PrepArgs& a, const int G, con
           const int c = col[h2];
           a.out.sp_meta[(r >> 7) * meta_rb_bytes + (r & 127) * 16 + (c >> 4) * 2048 + (c & 15)] =
               static_cast<uint8_t>(Z >> 16);
-          if (a.out.gemv != nullptr) {
+          if (a.out.gemv != nullptr && !a.out.gemv_code6) {
             // per group: the two kept 2-bit codes (01 = +1, 11 = -1) low, the
             // metadata nibble high; the vector's two bytes go to its lane slot
             // of the interleaved decode pack (16-row x 128-k units of 512
@@ -841,6 +841,44 @@ __device__ __forceinline__ void prepare_body(const PrepArgs& a, const int G, con
             uint8_t* unit = a.out.gemv + ((r >> 4) * a.out.gemv_upr + (c >> 4)) * int64_t(512);
             *reinterpret_cast<uint16_t*>(unit + lane_d * 16 + ((r >> 3) & 1) * 8 + (c & 3) * 2) =
                 static_cast<uint16_t>(__byte_perm(t, 0u, 0x3320) | nibs);
+          }
+        }
+      }
+      if (M == 4 && n == 2 && a.out.gemv_code6) {  // uniform per launch; gemv != nullptr
+        // The 6-bit states of the vector's two groups: 9 p + 3 d0 + d1 with p
+        // the rank of the kept pair (from the metadata nibble i0 | i1 << 2)
+        // and d the kept codes mod 3 (the int8 code's low two bits 0, 1, 3
+        // less their upper bit: 0, 1, 2).
+        constexpr uint64_t kPairRank = (1ull << 32) | (2ull << 48) | (3ull << 36) | (4ull << 52) | (5ull << 56);
+        const uint32_t vals = codes_of_high_bytes(__byte_perm(hb_lo, hb_hi, W));
+        const uint32_t t2 = vals & 0x03030303u;
+        const uint32_t d = t2 - ((t2 >> 1) & 0x01010101u);
+        const uint32_t p0 = static_cast<uint32_t>(kPairRank >> (4 * ((Z >> 16) & 0xFu))) & 0xFu;
+        const uint32_t p1 = static_cast<uint32_t>(kPairRank >> (4 * ((Z >> 20) & 0xFu))) & 0xFu;
+        const uint32_t s0 = 9u * p0 + 3u * (d & 0xFFu) + ((d >> 8) & 0xFFu);
+        const uint32_t s1 = 9u * p1 + 3u * ((d >> 16) & 0xFFu) + (d >> 24);
+        const uint32_t f = active ? (s0 | (s1 << 6)) : 0u;
+        // Four consecutive vectors of a row (groups 0..7 of one lane slot of
+        // a unit) sit in four consecutive lanes; the first gathers their 48
+        // bits and writes them: row g's to plane 0 and the low half of plane
+        // 1, row g + 8's to the high half of plane 1 and plane 2.
+        const uint32_t f1 = __shfl_down_sync(0xffffffffu, f, 1), f2 = __shfl_down_sync(0xffffffffu, f, 2),
+                       f3 = __shfl_down_sync(0xffffffffu, f, 3);
+        if (active && (lane & 3) == 0) {
+          const uint64_t bits = uint64_t(f) | (uint64_t(f1) << 12) | (uint64_t(f2) << 24) | (uint64_t(f3) << 36);
+          const int64_t r = row[h2];
+          const int c = col[h2];
+          const int lane_d = static_cast<int>(r & 7) * 4 + ((c >> 2) & 3);
+          uint8_t* unit = a.out.gemv + ((r >> 4) * a.out.gemv_upr + (c >> 4)) * int64_t(384);
+          uint32_t* w0 = reinterpret_cast<uint32_t*>(unit) + lane_d;
+          uint16_t* w1 = reinterpret_cast<uint16_t*>(unit + 128) + 2 * lane_d;
+          uint32_t* w2 = reinterpret_cast<uint32_t*>(unit + 256) + lane_d;
+          if (((r >> 3) & 1) == 0) {
+            *w0 = static_cast<uint32_t>(bits);
+            w1[0] = static_cast<uint16_t>(bits >> 32);
+          } else {
+            w1[1] = static_cast<uint16_t>(bits);
+            *w2 = static_cast<uint32_t>(bits >> 16);
           }
         }
       }
@@ -979,6 +1017,7 @@ static cudaError_t prep_args(const uint16_t* w, int64_t n_out, int64_t k, int n,
   a.out.gemv_cb = (2 * a.out.gemv_n8 + 3) / 4 * 4;
   a.out.gemv_unit_bytes = (a.out.gemv_n8 < 8 ? 256 : 0) + 32 * a.out.gemv_cb;
   a.out.gemv_upr = static_cast<int>((k + 127) / 128);
+  a.out.gemv_code6 = (L.gemv != 0 && (flags & SBL_PACK_GEMV_6BIT)) ? 1 : 0;
   if (mode != kPrepSumOnly && L.gemv && (n_out % 16 != 0 || k % 128 != 0)) {
     // the interleaved pack covers whole 16-row, 128-k units: what no weight
     // fills is zero

@@ -19,7 +19,7 @@ void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 namespace {
 
 constexpr int64_t kMaxK = 131072;  // keeps |acc| <= 127 * k below 2^24: (float)acc is exact
-constexpr uint32_t kLayerFlags = SBL_PACK_GEMV | SBL_MASK_FROM_QUANT;
+constexpr uint32_t kLayerFlags = SBL_PACK_GEMV | SBL_MASK_FROM_QUANT | SBL_PACK_GEMV_6BIT | SBL_FUSE_ACT_QUANT;
 constexpr uint32_t kBackwardFlags = SBL_GRAD_F32 | SBL_NO_DX | SBL_NO_DW | SBL_MASKED_GRAD | SBL_DW_QUANT_X;
 
 struct DeviceInfo {
@@ -54,6 +54,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 sbl_status check_shape(int64_t n_out, int64_t k, int n, int m, uint32_t flags) {
   if ((flags & ~kLayerFlags) != 0u) return SBL_ERR_INVALID_ARG;
   if (!(m == 2 || m == 4 || m == 8) || n < 1 || n > m) return SBL_ERR_UNSUPPORTED_NM;
+  if (flags & SBL_PACK_GEMV_6BIT) {  // a form of the 2:4 decode pack
+    if (!(flags & SBL_PACK_GEMV)) return SBL_ERR_INVALID_ARG;
+    if (!(n == 2 && m == 4)) return SBL_ERR_UNSUPPORTED_NM;
+  }
   if (n_out < 8 || n_out % 8 != 0 || k < 64 || k % 64 != 0) return SBL_ERR_SHAPE;
   if (k > kMaxK || n_out > (int64_t(1) << 30) || n_out * k > (int64_t(1) << 40)) return SBL_ERR_SHAPE;
   return SBL_OK;
@@ -67,10 +71,13 @@ sbl_status check_layer(const sbl_layer* layer, sbl_blob_layout* L) {
   return sbl_prepared_layout(layer->n_out, layer->k, layer->n, layer->m, layer->flags, L);
 }
 
+bool code6(const sbl_layer* layer) { return (layer->flags & SBL_PACK_GEMV_6BIT) != 0u; }
+
 // The decode kernel takes the call when the layer has the decode pack and the
 // token rows fit its shared memory.
 bool uses_decode(const sbl_layer* layer, const sbl_blob_layout& L, int64_t t) {
-  return L.gemv != 0 && gemv_fits(t, layer->k, layer->n, layer->m) && gemv_preferred(t, layer->n_out, layer->k);
+  return L.gemv != 0 && gemv_fits(t, layer->k, layer->n, layer->m, code6(layer)) &&
+         gemv_preferred(t, layer->n_out, layer->k);
 }
 
 template <class T>
@@ -118,7 +125,7 @@ sbl_status sbl_prepared_layout(int64_t n_out, int64_t k, int n, int m, uint32_t 
     L.codes = take(uint64_t(n_out) * uint64_t(k));
   }
   if (flags & SBL_PACK_GEMV) {
-    L.gemv_bytes = decode_pack_bytes(n_out, k, n, m);
+    L.gemv_bytes = decode_pack_bytes(n_out, k, n, m, (flags & SBL_PACK_GEMV_6BIT) != 0u);
     L.gemv = take(L.gemv_bytes);
   }
   L.total_bytes = off;
@@ -137,7 +144,8 @@ size_t sbl_prepared_bytes(int64_t n_out, int64_t k, int n, int m, uint32_t flags
 
 size_t sbl_workspace_bytes(int64_t t, int64_t k) {
   if (t < 0 || k < 0) return 0;
-  return static_cast<size_t>(align_up(uint64_t(t) * uint64_t(k), 256) + align_up(uint64_t(t) * 4, 256));
+  return static_cast<size_t>(align_up(uint64_t(t) * uint64_t(k), 256) + align_up(uint64_t(t) * 4, 256) +
+                             align_up(uint64_t(forward_tile_counters(t)) * 4, 256));
 }
 
 sbl_status sbl_prepare_weights(const sbl_layer* layer, const void* w_master, sbl_stream_t stream) {
@@ -224,9 +232,14 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
   if (xq == nullptr || ap == nullptr) {
     if (workspace == nullptr) return SBL_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SBL_ERR_ALIGN;
+  }
+  uint32_t* ready = nullptr;  // token-tile counters of the in-launch quantisation
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint64_t codes_bytes = align_up(uint64_t(t) * uint64_t(layer->k), 256);
     if (xq == nullptr) xq = reinterpret_cast<int8_t*>(ws);
-    if (ap == nullptr) ap = reinterpret_cast<float*>(ws + align_up(uint64_t(t) * uint64_t(layer->k), 256));
+    if (ap == nullptr) ap = reinterpret_cast<float*>(ws + codes_bytes);
+    ready = reinterpret_cast<uint32_t*>(ws + codes_bytes + align_up(uint64_t(t) * 4, 256));
   }
   if (!aligned16(x) || !aligned16(y) || !aligned16(xq) || !aligned16(ap) || !aligned16(acc_debug))
     return SBL_ERR_ALIGN;
@@ -242,24 +255,31 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
         launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true) != cudaSuccess)
       return SBL_ERR_CUDA;
     const cudaError_t e =
-        launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, static_cast<const uint16_t*>(x),
+        launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, code6(layer),
+                            static_cast<const uint16_t*>(x),
                             fused ? nullptr : xq, ap, g,
                             layer->n_out, t, layer->k, y, acc_debug, fused ? xq_out : nullptr,
                             fused ? xscale_out : nullptr, status, sms, s);
     return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
   }
-  // the forward GEMM is launched with programmatic dependent launch and waits
-  // for the quantiser's outputs itself, so the quantiser lets it launch early
-  cudaError_t e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true);
-  if (e != cudaSuccess) return SBL_ERR_CUDA;
+  // SBL_FUSE_ACT_QUANT: the GEMM launch quantises the activations itself
+  // (rows up to kFusedActQuantMaxK, counters in the workspace)
+  const bool fuse = (layer->flags & SBL_FUSE_ACT_QUANT) && ready != nullptr && layer->k <= kFusedActQuantMaxK;
+  const uint16_t* xq_src = fuse ? static_cast<const uint16_t*>(x) : nullptr;
+  cudaError_t e = cudaSuccess;
+  if (!fuse) {
+    // the forward GEMM is launched with programmatic dependent launch and waits
+    // for the quantiser's outputs itself, so the quantiser lets it launch early
+    e = launch_act_quant(static_cast<const uint16_t*>(x), t, layer->k, xq, ap, status, sms, s, true);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+  }
   if (is_24(layer->n, layer->m)) {
     e = launch_forward_gemm(true, at<const int8_t>(layer, L.sp_values), at<const uint8_t>(layer, L.sp_meta),
                             static_cast<int>(meta_k_padded(layer->k) / 128), L.sp_meta_bytes, xq, ap, g, layer->n_out,
-                            t, layer->k, y,
-                            acc_debug, status, sms, s);
+                            t, layer->k, y, acc_debug, status, sms, s, xq_src, ready);
   } else {
     e = launch_forward_gemm(false, at<const int8_t>(layer, L.codes), nullptr, 0, 0, xq, ap, g, layer->n_out, t, layer->k,
-                            y, acc_debug, status, sms, s);
+                            y, acc_debug, status, sms, s, xq_src, ready);
   }
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
@@ -280,7 +300,7 @@ sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const
   const float* g = at<const float>(layer, L.g);
   cudaError_t e;
   if (uses_decode(layer, L, t)) {
-    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, nullptr, xq, xscale, g,
+    e = launch_forward_gemv(at<const uint8_t>(layer, L.gemv), layer->n, layer->m, code6(layer), nullptr, xq, xscale, g,
                             layer->n_out, t, layer->k, y,
                             acc_debug, nullptr, nullptr, status, sms, s);
   } else if (is_24(layer->n, layer->m)) {

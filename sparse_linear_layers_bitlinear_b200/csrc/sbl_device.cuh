@@ -94,6 +94,42 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Counters in global memory that other CTAs of the launch raise (release:
+// each writer fences its data, then adds; acquire: the reader's loads below
+// see the data behind the count it read).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Orders this thread's generic-proxy global accesses with its async-proxy
+// (TMA) ones: data written by plain stores and then read by a TMA load.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until *ctr reaches `target`, bounded like mbar_wait.
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target, volatile int* abort_flag,
+                                           uint32_t* status) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    __nanosleep(64);
+    if ((it & 15u) == 15u) {
+      if (*abort_flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_status(status, SBL_STATUS_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialisation may start before its predecessor on the stream finishes;

@@ -48,6 +48,7 @@ struct PackOut {
   // decode pack of patterns other than 2:4 (gemv != nullptr): kept codes per
   // block of 8, code bytes per lane and unit, unit bytes, units per row
   int gemv_n8, gemv_cb, gemv_unit_bytes, gemv_upr;
+  int gemv_code6;  // 2:4: the 6-bit group states instead of a byte per group
 };
 
 // mode 0: the whole preparation; 1: only the exact sum of |w| (SBL_SUM_WORDS
@@ -82,23 +83,28 @@ cudaError_t launch_act_dequant(const uint16_t* x, int64_t t, int64_t k, uint16_t
 
 // Forward GEMM + dequant.  sparse: codes = 2:4 kept values [n_out][k/2] and
 // meta = tensor-core metadata; dense: codes = W_eff int8 [n_out][k].
+// x_quantise (optional, bf16 [t][k], k <= 3072): the launch quantises the
+// activations itself, writing xq and a_prime before its GEMM reads them, with
+// forward_tile_counters(t) uint32 counters at `ready` (zeroed by this call).
 cudaError_t launch_forward_gemm(bool sparse, const int8_t* codes, const uint8_t* meta, int meta_kblocks,
                                 uint64_t meta_bytes, const int8_t* xq, const float* a_prime, const float* g, int64_t n_out, int64_t t,
                                 int64_t k, float* y, int32_t* acc_out, uint32_t* status, int num_sms,
-                                cudaStream_t s);
+                                cudaStream_t s, const uint16_t* x_quantise = nullptr, uint32_t* ready = nullptr);
+int64_t forward_tile_counters(int64_t t);
+constexpr int64_t kFusedActQuantMaxK = 3072;
 
 // Decode forward for 1 <= t <= 32 tokens over the decode pack (2:4: one byte
-// per group of four; other N:M: the interleaved compressed-index pack, see
-// gemv.cu).  For t up to 4 the kernel quantises the activations itself
+// per group of four, or with code6 a 6-bit state per group; other N:M: the
+// interleaved compressed-index pack, see gemv.cu).  For t up to 4 the kernel quantises the activations itself
 // (xq_out / ap_out, when given, receive the codes and scales); otherwise, or
 // when x is NULL, xq_in / ap_in hold the codes (the act-quant kernel runs
 // first with its early trigger).  gemv_fits() says whether the token rows fit
 // the kernel's shared memory.
-uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m);
-bool gemv_fits(int64_t t, int64_t k, int n, int m);
+uint64_t decode_pack_bytes(int64_t n_out, int64_t k, int n, int m, bool code6);
+bool gemv_fits(int64_t t, int64_t k, int n, int m, bool code6);
 bool gemv_preferred(int64_t t, int64_t n_out, int64_t k);
 bool gemv_fuses_act_quant(int64_t t);
-cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, const uint16_t* x, const int8_t* xq_in,
+cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, bool code6, const uint16_t* x, const int8_t* xq_in,
                                 const float* ap_in, const float* g, int64_t n_out, int64_t t, int64_t k, float* y,
                                 int32_t* acc_out, int8_t* xq_out, float* ap_out, uint32_t* status, int num_sms,
                                 cudaStream_t s);

@@ -34,6 +34,8 @@ NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 # layer flags
 SBL_PACK_GEMV = 1 << 0
 SBL_MASK_FROM_QUANT = 1 << 1
+SBL_PACK_GEMV_6BIT = 1 << 2
+SBL_FUSE_ACT_QUANT = 1 << 3
 # backward flags
 SBL_GRAD_F32 = 1 << 1
 SBL_NO_DX = 1 << 2

@@ -83,6 +83,24 @@ def gemv_bytes(layer):
     return full[:n_out, :k // 4], pad
 
 
+def gemv_code6(layer):
+    """The 6-bit 2:4 decode pack of a layer re-laid out as the oracle's
+    per-row streams [n_out, 3k/16] (units of 16 rows x 128 k, 384 bytes: word
+    j of slot 4 (row % 8) + t in plane j; a slot's 96 bits are the 48 of row r
+    for groups 8t..8t+7, then the 48 of row r + 8), plus every byte outside the
+    matrix."""
+    n_out, k = layer.n_out, layer.k
+    tiles, upr = (n_out + 15) // 16, (k + 127) // 128
+    L = layer.layout()
+    assert L.gemv_bytes == tiles * upr * 384
+    raw = section(layer, "gemv", int(L.gemv_bytes)).reshape(tiles, upr, 3, 32, 4)  # tile, unit, plane, slot, byte
+    slots = raw.transpose(0, 1, 3, 2, 4).reshape(tiles, upr, 8, 4, 2, 6)  # tile, unit, g, t, hi, byte
+    full = slots.transpose(0, 4, 2, 1, 3, 5).reshape(tiles * 16, upr * 24)
+    row_bytes = 3 * k // 16
+    pad = np.concatenate([full[n_out:].ravel(), full[:n_out, row_bytes:].ravel()])
+    return full[:n_out, :row_bytes], pad
+
+
 def decode_gemv(gb):
     """(meta nibble [n_out, k/4], code0, code1) from the 2-bit decode packing."""
     nib = (gb >> 4) & 0xF

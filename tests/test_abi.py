@@ -57,17 +57,19 @@ def test_version(lib):
 
 def test_layout_sections_are_aligned_and_disjoint(lib):
     g = sbl.SBL_PACK_GEMV
+    g6 = g | sbl.SBL_PACK_GEMV_6BIT
     for (n_out, k, n, m, flags) in [(6912, 2560, 2, 4, 0), (2560, 6912, 6, 8, 0), (264, 320, 2, 4, g),
                                     (8, 64, 1, 2, 0), (2560, 6912, 6, 8, g), (264, 320, 3, 8, g), (8, 64, 1, 2, g),
-                                    (136, 448, 8, 8, g)]:
+                                    (136, 448, 8, 8, g), (264, 320, 2, 4, g6), (6912, 2560, 2, 4, g6)]:
         L = sbl.prepared_layout(n_out, k, n, m, flags)
         spans = [("header", L.header, 4096), ("scratch", L.scratch, 1024 * 40 * 8 + 1024 * 32 + 256), ("mask", L.mask, n_out * k // m), ("weff_bf16", L.weff_bf16, 2 * n_out * k)]
         if (n, m) == (2, 4):
             spans += [("sp_values", L.sp_values, n_out * k // 2), ("sp_meta", L.sp_meta, L.sp_meta_bytes)]
             assert L.sp_meta_bytes == ((n_out + 255) // 256 * 256) * ((k + 255) // 256 * 256) // 8
             assert L.codes == 0
-            if flags & sbl.SBL_PACK_GEMV:
-                assert L.gemv_bytes == ((n_out + 15) // 16) * ((k + 127) // 128) * 512  # interleaved units
+            if flags & sbl.SBL_PACK_GEMV:  # interleaved units: a byte or 6 bits a group of four
+                unit = 384 if flags & sbl.SBL_PACK_GEMV_6BIT else 512
+                assert L.gemv_bytes == ((n_out + 15) // 16) * ((k + 127) // 128) * unit
         else:
             spans.append(("codes", L.codes, n_out * k))
             assert L.sp_values == 0 and L.sp_meta == 0
@@ -112,6 +114,13 @@ def test_forward_dispatch_query(lib):
     assert not uses(2560, 6912, 6, 8, 0, 1)
     assert not uses(6912, 2560, 2, 4, g, 0)
     assert not uses(6912, 2560, 6, 4, g, 1)     # not a valid layer
+    g6 = g | sbl.SBL_PACK_GEMV_6BIT
+    for t in (1, 4, 16, 32):
+        # its 4 KB table (against 16 KB for the byte pack) leaves room for 32 rows of k = 6912
+        assert uses(6912, 2560, 2, 4, g6, t) and uses(2560, 6912, 2, 4, g6, t)
+        assert uses(2560, 6912, 2, 4, g, t) == (t <= 16)
+    assert not uses(6912, 2560, 2, 4, g6, 33)
+    assert not uses(2560, 2560, 6, 8, g6, 1)     # the 6-bit code is a 2:4 pack only
 
 
 def test_backward_workspace_for_the_quantised_x_operand(lib):
@@ -139,6 +148,9 @@ def test_backward_workspace_for_the_quantised_x_operand(lib):
     ((250, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),
     ((0, 256, 2, 4, 0), sbl.SBL_ERR_SHAPE),
     ((256, 256, 2, 4, 1 << 9), sbl.SBL_ERR_INVALID_ARG),
+    ((256, 256, 2, 4, sbl.SBL_PACK_GEMV_6BIT), sbl.SBL_ERR_INVALID_ARG),  # needs the decode pack
+    ((256, 256, 6, 8, sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT), sbl.SBL_ERR_UNSUPPORTED_NM),
+    ((256, 256, 4, 8, sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT), sbl.SBL_ERR_UNSUPPORTED_NM),
 ])
 def test_layout_rejects_bad_arguments(lib, args, code):
     out = sbl.sbl_blob_layout()
@@ -147,8 +159,10 @@ def test_layout_rejects_bad_arguments(lib, args, code):
 
 
 def test_workspace_bytes(lib):
-    assert sbl.workspace_bytes(4096, 2560) == 4096 * 2560 + 4096 * 4
-    assert sbl.workspace_bytes(3, 64) == 256 + 256
+    # codes, scales, then one counter per 16 tokens, each piece 256-byte aligned
+    assert sbl.workspace_bytes(4096, 2560) == 4096 * 2560 + 4096 * 4 + 1024
+    assert sbl.workspace_bytes(3, 64) == 256 + 256 + 256
+    assert sbl.workspace_bytes(300, 64) == 19200 + 1280 + 256
     assert sbl.workspace_bytes(0, 64) == 0
 
 

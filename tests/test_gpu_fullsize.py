@@ -139,17 +139,45 @@ def test_fullsize_gradients_whole_arrays(name, n_out, k, n, m, t, f32):
     assert np.allclose(dw_ref[oi, ki], dwr, rtol=1e-12, atol=1e-12)
 
 
+def test_fullsize_fused_act_quant_forward():
+    """The prefill 2:4 workload (T = 4096, K = 2560, N_out = 6912) with the
+    activations quantised inside the GEMM launch: every code, scale,
+    accumulator and output."""
+    n_out, k, t = 6912, 2560, 4096
+    w_d = synth.master_weights(n_out, k, 0, device="cuda")
+    x_d = synth.activations(t, k, 1, device="cuda")
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_FUSE_ACT_QUANT)
+    sbl.prepare_weights(layer, w_d)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, x_d, t, y, xq, ap, acc, workspace=ws)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    ref = oracle.prepare(w_d.cpu(), 2, 4)
+    xq_ref, ap_ref = oracle.act_quant(x_d.cpu())
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    acc_full = (xq_ref.astype(np.float64) @ ref["weff"].astype(np.float64).T).astype(np.int32)
+    assert np.array_equal(acc.cpu().numpy(), acc_full)
+    y_ref = oracle.dequant(acc_full, ap_ref, ref["g"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), y_ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("t", [1, 4, 16, 32])
 @pytest.mark.parametrize("n_out", [2560, 6912])
-@pytest.mark.parametrize("n,m", [(2, 4), (6, 8)])
-def test_decode_gemv_fullsize(t, n_out, n, m):
+@pytest.mark.parametrize("n,m,flags", [(2, 4, sbl.SBL_PACK_GEMV), (6, 8, sbl.SBL_PACK_GEMV),
+                                       (2, 4, sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT)])
+def test_decode_gemv_fullsize(t, n_out, n, m, flags):
     """The decode workload (k = 2560, n_out 2560 or 6912) through the decode
-    kernel, 2:4 on its 2-bit pack and 6:8 on the compressed-index pack: every
-    accumulator and output, bit for bit."""
+    kernel, 2:4 on its 2-bit pack or its 6-bit group code and 6:8 on the
+    compressed-index pack: every accumulator and output, bit for bit."""
     k = 2560
     w_d = synth.master_weights(n_out, k, 10, device="cuda")
     x_d = synth.activations(t, k, 11, device="cuda")
-    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
+    layer = sbl.Layer.allocate(n_out, k, n, m, flags)
     assert sbl.forward_uses_gemv(layer, t)
     sbl.prepare_weights(layer, w_d)
     y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")

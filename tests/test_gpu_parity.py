@@ -34,7 +34,7 @@ def _close(gpu, ref, rtol=RTOL, atol=ATOL):
 
 
 def _check_prepared(layer, w, n, m):
-    ref = oracle.prepare(w, n, m)
+    ref = oracle.prepare(w, n, m, mask_from_codes=bool(layer.flags & sbl.SBL_MASK_FROM_QUANT))
     gamma, g, status = bd.header_scalars(layer)
     assert status == 0
     assert np.float32(gamma).view(np.uint32) == np.float32(ref["gamma"]).view(np.uint32)
@@ -47,7 +47,11 @@ def _check_prepared(layer, w, n, m):
         canon, pad_rows, pad_cols = bd.sp_meta_canonical(layer)
         assert np.array_equal(canon, meta)
         assert (pad_rows == 0x44).all() and (pad_cols == 0x44).all()
-        if layer.flags & sbl.SBL_PACK_GEMV:
+        if layer.flags & sbl.SBL_PACK_GEMV_6BIT:
+            got, pad = bd.gemv_code6(layer)
+            assert not pad.any(), "bytes outside the matrix must be zero"
+            assert np.array_equal(got, oracle.pack24_code6(ref["weff"], ref["mask"]))
+        elif layer.flags & sbl.SBL_PACK_GEMV:
             gb, pad = bd.gemv_bytes(layer)
             assert not pad.any(), "bytes outside the matrix must be zero"
             nib, c0, c1 = bd.decode_gemv(gb)
@@ -710,14 +714,14 @@ def test_decode_dispatch_both_paths_bit_exact(t):
 NM_PATTERNS = [(6, 8), (4, 8), (3, 8), (1, 8), (2, 8), (5, 8), (7, 8), (8, 8), (1, 4), (3, 4), (4, 4), (1, 2), (2, 2)]
 
 
-def _decode_check(n_out, k, n, m, t, seed, with_codes=True):
+def _decode_check(n_out, k, n, m, t, seed, with_codes=True, flags=sbl.SBL_PACK_GEMV):
     """Prepare with the decode pack (its bytes checked against the oracle's
     pack), run sbl_forward at t tokens through the decode kernel and compare
     the int32 accumulators and y bit for bit (and the codes and scales it
     hands back)."""
     w = synth.master_weights(n_out, k, seed)
     x = synth.activations(t, k, seed + 1)
-    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_PACK_GEMV)
+    layer = sbl.Layer.allocate(n_out, k, n, m, flags)
     sbl.prepare_weights(layer, _dev(w))
     torch.cuda.synchronize()
     ref = _check_prepared(layer, w, n, m)
@@ -759,6 +763,107 @@ def test_decode_smallest_layer(n, m, t):
     """The smallest layer the library takes (8 rows, k = 64): half a row tile
     and half a k unit, every other lane's weights padding."""
     _decode_check(8, 64, n, m, t, seed=760 + 8 * n + m + t)
+
+
+CODE6 = sbl.SBL_PACK_GEMV | sbl.SBL_PACK_GEMV_6BIT
+
+
+@pytest.mark.parametrize("n_out,k", [(136, 448), (8, 64), (264, 320)])
+@pytest.mark.parametrize("t", [1, 3, 4, 5, 8, 9, 16, 32])
+def test_decode_6bit_code(n_out, k, t):
+    """2:4 layers with the 6-bit group code: the pack matches the oracle's
+    streams and the decode kernel's accumulators and y match bit for bit, on
+    ragged row tiles and half k units."""
+    _decode_check(n_out, k, 2, 4, t, seed=1200 + n_out + t, flags=CODE6)
+
+
+@pytest.mark.parametrize("n_out,k,t", [(11200, 640, 4), (11200, 640, 20), (16, 16384, 1), (16, 10240, 9)])
+def test_decode_6bit_code_many_tiles_and_long_rows(n_out, k, t):
+    _decode_check(n_out, k, 2, 4, t, seed=1300 + t, with_codes=False, flags=CODE6)
+
+
+def test_decode_6bit_code_under_the_mask_from_codes_ablation():
+    _decode_check(264, 320, 2, 4, 3, seed=1310, flags=CODE6 | sbl.SBL_MASK_FROM_QUANT)
+
+
+FUSED_CASES = [
+    # n_out, k, n, m, t
+    (264, 320, 2, 4, 300),     # two 240-token tiles, the second ragged
+    (256, 256, 2, 4, 16),
+    (8, 64, 2, 4, 5),
+    (520, 192, 1, 4, 33),
+    (136, 448, 6, 8, 77),
+    (384, 512, 8, 8, 260),
+    (200, 128, 1, 2, 50),
+    (264, 3072, 2, 4, 481),    # the longest rows the launch quantises itself
+    (512, 1024, 4, 8, 1000),   # dense tiles of 192 or 256 tokens
+]
+
+
+@pytest.mark.parametrize("n_out,k,n,m,t", FUSED_CASES)
+def test_fused_act_quant_forward(n_out, k, n, m, t):
+    """SBL_FUSE_ACT_QUANT: one launch quantises the activations and runs the
+    GEMM; codes, scales, accumulators and y match the oracle bit for bit."""
+    w = synth.master_weights(n_out, k, 1400 + n_out + t)
+    x = synth.activations(t, k, 1401 + t)
+    layer = sbl.Layer.allocate(n_out, k, n, m, sbl.SBL_FUSE_ACT_QUANT)
+    sbl.prepare_weights(layer, _dev(w))
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    ws = torch.full((sbl.workspace_bytes(t, k),), 0x5A, dtype=torch.uint8, device="cuda")  # stale counters
+    c0 = sbl.launch_count()
+    sbl.forward(layer, _dev(x), t, y, xq, ap, acc, workspace=ws)
+    launched = sbl.launch_count() - c0
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    assert launched == 1  # the GEMM launch alone
+    ref = oracle.forward(w, x, n, m)
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+    # the codes in the workspace path too, and again over the counters it left
+    y2 = torch.empty_like(y)
+    for _ in range(2):
+        sbl.forward(layer, _dev(x), t, y2, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+
+
+def test_fused_act_quant_falls_back_without_a_workspace_or_on_long_rows():
+    """Without a workspace (explicit code buffers) or with rows longer than
+    3072 the flag leaves the two-launch path in place; same bits."""
+    for (n_out, k, t, use_ws) in ((256, 512, 40, False), (256, 3584, 40, True)):
+        w = synth.master_weights(n_out, k, 1450 + k)
+        x = synth.activations(t, k, 1451)
+        layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_FUSE_ACT_QUANT)
+        sbl.prepare_weights(layer, _dev(w))
+        y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+        xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+        ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+        ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda") if use_ws else None
+        c0 = sbl.launch_count()
+        sbl.forward(layer, _dev(x), t, y, xq, ap, workspace=ws)
+        assert sbl.launch_count() - c0 == 2
+        torch.cuda.synchronize()
+        ref = oracle.forward(w, x, 2, 4)
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+
+
+def test_fused_act_quant_flags_nonfinite_activations():
+    n_out, k, t = 256, 2560, 300
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_FUSE_ACT_QUANT)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 1460)))
+    x = synth.activations(t, k, 1461)
+    x[250, 7] = float("nan")
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, workspace=ws)
+    code, bits = sbl.read_status(layer)
+    assert code == sbl.SBL_ERR_NONFINITE and bits & sbl.SBL_STATUS_NONFINITE_X
 
 
 @pytest.mark.parametrize("t,k", [(1, 2560), (3, 2560), (9, 2560), (2, 6912)])
