@@ -586,6 +586,59 @@ def bench_nm_sweep(dev, peaks, steps=10):
             "timing": f"CUDA events around each phase, mean of {steps} steps after 3", "points": out}
 
 
+def bench_fused_act_quant(dev, steps=40, reps=4):
+    """A/B of SBL_FUSE_ACT_QUANT on the prefill 2:4 step (T=4096, K=2560,
+    N_out=6912): the same step (prepare, forward, backward) with the
+    activations quantised by their own kernel or inside the GEMM launch,
+    alternated `reps` times on the same inputs; medians of the per-step time
+    and of the prepare + forward part."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    T, K, N = 4096, 2560, 6912
+    sets = [(synth.master_weights(N, K, 40 + 10 * r, device=dev), synth.activations(T, K, 41 + 10 * r, device=dev),
+             synth.upstream_grad(T, N, 42 + 10 * r, device=dev)) for r in range(ROTATE)]
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    arms = {"separate kernel": 0, "inside the GEMM launch": sbl.SBL_FUSE_ACT_QUANT}
+    layers = {name: sbl.Layer.allocate(N, K, 2, 4, f, device=dev) for name, f in arms.items()}
+    step_us = {name: [] for name in arms}
+    fwd_us = {name: [] for name in arms}
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(steps):
+            fn(i)
+        b.record()
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / steps * 1e3
+
+    for _ in range(reps):
+        for name, L in layers.items():
+            def prep_fwd(i, L=L):
+                w, x, _ = sets[i % ROTATE]
+                sbl.prepare_weights(L, w)
+                sbl.forward(L, x, T, y, workspace=ws)
+
+            def step(i, L=L):
+                prep_fwd(i)
+                sbl.backward(L, sets[i % ROTATE][1], sets[i % ROTATE][2], T, dx, dw, 0)
+
+            for i in range(3):
+                step(i)
+            step_us[name].append(timed(step))
+            fwd_us[name].append(timed(prep_fwd))
+            code, bits = sbl.read_status(L)
+            assert code == sbl.SBL_OK, (code, bits)
+    return {"workload": "prefill 2:4 step, T=4096, K=2560, N_out=6912", "steps_per_rep": steps, "reps": reps,
+            "arms": {name: {"step_us": statistics.median(step_us[name]), "prepare_forward_us":
+                            statistics.median(fwd_us[name]), "step_us_each": step_us[name]} for name in arms}}
+
+
 def bench_ablations(dev, steps=10):
     """The pages' ablations and the STE reading variant as flags, on the
     prefill 2:4 workload: the plain step, the mask from the ternary codes
@@ -1124,6 +1177,7 @@ def main():
         line["train_step"] = [bench_train_step(dev, peaks, 2, 4), bench_train_step(dev, peaks, 4, 8)]
         line["nm_sweep"] = bench_nm_sweep(dev, peaks)
         line["ablations"] = bench_ablations(dev)
+        line["fused_act_quant_ab"] = bench_fused_act_quant(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T, K, N, n, m)
     if rank == 0:
