@@ -896,7 +896,33 @@ def profile_grouped_prepare():
     torch.cuda.synchronize()
 
 
-PROFILE_CASES = {"decode": profile_decode, "prefill68": profile_prefill68, "grouped_prepare": profile_grouped_prepare}
+def profile_prefill24():
+    """The prefill 2:4 step (T = 4096, K = 2560, N_out = 6912, the benchmark's
+    seeds): prepare, forward (act-quant and 2:4 GEMM) and backward, three steps
+    on one input set: twelve launches."""
+    import torch
+
+    from sparse_linear_layers_bitlinear_b200 import sbl, synth
+
+    dev = torch.device("cuda", 0)
+    T, K, N = WORKLOAD["tokens"], WORKLOAD["k"], WORKLOAD["n_out"]
+    w = synth.master_weights(N, K, 0, device=dev)
+    x = synth.activations(T, K, 1, device=dev)
+    dy = synth.upstream_grad(T, N, 2, device=dev)
+    L = sbl.Layer.allocate(N, K, 2, 4, device=dev)
+    y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbl.workspace_bytes(T, K), dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        sbl.prepare_weights(L, w)
+        sbl.forward(L, x, T, y, workspace=ws)
+        sbl.backward(L, x, dy, T, dx, dw, 0)
+    torch.cuda.synchronize()
+
+
+PROFILE_CASES = {"decode": profile_decode, "prefill68": profile_prefill68, "grouped_prepare": profile_grouped_prepare,
+                 "prefill24": profile_prefill24}
 
 
 # ---------------------------------------------------------------------------
