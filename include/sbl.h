@@ -254,6 +254,19 @@ sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* 
 sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const float* xscale, int64_t t, float* y,
                                  int32_t* acc_debug, sbl_stream_t stream);
 
+/* Step 4's activation quantisation alone: x (bf16 [t, k]) -> xq_out (int8
+ * [t, k]) and xscale_out (fp32 [t], the a'_i), the same bits sbl_forward
+ * computes, for sbl_forward_quantized later (e.g. on another stream, ahead of
+ * the layer's weight preparation).  A non-finite activation ORs
+ * SBL_STATUS_NONFINITE_X into *status_dev (a caller-owned device uint32, not
+ * the layer's word, so that a prepare of the layer does not clear it).
+ * Errors: SBL_ERR_SHAPE (k not a multiple of 64 in 64..131072, t out of
+ * range), SBL_ERR_INVALID_ARG (a NULL pointer when t > 0), SBL_ERR_ALIGN
+ * (x, xq_out, xscale_out not 16-byte aligned, status_dev not 4-byte
+ * aligned), SBL_ERR_DEVICE, SBL_ERR_CUDA. */
+sbl_status sbl_quantize_activations(const void* x, int64_t t, int64_t k, int8_t* xq_out, float* xscale_out,
+                                    uint32_t* status_dev, sbl_stream_t stream);
+
 /* 1 when sbl_forward on this layer with t tokens takes the decode kernel
  * over the decode pack, 0 when it takes a tensor-core GEMM (or the arguments
  * are invalid).  Host only, no device access. */

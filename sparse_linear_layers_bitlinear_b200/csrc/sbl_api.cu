@@ -314,6 +314,22 @@ sbl_status sbl_forward_quantized(const sbl_layer* layer, const int8_t* xq, const
   return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
 }
 
+sbl_status sbl_quantize_activations(const void* x, int64_t t, int64_t k, int8_t* xq_out, float* xscale_out,
+                                    uint32_t* status_dev, sbl_stream_t stream) {
+  if (t < 0 || t > (int64_t(1) << 30) || k < 64 || k % 64 != 0 || k > kMaxK) return SBL_ERR_SHAPE;
+  if (t == 0) return SBL_OK;
+  if (x == nullptr || xq_out == nullptr || xscale_out == nullptr || status_dev == nullptr) return SBL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq_out) || !aligned16(xscale_out) || (reinterpret_cast<uintptr_t>(status_dev) & 3u))
+    return SBL_ERR_ALIGN;
+  int sms = 0;
+  const sbl_status st = current_device(&sms);
+  if (st != SBL_OK) return st;
+  return launch_act_quant(static_cast<const uint16_t*>(x), t, k, xq_out, xscale_out, status_dev, sms,
+                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SBL_OK
+             : SBL_ERR_CUDA;
+}
+
 size_t sbl_backward_workspace_bytes(int64_t t, int64_t k, uint32_t flags) {
   if (t <= 0 || k <= 0 || (flags & SBL_NO_DW) || !(flags & SBL_DW_QUANT_X)) return 0;
   return size_t(t) * size_t(k) * 2;

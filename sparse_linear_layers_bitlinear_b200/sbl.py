@@ -90,6 +90,7 @@ SIGNATURES = {
     "sbl_read_scale": (_I32, [_LP, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "sbl_selftest_wait_timeout": (_I32, [_P, _U64, _P]),
     "sbl_selftest_chain_floor": (_I32, [_I32, _P]),
+    "sbl_quantize_activations": (_I32, [_P, _I64, _I64, _P, _P, _P, _P]),
     "sbl_selftest_mma_rate": (_I32, [_I32, _I32, _I32, _P, ctypes.POINTER(ctypes.c_int64), _P]),
     "sbl_version": (ctypes.c_char_p, []),
     "sbl_launch_count": (ctypes.c_uint64, []),
@@ -254,6 +255,13 @@ def forward_quantized(layer: Layer, xq, xscale, t: int, y, acc_debug=None, strea
     cl = layer.c()
     _check(lib().sbl_forward_quantized(ctypes.byref(cl), _ptr(xq), _ptr(xscale), t, _ptr(y), _ptr(acc_debug),
                                        _stream(stream)), "sbl_forward_quantized")
+
+
+def quantize_activations(x, t: int, k: int, xq, xscale, status, stream=None):
+    """sbl_quantize_activations: the forward's activation codes and scales
+    alone; `status` is a device int32 tensor that receives the non-finite bit."""
+    _check(lib().sbl_quantize_activations(_ptr(x), t, k, _ptr(xq), _ptr(xscale), _ptr(status), _stream(stream)),
+           "sbl_quantize_activations")
 
 
 def forward_noalloc(layer: Layer, x, t: int, y, acc_debug=None, stream=None):

@@ -186,6 +186,14 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 0, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_backward(ctypes.byref(layer), None, None, 4, None, None, 1 << 7, None) == sbl.SBL_ERR_INVALID_ARG
     assert lib.sbl_selftest_wait_timeout(None, 1000, None) == sbl.SBL_ERR_INVALID_ARG
+    q = lib.sbl_quantize_activations
+    P = ctypes.c_void_p
+    assert q(P(0x1000), 4, 100, P(0x2000), P(0x3000), P(0x4000), None) == sbl.SBL_ERR_SHAPE
+    assert q(P(0x1000), -1, 128, P(0x2000), P(0x3000), P(0x4000), None) == sbl.SBL_ERR_SHAPE
+    assert q(None, 0, 128, None, None, None, None) == sbl.SBL_OK
+    assert q(P(0x1000), 4, 128, P(0x2000), P(0x3000), None, None) == sbl.SBL_ERR_INVALID_ARG
+    assert q(P(0x1008), 4, 128, P(0x2000), P(0x3000), P(0x4000), None) == sbl.SBL_ERR_ALIGN
+    assert q(P(0x1000), 4, 128, P(0x2000), P(0x3000), P(0x4002), None) == sbl.SBL_ERR_ALIGN
     st = ctypes.c_void_p(0x5000)
     for kind, stages, pairs, status in ((3, 16, 1, st), (-1, 16, 1, st), (0, 0, 1, st), (0, (1 << 20) + 1, 1, st),
                                         (0, 16, 0, st), (0, 16, 1, None)):

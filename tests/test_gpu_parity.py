@@ -833,6 +833,36 @@ def test_fused_act_quant_forward(n_out, k, n, m, t):
         assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
 
 
+@pytest.mark.parametrize("t,k", [(300, 2560), (33, 6912), (5, 64), (4096, 2560)])
+def test_quantize_activations_alone_then_forward_from_codes(t, k):
+    """sbl_quantize_activations gives the oracle's codes and scales; the
+    forward from them gives sbl_forward's y; a NaN sets the caller's word."""
+    x = synth.activations(t, k, 1480 + t)
+    xq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    ap = torch.empty((t,), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sbl.quantize_activations(_dev(x), t, k, xq, ap, status)
+    torch.cuda.synchronize()
+    xq_ref, ap_ref = oracle.act_quant(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(ap.cpu().numpy().view(np.uint32), ap_ref.view(np.uint32))
+    assert int(status.item()) == 0
+    n_out = 256
+    layer = sbl.Layer.allocate(n_out, k, 2, 4)
+    sbl.prepare_weights(layer, _dev(synth.master_weights(n_out, k, 1481)))
+    y1 = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    y2 = torch.empty_like(y1)
+    sbl.forward_quantized(layer, xq, ap, t, y1)
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y2, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+    x[t // 2, k - 1] = float("nan")
+    sbl.quantize_activations(_dev(x), t, k, xq, ap, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & sbl.SBL_STATUS_NONFINITE_X
+
+
 def test_fused_act_quant_falls_back_without_a_workspace_or_on_long_rows():
     """Without a workspace (explicit code buffers) or with rows longer than
     3072 the flag leaves the two-launch path in place; same bits."""
