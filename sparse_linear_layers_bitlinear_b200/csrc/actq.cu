@@ -18,7 +18,7 @@
 // Launched with programmatic stream serialisation: its launch overlaps the
 // kernel before it, and it waits for that kernel (which may have written x,
 // or reset the status word) before it reads anything.  With early_trigger it
-// then lets the next kernel (the decode GEMV) launch at once.
+// then lets the next kernel (the GEMM or the decode kernel) launch at once.
 //
 // DEQ = true is the same pass writing the dequantised activations
 // xhat = RN_bf16(xq * a' / 127) instead of the codes: the dW operand of the

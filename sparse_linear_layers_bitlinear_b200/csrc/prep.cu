@@ -818,7 +818,7 @@ __device__ __forceinline__ void prepare_body(const PrepArgs& a, const int G, con
         }
         weff_c[u] = make_uint4(weff[0], weff[1], weff[2], weff[3]);
         if (codes_c != nullptr) codes_c[u] = make_uint2(codes_of_high_bytes(hb_lo), codes_of_high_bytes(hb_hi));
-        if (M == 4 && spv_c != nullptr) {  // 2:4: kept values, metadata, optional GEMV bytes
+        if (M == 4 && spv_c != nullptr) {  // 2:4: kept values, metadata, optional decode pack
           const uint32_t vals = codes_of_high_bytes(__byte_perm(hb_lo, hb_hi, W));  // the kept codes, index order
           spv_c[u] = vals;
           // tensor-core metadata: [row_block][k_block][128 rows][16 bytes];
