@@ -657,9 +657,20 @@ cudaError_t launch_forward_gemv(const uint8_t* gemv, int n, int m, bool code6, c
   const int fmt = decode_fmt(n, m, code6), nt = decode_nt(t);
   // codes from the caller (x == NULL), else quantised here for few tokens
   const bool fused = x != nullptr && gemv_fuses_act_quant(t);
-  // As many blocks as fit two per SM; each takes an equal run of tiles.
+  // Each block takes an equal run of tiles.  Up to 8 tokens, as many blocks
+  // as fit two per SM: a call is a short chain, and more blocks split the
+  // weight stream over more warps.  From 9 tokens, one block per SM while
+  // that leaves at most three tiles a block (two above 16 tokens, where a
+  // tile's products weigh more): every block stages all t rows of codes, so
+  // fewer blocks stage fewer bytes.
+  // Measured per call in a graph (K = 2560), one against two blocks per SM:
+  // t = 16 at 2560 rows 5.65 against 5.85-6.35 us, at 6912 rows 6.72 against
+  // 7.17-7.46; t = 32 at 2560 rows 7.3 against 8.4-9.0; t = 32 at 6912 rows
+  // (three tiles a block) 11.6-12.4 against 10.5-11.0; t = 1 at 6912 rows
+  // 5.37 against 4.78.
   const size_t smem1 = decode_smem(fmt, nt, t, k, 1);
-  const int per_sm = smem1 * 2 + 2048 <= 228 * 1024 ? 2 : 1;
+  int per_sm = smem1 * 2 + 2048 <= 228 * 1024 ? 2 : 1;
+  if (t > 8 && a.tiles <= (t <= 16 ? 3 : 2) * num_sms) per_sm = 1;
   int tpb = (a.tiles + num_sms * per_sm - 1) / (num_sms * per_sm);
   while (decode_smem(fmt, nt, t, k, tpb) > kDecMaxSmem && tpb > 1) --tpb;
   const size_t smem = decode_smem(fmt, nt, t, k, tpb);
