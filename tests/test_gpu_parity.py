@@ -883,6 +883,28 @@ def test_fused_act_quant_falls_back_without_a_workspace_or_on_long_rows():
         assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
 
 
+@pytest.mark.parametrize("t", [3, 40, 300])
+def test_fused_act_quant_with_the_decode_pack(t):
+    """A layer with both SBL_FUSE_ACT_QUANT and SBL_PACK_GEMV: decode-sized
+    calls take the decode kernel, larger ones the GEMM that quantises in its
+    own launch; the same bits either way."""
+    n_out, k = 264, 1024
+    w = synth.master_weights(n_out, k, 1470)
+    x = synth.activations(t, k, 1471 + t)
+    layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_FUSE_ACT_QUANT | sbl.SBL_PACK_GEMV)
+    sbl.prepare_weights(layer, _dev(w))
+    assert sbl.forward_uses_gemv(layer, t) == (t <= 32)
+    y = torch.empty((t, n_out), dtype=torch.float32, device="cuda")
+    acc = torch.empty((t, n_out), dtype=torch.int32, device="cuda")
+    ws = torch.empty(sbl.workspace_bytes(t, k), dtype=torch.uint8, device="cuda")
+    sbl.forward(layer, _dev(x), t, y, acc_debug=acc, workspace=ws)
+    torch.cuda.synchronize()
+    assert sbl.read_status(layer)[0] == sbl.SBL_OK
+    ref = oracle.forward(w, x, 2, 4)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), ref["y"].view(np.uint32))
+
+
 def test_fused_act_quant_flags_nonfinite_activations():
     n_out, k, t = 256, 2560, 300
     layer = sbl.Layer.allocate(n_out, k, 2, 4, sbl.SBL_FUSE_ACT_QUANT)
