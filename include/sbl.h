@@ -32,13 +32,16 @@
  *  - The caller owns and allocates every buffer (cudaMalloc, torch, ...).  The
  *    library allocates no device memory and keeps no state between calls.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
- *    stream).  Calls do not synchronise, except sbl_read_status.
+ *    stream).  Calls do not synchronise, except sbl_read_status and
+ *    sbl_read_scale (and the first sbl_forward_noalloc on a device, see
+ *    there).
  *  - Arguments are validated before anything is enqueued; a rejected call
  *    returns an error code and enqueues nothing.
  *  - Errors that only the device can see (non-finite inputs, a bounded wait
  *    that ran out) are OR-ed into the status word inside the prepared blob and
- *    reported by sbl_read_status.  Outputs of a call that raised a device
- *    error are unspecified.
+ *    reported by sbl_read_status (sbl_quantize_activations and the self tests
+ *    take a caller-owned status word instead).  Outputs of a call that raised
+ *    a device error are unspecified.
  */
 #ifndef SBL_H
 #define SBL_H
@@ -240,7 +243,10 @@ sbl_status sbl_prepare_weights_from_sum(const sbl_layer* layer, const void* w_ma
  * pack instead for t <= 32 tokens, when that many token rows of k codes fit
  * the kernel's shared memory (sbl_forward_uses_gemv says which path a call
  * takes); for t <= 4 the decode kernel also quantises the activations
- * itself, so the call is one launch.  The outputs are the same bits on every
+ * itself, so the call is one launch.  On the GEMM path a layer with
+ * SBL_FUSE_ACT_QUANT quantises inside the GEMM's launch when the call passes
+ * a workspace and k <= 3072 (the workspace's counters are used even when
+ * xq_out and xscale_out are given).  The outputs are the same bits on every
  * path. */
 sbl_status sbl_forward(const sbl_layer* layer, const void* x, int64_t t, float* y, int8_t* xq_out,
                        float* xscale_out, int32_t* acc_debug, void* workspace, sbl_stream_t stream);
