@@ -667,3 +667,72 @@ def test_grad_w_quant_x_uses_the_dequantised_operand():
     assert np.allclose(dw_q, ref, rtol=1e-12, atol=1e-12)
     # and it is not the raw-X gradient
     assert not np.allclose(dw_q, oracle.grad_w(dy, x), rtol=1e-4, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# Property checks over random small cases (hypothesis): the packs decode back
+# to W_eff whatever the pattern, shape and codes, and the mask keeps the
+# largest magnitudes.
+# ---------------------------------------------------------------------------
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+_NM = [(1, 2), (2, 2), (1, 4), (2, 4), (3, 4), (4, 4), (1, 8), (2, 8), (3, 8), (4, 8), (5, 8), (6, 8), (7, 8), (8, 8)]
+
+
+@st.composite
+def _masked_codes(draw):
+    n, m = draw(st.sampled_from(_NM))
+    rows = draw(st.integers(1, 4))
+    k = 64 * draw(st.integers(1, 2))
+    seed = draw(st.integers(0, 2**31 - 1))
+    rng = np.random.default_rng(seed)
+    mask = np.zeros((rows, k // m), dtype=np.uint8)
+    for r in range(rows):
+        for g in range(k // m):
+            for j in rng.choice(m, size=n, replace=False):
+                mask[r, g] |= 1 << int(j)
+    codes = rng.integers(-1, 2, size=(rows, k)).astype(np.int8)
+    keep = np.unpackbits(mask[..., None], axis=-1, bitorder="little")[..., :m].reshape(rows, k).astype(bool)
+    return n, m, np.where(keep, codes, 0).astype(np.int8), mask
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(_masked_codes())
+def test_pack_nm_round_trip_on_random_masks(case):
+    n, m, weff, mask = case
+    masks8, codes = oracle.pack_nm(weff, mask, n, m)
+    assert np.array_equal(_unpack_nm(masks8, codes, n, m, weff.shape[1]), weff)
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(_masked_codes().filter(lambda c: (c[0], c[1]) == (2, 4)))
+def test_pack24_code6_round_trip_on_random_masks(case):
+    _, _, weff, mask = case
+    back, masks = _unpack_code6(oracle.pack24_code6(weff, mask), weff.shape[1])
+    assert np.array_equal(back, weff) and np.array_equal(masks, mask)
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(st.sampled_from(_NM), st.integers(0, 2**31 - 1))
+def test_mask_keeps_the_largest_magnitudes(nm, seed):
+    """Every kept magnitude is at least every dropped one in its group, and a
+    drop of an equal magnitude only happens to a higher index (ties to the
+    lowest index)."""
+    n, m = nm
+    rng = np.random.default_rng(seed)
+    k = 64
+    # few distinct magnitudes, so that ties are common
+    w = (rng.integers(-3, 4, size=(2, k)) * 0.25).astype(np.float32)
+    wb = synth.bits(torch.from_numpy(w).to(torch.bfloat16))
+    mask = oracle.nm_mask(wb, n, m)
+    mags = np.abs(w)
+    for r in range(2):
+        for g in range(k // m):
+            bits = [(int(mask[r, g]) >> j) & 1 for j in range(m)]
+            assert sum(bits) == n
+            for a in range(m):
+                for b in range(m):
+                    if bits[a] and not bits[b]:
+                        ma, mb = mags[r, g * m + a], mags[r, g * m + b]
+                        assert ma > mb or (ma == mb and a < b)
